@@ -1,0 +1,534 @@
+"""Benchmark of the quantized-KV decode step (KVQuant hot path) on B200.
+
+One step = for every layer: quantize-append one new token (K and V) into the
+3-bit cache, then decode attention of one query per sequence over the whole
+cache (QK with NUQ lookup + RoPE + key outliers, split-K softmax merge, PV with
+value outliers).  Default workload: LLaMA-7B shape, 32 layers x 32 heads x
+head_dim 128, 1,048,576 cached tokens, batch 1, 3-bit NUQ, 0.5% outliers,
+synthetic seeded inputs.  Prints one JSON line (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KV tokens/s in quantized decode attention; achieved HBM GB/s vs peak"
+UNIT = "KV tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=30)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--workload", default="llama7b_1m_32layers")
+    p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    p.add_argument("--splits", type=int, default=0)
+    p.add_argument("--path", default="split", choices=["split", "fused"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-fp16", action="store_true")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def src_hash(kernel_file):
+    with open(os.path.join(ROOT, "long_context_decode_nuq_b200", "csrc", kernel_file), "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()[:16]
+
+
+def traffic_for(kernel, units):
+    """Per-launch DRAM bytes from the committed ncu summary, if the kernel is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        d = json.load(fh)
+    e = d.get(kernel)
+    if not e or e.get("src_sha") != src_hash(e["file"]):
+        return None
+    return e["dram_bytes_per_unit"] * units
+
+
+# ----------------------------------------------------------------------------- algorithmic bytes
+
+def bytes_model(w, T, kcount, vcount, path):
+    """Algorithmic bytes of one layer's decode (attention part) over T tokens.
+
+    Key side (QK): packed key codes, key-outlier entries (4 B position + 2 B value),
+    key chunk pointers; value side (PV): packed value codes, value-outlier entries,
+    value token params (8 B/token), value chunk pointers.  The split path also
+    writes and reads fp32 logits (4 B per token per query head, each way).
+    """
+    code_row = w.Hkv * w.D * w.bits // 8
+    nch = (T + 63) // 64 + 1
+    k_bytes = T * code_row + 6 * kcount + 4 * nch
+    v_bytes = T * code_row + 6 * vcount + 8 * T + 4 * nch
+    logit = 4 * w.Hq * T
+    if path == "split":
+        return {"qk": k_bytes + logit, "pv": v_bytes + logit, "total": k_bytes + v_bytes + 2 * logit}
+    return {"attn": k_bytes + v_bytes, "total": k_bytes + v_bytes}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def cpu_oracle_sample(w, budget_s=12.0, layer=0):
+    """Time the CPU oracle's decode (dequantize + binary64 attention) on a bounded
+    sample of the workload: one layer, all heads, T_s tokens; returns KV tokens/s."""
+    import oracle as O
+    import synth
+    T_s = 1024 if w.Hkv >= 16 else 4096
+    ws = synth.workload(w.name, B=1, T=T_s)
+    idx = (np.zeros((1, 1, 1, 1), dtype=np.int64), np.arange(T_s)[None, :, None, None],
+           np.arange(w.Hkv)[None, None, :, None], np.arange(w.D)[None, None, None, :])
+    K16 = synth.gen_k(ws, layer, *idx)
+    V16 = synth.gen_v(ws, layer, *idx)
+    cbK = O.fit_codebook(synth.codebook_samples_k(ws, layer), w.f, w.bits)
+    cbV = O.fit_codebook(synth.codebook_samples_v(ws, layer), w.f, w.bits)
+    c = O.QuantizedCache(1, w.Hkv, w.bits, T_s, w.f, T_s * w.Hkv * w.D, T_s * w.Hkv * w.D)
+    c.prefill(K16, V16, [T_s], cbK, cbV)
+    q = synth.gen_q(ws, layer)[0]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        Kh, Vh = c.dequantize(0, cbK, cbV)
+        O.decode_attention(q, T_s, Kh, Vh, w.rope_theta)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return reps * T_s / el, f"1 layer x {w.Hkv} kv heads x {T_s} tokens, {reps} repetitions, {el:.1f} s"
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((i.get("num_threads", 1) for i in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import synth
+    w = synth.workload(args.workload)
+    steps_t = []
+    samples = []
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, budget_s=2.0)
+    for _ in range(args.steps):
+        v, smp = cpu_oracle_sample(w, budget_s=4.0)
+        steps_t.append(v)
+        samples.append(smp)
+    val = statistics.median(steps_t)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Philox4x32-10, LLaMA-shaped)",
+        "config": {"workload": w.name, "layers": w.layers, "B": w.B, "kv_heads": w.Hkv,
+                   "head_dim": w.D, "T": w.T, "bits": w.bits, "outlier_frac": w.f},
+        "cpu_baseline": {"value": val, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": samples[-1]},
+        "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_kvq(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    import long_context_decode_nuq_b200 as K
+    import synth
+    from synth.gpu import DeviceGen
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    w = synth.workload(args.workload)
+    steps_total = args.warmup + args.steps
+    if w.T + steps_total + 16 > w.T_gen:
+        w = synth.workload(args.workload, appends=1, steps=steps_total + 16)
+    layers = w.layers
+    T0 = w.T
+    e2e_steps = min(args.steps, 10)
+    T_max = T0 + steps_total + e2e_steps + 64
+    kout_cap = int(T_max * max(w.f * w.n * 1.5, 4) + 4096)
+    vout_cap = int(T_max * (2 * math.floor(w.f * w.n / 2 + 0.5) + 2) + 4096)
+    cfg = K.make_cfg(w.B, w.Hq, w.Hkv, w.bits, T_max, w.f, w.rope_theta, kout_cap, vout_cap)
+    # a different synthetic sequence per rank (weak scaling): layer key offset by rank
+    layer_key = lambda l: l + 4096 * rank  # noqa: E731
+
+    # replicas of the whole cache so that the timed inputs exceed L2 by a wide margin
+    one_cache_bytes = sum(K.kvq_layout(cfg).values()) * layers
+    R = 1 if one_cache_bytes * 1 > 4 * L2_BYTES else int(math.ceil(4 * L2_BYTES / one_cache_bytes))
+
+    t_setup = time.time()
+    kstage = torch.empty((w.B, T0, w.Hkv, w.D), dtype=torch.float16, device=dev)
+    vstage = torch.empty_like(kstage)
+    caches, cbs = [], []
+    kfirst = None
+    fit_ws = torch.empty(K.kvq_fit_workspace(32, 128), dtype=torch.uint8, device=dev)
+    qws = torch.empty(K.kvq_quantize_workspace(cfg, T0, 1), dtype=torch.uint8, device=dev)
+    prefill_ms = []
+    for r in range(R):
+        for l in range(layers):
+            gen = DeviceGen(w, layer_key(l) + 100000 * r, device=dev)
+            gen.fill_k(kstage, 0, T0)
+            gen.fill_v(vstage, 0, T0)
+            cb = []
+            for samples in (synth.codebook_samples_k(w, layer_key(l)),
+                            synth.codebook_samples_v(w, layer_key(l))):
+                s = torch.from_numpy(samples.view(np.int16).copy()).to(dev)
+                lev = torch.empty(1 << w.bits, dtype=torch.float32, device=dev)
+                bnd = torch.empty((1 << w.bits) - 1, dtype=torch.float32, device=dev)
+                K.kvq_fit_codebook(s, w.f, w.bits, lev, bnd,
+                                   torch.empty(K.kvq_fit_workspace(*samples.shape),
+                                               dtype=torch.uint8, device=dev))
+                cb.append(K.Codebook(lev, bnd))
+            c = K.Cache(cfg, device=dev)
+            K.kvq_cache_reset(c)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            K.kvq_quantize_append(c, cb[0], cb[1], kstage, vstage, T0, None, 1, qws)
+            e1.record()
+            torch.cuda.synchronize()
+            prefill_ms.append(e0.elapsed_time(e1))
+            st = K.kvq_get_status(c)
+            if st:
+                raise RuntimeError(f"cache status {st} after prefill of layer {l}")
+            caches.append(c)
+            cbs.append(cb)
+    setup_s = time.time() - t_setup
+    kcount = int(caches[0].kcount.cpu()[0])
+    vcount = int(caches[0].vcount.cpu()[0])
+
+    # per-step inputs: appended token K/V and queries, per layer (device and pinned host)
+    nL = layers * R
+    knew = torch.empty((nL, steps_total, w.B, 1, w.Hkv, w.D), dtype=torch.float16, device=dev)
+    vnew = torch.empty_like(knew)
+    qall = torch.empty((nL, steps_total, w.B, w.Hq, w.D), dtype=torch.float16, device=dev)
+    for i in range(nL):
+        r, l = divmod(i, layers)
+        gen = DeviceGen(w, layer_key(l) + 100000 * r, device=dev)
+        for s in range(steps_total):
+            tmp = torch.empty((w.B, 1, w.Hkv, w.D), dtype=torch.float16, device=dev)
+            gen.fill_k(tmp, T0 + s, 1)
+            knew[i, s] = tmp
+            gen.fill_v(tmp, T0 + s, 1)
+            vnew[i, s] = tmp
+            gen.fill_q(qall[i, s], step=s)
+    qpos = torch.tensor([[T0 + s] * w.B for s in range(steps_total)], dtype=torch.int32,
+                        device=dev)
+    S = args.splits or K.kvq_decode_splits(cfg, T_max)
+    aws = torch.empty(K.kvq_quantize_workspace(cfg, 1, 0), dtype=torch.uint8, device=dev)
+    dws = torch.empty(K.kvq_decode_workspace(cfg, T_max, S), dtype=torch.uint8, device=dev)
+    BH = w.B * w.Hq
+    logits = torch.empty((w.B, w.Hq, T_max), dtype=torch.float32, device=dev)
+    stats = torch.empty((w.B, w.Hq, S, 2), dtype=torch.float32, device=dev)
+    mlb = torch.empty((w.B, w.Hq, 2), dtype=torch.float32, device=dev)
+    part = torch.empty((w.B, w.Hq, S, w.D), dtype=torch.float32, device=dev)
+    outs = torch.empty((nL, w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    ev_pool = []
+
+    def ev():
+        e = torch.cuda.Event(enable_timing=True)
+        ev_pool.append(e)
+        return e
+
+    def layer_step(i, s, timing):
+        c = caches[i]
+        cbK, cbV = cbs[i]
+        max_len = T0 + s + 1
+        marks = [ev(), ev(), ev(), ev(), ev()] if timing else None
+        if timing:
+            marks[0].record()
+        K.kvq_quantize_append(c, cbK, cbV, knew[i, s], vnew[i, s], 1, None, 0, aws)
+        if timing:
+            marks[1].record()
+        if args.path == "split":
+            K.kvq_decode_qk(c, cbK, qall[i, s], qpos[s], max_len, logits, stats, S)
+            if timing:
+                marks[2].record()
+            K.kvq_softmax_merge(cfg, stats, S, mlb)
+            if timing:
+                marks[3].record()
+            K.kvq_decode_pv(c, cbV, logits, mlb, max_len, outs[i], part, S)
+        else:
+            if timing:
+                marks[2].record()
+                marks[3].record()
+            K.kvq_decode_attention(c, cbK, cbV, qall[i, s], qpos[s], max_len, outs[i], dws, S)
+        if timing:
+            marks[4].record()
+        return marks
+
+    # warm-up
+    for s in range(args.warmup):
+        for i in range(nL):
+            layer_step(i, s, False)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    marks = []
+    with ClockSampler(dev.index) as clk:
+        t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t_start.record()
+        for s in range(args.warmup, steps_total):
+            rep = s % R
+            for i in range(rep * layers, (rep + 1) * layers):
+                marks.append(layer_step(i, s, True))
+        t_end.record()
+        torch.cuda.synchronize()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        dist.barrier()
+    n_layer_steps = len(marks)
+    tok_per_layer_step = [T0 + s + 1 for s in range(args.warmup, steps_total) for _ in range(layers)]
+    kv_tokens = w.B * sum(tok_per_layer_step) * world
+    value = kv_tokens / (elapsed_ms / 1e3)
+    # per-kernel times
+    t_app = sum(m[0].elapsed_time(m[1]) for m in marks)
+    t_qk = sum(m[1].elapsed_time(m[2]) for m in marks)
+    t_merge = sum(m[2].elapsed_time(m[3]) for m in marks)
+    t_pv = sum(m[3].elapsed_time(m[4]) for m in marks)
+    Tmid = T0 + args.warmup + args.steps // 2 + 1
+    bm = bytes_model(w, Tmid, kcount, vcount, args.path)
+    hbm, peak_kind = peaks()
+    if args.path == "split":
+        kernels = {"k_qk": (t_qk, bm["qk"], "kvq_decode.cu"), "k_pv": (t_pv, bm["pv"], "kvq_decode.cu")}
+    else:
+        kernels = {"k_attn": (t_pv, bm["attn"], "kvq_decode.cu")}
+    dom = max(kernels, key=lambda k: kernels[k][0])
+    dom_ms = kernels[dom][0] / n_layer_steps
+    dom_bytes = kernels[dom][1]
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    step_attn_ms = (t_qk + t_merge + t_pv) / n_layer_steps
+    attn_gbs = bm["total"] / (step_attn_ms / 1e3) / 1e9
+
+    # ---- end-to-end through the public API with host buffers
+    h_q = torch.empty_like(qall, device="cpu").pin_memory()
+    h_k = torch.empty_like(knew, device="cpu").pin_memory()
+    h_v = torch.empty_like(vnew, device="cpu").pin_memory()
+    h_q.copy_(qall)
+    h_k.copy_(knew)
+    h_v.copy_(vnew)
+    h_out = torch.empty((nL, w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
+    d_q = torch.empty((nL, w.B, w.Hq, w.D), dtype=torch.float16, device=dev)
+    d_k = torch.empty((nL, w.B, 1, w.Hkv, w.D), dtype=torch.float16, device=dev)
+    d_v = torch.empty_like(d_k)
+    # the e2e leg appends at fresh positions after the timed steps (replica 0)
+    qpos_e2e = torch.tensor([[T0 + steps_total + j] * w.B for j in range(e2e_steps)],
+                            dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h2d = d2h = 0
+    e_s.record()
+    for j in range(e2e_steps):
+        s = args.warmup + j
+        ml_len = T0 + steps_total + j + 1
+        d_q.copy_(h_q[:, s], non_blocking=True)
+        d_k.copy_(h_k[:, s], non_blocking=True)
+        d_v.copy_(h_v[:, s], non_blocking=True)
+        for i in range(layers):
+            c = caches[i]
+            K.kvq_quantize_append(c, cbs[i][0], cbs[i][1], d_k[i], d_v[i], 1, None, 0, aws)
+            if args.path == "split":
+                K.kvq_decode_qk(c, cbs[i][0], d_q[i], qpos_e2e[j], ml_len, logits, stats, S)
+                K.kvq_softmax_merge(cfg, stats, S, mlb)
+                K.kvq_decode_pv(c, cbs[i][1], logits, mlb, ml_len, outs[i], part, S)
+            else:
+                K.kvq_decode_attention(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j], ml_len,
+                                       outs[i], dws, S)
+        h_out.copy_(outs, non_blocking=True)
+        h2d = (d_q[:layers].numel() + d_k[:layers].numel() + d_v[:layers].numel()) * 2
+        d2h = h_out[:layers].numel() * 4
+    e_e.record()
+    torch.cuda.synchronize()
+    e2e_ms = e_s.elapsed_time(e_e)
+    e2e_tokens = w.B * sum(T0 + steps_total + j + 1 for j in range(e2e_steps)) * layers
+    e2e_value = e2e_tokens / (e2e_ms / 1e3) * world
+
+    # ---- uncompressed fp16 comparison kernel on one layer (last staged K/V)
+    fp16 = None
+    if not args.no_fp16:
+        lens = torch.full((w.B,), T0, dtype=torch.int32, device=dev)
+        fws = torch.empty(K.kvq_decode_workspace(cfg, T0, S), dtype=torch.uint8, device=dev)
+        fout = torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
+        qp0 = torch.full((w.B,), T0, dtype=torch.int32, device=dev)
+        for _ in range(3):
+            K.kvq_fp16_decode_attention(cfg, kstage, vstage, T0, lens, qall[0, 0], qp0, T0, fout,
+                                        fws, S)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nrep = 5
+        f0.record()
+        for _ in range(nrep):
+            K.kvq_fp16_decode_attention(cfg, kstage, vstage, T0, lens, qall[0, 0], qp0, T0, fout,
+                                        fws, S)
+        f1.record()
+        torch.cuda.synchronize()
+        fms = f0.elapsed_time(f1) / nrep
+        fbytes = 2 * w.B * T0 * w.Hkv * w.D * 2
+        fp16 = {"ms_per_layer": fms, "GB/s": fbytes / (fms / 1e3) / 1e9,
+                "kv_tokens_per_s": w.B * T0 / (fms / 1e3),
+                "quantized_ms_per_layer": step_attn_ms,
+                "speedup_quantized_vs_fp16": fms / step_attn_ms}
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v_cpu, smp = cpu_oracle_sample(w)
+        cpu = {"value": v_cpu, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": smp}
+
+    if rank != 0:
+        return 0
+    launches_per_layer_step = 8 if args.path == "split" else 6
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded Philox4x32-10; LLaMA-7B-shaped K/V distributions)",
+        "config": {"workload": w.name, "layers": layers, "B": w.B, "q_heads": w.Hq,
+                   "kv_heads": w.Hkv, "head_dim": w.D, "T_cached": T0, "bits": w.bits,
+                   "outlier_frac": w.f, "rope_theta": w.rope_theta, "path": args.path,
+                   "splits": S, "cache_replicas": R,
+                   "l2": f"inputs {one_cache_bytes * R / 1e9:.1f} GB > 126 MB L2, not flushed"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_kind,
+                     "traffic": traffic_for(dom, Tmid),
+                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "avg_launch_ms": dom_ms},
+        "attention_step": {"ms_per_layer": step_attn_ms, "GB/s": attn_gbs,
+                           "frac_of_peak": attn_gbs / hbm, "bytes_per_layer": bm["total"]},
+        "kernels_ms_per_layer": {"append": t_app / n_layer_steps, "qk": t_qk / n_layer_steps,
+                                 "merge": t_merge / n_layer_steps, "pv": t_pv / n_layer_steps},
+        "prefill": {"ms_per_layer": statistics.median(prefill_ms), "tokens": T0,
+                    "setup_s": setup_s},
+        "outliers_per_layer": {"k": kcount, "v": vcount},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "fp16_attention": fp16,
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_layer_step * n_layer_steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    try:
+        return run_kvq(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,274 @@
+/*
+ * kvq.h -- C ABI of libkvq.so: a sub-4-bit KVQuant KV cache on NVIDIA B200 (sm_100a).
+ *
+ * The library implements the decode-time hot path of KVQuant ("KVQuant: Towards
+ * 10 Million Context Length LLM Inference with KV Cache Quantization", arXiv
+ * 2401.18079):
+ *   - the append-time quantizer that writes the cache, using (i) per-channel key
+ *     quantization, (ii) pre-RoPE keys, (iii) a per-layer non-uniform (NUQ)
+ *     datatype and (iv) per-vector dense-and-sparse outliers (study.space
+ *     summary, techniques (i)-(iv); phantomic12 research note, components (1)-(4));
+ *   - decode attention read directly from that cache: QK with on-the-fly NUQ
+ *     lookup, RoPE and sparse outlier correction, a split-K softmax with a
+ *     max/sum merge, and the probability-weighted value sum (study.space
+ *     summary: custom kernels replacing the fp16 matrix-vector products of
+ *     memory- and bandwidth-bound long-context decode).
+ *
+ * Conventions (every entry point):
+ *   - Buffers are DEVICE pointers owned by the caller unless a parameter says
+ *     "host".  Cache and workspace buffers must be 16-byte aligned.  The library
+ *     allocates no memory and keeps no global state.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls only enqueue work; none synchronizes except kvq_get_status.
+ *   - Return value: KVQ_OK (0) or a negative KVQ_ERR_* code.  Argument checks are
+ *     synchronous and nothing is launched when one fails.  KVQ_ERR_CUDA reports
+ *     a failed launch; the CUDA error string is available via kvq_strerror.
+ *   - Conditions only the device can see (an outlier list that is full, a length
+ *     past T_max) set bits in the sticky int32 `status` word of the cache and the
+ *     kernel carries on without trapping; read it with kvq_get_status.
+ *   - fp16 values travel as their uint16_t bit patterns.
+ *   - Only head_dim D = 128 and bits in {2, 3, 4} are supported.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_ABI_VERSION 1
+
+enum {
+    KVQ_OK = 0,
+    KVQ_ERR_NULL = -1,        /* a required pointer is NULL */
+    KVQ_ERR_ALIGN = -2,       /* a device pointer is not 16-byte aligned */
+    KVQ_ERR_SHAPE = -3,       /* a dimension or count is out of range */
+    KVQ_ERR_UNSUPPORTED = -4, /* bits or head_dim not supported */
+    KVQ_ERR_RANGE = -5,       /* token range beyond T_max / split count out of range */
+    KVQ_ERR_WORKSPACE = -6,   /* workspace smaller than the size query returned */
+    KVQ_ERR_CUDA = -7,        /* a CUDA launch or runtime call failed */
+};
+
+/* Sticky device status bits (cache->status). */
+#define KVQ_STATUS_OUTLIER_OVERFLOW 1 /* outliers of some tokens did not fit and were dropped */
+#define KVQ_STATUS_LEN_OVERFLOW 2     /* a write past T_max (or a length past max_len) was skipped */
+#define KVQ_STATUS_NOT_EMPTY 4        /* a calibrating prefill met a non-empty sequence; skipped */
+
+#define KVQ_CHUNK 64 /* tokens per outlier chunk */
+
+/* Geometry of one layer's cache.  n = Hkv * D channels per token. */
+typedef struct kvq_cfg {
+    int32_t B;          /* sequences (batch) */
+    int32_t Hq;         /* query heads; a multiple of Hkv */
+    int32_t Hkv;        /* key/value heads */
+    int32_t D;          /* head dimension; must be 128 */
+    int32_t bits;       /* NUQ code width: 2, 3 or 4 */
+    int32_t T_max;      /* token capacity per sequence, 1 .. 16,777,216 */
+    int32_t out_cap_k;  /* key-outlier list capacity per sequence (entries) */
+    int32_t out_cap_v;  /* value-outlier list capacity per sequence (entries) */
+    double outlier_frac;/* f: per vector, k = floor(f*N/2 + 1/2) outliers per side */
+    double rope_theta;  /* RoPE base; theta_i = rope_theta^(-2i/D) */
+} kvq_cfg;
+
+/*
+ * Device arrays of one layer's cache (all caller-allocated; sizes from kvq_layout).
+ * W = 4*bits words per (token, kv head) row.  Layouts:
+ *  kcodes  uint32 [B][T_max][Hkv][W]   key row: 64 rotate-half pairs (p, p+64);
+ *          pair-group g = p/16 is `bits` words; pair p is the 2*bits-wide field
+ *          code[p] | code[p+64] << bits at bit 2*bits*(p%16) of the group's
+ *          little-endian bit string.
+ *  vcodes  uint32 [B][T_max][Hkv][W]   value row: channel group g (c = 32g+k) is
+ *          `bits` words in nibble format (3 bits: k < 24 -> bits 0-2 of nibble
+ *          k%8 of word k/8; k = 24+j -> bit m of the code in bit 3 of nibble j of
+ *          word m; 2 bits: word k/16, nibble (k%16)%8, bit pair (k%16)/8;
+ *          4 bits: word k/8, nibble k%8).
+ *  kthr    uint16 [B][n][2]  fp16 key thresholds (t_lo, t_hi) per channel
+ *  kparams float  [B][n][2]  key channel (off, half)
+ *  vparams float  [B][T_max][2] value token (off, half)
+ *  k/vout_pos uint32 [B][cap]  outlier entry ((t % 64) << 16) | (h*D + c),
+ *          sorted by (t, h*D + c); k/vout_val uint16 [B][cap] its fp16 bits
+ *  k/vchunk uint32 [B][ceil(T_max/64)+1]  entries of tokens [64m, 64m+64) are
+ *          [chunk[m], chunk[m+1])
+ *  k/vcount uint32 [B]  entries in use;  len int32 [B]  tokens in the cache
+ *  status  int32 [1]  sticky KVQ_STATUS_* bits
+ */
+typedef struct kvq_cache {
+    uint32_t* kcodes;
+    uint32_t* vcodes;
+    uint16_t* kthr;
+    float* kparams;
+    float* vparams;
+    uint32_t* kout_pos;
+    uint16_t* kout_val;
+    uint32_t* vout_pos;
+    uint16_t* vout_val;
+    uint32_t* kchunk;
+    uint32_t* vchunk;
+    uint32_t* kcount;
+    uint32_t* vcount;
+    int32_t* len;
+    int32_t* status;
+} kvq_cache;
+
+/* A per-layer NUQ datatype (device arrays): levels[2^bits] ascending binary32
+ * values whose bit patterns are (u << 16) | u, and the decision bounds
+ * bounds[2^bits - 1] = binary32((levels[j] + levels[j+1]) / 2). */
+typedef struct kvq_codebook {
+    const float* levels;
+    const float* bounds;
+} kvq_codebook;
+
+/* Byte size of every cache array of kvq_cache, same field names. */
+typedef struct kvq_sizes {
+    size_t kcodes, vcodes, kthr, kparams, vparams;
+    size_t kout_pos, kout_val, vout_pos, vout_val;
+    size_t kchunk, vchunk, kcount, vcount, len, status;
+} kvq_sizes;
+
+/* ABI version (KVQ_ABI_VERSION). */
+int kvq_abi_version(void);
+
+/* Static message for a KVQ_* code; for KVQ_ERR_CUDA the last CUDA error's text.
+ * The pointer is owned by the library and valid until the next call. */
+const char* kvq_strerror(int code);
+
+/* Check a configuration.  KVQ_OK, KVQ_ERR_NULL, KVQ_ERR_SHAPE or KVQ_ERR_UNSUPPORTED. */
+int kvq_validate_cfg(const kvq_cfg* cfg);
+
+/* Fill *out (host) with the byte size of each cache array for cfg. */
+int kvq_layout(const kvq_cfg* cfg, kvq_sizes* out);
+
+/* Empty the cache: zero len, counts, chunk pointers and status (async on stream). */
+int kvq_cache_reset(const kvq_cfg* cfg, const kvq_cache* cache, void* stream);
+
+/* Workspace bytes for kvq_quantize_append with this many tokens per sequence. */
+int kvq_quantize_workspace(const kvq_cfg* cfg, int32_t n_new, int32_t calibrate, size_t* bytes);
+
+/*
+ * Quantize and append tokens (technique (i)-(iv) on the write side).
+ *   k, v     fp16 [B][n_new][Hkv][D] pre-RoPE keys and values (device)
+ *   plen     int32 [B] tokens of sequence b to take from the block (<= n_new),
+ *            or NULL for n_new each (device)
+ *   calibrate 1: prefill -- the sequence must be empty; per key channel the
+ *            thresholds t_lo = s[k], t_hi = s[N-1-k] of its N = plen[b] values
+ *            (ascending in IEEE total order, k = floor(f*N/2 + 1/2) capped at
+ *            (N-1)/2) and off = (t_lo+t_hi)*0.5, half = (t_hi-t_lo)*0.5 (binary32)
+ *            are computed first.  0: append at positions len[b] onwards with the
+ *            existing key calibration.
+ *   Per token: value thresholds/scales over its n values as above; an entry is
+ *   an outlier iff x < t_lo or x > t_hi; outliers go to the lists unchanged and
+ *   are encoded as 0; xn = (x - off)/half (0 if half == 0); code = #{j: xn >
+ *   bounds[j]}.  Tokens whose outliers would exceed the list capacity (counting
+ *   from the start of this call, in token order) drop their outliers and set
+ *   KVQ_STATUS_OUTLIER_OVERFLOW.
+ *   workspace: device scratch of kvq_quantize_workspace bytes, 16-byte aligned.
+ */
+int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
+                        const kvq_codebook* cbV, const uint16_t* k, const uint16_t* v,
+                        int32_t n_new, const int32_t* plen, int32_t calibrate, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/*
+ * Decode QK (technique (ii) read side): for every query head hq (kv head
+ * h = hq / (Hq/Hkv)) and cached token t < len[b]:
+ *   logits[b][hq][t] = (R(qpos[b]) q) . (R(t) khat_t,h) / sqrt(D)
+ * with rotate-half RoPE R and khat the dequantized key (dense off + half*L[code],
+ * outliers replaced by their stored value).  Also writes per split s (tokens
+ * [s*Ls, (s+1)*Ls), Ls = the split length chosen from max_len and `splits`):
+ *   stats[b][hq][s] = (m_s, l_s), m_s = max logit, l_s = sum exp(logit - m_s)
+ * (m_s = -inf, l_s = 0 for an empty split).
+ *   q       fp16 [B][Hq][D] pre-RoPE query;  qpos int32 [B] its position
+ *   max_len host upper bound on len[b] (sizes the grid); a longer sequence is
+ *           clipped and sets KVQ_STATUS_LEN_OVERFLOW
+ *   logits  float [B][Hq][T_max];  stats float2 [B][Hq][splits]
+ *   splits  1 .. 4096, or 0 to let the library choose (kvq_decode_splits)
+ */
+int kvq_decode_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
+                  const uint16_t* q, const int32_t* qpos, int32_t max_len, float* logits,
+                  float* stats, int32_t splits, void* stream);
+
+/* The split count the library uses for `splits = 0`. */
+int kvq_decode_splits(const kvq_cfg* cfg, int32_t max_len);
+
+/* Split-K softmax merge: ml[b][hq] = (M, L), M = max_s m_s, L = sum_s l_s e^(m_s - M).
+ * stats float2 [B][Hq][splits] from kvq_decode_qk; ml float2 [B][Hq]. */
+int kvq_softmax_merge(const kvq_cfg* cfg, const float* stats, int32_t splits, float* ml,
+                      void* stream);
+
+/*
+ * Decode PV: out[b][hq][:] = sum_t p_t * vhat_t,h with p_t = exp(logits - M)/L and
+ * vhat the dequantized value (off_t + half_t*L[code], outliers replaced).
+ *   logits, ml from the two calls above; out float [B][Hq][D]
+ *   part   float scratch [B][Hq][splits][D] (per-split partial sums, summed in
+ *          split order)
+ */
+int kvq_decode_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbV,
+                  const float* logits, const float* ml, int32_t max_len, float* out, float* part,
+                  int32_t splits, void* stream);
+
+/* Workspace bytes of kvq_decode_attention for max_len and splits (0 = auto). */
+int kvq_decode_workspace(const kvq_cfg* cfg, int32_t max_len, int32_t splits, size_t* bytes);
+
+/*
+ * Fused single-pass decode attention: the same result as kvq_decode_qk +
+ * kvq_softmax_merge + kvq_decode_pv, computed with an online softmax per split
+ * (no logits written) and one merge; out float [B][Hq][D].
+ *   workspace  device scratch of kvq_decode_workspace bytes
+ */
+int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
+                         const kvq_codebook* cbV, const uint16_t* q, const int32_t* qpos,
+                         int32_t max_len, float* out, void* workspace, size_t workspace_bytes,
+                         int32_t splits, void* stream);
+
+/*
+ * Dequantize rows [t0, t0 + nt) of every sequence (test support):
+ *   khat, vhat fp16 [B][nt][Hkv][D] (keys pre-RoPE): dense fp16(off + half*L[code])
+ *   (binary32 multiply, then add, then round to fp16), outliers replaced by their
+ *   stored fp16 value.  Rows at or past len[b] are written as 0.
+ */
+int kvq_dequantize(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
+                   const kvq_codebook* cbV, int32_t t0, int32_t nt, uint16_t* khat,
+                   uint16_t* vhat, void* stream);
+
+/*
+ * Uncompressed comparison kernel: decode attention over an fp16 cache.
+ *   K, V fp16 [B][T_stride][Hkv][D] (keys pre-RoPE, RoPE applied on the fly);
+ *   len int32 [B]; q, qpos as kvq_decode_qk; out float [B][Hq][D];
+ *   workspace of kvq_decode_workspace bytes for the same cfg/max_len/splits.
+ */
+int kvq_fp16_decode_attention(const kvq_cfg* cfg, const uint16_t* K, const uint16_t* V,
+                              int32_t T_stride, const int32_t* len, const uint16_t* q,
+                              const int32_t* qpos, int32_t max_len, float* out, void* workspace,
+                              size_t workspace_bytes, int32_t splits, void* stream);
+
+/* Workspace bytes of kvq_fit_codebook. */
+int kvq_fit_workspace(int32_t n_vec, int32_t vec_len, size_t* bytes);
+
+/*
+ * Fit a per-layer NUQ datatype (technique (iii)) on the device.
+ *   samples fp16 [n_vec][vec_len]: each vector is thresholded and normalized by
+ *   its own order statistics (as in kvq_quantize_append), its outliers are
+ *   dropped, and the pooled normalized values (binary64) are fitted by weighted
+ *   1-D Lloyd k-means with 2^bits centroids: init at weighted quantiles
+ *   (j+1/2)/K, nearest centroid with ties to the lower index, weighted-mean
+ *   update (an empty cell keeps its value), stop when the assignment repeats or
+ *   after max_iter iterations.  Centroids are sorted, rounded to the nearest
+ *   (u << 16) | u binary32 value and bounds are binary32 midpoints.
+ *   weights  binary64 [n_vec][vec_len] sensitivity weights, or NULL for 1
+ *   levels   float [2^bits], bounds float [2^bits - 1] (device outputs)
+ *   n_vec * vec_len <= 16384.  Runs as one thread block.
+ */
+int kvq_fit_codebook(const uint16_t* samples, int32_t n_vec, int32_t vec_len, double f,
+                     const double* weights, int32_t bits, int32_t max_iter, float* levels,
+                     float* bounds, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Read the sticky status word into *out (host).  Synchronizes `stream`. */
+int kvq_get_status(const kvq_cache* cache, int32_t* out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H */

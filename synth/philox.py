@@ -144,6 +144,14 @@ def _four_normals(lo, hi, stream, tag, seed, layer):
 def normals(seed, layer, stream, e):
     """Standard normal deviates (binary64) for flat element indices ``e``."""
     e = np.asarray(e, dtype=np.uint64)
+    flat = e.ravel()
+    if flat.size >= 4 and flat.size % 4 == 0 and int(flat[0]) % 4 == 0:
+        groups = flat.reshape(-1, 4)
+        if np.array_equal(groups - groups[:, :1], np.broadcast_to(
+                np.arange(4, dtype=np.uint64), groups.shape)):
+            lo, hi = _split64(groups[:, 0] >> np.uint64(2))
+            z = _four_normals(lo, hi, stream, 0, seed, layer)
+            return np.stack(z, axis=1).reshape(e.shape)
     lo, hi = _split64(e >> np.uint64(2))
     z = _four_normals(lo, hi, stream, 0, seed, layer)
     lane = (e & np.uint64(3)).astype(np.int64)

@@ -1,0 +1,82 @@
+"""The C-ABI library loads, exports every declared symbol and rejects bad arguments
+before touching the GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_decode_nuq_b200 as K
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "kvq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = K.load()
+    names = _declared()
+    assert len(names) >= 18
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(K.EXPORTS)
+    assert K.kvq_abi_version() == 1
+
+
+def test_cfg_validation():
+    ok = K.make_cfg(1, 32, 32, 3, 4096, 0.01, 1e4, 100, 100)
+    assert K.kvq_validate_cfg(ok) == 0
+    bad = [
+        dict(bits=5), dict(bits=1), dict(D=64), dict(Hq=30), dict(B=0), dict(T_max=0),
+        dict(outlier_frac=1.5), dict(rope_theta=0.5), dict(out_cap_k=-1),
+    ]
+    for kw in bad:
+        args = dict(B=1, Hq=32, Hkv=32, bits=3, T_max=4096, outlier_frac=0.01, rope_theta=1e4,
+                    out_cap_k=100, out_cap_v=100, D=128)
+        args.update(kw)
+        assert K.kvq_validate_cfg(K.make_cfg(**args)) < 0, kw
+    assert K.load().kvq_validate_cfg(None) == -1
+
+
+def test_layout_sizes():
+    cfg = K.make_cfg(2, 8, 4, 3, 1000, 0.01, 1e4, 50, 70)
+    s = K.kvq_layout(cfg)
+    assert s["kcodes"] == 2 * 1000 * 4 * 12 * 4
+    assert s["vparams"] == 2 * 1000 * 2 * 4
+    assert s["kout_pos"] == 2 * 50 * 4 and s["vout_val"] == 2 * 70 * 2
+    assert s["kchunk"] == 2 * (16 + 1) * 4
+    assert K.kvq_quantize_workspace(cfg, 100, 1) > K.kvq_quantize_workspace(cfg, 100, 0)
+    assert K.kvq_decode_splits(cfg, 1000) >= 1
+
+
+def test_argument_errors_without_gpu():
+    lib = K.load()
+    cfg = K.make_cfg(1, 4, 4, 3, 256, 0.01, 1e4, 64, 64)
+    empty = K.CacheStruct()
+    cb = K.CodebookStruct(None, None)
+    null = None
+    # NULL cache arrays are rejected synchronously
+    rc = lib.kvq_quantize_append(ctypes.byref(cfg), ctypes.byref(empty), ctypes.byref(cb),
+                                 ctypes.byref(cb), null, null, 1, null, 0, null, 0, null)
+    assert rc == -1
+    # misaligned (never dereferenced) pointers are rejected
+    fake = K.CacheStruct(*([0x1000] * 15))
+    fake.kcodes = 0x1001
+    rc = lib.kvq_cache_reset(ctypes.byref(cfg), ctypes.byref(fake), null)
+    assert rc == -2
+    # unsupported head_dim is reported before anything else
+    cfg64 = K.make_cfg(1, 4, 4, 3, 256, 0.01, 1e4, 64, 64, D=64)
+    assert lib.kvq_cache_reset(ctypes.byref(cfg64), ctypes.byref(fake), null) == -4
+    # split count out of range
+    fake.kcodes = 0x1000
+    cbf = K.CodebookStruct(0x1000, 0x1000)
+    rc = lib.kvq_decode_qk(ctypes.byref(cfg), ctypes.byref(fake), ctypes.byref(cbf), 0x1000,
+                           0x1000, 100, 0x1000, 0x1000, 5000, null)
+    assert rc == -5
+    # fit: too many samples
+    assert lib.kvq_fit_workspace(5, 5000, ctypes.byref(ctypes.c_size_t())) == -3
+    assert K.load().kvq_strerror(-6) == b"workspace too small"
