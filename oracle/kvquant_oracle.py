@@ -27,7 +27,10 @@ listed in the design doc with its ID):
   R4 normalization: off = (t_lo + t_hi)*0.5, half = (t_hi - t_lo)*0.5,
      xn = (x - off)/half, all binary32 round-to-nearest; xn = 0 if half == 0.
   R5 dense remainder: outlier positions are set to 0 before encoding;
-     reconstruction replaces them with the stored fp16 value.
+     reconstruction replaces them with the stored fp16 value.  The
+     reconstruction used by attention is exact: x = off + half * L[code] in real
+     arithmetic on the stored binary32 values (binary64 here); rounding it to
+     fp16 is only the format of the dequantized-cache output.
   R6 encode: code = #{j : xn > bounds[j]} (ties go to the lower code).
   R7 codebook: weighted 1-D Lloyd k-means in binary64 (init at weighted
      quantiles (j+1/2)/K, nearest-centroid assignment with ties to the lower
@@ -439,6 +442,21 @@ class QuantizedCache:
                 p = int(self.out_pos[s][b, i])
                 out.append((m * CHUNK + (p >> 16), p & 0xFFFF, int(self.out_val[s][b, i])))
         return out
+
+    def reconstruct(self, b, cbK, cbV):
+        """Exact binary64 K-hat, V-hat [T, Hkv, D] of sequence b, the attention input (R5)."""
+        L = int(self.len[b])
+        levK = np.asarray(cbK[0], dtype=np.float64)
+        levV = np.asarray(cbV[0], dtype=np.float64)
+        kp = self.kparams[b].astype(np.float64)
+        vp = self.vparams[b, :L].astype(np.float64)
+        Kx = kp[:, 0] + kp[:, 1] * levK[self.kc[b, :L].astype(np.int64)]
+        Vx = vp[:, 0:1] + vp[:, 1:2] * levV[self.vc[b, :L].astype(np.int64)]
+        for s, X in (("k", Kx), ("v", Vx)):
+            for t, j, bits in self.outlier_entries(s, b):
+                if t < L:
+                    X[t, j] = float(np.uint16(bits).view(np.float16))
+        return Kx.reshape(L, self.Hkv, self.D), Vx.reshape(L, self.Hkv, self.D)
 
     def dequantize(self, b, cbK, cbV, t_range=None):
         """fp16 K-hat, V-hat [T, Hkv, D] (keys pre-RoPE) of sequence b."""

@@ -52,8 +52,8 @@ def _setup(name, over, T, plen, appends):
         if o.len[b] == 0:
             refs.append(None)
             continue
-        Kh, Vh = o.dequantize(b, cbK, cbV)
-        refs.append(O.decode_attention(q16[b], int(qpos[b]), Kh, Vh, w.rope_theta))
+        Kx, Vx = o.reconstruct(b, cbK, cbV)
+        refs.append(O.decode_attention(q16[b], int(qpos[b]), Kx, Vx, w.rope_theta))
     dq = torch.from_numpy(q16).cuda()
     dpos = torch.from_numpy(qpos).cuda()
     return w, o, g, dK, dV, dq, dpos, refs, K16, V16

@@ -520,3 +520,26 @@ def test_dequantize_then_attend_end_to_end():
     assert np.isfinite(o).all() and abs(p.sum() - 1) < 1e-12
     # 3-bit + 1% outliers stays close to the unquantized attention
     assert np.corrcoef(lg[0], lgx[0])[0, 1] > 0.98
+
+
+def test_reconstruct_is_exact_affine_and_rounds_to_dequantize():
+    """Exact reconstruction: off + half * L in binary64; rounding it gives the fp16 dequant
+    except where binary32 multiply-then-add rounding differs (double rounding), and the
+    outliers are identical in both."""
+    w = synth.workload("llama7b_layer_32k", Hq=2, Hkv=2)
+    T = 200
+    c, K, V, cbK, cbV = _small_cache(w, T)
+    Kx, Vx = c.reconstruct(0, cbK, cbV)
+    Kh, Vh = c.dequantize(0, cbK, cbV)
+    j = 77
+    t = 13
+    code = int(c.kc[0, t, j])
+    want = float(c.kparams[0, j, 0]) + float(c.kparams[0, j, 1]) * float(cbK[0][code])
+    if not any(tt == t and jj == j for tt, jj, _ in c.outlier_entries("k", 0)):
+        assert Kx.reshape(T, -1)[t, j] == want
+    for X, H in ((Kx, Kh), (Vx, Vh)):
+        r = X.astype(np.float32).astype(np.float16)
+        assert np.mean(r == H) > 0.999
+        assert np.abs(X - H.astype(np.float64)).max() <= np.abs(X).max() * 2 ** -10
+    for t_, j_, bits in c.outlier_entries("v", 0):
+        assert Vx.reshape(T, -1)[t_, j_] == float(np.uint16(bits).view(np.float16))
