@@ -44,6 +44,8 @@ def parse():
     p.add_argument("--path", default="split", choices=["split", "fused"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-fp16", action="store_true")
+    p.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
+    p.add_argument("--tokens", type=int, default=0, help="override the cached token count")
     return p.parse_args()
 
 
@@ -234,10 +236,15 @@ def run_kvq(args, rank, world):
 
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
     torch.cuda.set_device(dev)
-    w = synth.workload(args.workload)
+    over = {}
+    if args.layers:
+        over["layers"] = args.layers
+    if args.tokens:
+        over["T"] = args.tokens
+    w = synth.workload(args.workload, **over)
     steps_total = args.warmup + args.steps
     if w.T + steps_total + 16 > w.T_gen:
-        w = synth.workload(args.workload, appends=1, steps=steps_total + 16)
+        w = synth.workload(args.workload, appends=1, steps=steps_total + 16, **over)
     layers = w.layers
     T0 = w.T
     e2e_steps = min(args.steps, 10)

@@ -83,8 +83,8 @@ int kvq_layout(const kvq_cfg* cfg, kvq_sizes* out) {
     const size_t B = cfg->B, T = cfg->T_max, n = (size_t)cfg->Hkv * cfg->D;
     const size_t W = kvq::row_words(cfg->bits);
     const size_t nch = kvq::nchunks(cfg->T_max) + 1;
-    out->kcodes = B * T * cfg->Hkv * W * 4;
-    out->vcodes = out->kcodes;
+    out->kcodes = B * (size_t)kvq::npairs(cfg->T_max) * cfg->Hkv * kvq::block_words(cfg->bits) * 4;
+    out->vcodes = B * T * cfg->Hkv * W * 4;
     out->kthr = B * n * 2 * 2;
     out->kparams = B * n * 2 * 4;
     out->vparams = B * T * 2 * 4;

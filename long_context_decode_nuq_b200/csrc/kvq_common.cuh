@@ -14,8 +14,10 @@ constexpr int kD = 128;          // head dimension (the only one supported)
 constexpr int kPairs = kD / 2;   // rotate-half pairs (p, p + 64)
 constexpr int kChunk = KVQ_CHUNK;
 
-__host__ __device__ inline int row_words(int bits) { return 4 * bits; }
+__host__ __device__ inline int row_words(int bits) { return 4 * bits; }    // value row
+__host__ __device__ inline int block_words(int bits) { return 8 * bits; }  // key block (2 tokens)
 __host__ __device__ inline int nchunks(int T_max) { return (T_max + kChunk - 1) / kChunk; }
+__host__ __device__ inline int npairs(int T_max) { return (T_max + 1) / 2; }
 
 // Outliers kept per side of an N-value vector: floor(f*N/2 + 1/2), capped at (N-1)/2.
 __host__ __device__ inline int vector_k(double f, int N) {
@@ -49,48 +51,36 @@ __device__ inline uint32_t encode(float xn, const float* bounds, int nb) {
     return c;
 }
 
-// ---- key row layout: pair p = (p, p+64) is a 2*bits field in pair-group p/16 ----
-__device__ inline uint32_t k_pair_field(const uint32_t* row, int bits, int p) {
-    const int g = p >> 4, j = p & 15;
-    const int o = 2 * bits * j;
-    const int w = o >> 5, s = o & 31;
-    const uint32_t* gw = row + g * bits;
-    uint32_t v = gw[w] >> s;
-    if (s + 2 * bits > 32) v |= gw[w + 1] << (32 - s);
-    return v & ((1u << (2 * bits)) - 1u);
+// ---- key block (token pair 2u, 2u+1; one kv head): channel c = j + 16m + 64s
+// (j in [0,16), m in [0,4), s in {0,1}) has the 2*bits field
+// code(2u, c) | code(2u+1, c) << bits at bit 16*bits*j + 2*bits*(2m + s).
+__host__ __device__ inline int k_field_index(int c) {
+    return 8 * (c & 15) + 2 * ((c & 63) >> 4) + (c >> 6);
+}
+// ---- value row (one token, one kv head): channel c < 64 and c + 64 share the field
+// code(c) | code(c+64) << bits at bit 16*bits*j + 2*bits*m for c = j + 8m.
+__host__ __device__ inline int v_field_index(int c) { return 8 * (c & 7) + ((c & 63) >> 3); }
+// channel of field f (key block: f = 8j + 2m + s; value row: f = 8j + m, channel < 64)
+__host__ __device__ inline int k_field_channel(int f) { return (f >> 3) + 16 * ((f >> 1) & 3) + 64 * (f & 1); }
+__host__ __device__ inline int v_field_channel(int f) { return (f >> 3) + 8 * (f & 7); }
+
+__device__ inline uint32_t get_field(const uint32_t* w, int f, int width) {
+    const int off = f * width;
+    const int wi = off >> 5, s = off & 31;
+    uint32_t v = w[wi] >> s;
+    if (s + width > 32) v |= w[wi + 1] << (32 - s);
+    return v & ((1u << width) - 1u);
 }
 
-// ---- value row layout: channel c = 32g + k in nibble format ----
-// Bit position (word within the group, bit) of bit m of code k.
-__host__ __device__ inline void v_bitpos(int bits, int k, int m, int* word, int* bit) {
-    if (bits == 3) {
-        if (k < 24) { *word = k >> 3; *bit = 4 * (k & 7) + m; }
-        else { *word = m; *bit = 4 * (k - 24) + 3; }
-    } else if (bits == 2) {
-        const int w = k >> 4, kk = k & 15;
-        *word = w; *bit = 4 * (kk & 7) + 2 * (kk >> 3) + m;
-    } else {
-        *word = k >> 3; *bit = 4 * (k & 7) + m;
-    }
+// Code of channel c of token (2u + parity) from a key block.
+__device__ inline uint32_t k_code(const uint32_t* block, int bits, int c, int parity) {
+    const uint32_t f = get_field(block, k_field_index(c), 2 * bits);
+    return parity ? (f >> bits) : (f & ((1u << bits) - 1u));
 }
 
+// Code of channel c from a value row.
 __device__ inline uint32_t v_code(const uint32_t* row, int bits, int c) {
-    const int g = c >> 5, k = c & 31;
-    const uint32_t* gw = row + g * bits;
-    if (bits == 3) {
-        if (k < 24) return (gw[k >> 3] >> (4 * (k & 7))) & 7u;
-        const int sh = 4 * (k - 24) + 3;
-        return ((gw[0] >> sh) & 1u) | (((gw[1] >> sh) & 1u) << 1) | (((gw[2] >> sh) & 1u) << 2);
-    }
-    if (bits == 2) {
-        const int kk = k & 15;
-        return (gw[k >> 4] >> (4 * (kk & 7) + 2 * (kk >> 3))) & 3u;
-    }
-    return (gw[k >> 3] >> (4 * (k & 7))) & 15u;
-}
-
-__device__ inline uint32_t k_code(const uint32_t* row, int bits, int c) {
-    const uint32_t f = k_pair_field(row, bits, c & 63);
+    const uint32_t f = get_field(row, v_field_index(c), 2 * bits);
     return (c < 64) ? (f & ((1u << bits) - 1u)) : (f >> bits);
 }
 

@@ -396,7 +396,9 @@ __global__ void __launch_bounds__(kScanThreads) k_tok_scan(kvq_cfg cfg, kvq_cach
 }
 
 // ---------------------------------------------------------------------------------
-// Per token: encode both rows, pack, and compact the outliers in (h*D + c) order.
+// Per token pair (2u, 2u+1): encode the tokens of this call in it, write their value
+// rows and outliers, then the pair's key blocks (whole when the even token is new,
+// else only the odd half merged into the existing block).
 __device__ void compact_outliers(int n, const uint8_t* flag, const uint16_t* x, uint32_t first,
                                  uint32_t tloc, uint32_t* pos, uint16_t* val, uint32_t* sm) {
     const int per = (n + blockDim.x - 1) / blockDim.x;
@@ -420,75 +422,98 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cach
                                                            const uint16_t* __restrict__ k,
                                                            const uint16_t* __restrict__ v,
                                                            int n_new, QuantWs ws) {
-    const int b = blockIdx.y, i = blockIdx.x;
-    if (i >= ws.ntok[b]) return;
+    const int b = blockIdx.y;
+    const int nt = ws.ntok[b], t0 = ws.t0[b];
+    if (nt == 0) return;
+    const int u = t0 / 2 + blockIdx.x;
+    const int ta = max(2 * u, t0), tb = min(2 * u + 1, t0 + nt - 1);
+    if (ta > tb) return;
     extern __shared__ uint8_t smem[];
     const int n = cfg.Hkv * kD;
-    const int bits = cfg.bits, W = row_words(bits), nbnd = (1 << bits) - 1;
-    uint8_t* kc = smem;
-    uint8_t* vc = kc + n;
-    uint8_t* kf = vc + n;
-    uint8_t* vf = kf + n;
+    const int bits = cfg.bits, W = row_words(bits), KW = block_words(bits), nbnd = (1 << bits) - 1;
+    uint8_t* kc = smem;            // [2][n] key codes of tokens 2u, 2u+1 (0 when absent)
+    uint8_t* vc = kc + 2 * n;      // [n]
+    uint8_t* kf = vc + n;          // [n]
+    uint8_t* vf = kf + n;          // [n]
     __shared__ float bK[16], bV[16];
     __shared__ uint32_t sm[32];
     if (threadIdx.x < nbnd) {
         bK[threadIdx.x] = cbK.bounds[threadIdx.x];
         bV[threadIdx.x] = cbV.bounds[threadIdx.x];
     }
+    for (int j = threadIdx.x; j < 2 * n; j += blockDim.x) kc[j] = 0;
     __syncthreads();
-    const int t = ws.t0[b] + i;
-    const uint16_t* vrow = v + ((size_t)b * n_new + i) * n;
-    const uint16_t* krow = k + ((size_t)b * n_new + i) * n;
-    const uint32_t vt = ws.vthr[(size_t)b * n_new + i];
-    const float vlo = h2f((uint16_t)(vt & 0xffffu)), vhi = h2f((uint16_t)(vt >> 16));
-    const float voff = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0];
-    const float vhalf = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1];
     const uint16_t* kt = c.kthr + (size_t)b * n * 2;
     const float* kp = c.kparams + (size_t)b * n * 2;
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-        const float xk = h2f(krow[j]);
-        const bool ok_ = xk < h2f(kt[2 * j]) || xk > h2f(kt[2 * j + 1]);
-        kf[j] = ok_;
-        kc[j] = (uint8_t)encode(normalize(ok_ ? 0.0f : xk, kp[2 * j], kp[2 * j + 1]), bK, nbnd);
-        const float xv = h2f(vrow[j]);
-        const bool ov = xv < vlo || xv > vhi;
-        vf[j] = ov;
-        vc[j] = (uint8_t)encode(normalize(ov ? 0.0f : xv, voff, vhalf), bV, nbnd);
-    }
-    __syncthreads();
-    const size_t rowbase = ((size_t)b * cfg.T_max + t) * cfg.Hkv * W;
-    for (int wi = threadIdx.x; wi < cfg.Hkv * W; wi += blockDim.x) {
-        const int h = wi / W, ww = wi % W;
-        const int g = ww / bits, wg = ww % bits;
-        const uint8_t* kh = kc + h * kD;
-        const uint8_t* vh = vc + h * kD;
-        uint32_t kw = 0, vw = 0;
-        for (int jf = 0; jf < 16; ++jf) {
-            const int o = 2 * bits * jf - 32 * wg;
-            if (o >= 32 || o + 2 * bits <= 0) continue;
-            const int p = g * 16 + jf;
-            const uint32_t field = (uint32_t)kh[p] | ((uint32_t)kh[p + 64] << bits);
-            kw |= (o >= 0) ? (field << o) : (field >> (-o));
+    for (int t = ta; t <= tb; ++t) {
+        const int i = t - t0;
+        const uint16_t* vrow = v + ((size_t)b * n_new + i) * n;
+        const uint16_t* krow = k + ((size_t)b * n_new + i) * n;
+        const uint32_t vt = ws.vthr[(size_t)b * n_new + i];
+        const float vlo = h2f((uint16_t)(vt & 0xffffu)), vhi = h2f((uint16_t)(vt >> 16));
+        const float voff = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0];
+        const float vhalf = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1];
+        uint8_t* kct = kc + (t & 1) * n;
+        for (int j = threadIdx.x; j < n; j += blockDim.x) {
+            const float xk = h2f(krow[j]);
+            const bool ok_ = xk < h2f(kt[2 * j]) || xk > h2f(kt[2 * j + 1]);
+            kf[j] = ok_;
+            kct[j] = (uint8_t)encode(normalize(ok_ ? 0.0f : xk, kp[2 * j], kp[2 * j + 1]), bK, nbnd);
+            const float xv = h2f(vrow[j]);
+            const bool ov = xv < vlo || xv > vhi;
+            vf[j] = ov;
+            vc[j] = (uint8_t)encode(normalize(ov ? 0.0f : xv, voff, vhalf), bV, nbnd);
         }
-        for (int kk = 0; kk < 32; ++kk) {
-            const uint32_t code = vh[g * 32 + kk];
-            for (int m = 0; m < bits; ++m) {
-                int wd, bt;
-                v_bitpos(bits, kk, m, &wd, &bt);
-                if (wd == wg) vw |= ((code >> m) & 1u) << bt;
+        __syncthreads();
+        // value rows of token t: field f of head h holds code(c) | code(c+64) << bits
+        const size_t vbase = ((size_t)b * cfg.T_max + t) * cfg.Hkv * W;
+        for (int wi = threadIdx.x; wi < cfg.Hkv * W; wi += blockDim.x) {
+            const int h = wi / W, ww = wi % W;
+            const uint8_t* vh = vc + h * kD;
+            const int w2 = 2 * bits;
+            uint32_t word = 0;
+            for (int f = max(0, (32 * ww) / w2 - 1); f < 64 && f * w2 < 32 * ww + 32; ++f) {
+                const int o = f * w2 - 32 * ww;
+                if (o + w2 <= 0) continue;
+                const int ch = v_field_channel(f);
+                const uint32_t field = (uint32_t)vh[ch] | ((uint32_t)vh[ch + 64] << bits);
+                word |= (o >= 0) ? (field << o) : (field >> (-o));
             }
+            c.vcodes[vbase + wi] = word;
         }
-        c.kcodes[rowbase + wi] = kw;
-        c.vcodes[rowbase + wi] = vw;
+        const uint32_t tloc = (uint32_t)(t % kChunk);
+        compact_outliers(n, kf, krow, ws.koff[(size_t)b * n_new + i], tloc,
+                         c.kout_pos + (size_t)b * cfg.out_cap_k,
+                         c.kout_val + (size_t)b * cfg.out_cap_k, sm);
+        __syncthreads();
+        compact_outliers(n, vf, vrow, ws.voff[(size_t)b * n_new + i], tloc,
+                         c.vout_pos + (size_t)b * cfg.out_cap_v,
+                         c.vout_val + (size_t)b * cfg.out_cap_v, sm);
+        __syncthreads();
     }
-    const uint32_t tloc = (uint32_t)(t % kChunk);
-    compact_outliers(n, kf, krow, ws.koff[(size_t)b * n_new + i], tloc,
-                     c.kout_pos + (size_t)b * cfg.out_cap_k, c.kout_val + (size_t)b * cfg.out_cap_k,
-                     sm);
-    __syncthreads();
-    compact_outliers(n, vf, vrow, ws.voff[(size_t)b * n_new + i], tloc,
-                     c.vout_pos + (size_t)b * cfg.out_cap_v, c.vout_val + (size_t)b * cfg.out_cap_v,
-                     sm);
+    // key blocks of pair u: whole block if the even token is written here, else odd half only
+    const bool fresh = (ta == 2 * u);
+    const size_t kbase = ((size_t)b * npairs(cfg.T_max) + u) * cfg.Hkv * KW;
+    for (int wi = threadIdx.x; wi < cfg.Hkv * KW; wi += blockDim.x) {
+        const int h = wi / KW, ww = wi % KW;
+        const int w2 = 2 * bits;
+        uint32_t word = 0, oddmask = 0;
+        for (int f = max(0, (32 * ww) / w2 - 1); f < 128 && f * w2 < 32 * ww + 32; ++f) {
+            const int o = f * w2 - 32 * ww;
+            if (o + w2 <= 0) continue;
+            const int ch = h * kD + k_field_channel(f);
+            const uint32_t field = (uint32_t)kc[ch] | ((uint32_t)kc[n + ch] << bits);
+            const uint32_t om = ((1u << bits) - 1u) << bits;
+            word |= (o >= 0) ? (field << o) : (field >> (-o));
+            oddmask |= (o >= 0) ? (om << o) : (om >> (-o));
+        }
+        if (fresh) {
+            c.kcodes[kbase + wi] = word;
+        } else {
+            const uint32_t old = c.kcodes[kbase + wi];
+            c.kcodes[kbase + wi] = (old & ~oddmask) | (word & oddmask);
+        }
+    }
 }
 
 }  // namespace
@@ -548,6 +573,7 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
     dim3 gt(n_new, C.B);
     k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
     k_tok_scan<<<C.B, kScanThreads, 0, st>>>(C, K, n_new, ws);
-    k_tok_write<<<gt, kTokThreads, 4 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
+    dim3 gw(n_new / 2 + 1, C.B);
+    k_tok_write<<<gw, kTokThreads, 5 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
     return record_cuda(cudaGetLastError());
 }

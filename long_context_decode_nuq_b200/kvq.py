@@ -154,7 +154,8 @@ class Cache:
         nch = (cfg.T_max + CHUNK - 1) // CHUNK + 1
         dev = torch.device(device)
         i32, f32, f16 = torch.int32, torch.float32, torch.float16
-        self.kcodes = torch.zeros((cfg.B, cfg.T_max, cfg.Hkv, W), dtype=i32, device=dev)
+        self.kcodes = torch.zeros((cfg.B, (cfg.T_max + 1) // 2, cfg.Hkv, 2 * W), dtype=i32,
+                                  device=dev)
         self.vcodes = torch.zeros((cfg.B, cfg.T_max, cfg.Hkv, W), dtype=i32, device=dev)
         self.kthr = torch.zeros((cfg.B, n, 2), dtype=f16, device=dev)
         self.kparams = torch.zeros((cfg.B, n, 2), dtype=f32, device=dev)

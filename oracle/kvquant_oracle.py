@@ -38,7 +38,7 @@ listed in the design doc with its ID):
      assignment repeats or after 100 iterations); levels are then rounded to
      the nearest "DB16" binary32 value (bit pattern (u << 16) | u) and
      bounds[j] = binary32((L_j + L_{j+1})/2).
-  R8 packing: see pack_k_row / pack_v_row.
+  R8 packing: see pack_k_block / pack_v_row (a layout of this implementation).
   R9 RoPE: rotate-half pairs (i, i + D/2), theta_i = base^(-2i/D), 0-based
      positions; the query is rotated at its own position.
   R10 scale 1/sqrt(D); every cached token is visible; kv head = hq // (Hq/Hkv).
@@ -220,100 +220,96 @@ def fit_codebook(samples16, f, bits, weights=None, max_iter=100):
 
 
 def row_words(bits: int, D: int = 128) -> int:
+    """Words of one value row (one token, one kv head)."""
     return D * bits // 32
 
 
-def pack_k_row(codes, bits):
-    """Key row: 64 rotate-half pairs (p, p+64) as 2*bits-wide fields.
+def block_words(bits: int, D: int = 128) -> int:
+    """Words of one key block (two tokens, one kv head)."""
+    return 2 * D * bits // 32
 
-    Four pair-groups of ``bits`` words; pair p sits in group p // 16, field
-    p % 16, at bit 2*bits*(p % 16) of the group's little-endian bit string;
-    the field is code[p] | code[p + 64] << bits.
+
+def _k_field_offsets(bits):
+    """Key block: (channel, bit offset of its 2*bits field) for the 128 channels.
+
+    Pair-group j in [0, 16) holds rotate-half pairs p = j + 16m (m in [0, 4)); the
+    field of channel c = p + 64s (s = 0, 1) sits at bit 16*bits*j + 2*bits*(2m + s)
+    and holds code(token 2u, c) | code(token 2u+1, c) << bits.
     """
-    codes = np.asarray(codes, dtype=np.uint64)
-    D = codes.shape[-1]
-    assert D == 128
-    out = np.zeros(codes.shape[:-1] + (4 * bits,), dtype=np.uint64)
-    for p in range(64):
-        g, j = divmod(p, 16)
-        field = codes[..., p] | (codes[..., p + 64] << np.uint64(bits))
-        o = 2 * bits * j
-        w, s = divmod(o, 32)
-        out[..., g * bits + w] |= (field << np.uint64(s)) & np.uint64(0xFFFFFFFF)
-        if s + 2 * bits > 32:
-            out[..., g * bits + w + 1] |= field >> np.uint64(32 - s)
+    out = []
+    for j in range(16):
+        for m in range(4):
+            for sh in range(2):
+                out.append((j + 16 * m + 64 * sh, 16 * bits * j + 2 * bits * (2 * m + sh)))
+    return out
+
+
+def _v_field_offsets(bits):
+    """Value row: (channel c < 64, bit offset) of the field code(c) | code(c+64) << bits.
+
+    Pair-group j in [0, 8) holds channels c = j + 8m (m in [0, 8)); the field sits at
+    bit 16*bits*j + 2*bits*m.
+    """
+    return [(j + 8 * m, 16 * bits * j + 2 * bits * m) for j in range(8) for m in range(8)]
+
+
+def _put_field(out, field, off, width):
+    w, s = divmod(off, 32)
+    out[..., w] |= (field << np.uint64(s)) & np.uint64(0xFFFFFFFF)
+    if s + width > 32:
+        out[..., w + 1] |= field >> np.uint64(32 - s)
+
+
+def _get_field(words, off, width):
+    w, s = divmod(off, 32)
+    v = words[..., w] >> np.uint64(s)
+    if s + width > 32:
+        v = v | (words[..., w + 1] << np.uint64(32 - s))
+    return v & np.uint64((1 << width) - 1)
+
+
+def pack_k_block(codes_even, codes_odd, bits):
+    """Key block of a token pair: codes_even/odd [..., 128] -> [..., 8*bits] words."""
+    ce = np.asarray(codes_even, dtype=np.uint64)
+    co = np.asarray(codes_odd, dtype=np.uint64)
+    assert ce.shape[-1] == 128 and co.shape == ce.shape
+    out = np.zeros(ce.shape[:-1] + (block_words(bits),), dtype=np.uint64)
+    for c, off in _k_field_offsets(bits):
+        _put_field(out, ce[..., c] | (co[..., c] << np.uint64(bits)), off, 2 * bits)
     return out.astype(np.uint32)
 
 
-def _v_bit_positions(bits):
-    """For a 32-code value group: list over codes of [(word, bit)] for each code bit."""
-    pos = []
-    for k in range(32):
-        if bits == 2:
-            w, kk = divmod(k, 16)
-            nib, hi = kk % 8, kk // 8
-            pos.append([(w, 4 * nib + 2 * hi + m) for m in range(2)])
-        elif bits == 3:
-            if k < 24:
-                w, nib = divmod(k, 8)
-                pos.append([(w, 4 * nib + m) for m in range(3)])
-            else:
-                j = k - 24
-                pos.append([(m, 4 * j + 3) for m in range(3)])
-        elif bits == 4:
-            w, nib = divmod(k, 8)
-            pos.append([(w, 4 * nib + m) for m in range(4)])
-        else:
-            raise ValueError(bits)
-    return pos
+def unpack_k_block(words, bits):
+    words = np.asarray(words, dtype=np.uint64)
+    ce = np.zeros(words.shape[:-1] + (128,), dtype=np.uint8)
+    co = np.zeros_like(ce)
+    mask = np.uint64((1 << bits) - 1)
+    for c, off in _k_field_offsets(bits):
+        f = _get_field(words, off, 2 * bits)
+        ce[..., c] = (f & mask).astype(np.uint8)
+        co[..., c] = ((f >> np.uint64(bits)) & mask).astype(np.uint8)
+    return ce, co
 
 
 def pack_v_row(codes, bits):
-    """Value row: four groups of 32 channels (c = 32g + k), ``bits`` words each.
-
-    Nibble format.  bits=3: codes k < 24 occupy bits 0-2 of nibble k % 8 of
-    word k // 8; code 24 + j stores its bit m in bit 3 of nibble j of word m.
-    bits=2: code k occupies bits 2*(k' // 8) .. +1 of nibble k' % 8 of word
-    k // 16 (k' = k % 16).  bits=4: code k is nibble k % 8 of word k // 8.
-    """
+    """Value row of one token: codes [..., 128] -> [..., 4*bits] words."""
     codes = np.asarray(codes, dtype=np.uint64)
     assert codes.shape[-1] == 128
-    out = np.zeros(codes.shape[:-1] + (4 * bits,), dtype=np.uint64)
-    pos = _v_bit_positions(bits)
-    for g in range(4):
-        for k in range(32):
-            c = codes[..., 32 * g + k]
-            for m, (w, b) in enumerate(pos[k]):
-                out[..., g * bits + w] |= ((c >> np.uint64(m)) & np.uint64(1)) << np.uint64(b)
+    out = np.zeros(codes.shape[:-1] + (row_words(bits),), dtype=np.uint64)
+    for c, off in _v_field_offsets(bits):
+        _put_field(out, codes[..., c] | (codes[..., c + 64] << np.uint64(bits)), off, 2 * bits)
     return out.astype(np.uint32)
-
-
-def unpack_k_row(words, bits):
-    words = np.asarray(words, dtype=np.uint64)
-    codes = np.zeros(words.shape[:-1] + (128,), dtype=np.uint8)
-    mask = np.uint64((1 << bits) - 1)
-    for p in range(64):
-        g, j = divmod(p, 16)
-        o = 2 * bits * j
-        w, s = divmod(o, 32)
-        v = words[..., g * bits + w] >> np.uint64(s)
-        if s + 2 * bits > 32:
-            v = v | (words[..., g * bits + w + 1] << np.uint64(32 - s))
-        codes[..., p] = (v & mask).astype(np.uint8)
-        codes[..., p + 64] = ((v >> np.uint64(bits)) & mask).astype(np.uint8)
-    return codes
 
 
 def unpack_v_row(words, bits):
     words = np.asarray(words, dtype=np.uint64)
-    codes = np.zeros(words.shape[:-1] + (128,), dtype=np.uint64)
-    pos = _v_bit_positions(bits)
-    for g in range(4):
-        for k in range(32):
-            for m, (w, b) in enumerate(pos[k]):
-                codes[..., 32 * g + k] |= ((words[..., g * bits + w] >> np.uint64(b))
-                                           & np.uint64(1)) << np.uint64(m)
-    return codes.astype(np.uint8)
+    codes = np.zeros(words.shape[:-1] + (128,), dtype=np.uint8)
+    mask = np.uint64((1 << bits) - 1)
+    for c, off in _v_field_offsets(bits):
+        f = _get_field(words, off, 2 * bits)
+        codes[..., c] = (f & mask).astype(np.uint8)
+        codes[..., c + 64] = ((f >> np.uint64(bits)) & mask).astype(np.uint8)
+    return codes
 
 
 # ----------------------------------------------------------------------------------------
@@ -340,7 +336,7 @@ class QuantizedCache:
         self.n = Hkv * D
         W = row_words(bits, D)
         self.nchunk = (T_max + CHUNK - 1) // CHUNK
-        self.kcodes = np.zeros((B, T_max, Hkv, W), dtype=np.uint32)
+        self.kcodes = np.zeros((B, (T_max + 1) // 2, Hkv, block_words(bits, D)), dtype=np.uint32)
         self.vcodes = np.zeros((B, T_max, Hkv, W), dtype=np.uint32)
         self.kthr = np.zeros((B, self.n, 2), dtype=np.uint16)
         self.kparams = np.zeros((B, self.n, 2), dtype=np.float32)
@@ -395,8 +391,13 @@ class QuantizedCache:
         self.vparams[b, ts, 1] = vhalf
         self.kc[b, ts] = kc
         self.vc[b, ts] = vc
-        self.kcodes[b, ts] = pack_k_row(kc.reshape(ntok, self.Hkv, self.D), self.bits)
         self.vcodes[b, ts] = pack_v_row(vc.reshape(ntok, self.Hkv, self.D), self.bits)
+        # key blocks of every token pair touched; a token not yet written has code 0
+        for u in sorted(set(int(t) // 2 for t in ts)):
+            even = self.kc[b, 2 * u].reshape(self.Hkv, self.D)
+            odd = (self.kc[b, 2 * u + 1] if 2 * u + 1 < self.T_max
+                   else np.zeros(self.n, dtype=np.uint8)).reshape(self.Hkv, self.D)
+            self.kcodes[b, u] = pack_k_block(even, odd, self.bits)
         for s, mask, X in (("k", kout, K), ("v", vout, V)):
             per_tok = mask.sum(axis=1)
             start = int(self.out_count[s][b])

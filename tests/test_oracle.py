@@ -179,6 +179,15 @@ def test_fitted_codebook_properties():
 
 # ---------------------------------------------------------------- packing (R8)
 
+def _spec(spec):
+    codes = np.zeros(128, dtype=np.uint8)
+    for item in spec.split(","):
+        if item:
+            ch, cd = item.split(":")
+            codes[int(ch)] = int(cd)
+    return codes
+
+
 def _golden_rows():
     rows = []
     with open(os.path.join(GOLDEN, "pack_rows.txt")) as fh:
@@ -187,12 +196,13 @@ def _golden_rows():
             if not line or line.startswith("#"):
                 continue
             lhs, rhs = line.split("|")
-            kind, bits, spec = lhs.split()
-            codes = np.zeros(128, dtype=np.uint8)
-            for item in spec.split(","):
-                ch, cd = item.split(":")
-                codes[int(ch)] = int(cd)
+            kind, bits, spec = lhs.split(None, 2)
             words = [int(x, 16) if x.startswith("0x") else int(x) for x in rhs.split()]
+            if kind == "k":
+                ev, od = spec.split("/")
+                codes = (_spec(ev.strip()), _spec(od.strip()))
+            else:
+                codes = _spec(spec.strip())
             rows.append((kind, int(bits), codes, np.array(words, dtype=np.uint32)))
     return rows
 
@@ -201,30 +211,40 @@ def test_pack_golden_rows():
     rows = _golden_rows()
     assert len(rows) >= 6
     for kind, bits, codes, words in rows:
-        pack = O.pack_k_row if kind == "k" else O.pack_v_row
-        got = pack(codes, bits)
-        assert got.shape == (4 * bits,)
+        if kind == "k":
+            got = O.pack_k_block(codes[0], codes[1], bits)
+            assert got.shape == (8 * bits,)
+        else:
+            got = O.pack_v_row(codes, bits)
+            assert got.shape == (4 * bits,)
         assert np.array_equal(got, words), (kind, bits, [hex(x) for x in got])
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_pack_roundtrip_and_bit_budget(bits):
     rng = np.random.default_rng(bits)
-    codes = rng.integers(0, 1 << bits, size=(50, 128)).astype(np.uint8)
-    for pack, unpack in ((O.pack_k_row, O.unpack_k_row), (O.pack_v_row, O.unpack_v_row)):
-        w = pack(codes, bits)
-        assert np.array_equal(unpack(w, bits), codes)
-        # every bit of the row is used exactly once: all-ones codes fill every word
-        full = pack(np.full(128, (1 << bits) - 1, dtype=np.uint8), bits)
-        assert np.all(full == 0xFFFFFFFF)
-        # single-channel codes touch disjoint bits
-        acc = np.zeros(4 * bits, dtype=np.uint64)
-        for ch in range(128):
-            one = np.zeros(128, dtype=np.uint8)
-            one[ch] = (1 << bits) - 1
-            wv = pack(one, bits).astype(np.uint64)
-            assert not np.any(acc & wv)
-            acc |= wv
+    ce = rng.integers(0, 1 << bits, size=(50, 128)).astype(np.uint8)
+    co = rng.integers(0, 1 << bits, size=(50, 128)).astype(np.uint8)
+    assert np.array_equal(O.unpack_v_row(O.pack_v_row(ce, bits), bits), ce)
+    e2, o2 = O.unpack_k_block(O.pack_k_block(ce, co, bits), bits)
+    assert np.array_equal(e2, ce) and np.array_equal(o2, co)
+    full = np.full(128, (1 << bits) - 1, dtype=np.uint8)
+    assert np.all(O.pack_v_row(full, bits) == 0xFFFFFFFF)
+    assert np.all(O.pack_k_block(full, full, bits) == 0xFFFFFFFF)
+    # single codes touch disjoint bits (each bit of a row/block is used exactly once)
+    zero = np.zeros(128, dtype=np.uint8)
+    acc_v = np.zeros(4 * bits, dtype=np.uint64)
+    acc_k = np.zeros(8 * bits, dtype=np.uint64)
+    for ch in range(128):
+        one = zero.copy()
+        one[ch] = (1 << bits) - 1
+        wv = O.pack_v_row(one, bits).astype(np.uint64)
+        assert not np.any(acc_v & wv)
+        acc_v |= wv
+        for ev, od in ((one, zero), (zero, one)):
+            wk = O.pack_k_block(ev, od, bits).astype(np.uint64)
+            assert not np.any(acc_k & wk)
+            acc_k |= wk
 
 
 # ---------------------------------------------------------------- quantizer invariants
