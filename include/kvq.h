@@ -17,7 +17,8 @@
  * Conventions (every entry point):
  *   - Buffers are DEVICE pointers owned by the caller unless a parameter says
  *     "host".  Cache and workspace buffers must be 16-byte aligned.  The library
- *     allocates no memory and keeps no global state.
+ *     allocates no memory; its only global state is the fixed scratch array of
+ *     kvq_quantize_append_noalloc and the per-thread text of the last CUDA error.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls only enqueue work; none synchronizes except kvq_get_status.
  *   - Return value: KVQ_OK (0) or a negative KVQ_ERR_* code.  Argument checks are
@@ -50,6 +51,7 @@ enum {
     KVQ_ERR_RANGE = -5,       /* token range beyond T_max / split count out of range */
     KVQ_ERR_WORKSPACE = -6,   /* workspace smaller than the size query returned */
     KVQ_ERR_CUDA = -7,        /* a CUDA launch or runtime call failed */
+    KVQ_ERR_SCRATCH_LIMIT = -8, /* request exceeds the fixed scratch of kvq_quantize_append_noalloc */
 };
 
 /* Sticky device status bits (cache->status). */
@@ -75,16 +77,15 @@ typedef struct kvq_cfg {
 
 /*
  * Device arrays of one layer's cache (all caller-allocated; sizes from kvq_layout).
- * W = 4*bits words per (token, kv head) row.  Layouts:
- *  kcodes  uint32 [B][T_max][Hkv][W]   key row: 64 rotate-half pairs (p, p+64);
- *          pair-group g = p/16 is `bits` words; pair p is the 2*bits-wide field
- *          code[p] | code[p+64] << bits at bit 2*bits*(p%16) of the group's
- *          little-endian bit string.
- *  vcodes  uint32 [B][T_max][Hkv][W]   value row: channel group g (c = 32g+k) is
- *          `bits` words in nibble format (3 bits: k < 24 -> bits 0-2 of nibble
- *          k%8 of word k/8; k = 24+j -> bit m of the code in bit 3 of nibble j of
- *          word m; 2 bits: word k/16, nibble (k%16)%8, bit pair (k%16)/8;
- *          4 bits: word k/8, nibble k%8).
+ * Layouts (codes are little-endian bit strings over consecutive uint32 words):
+ *  kcodes  uint32 [B][ceil(T_max/2)][Hkv][8*bits]  key block of the token pair
+ *          (2u, 2u+1) of one kv head: channel c = j + 16m + 64s (j < 16, m < 4,
+ *          s in {0,1}) is the 2*bits-wide field code(2u, c) | code(2u+1, c) << bits
+ *          at bit 16*bits*j + 2*bits*(2m + s).  A block whose odd token is not yet
+ *          written holds 0 in the odd half of every field.
+ *  vcodes  uint32 [B][T_max][Hkv][4*bits]  value row of one token and kv head:
+ *          channels c and c + 64 (c = j + 8m < 64, j < 8, m < 8) share the field
+ *          code(c) | code(c + 64) << bits at bit 16*bits*j + 2*bits*m.
  *  kthr    uint16 [B][n][2]  fp16 key thresholds (t_lo, t_hi) per channel
  *  kparams float  [B][n][2]  key channel (off, half)
  *  vparams float  [B][T_max][2] value token (off, half)
@@ -264,6 +265,37 @@ int kvq_fit_workspace(int32_t n_vec, int32_t vec_len, size_t* bytes);
 int kvq_fit_codebook(const uint16_t* samples, int32_t n_vec, int32_t vec_len, double f,
                      const double* weights, int32_t bits, int32_t max_iter, float* levels,
                      float* bounds, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Append tokens without any device allocation and without a workspace argument.
+ * (No counterpart in the KVQuant pages: this is a deployment convenience of this library.)
+ *
+ * For callers that must not allocate device memory on their decode path: serving loops
+ * that keep the allocator out of the per-token step for latency, runtimes that reserve a
+ * fixed device-memory budget up front and hand plug-ins only pre-sized buffers, or code
+ * that has no access to an allocator at all.  It does exactly what
+ * kvq_quantize_append(..., calibrate = 0, ...) does, with its scratch taken from a
+ * file-scope device array of KVQ_NOALLOC_SCRATCH_BYTES that the library owns; every GPU
+ * that loads libkvq.so holds that array until the process exits.
+ *   - Limit: the scratch that kvq_quantize_workspace(cfg, n_new, 0) reports must fit in
+ *     KVQ_NOALLOC_SCRATCH_BYTES (1 MiB, about 20 bytes per (sequence, new token): some
+ *     52,000 of them, e.g. B = 256 sequences appending up to 200 tokens each); larger
+ *     requests return KVQ_ERR_SCRATCH_LIMIT and launch nothing.  Use
+ *     kvq_quantize_append with a caller workspace for prefills.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture begins.
+ *   - All calls share the one array: calls that may run concurrently on the same GPU
+ *     (different streams without ordering) race on it and must not be issued that way.
+ *     Each call writes every scratch entry before reading it, so nothing needs clearing
+ *     between calls.
+ * Arguments, layouts and device-side status behaviour are those of kvq_quantize_append.
+ */
+#define KVQ_NOALLOC_SCRATCH_BYTES (1u << 20)
+int kvq_quantize_append_noalloc(const kvq_cfg* cfg, const kvq_cache* cache,
+                                const kvq_codebook* cbK, const kvq_codebook* cbV,
+                                const uint16_t* k, const uint16_t* v, int32_t n_new,
+                                const int32_t* plen, void* stream);
 
 /* Read the sticky status word into *out (host).  Synchronizes `stream`. */
 int kvq_get_status(const kvq_cache* cache, int32_t* out, void* stream);

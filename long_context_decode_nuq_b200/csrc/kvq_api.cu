@@ -70,6 +70,8 @@ const char* kvq_strerror(int code) {
         case KVQ_ERR_RANGE: return "token range or split count out of range";
         case KVQ_ERR_WORKSPACE: return "workspace too small";
         case KVQ_ERR_CUDA: return g_cuda_msg;
+        case KVQ_ERR_SCRATCH_LIMIT:
+            return "request needs more scratch than the fixed no-alloc array holds";
         default: return "unknown kvq error code";
     }
 }

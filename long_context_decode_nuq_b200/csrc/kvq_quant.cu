@@ -11,6 +11,8 @@
 //   k_tok_scan     per sequence: outlier offsets, the capacity rule, chunk pointers,
 //                  counts and len
 //   k_tok_write    per token: encode, bit-pack both rows, compact the outliers
+#include <mutex>
+
 #include "kvq_common.cuh"
 
 using namespace kvq;
@@ -570,6 +572,63 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
         k_calib_hist<<<gh, 256, kCalCols * 512 * 4, st>>>(C, k, n_new, ws, 2);
         k_calib_select<<<gs, 128, 0, st>>>(C, K, ws, 2);
     }
+    dim3 gt(n_new, C.B);
+    k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
+    k_tok_scan<<<C.B, kScanThreads, 0, st>>>(C, K, n_new, ws);
+    dim3 gw(n_new / 2 + 1, C.B);
+    k_tok_write<<<gw, kTokThreads, 5 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
+    return record_cuda(cudaGetLastError());
+}
+
+// ---------------------------------------------------------------------------------
+// Append without allocation: the scratch lives in this file-scope device array.  Host code
+// must not use the symbol itself as a device address; the address is looked up once per
+// device (with that device current) and passed to the kernels.
+static __device__ __align__(256) unsigned char g_append_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce) return record_cuda(ce);
+    if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_RANGE;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        ce = cudaGetSymbolAddress(&p, g_append_scratch);
+        if (ce) return record_cuda(ce);
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return KVQ_OK;
+}
+}  // namespace
+
+extern "C" int kvq_quantize_append_noalloc(const kvq_cfg* cfg, const kvq_cache* cache,
+                                           const kvq_codebook* cbK, const kvq_codebook* cbV,
+                                           const uint16_t* k, const uint16_t* v, int32_t n_new,
+                                           const int32_t* plen, void* stream) {
+    int e = check_cfg(cfg);
+    if (e) return e;
+    if ((e = check_cache(cfg, cache))) return e;
+    if ((e = check_codebook(cbK)) || (e = check_codebook(cbV))) return e;
+    if (n_new < 0 || n_new > cfg->T_max) return KVQ_ERR_RANGE;
+    if (n_new == 0) return KVQ_OK;
+    if (!k || !v) return KVQ_ERR_NULL;
+    const WsPlan p = plan_ws(*cfg, n_new, 0);
+    if (p.total > (size_t)KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_SCRATCH_LIMIT;
+    void* scratch = nullptr;
+    if ((e = noalloc_scratch(&scratch))) return e;
+    QuantWs ws = bind_ws((char*)scratch, p);
+    cudaStream_t st = (cudaStream_t)stream;
+    const kvq_cfg C = *cfg;
+    const kvq_cache K = *cache;
+    const int n = C.Hkv * kD;
+    k_begin<<<(C.B + 127) / 128, 128, 0, st>>>(C, K, plen, n_new, 0, ws);
     dim3 gt(n_new, C.B);
     k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
     k_tok_scan<<<C.B, kScanThreads, 0, st>>>(C, K, n_new, ws);

@@ -19,13 +19,14 @@ KVQ_STATUS_OUTLIER_OVERFLOW = 1
 KVQ_STATUS_LEN_OVERFLOW = 2
 KVQ_STATUS_NOT_EMPTY = 4
 CHUNK = 64
+NOALLOC_SCRATCH_BYTES = 1 << 20  # KVQ_NOALLOC_SCRATCH_BYTES
 
 EXPORTS = (
     "kvq_abi_version", "kvq_strerror", "kvq_validate_cfg", "kvq_layout", "kvq_cache_reset",
     "kvq_quantize_workspace", "kvq_quantize_append", "kvq_decode_qk", "kvq_decode_splits",
     "kvq_softmax_merge", "kvq_decode_pv", "kvq_decode_workspace", "kvq_decode_attention",
     "kvq_dequantize", "kvq_fp16_decode_attention", "kvq_fit_workspace", "kvq_fit_codebook",
-    "kvq_get_status",
+    "kvq_get_status", "kvq_quantize_append_noalloc",
 )
 
 
@@ -99,6 +100,9 @@ def load():
         "kvq_fit_codebook": ([P, c_int32, c_int32, c_double, P, c_int32, c_int32, P, P, P,
                               c_size_t, P], c_int),
         "kvq_get_status": ([POINTER(CacheStruct), POINTER(c_int32), P], c_int),
+        "kvq_quantize_append_noalloc": ([POINTER(Cfg), POINTER(CacheStruct),
+                                         POINTER(CodebookStruct), POINTER(CodebookStruct), P, P,
+                                         c_int32, P, P], c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -277,6 +281,15 @@ def kvq_fit_codebook(samples, f: float, bits: int, levels, bounds, workspace, we
                                    max_iter, _ptr(levels), _ptr(bounds), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)),
            "kvq_fit_codebook")
+
+
+def kvq_quantize_append_noalloc(cache: Cache, cbK: Codebook, cbV: Codebook, k, v, n_new: int,
+                                plen=None, stream=None) -> None:
+    """Append without a workspace: the library's own fixed device scratch is used instead."""
+    _check(load().kvq_quantize_append_noalloc(
+        ctypes.byref(cache.cfg), ctypes.byref(cache.struct), ctypes.byref(cbK.struct),
+        ctypes.byref(cbV.struct), _ptr(k), _ptr(v), n_new, _ptr(plen), _stream(stream)),
+        "kvq_quantize_append_noalloc")
 
 
 def kvq_get_status(cache: Cache, stream=None) -> int:

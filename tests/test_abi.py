@@ -80,3 +80,26 @@ def test_argument_errors_without_gpu():
     # fit: too many samples
     assert lib.kvq_fit_workspace(5, 5000, ctypes.byref(ctypes.c_size_t())) == -3
     assert K.load().kvq_strerror(-6) == b"workspace too small"
+
+
+def test_noalloc_append_argument_errors_without_gpu():
+    lib = K.load()
+    null = None
+    cfg = K.make_cfg(1, 4, 4, 3, 256, 0.01, 1e4, 64, 64)
+    cb = K.CodebookStruct(0x1000, 0x1000)
+    empty = K.CacheStruct()
+    rc = lib.kvq_quantize_append_noalloc(ctypes.byref(cfg), ctypes.byref(empty), ctypes.byref(cb),
+                                         ctypes.byref(cb), 0x1000, 0x1000, 1, null, null)
+    assert rc == -1
+    # a request whose scratch exceeds the fixed array is refused before any device work
+    big = K.make_cfg(64, 32, 32, 3, 8192, 0.01, 1e4, 64, 64)
+    assert K.kvq_quantize_workspace(big, 4096, 0) > K.NOALLOC_SCRATCH_BYTES
+    fake = K.CacheStruct(*([0x1000] * 15))
+    rc = lib.kvq_quantize_append_noalloc(ctypes.byref(big), ctypes.byref(fake), ctypes.byref(cb),
+                                         ctypes.byref(cb), 0x1000, 0x1000, 4096, null, null)
+    assert rc == -8
+    assert b"scratch" in lib.kvq_strerror(-8)
+    # n_new beyond T_max is a range error, checked before the scratch size
+    rc = lib.kvq_quantize_append_noalloc(ctypes.byref(cfg), ctypes.byref(fake), ctypes.byref(cb),
+                                         ctypes.byref(cb), 0x1000, 0x1000, 257, null, null)
+    assert rc == -5
