@@ -58,6 +58,8 @@ enum {
 #define KVQ_STATUS_OUTLIER_OVERFLOW 1 /* outliers of some tokens did not fit and were dropped */
 #define KVQ_STATUS_LEN_OVERFLOW 2     /* a write past T_max (or a length past max_len) was skipped */
 #define KVQ_STATUS_NOT_EMPTY 4        /* a calibrating prefill met a non-empty sequence; skipped */
+#define KVQ_STATUS_WAIT_TIMEOUT 8     /* a decode kernel gave up waiting for its bulk copies; its
+                                         outputs of that call are invalid */
 
 #define KVQ_CHUNK 64 /* tokens per outlier chunk */
 

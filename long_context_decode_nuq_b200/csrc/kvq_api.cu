@@ -83,10 +83,9 @@ int kvq_layout(const kvq_cfg* cfg, kvq_sizes* out) {
     if (e) return e;
     if (!out) return KVQ_ERR_NULL;
     const size_t B = cfg->B, T = cfg->T_max, n = (size_t)cfg->Hkv * cfg->D;
-    const size_t W = kvq::row_words(cfg->bits);
     const size_t nch = kvq::nchunks(cfg->T_max) + 1;
-    out->kcodes = B * (size_t)kvq::npairs(cfg->T_max) * cfg->Hkv * kvq::block_words(cfg->bits) * 4;
-    out->vcodes = B * T * cfg->Hkv * W * 4;
+    out->kcodes = B * (size_t)kvq::nquads(cfg->T_max) * cfg->Hkv * kvq::block_words(cfg->bits) * 4;
+    out->vcodes = out->kcodes;
     out->kthr = B * n * 2 * 2;
     out->kparams = B * n * 2 * 4;
     out->vparams = B * T * 2 * 4;

@@ -14,10 +14,9 @@ constexpr int kD = 128;          // head dimension (the only one supported)
 constexpr int kPairs = kD / 2;   // rotate-half pairs (p, p + 64)
 constexpr int kChunk = KVQ_CHUNK;
 
-__host__ __device__ inline int row_words(int bits) { return 4 * bits; }    // value row
-__host__ __device__ inline int block_words(int bits) { return 8 * bits; }  // key block (2 tokens)
+__host__ __device__ inline int block_words(int bits) { return 16 * bits; }  // code block (4 tokens)
 __host__ __device__ inline int nchunks(int T_max) { return (T_max + kChunk - 1) / kChunk; }
-__host__ __device__ inline int npairs(int T_max) { return (T_max + 1) / 2; }
+__host__ __device__ inline int nquads(int T_max) { return (T_max + 3) / 4; }
 
 // Outliers kept per side of an N-value vector: floor(f*N/2 + 1/2), capped at (N-1)/2.
 __host__ __device__ inline int vector_k(double f, int N) {
@@ -51,36 +50,25 @@ __device__ inline uint32_t encode(float xn, const float* bounds, int nb) {
     return c;
 }
 
-// ---- key block (token pair 2u, 2u+1; one kv head): channel c = j + 16m + 64s
-// (j in [0,16), m in [0,4), s in {0,1}) has the 2*bits field
-// code(2u, c) | code(2u+1, c) << bits at bit 16*bits*j + 2*bits*(2m + s).
-__host__ __device__ inline int k_field_index(int c) {
-    return 8 * (c & 15) + 2 * ((c & 63) >> 4) + (c >> 6);
+// ---- code block (token quad 4u .. 4u+3; one kv head; keys and values alike): lane group
+// i in [0,16) owns words [bits*i, bits*i + bits) and the rotate-half pairs (c, c + 64) for
+// c = i + 16k (k in [0,4)); the 2*bits field code(4u+j, c) | code(4u+j, c+64) << bits of
+// token j sits in slot s = j ^ (i >> 2), at bit 2*bits*(4k + s) of the group's bit string.
+__host__ __device__ inline int field_offset(int bits, int c, int j) {
+    const int i = c & 15;
+    return 32 * bits * i + 2 * bits * (4 * (c >> 4) + (j ^ (i >> 2)));
 }
-// ---- value row (one token, one kv head): channel c < 64 and c + 64 share the field
-// code(c) | code(c+64) << bits at bit 16*bits*j + 2*bits*m for c = j + 8m.
-__host__ __device__ inline int v_field_index(int c) { return 8 * (c & 7) + ((c & 63) >> 3); }
-// channel of field f (key block: f = 8j + 2m + s; value row: f = 8j + m, channel < 64)
-__host__ __device__ inline int k_field_channel(int f) { return (f >> 3) + 16 * ((f >> 1) & 3) + 64 * (f & 1); }
-__host__ __device__ inline int v_field_channel(int f) { return (f >> 3) + 8 * (f & 7); }
 
-__device__ inline uint32_t get_field(const uint32_t* w, int f, int width) {
-    const int off = f * width;
+__device__ inline uint32_t get_bits(const uint32_t* w, int off, int width) {
     const int wi = off >> 5, s = off & 31;
     uint32_t v = w[wi] >> s;
     if (s + width > 32) v |= w[wi + 1] << (32 - s);
     return v & ((1u << width) - 1u);
 }
 
-// Code of channel c of token (2u + parity) from a key block.
-__device__ inline uint32_t k_code(const uint32_t* block, int bits, int c, int parity) {
-    const uint32_t f = get_field(block, k_field_index(c), 2 * bits);
-    return parity ? (f >> bits) : (f & ((1u << bits) - 1u));
-}
-
-// Code of channel c from a value row.
-__device__ inline uint32_t v_code(const uint32_t* row, int bits, int c) {
-    const uint32_t f = get_field(row, v_field_index(c), 2 * bits);
+// Code of channel c (0 .. 127) of token j of the quad.
+__device__ inline uint32_t block_code(const uint32_t* block, int bits, int c, int j) {
+    const uint32_t f = get_bits(block, field_offset(bits, c & 63, j), 2 * bits);
     return (c < 64) ? (f & ((1u << bits) - 1u)) : (f >> bits);
 }
 

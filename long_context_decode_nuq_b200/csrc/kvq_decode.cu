@@ -2,6 +2,15 @@
 // QK with NUQ lookup + on-the-fly RoPE + key-outlier correction, split-K softmax
 // statistics and merge, and the probability-weighted value sum with value-outlier
 // replacement.  Also the uncompressed fp16 comparison kernel.
+//
+// The two quantized kernels share one shape.  A CTA covers HPC query heads over one split
+// of the tokens and walks it in 64-token chunks.  The chunk's 4-token code blocks (for the
+// kv heads of those query heads) arrive in a ring of shared-memory stages filled by bulk
+// copies (cp.async.bulk, completion counted on an mbarrier; no multicast).  Half-warp qd
+// of the CTA takes token quad qd of the chunk and lane i of the half-warp the rotate-half
+// pairs (c, c + 64), c = i + 16k: exactly the lane group i of the code block, whose token
+// slot s holds token s ^ (i >> 2) (the rotation that lets QK reduce its 16 partials per
+// lane across the half-warp with plain shuffles).
 #include "kvq_common.cuh"
 
 using namespace kvq;
@@ -10,6 +19,11 @@ namespace {
 
 constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
 constexpr int kMaxG = 16;                          // query heads per kv head
+constexpr int kThreads = 256;                      // 8 warps = 16 half-warps
+constexpr int kQuads = kThreads / 16;              // token quads per chunk (64 tokens)
+constexpr int kStages = 4;                         // chunks in the bulk-copy ring
+constexpr int kPitchPad = 64;                      // bytes after each quad row of a stage
+constexpr uint32_t kWaitLimit = 1u << 24;          // mbarrier polls before giving up
 
 __device__ inline float warp_sum(float v) {
 #pragma unroll
@@ -22,6 +36,52 @@ __host__ __device__ inline int split_len(int max_len, int S) {
     int per = (max_len + S - 1) / S;
     per = (per + kChunk - 1) / kChunk * kChunk;
     return per < kChunk ? kChunk : per;
+}
+
+// ---------------------------------------------------------------------------------
+// mbarrier + bulk copy (PTX).
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+                 : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait for the phase with the given parity; false when the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kWaitLimit; ++it)
+        if (mbar_try_wait(bar, parity)) return true;
+    return false;
+}
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // ---------------------------------------------------------------------------------
@@ -45,56 +105,44 @@ __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigne
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
 }
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+    return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
+}
+// (c, s) <- (c, s) rotated by the angle whose (cos, sin) is (rc, rs), in binary64.
+__device__ __forceinline__ void rot64(double& c, double& s, double rc, double rs) {
+    const double nc = c * rc - s * rs, ns = s * rc + c * rs;
+    c = nc;
+    s = ns;
+}
 
 template <int BITS>
 struct Fmt {
-    static constexpr int FW = 2 * BITS;      // field width (two codes)
-    static constexpr int NT = 1 << FW;       // pair-table entries
-    static constexpr int GB = 16 * BITS;     // bits of one lane group
-    static constexpr int KBW = 8 * BITS;     // words of a key block
-    static constexpr int VRW = 4 * BITS;     // words of a value row
+    static constexpr int FW = 2 * BITS;  // field width (codes of c and c + 64)
+    static constexpr int NT = 1 << FW;   // entries of a pair table
+    static constexpr int BW = 16 * BITS; // words of a code block
 };
 
-// First word index and bit shift of lane group j (GB bits at bit GB*j).
-template <int BITS>
-__device__ __forceinline__ void group_pos(int j, int& w, int& sh) {
-    const int bit0 = Fmt<BITS>::GB * j;
-    w = bit0 >> 5;
-    sh = bit0 & 31;
-}
-
-// Align the two words of a lane group so that the group starts at bit 0 of lo.
-template <int BITS>
-__device__ __forceinline__ void group_align(uint32_t w0, uint32_t w1, int sh, uint32_t& lo,
-                                            uint32_t& hi) {
-    if (Fmt<BITS>::GB <= 32) {
-        lo = w0;
-        hi = 0u;
+// A word holding slot F's field (bit FW*F of the lane group's string w[0 .. BITS)) at bit P
+// (the other bits are junk, masked by the caller).
+template <int BITS, int F, int P>
+__device__ __forceinline__ uint32_t field_to(const uint32_t (&w)[BITS]) {
+    constexpr int FW = 2 * BITS;
+    constexpr int O = FW * F;
+    constexpr int wi = O >> 5, sh = O & 31;
+    if constexpr (sh + FW <= 32) {
+        if constexpr (sh >= P)
+            return w[wi] >> (sh - P);
+        else
+            return w[wi] << (P - sh);
     } else {
-        lo = __funnelshift_r(w0, w1, sh);
-        hi = w1 >> sh;
+        static_assert(sh >= P, "a field that crosses words starts above bit P");
+        return __funnelshift_r(w[wi], w[wi + 1], sh - P);
     }
 }
 
-// A word holding the field at bit O of (hi:lo) in bits [7, 7 + FW) (other bits: junk).
-template <int O>
-__device__ __forceinline__ uint32_t field_at7(uint32_t lo, uint32_t hi) {
-    if constexpr (O < 7) {
-        return lo << (7 - O);
-    } else if constexpr (O - 7 < 32) {
-        return __funnelshift_r(lo, hi, O - 7);
-    } else {
-        return hi >> (O - 39);
-    }
-}
-
-template <int BITS>
-__device__ void build_pair_table(const float* levels, float2* tab) {
-    constexpr int NT = Fmt<BITS>::NT;
-    for (int e = threadIdx.x; e < NT * 16; e += blockDim.x) {
-        const int idx = e >> 4;
-        tab[e] = make_float2(levels[idx & ((1 << BITS) - 1)], levels[idx >> BITS]);
-    }
+// Shared-memory table load at a byte offset.
+__device__ __forceinline__ unsigned long long tld(const uint8_t* tab, uint32_t off) {
+    return *reinterpret_cast<const unsigned long long*>(tab + off);
 }
 
 // zhat = off + half * L[encode((0 - off)/half)]: the dense value stored at an outlier.
@@ -104,100 +152,124 @@ __device__ __forceinline__ float zero_code_value(float off, float half, const fl
     return off + half * levels[encode(xn, bounds, nb)];
 }
 
-// Pair-table load: `tab` is a shared-memory table, `off` a byte offset into it.
-__device__ __forceinline__ unsigned long long tld(const unsigned long long* tab, uint32_t off) {
-    return *reinterpret_cast<const unsigned long long*>(reinterpret_cast<const char*>(tab) + off);
+// Head slot of lane i's result after the half-warp reduction, and whether lane i is the
+// one lane (of the lanes holding that result) that writes it.
+template <int HPC>
+__device__ __forceinline__ int out_head(int i) {
+    return HPC == 4 ? (i & 3) : (HPC == 2 ? ((i >> 1) & 1) : 0);
 }
-
-// Byte offset of the pair-table entry of the field at bit O of (hi:lo): rows of 16 lane
-// copies of 8 bytes (128 B per entry), copy `lane16` for this lane: (idx << 7) | lane16 << 3.
-template <int BITS, int O>
-__device__ __forceinline__ uint32_t tab_off(uint32_t lo, uint32_t hi, uint32_t lanebits) {
-    constexpr uint32_t MASK = (uint32_t)(Fmt<BITS>::NT - 1) << 7;
-    return (field_at7<O>(lo, hi) & MASK) | lanebits;
-}
-
-// One rotate-half pair m of a token pair: contribution of channels a = p, b = p + 64
-// (p = j + 16m) to the two tokens' logits,
-//   X = C1 + A1 La + B1 Lb,  Y = C2 + A2 La + B2 Lb,  acc += cos X + sin Y,
-// evaluated for both tokens at once in the two f32x2 lanes.
-template <int BITS, int M>
-__device__ __forceinline__ void qk_step(const unsigned long long* tab, uint32_t lo, uint32_t hi,
-                                        uint32_t lanebits, const float4* csrow,
-                                        const unsigned long long* cf, unsigned long long& acc) {
-    constexpr int FW = Fmt<BITS>::FW;
-    const unsigned long long La = tld(tab, tab_off<BITS, FW * (2 * M)>(lo, hi, lanebits));
-    const unsigned long long Lb = tld(tab, tab_off<BITS, FW * (2 * M + 1)>(lo, hi, lanebits));
-    const float4 cs = csrow[16 * M];
-    unsigned long long X = fma2(cf[6 * M + 0], La, cf[6 * M + 2]);
-    X = fma2(cf[6 * M + 1], Lb, X);
-    unsigned long long Y = fma2(cf[6 * M + 3], La, cf[6 * M + 5]);
-    Y = fma2(cf[6 * M + 4], Lb, Y);
-    acc = fma2(pk(cs.x, cs.y), X, acc);
-    acc = fma2(pk(cs.z, cs.w), Y, acc);
-}
-
-// One value field m of a token: (o_c, o_c+64) += w * (L[code c], L[code c+64]).
-template <int BITS, int M>
-__device__ __forceinline__ void pv_step(const unsigned long long* tab, uint32_t lo, uint32_t hi,
-                                        uint32_t lanebits, unsigned long long w,
-                                        unsigned long long* o) {
-    constexpr int FW = Fmt<BITS>::FW;
-    o[M] = fma2(w, tld(tab, tab_off<BITS, FW * M>(lo, hi, lanebits)), o[M]);
+template <int HPC>
+__device__ __forceinline__ bool out_owner(int i) {
+    return HPC == 4 ? true : (HPC == 2 ? !(i & 1) : !(i & 3));
 }
 
 // ---------------------------------------------------------------------------------
-// QK: CTA = (split, sequence, group of 16 query heads); a half-warp per query head,
-// lane j of it owns rotate-half pairs p = j + 16m (m < 4) of every token pair.
-constexpr int kQKHeads = 16;
-constexpr int kQKThreads = 256;
-constexpr int kRedStride = 176;  // floats per half-warp reduction region (bank skew)
-
-struct QKSmem {  // dynamic part (the pair table is static)
-    static constexpr size_t cs4 = 0;                              // [32 token pairs][64] float4
-    static constexpr size_t s8 = cs4 + 32 * 64 * 16;              // [8][64] float2 (8a*theta)
-    static constexpr size_t s1 = s8 + 8 * 64 * 8;                 // [8][64] float2 (b*theta)
-    static constexpr size_t b8 = s1 + 8 * 64 * 8;                 // [8][64] float2 per chunk
-    static constexpr size_t qr = b8 + 8 * 64 * 8;                 // [16][128] rotated query
-    static constexpr size_t zh = qr + kQKHeads * kD * 4;          // [16][128] zhat per channel
-    static constexpr size_t lg = zh + kQKHeads * kD * 4;          // [64][16] chunk logits
-    static constexpr size_t red = lg + 64 * kQKHeads * 4;         // reduction scratch
-    static constexpr size_t base = red + (kQKThreads / 16) * kRedStride * 4;  // [64] double2
-    static constexpr size_t step = base + 64 * 16;                // [64] double2 (64*theta)
-    static constexpr size_t kb = step + 64 * 16;                  // bounds
-    static constexpr size_t total = kb + 16 * 4;
+// Shared-memory plans (host and device).
+struct QKPlan {
+    int tab, ring, pitch, base, r8, r1, qr, zh, corr, red, kb, bar, flag, total;
 };
+__host__ __device__ inline QKPlan qk_plan(int bits, int hpc, int kvb) {
+    QKPlan p;
+    int o = 0;
+    p.tab = o;  o += hpc * 64 * (1 << (2 * bits)) * 8;       // [entry][head][pair] (X, Y)
+    p.pitch = kvb * 16 * bits * 4 + kPitchPad;
+    p.ring = o; o += kStages * kQuads * p.pitch;
+    p.base = o; o += 3 * 64 * 8;                              // [3][64] (cos, sin) at chunk start
+    p.r8 = o;   o += 8 * 64 * 8;                              // [8][64] rotation by 8a tokens
+    p.r1 = o;   o += 8 * 64 * 8;                              // [8][64] rotation by a tokens
+    p.qr = o;   o += hpc * 128 * 4;                           // rotated, scaled queries
+    p.zh = o;   o += hpc * 128 * 4;                           // dense value at a key outlier
+    p.corr = o; o += 3 * 64 * hpc * 4;                        // [3][64][hpc] outlier corrections
+    p.red = o;  o += kThreads * 8;
+    p.kb = o;   o += 16 * 4;
+    p.bar = o;  o += kStages * 8;
+    p.flag = o; o += 16;
+    p.total = o;
+    return p;
+}
 
-template <int BITS>
-__global__ void __launch_bounds__(kQKThreads, 2) k_qk2(kvq_cfg cfg, kvq_cache c, kvq_codebook cb,
-                                                       const uint16_t* __restrict__ q,
-                                                       const int32_t* __restrict__ qpos, int Ls,
-                                                       int S, int max_len,
-                                                       float* __restrict__ logits,
-                                                       float2* __restrict__ stats) {
+struct PVPlan {
+    int tab, ring, pitch, wsm, psm, vsm, corr, pored, posum, vb, bar, flag, total;
+};
+__host__ __device__ inline PVPlan pv_plan(int bits, int hpc, int kvb) {
+    PVPlan p;
+    int o = 0;
+    p.tab = o;  o += (1 << (2 * bits)) * 16 * 8;              // [entry][16 lane copies] (La, Lb)
+    p.pitch = kvb * 16 * bits * 4 + kPitchPad;
+    p.ring = o;
+    {
+        const int ring = kStages * kQuads * p.pitch, red = kQuads * hpc * 128 * 4;
+        o += ring > red ? ring : red;                         // reused by the final reduction
+    }
+    p.wsm = o;  o += kQuads * 4 * hpc * 8;                    // [quad][token][head] (w, w)
+    p.psm = o;  o += 2 * 64 * hpc * 4;                        // [2][64][hpc] probabilities
+    p.vsm = o;  o += 2 * 64 * 8;                              // [2][64] value (off, half)
+    p.corr = o; o += hpc * 128 * 4;                           // value-outlier corrections
+    p.pored = o; o += kThreads * 4;
+    p.posum = o; o += 16 * 4;
+    p.vb = o;   o += 16 * 4;
+    p.bar = o;  o += kStages * 8;
+    p.flag = o; o += 16;
+    p.total = o;
+    return p;
+}
+
+// Issue the bulk copies of chunk `cc` (quads of [tc, min(tc + 64, t_end)) for the CTA's kv
+// heads) into its ring stage.  One thread.
+__device__ inline void issue_chunk(uint8_t* ring, int pitch, uint64_t* bars, const uint32_t* src0,
+                                   size_t quad_stride, uint32_t row_bytes, int t_begin, int t_end,
+                                   int cc) {
+    const int tc = t_begin + cc * kChunk;
+    const int q0 = tc >> 2, q1 = (min(tc + kChunk, t_end) + 3) >> 2;
+    uint64_t* bar = bars + cc % kStages;
+    uint8_t* dst = ring + (size_t)(cc % kStages) * kQuads * pitch;
+    mbar_arrive_expect_tx(bar, (uint32_t)(q1 - q0) * row_bytes);
+    for (int qq = q0; qq < q1; ++qq)
+        bulk_load(dst + (size_t)(qq - q0) * pitch, src0 + (size_t)qq * quad_stride, row_bytes, bar);
+}
+
+// After an abandoned wait: let every copy still in flight land before the CTA exits.
+__device__ inline void drain_chunks(uint64_t* bars, int from, int to) {
+    for (int cc = from; cc < to; ++cc) mbar_wait(bars + cc % kStages, (cc / kStages) & 1);
+}
+
+// ---------------------------------------------------------------------------------
+// QK.  Per head slot and pair p the CTA tabulates, for every code pair e = (xa, xb),
+//   X = qa (off_a + half_a L[xa]) + qb (off_b + half_b L[xb]),
+//   Y = qb (off_a + half_a L[xa]) - qa (off_b + half_b L[xb])
+// (q the query rotated to its own position and scaled by 1/sqrt(D)); the logit of token t
+// is then sum_p cos(t theta_p) X + sin(t theta_p) Y, one f32x2 FMA per pair and token.
+// The (cos, sin) of a lane's tokens come from the chunk's binary64-derived base times fixed
+// per-lane rotations.  Lane i's accumulator slot (token s, head h) holds token s ^ (i >> 2),
+// head h ^ hperm(i), so the 16 (or 8, 4) partials reduce across the half-warp by halving.
+template <int BITS, int HPC, bool SHARE>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_qk(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const uint16_t* __restrict__ q,
+         const int32_t* __restrict__ qpos, int Ls, int S, int max_len, int kvb,
+         float* __restrict__ logits, float2* __restrict__ stats) {
     using F = Fmt<BITS>;
-    using L = QKSmem;
-    __shared__ __align__(16) unsigned long long ktab[F::NT * 16];
-    extern __shared__ __align__(16) uint8_t sm[];
-    float4* cs4 = (float4*)(sm + L::cs4);
-    float2* s8 = (float2*)(sm + L::s8);
-    float2* s1 = (float2*)(sm + L::s1);
-    float2* b8 = (float2*)(sm + L::b8);
-    float* qr = (float*)(sm + L::qr);
-    float* zh = (float*)(sm + L::zh);
-    float* lg = (float*)(sm + L::lg);
-    float* red = (float*)(sm + L::red);
-    double2* base = (double2*)(sm + L::base);
-    double2* step = (double2*)(sm + L::step);
-    float* kb = (float*)(sm + L::kb);
+    constexpr int LH = HPC == 4 ? 2 : (HPC == 2 ? 1 : 0);
+    constexpr int P = 9 + LH;  // bit of the entry index in a table byte offset
+    constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << P;
+    constexpr int NW = SHARE ? 1 : HPC;
+    constexpr int V = 4 * HPC;  // partials per lane
+    extern __shared__ __align__(128) uint8_t sm[];
+    const QKPlan L = qk_plan(BITS, HPC, kvb);
+    uint8_t* tab = sm + L.tab;
+    uint8_t* ring = sm + L.ring;
+    float2* base = (float2*)(sm + L.base);
+    float2* r8 = (float2*)(sm + L.r8);
+    float2* r1 = (float2*)(sm + L.r1);
+    float* qr = (float*)(sm + L.qr);
+    float* zh = (float*)(sm + L.zh);
+    float* corr = (float*)(sm + L.corr);
+    float* kb = (float*)(sm + L.kb);
+    uint64_t* bars = (uint64_t*)(sm + L.bar);
+    int* flag = (int*)(sm + L.flag);
 
-    const int s = blockIdx.x, b = blockIdx.y, hq0 = blockIdx.z * kQKHeads;
+    const int tid = threadIdx.x, i = tid & 15, qd = tid >> 4, x = i >> 2;
+    const int s = blockIdx.x, b = blockIdx.y, hq0 = blockIdx.z * HPC;
     const int Hq = cfg.Hq, Hkv = cfg.Hkv, g = Hq / Hkv;
-    const int nh = min(kQKHeads, Hq - hq0);
-    const int tid = threadIdx.x, hh = tid >> 4, j = tid & 15;
-    const bool active = hh < nh;
-    const int hq = hq0 + (active ? hh : 0);
-    const int h = hq / g;
     int len = c.len[b];
     if (len > max_len) {
         if (tid == 0 && s == 0 && blockIdx.z == 0) set_status(c.status, KVQ_STATUS_LEN_OVERFLOW);
@@ -205,375 +277,443 @@ __global__ void __launch_bounds__(kQKThreads, 2) k_qk2(kvq_cfg cfg, kvq_cache c,
     }
     const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
     if (t_begin >= t_end) {
-        if (active && j == 0) stats[((size_t)b * Hq + hq) * S + s] = make_float2(-INFINITY, 0.0f);
+        if (tid < HPC) stats[((size_t)b * Hq + hq0 + tid) * S + s] = make_float2(-INFINITY, 0.0f);
         return;
+    }
+    const int nch = (t_end - t_begin + kChunk - 1) / kChunk;
+    const int kv_first = min(hq0 / g, Hkv - kvb);
+    const size_t NQ = nquads(cfg.T_max);
+    const uint32_t* src0 = c.kcodes + ((size_t)b * NQ * Hkv + kv_first) * F::BW;
+    const size_t quad_stride = (size_t)Hkv * F::BW;
+    const uint32_t row_bytes = (uint32_t)kvb * F::BW * 4;
+    if (tid == 0) {
+        for (int k = 0; k < kStages; ++k) mbar_init(bars + k, 1);
+        *flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    int issued = 0;
+    if (tid == 0) {
+        for (; issued < min(kStages, nch); ++issued)
+            issue_chunk(ring, L.pitch, bars, src0, quad_stride, row_bytes, t_begin, t_end, issued);
     }
     // ---- per-CTA tables
     const int nb = (1 << BITS) - 1;
     if (tid < nb) kb[tid] = cb.bounds[tid];
-    for (int e = tid; e < F::NT * 16; e += blockDim.x) {
-        const int idx = e >> 4;
-        ktab[e] = pk(cb.levels[idx & ((1 << BITS) - 1)], cb.levels[idx >> BITS]);
-    }
+    double bc = 0.0, bs = 0.0, sc64 = 1.0, ss64 = 0.0;  // threads < 64: next chunk base
     if (tid < 64) {
         const double th = rope_freq(cfg.rope_theta, tid);
         double cq, sq;
-        rope_cs64((double)t_begin, th, &cq, &sq);
-        base[tid] = make_double2(cq, sq);
-        rope_cs64((double)kChunk, th, &cq, &sq);
-        step[tid] = make_double2(cq, sq);
-        // rotated, scaled query of every head of the CTA at position qpos
         rope_cs64((double)qpos[b], th, &cq, &sq);
-        for (int hh2 = 0; hh2 < nh; ++hh2) {
-            const uint16_t* qv = q + ((size_t)b * Hq + hq0 + hh2) * kD;
+        for (int h = 0; h < HPC; ++h) {
+            const uint16_t* qv = q + ((size_t)b * Hq + hq0 + h) * kD;
             const double qa = (double)h2f(qv[tid]), qb = (double)h2f(qv[tid + 64]);
-            qr[hh2 * kD + tid] = (float)((qa * cq - qb * sq) * (double)kInvSqrtD);
-            qr[hh2 * kD + tid + 64] = (float)((qa * sq + qb * cq) * (double)kInvSqrtD);
+            qr[h * kD + tid] = (float)((qa * cq - qb * sq) * (double)kInvSqrtD);
+            qr[h * kD + tid + 64] = (float)((qa * sq + qb * cq) * (double)kInvSqrtD);
         }
-        const float thf = (float)th;
-        for (int a8 = 0; a8 < 8; ++a8) {
-            float sn, cn;
-            sincosf((float)(8 * a8) * thf, &sn, &cn);
-            s8[a8 * 64 + tid] = make_float2(cn, sn);
-            sincosf((float)a8 * thf, &sn, &cn);
-            s1[a8 * 64 + tid] = make_float2(cn, sn);
+        for (int a = 0; a < 8; ++a) {
+            double cc, ss;
+            rope_cs64((double)(8 * a), th, &cc, &ss);
+            r8[a * 64 + tid] = make_float2((float)cc, (float)ss);
+            rope_cs64((double)a, th, &cc, &ss);
+            r1[a * 64 + tid] = make_float2((float)cc, (float)ss);
         }
+        rope_cs64((double)kChunk, th, &sc64, &ss64);
+        rope_cs64((double)t_begin, th, &bc, &bs);
+        base[tid] = make_float2((float)bc, (float)bs);
+        rot64(bc, bs, sc64, ss64);
+        base[64 + tid] = make_float2((float)bc, (float)bs);
     }
+    for (int e = tid; e < 3 * 64 * HPC; e += kThreads) corr[e] = 0.0f;
     __syncthreads();
     const float* kp = c.kparams + (size_t)b * Hkv * kD * 2;
-    for (int e = tid; e < nh * kD; e += blockDim.x) {
-        const int hh2 = e >> 7, ch = e & 127;
-        const float* p = kp + ((size_t)((hq0 + hh2) / g) * kD + ch) * 2;
-        zh[e] = zero_code_value(p[0], p[1], cb.levels, kb, nb);
+    for (int e = tid; e < HPC * kD; e += kThreads) {
+        const int h = e >> 7, ch = e & 127;
+        const float* pp = kp + ((size_t)((hq0 + h) / g) * kD + ch) * 2;
+        zh[e] = zero_code_value(pp[0], pp[1], cb.levels, kb, nb);
     }
-    // ---- per-lane coefficients, duplicated into both f32x2 halves (one per token)
-    unsigned long long cf[24];
-#pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const int p = j + 16 * m;
-        const float* pa = kp + ((size_t)h * kD + p) * 2;
-        const float* pb = kp + ((size_t)h * kD + p + 64) * 2;
+    for (int e = tid; e < HPC * 64 * F::NT; e += kThreads) {
+        const int p = e & 63, h = (e >> 6) & (HPC - 1), idx = e >> (6 + LH);
+        const int kvh = (hq0 + h) / g;
+        const float* pa = kp + ((size_t)kvh * kD + p) * 2;
+        const float* pb = kp + ((size_t)kvh * kD + p + 64) * 2;
         const float offa = pa[0], halfa = pa[1], offb = pb[0], halfb = pb[1];
-        const float qa = qr[hh * kD + p], qb = qr[hh * kD + p + 64];
+        const float qa = qr[h * kD + p], qb = qr[h * kD + p + 64];
+        const float La = cb.levels[idx & nb], Lb = cb.levels[idx >> BITS];
         const float A1 = qa * halfa, B1 = qb * halfb, C1 = qa * offa + qb * offb;
         const float A2 = qb * halfa, B2 = -qa * halfb, C2 = qb * offa - qa * offb;
-        cf[6 * m + 0] = pk(A1, A1);
-        cf[6 * m + 1] = pk(B1, B1);
-        cf[6 * m + 2] = pk(C1, C1);
-        cf[6 * m + 3] = pk(A2, A2);
-        cf[6 * m + 4] = pk(B2, B2);
-        cf[6 * m + 5] = pk(C2, C2);
+        const float X = fmaf(B1, Lb, fmaf(A1, La, C1));
+        const float Y = fmaf(B2, Lb, fmaf(A2, La, C2));
+        reinterpret_cast<unsigned long long*>(tab)[e] = pk(X, Y);
     }
+    // ---- per-lane constants
+    const int hperm = out_head<HPC>(i);
+    uint32_t lb[HPC];
+#pragma unroll
+    for (int h = 0; h < HPC; ++h) lb[h] = ((uint32_t)(h ^ hperm) << 9) | ((uint32_t)i << 3);
+    uint32_t woff[NW];
+#pragma unroll
+    for (int h = 0; h < NW; ++h) {
+        const int kvs = SHARE ? 0 : (hq0 + (h ^ hperm)) / g - kv_first;
+        woff[h] = (uint32_t)(qd * L.pitch + kvs * F::BW * 4 + i * BITS * 4);
+    }
+    const int khlo = hq0 / g, khhi = (hq0 + HPC - 1) / g;
     const int nch1 = nchunks(cfg.T_max) + 1;
-    const uint32_t* chunk = c.kchunk + (size_t)b * nch1;
+    const uint32_t* kchunk = c.kchunk + (size_t)b * nch1;
     const uint32_t kcount = c.kcount[b];
     const uint32_t* opos = c.kout_pos + (size_t)b * cfg.out_cap_k;
     const uint16_t* oval = c.kout_val + (size_t)b * cfg.out_cap_k;
-    const size_t pair_stride = (size_t)Hkv * F::KBW;
-    int gw_, gsh;
-    group_pos<BITS>(j, gw_, gsh);
-    const uint32_t* kb_lane =
-        c.kcodes + (size_t)b * npairs(cfg.T_max) * pair_stride + (size_t)h * F::KBW + gw_;
-    const uint32_t lanebits = (uint32_t)j << 3;
-    float* myred = red + (tid >> 4) * kRedStride;
+    // key outliers of chunk cc: logit(t, h) += (x - zhat) * (component of q rotated to t)
+    auto outliers = [&](int cc) {
+        const int m = (t_begin + cc * kChunk) / kChunk;
+        const uint32_t lo = min(kchunk[m], kcount), hi = min(kchunk[m + 1], kcount);
+        const float2* bse = base + (cc % 3) * 64;
+        float* cr = corr + (cc % 3) * 64 * HPC;
+        for (uint32_t e = lo + tid; e < hi; e += kThreads) {
+            const uint32_t pw = opos[e];
+            const int tl = (int)(pw >> 16), jf = (int)(pw & 0xffffu);
+            const int kh = jf >> 7, chn = jf & 127;
+            if (tl >= kChunk || kh < khlo || kh > khhi) continue;
+            const int pp = chn & 63;
+            const float2 cs = cmul(cmul(bse[pp], r8[(tl >> 3) * 64 + pp]), r1[(tl & 7) * 64 + pp]);
+            const float xv = h2f(oval[e]);
+#pragma unroll
+            for (int h = 0; h < HPC; ++h) {
+                if ((hq0 + h) / g != kh) continue;
+                const float d = xv - zh[h * kD + chn];
+                const float qa = qr[h * kD + pp], qb = qr[h * kD + pp + 64];
+                const float r = (chn < 64) ? (cs.x * qa + cs.y * qb) : (cs.x * qb - cs.y * qa);
+                atomicAdd(&cr[tl * HPC + h], d * r);
+            }
+        }
+    };
+    __syncthreads();  // tables complete
+    float2 RS[4][4];  // rotation from the chunk start to token 4 qd + (s ^ x), pair i + 16k
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) {
+            const int tau = 4 * qd + (sl ^ x), p = i + 16 * k;
+            RS[k][sl] = cmul(r8[(tau >> 3) * 64 + p], r1[(tau & 7) * 64 + p]);
+        }
+    outliers(0);
+    __syncthreads();
+    const int hs_out = out_head<HPC>(i);
+    const bool owner = out_owner<HPC>(i);
+    const int tq = 4 * qd + x;
     float run_m = -INFINITY, run_l = 0.0f;
-    uint32_t nw0[4], nw1[4];
-    {
-        const uint32_t* cp0 = kb_lane + (size_t)(t_begin >> 1) * pair_stride;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-            const bool ok = active && (t_begin + 2 * qq < t_end);
-            nw0[qq] = ok ? __ldg(cp0 + (size_t)qq * pair_stride) : 0u;
-            nw1[qq] = (ok && F::GB > 32) ? __ldg(cp0 + (size_t)qq * pair_stride + 1) : 0u;
+    int ch = 0;
+    for (; ch < nch; ++ch) {
+        const int tc = t_begin + ch * kChunk;
+        const int slot = ch % kStages;
+        if (!mbar_wait(bars + slot, (uint32_t)(ch / kStages) & 1u)) {
+            atomicOr(flag, 1);
+            set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
         }
-    }
-    for (int tc = t_begin; tc < t_end; tc += kChunk) {
-        // RoPE table of the chunk: cs(tc + d) = base (x) s8[d >> 3] (x) s1[d & 7]
-        __syncthreads();
-        for (int e = tid; e < 8 * 64; e += blockDim.x) {
-            const int i = e & 63;
-            const double2 bb = base[i];
-            const float2 a8 = s8[e];
-            const float bc = (float)bb.x, bs = (float)bb.y;
-            b8[e] = make_float2(bc * a8.x - bs * a8.y, bs * a8.x + bc * a8.y);
-        }
-        __syncthreads();
-        for (int e = tid; e < 32 * 64; e += blockDim.x) {
-            const int u = e >> 6, i = e & 63;
-            const int d0 = 2 * u, d1 = 2 * u + 1;
-            const float2 p0 = b8[(d0 >> 3) * 64 + i], q0 = s1[(d0 & 7) * 64 + i];
-            const float2 p1 = b8[(d1 >> 3) * 64 + i], q1 = s1[(d1 & 7) * 64 + i];
-            cs4[e] = make_float4(p0.x * q0.x - p0.y * q0.y, p1.x * q1.x - p1.y * q1.y,
-                                 p0.y * q0.x + p0.x * q0.y, p1.y * q1.x + p1.x * q1.y);
-        }
-        if (tid < 64) {  // advance the binary64 base angle by 64 tokens for the next chunk
-            const double2 bb = base[tid], st = step[tid];
-            base[tid] = make_double2(bb.x * st.x - bb.y * st.y, bb.y * st.x + bb.x * st.y);
-        }
-        __syncthreads();
-        const int ntok = min(kChunk, t_end - tc);
-        const int npr = (ntok + 1) >> 1;
-        const uint32_t* cp = kb_lane + (size_t)(tc >> 1) * pair_stride;
-        for (int u4 = 0; u4 < npr; u4 += 4) {
-            uint32_t w0[4], w1[4];
+        const uint8_t* stage = ring + (size_t)slot * kQuads * L.pitch;
+        uint32_t w[NW][BITS];
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                w0[qq] = nw0[qq];
-                w1[qq] = nw1[qq];
-                const int un = u4 + 4 + qq;
-                const uint32_t* src = (un < npr) ? cp + (size_t)un * pair_stride
-                                                 : cp + (size_t)(32 + qq) * pair_stride;
-                const bool ok = active && ((un < npr) || (tc + kChunk + 2 * qq < t_end));
-                nw0[qq] = ok ? __ldg(src) : 0u;
-                nw1[qq] = (ok && F::GB > 32) ? __ldg(src + 1) : 0u;
-            }
-            unsigned long long acc[4];
+        for (int h = 0; h < NW; ++h)
 #pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                uint32_t lo, hi;
-                group_align<BITS>(w0[qq], w1[qq], gsh, lo, hi);
-                const float4* csrow = cs4 + (u4 + qq) * 64 + j;
-                unsigned long long a = 0ull;
-                qk_step<BITS, 0>(ktab, lo, hi, lanebits, csrow, cf, a);
-                qk_step<BITS, 1>(ktab, lo, hi, lanebits, csrow, cf, a);
-                qk_step<BITS, 2>(ktab, lo, hi, lanebits, csrow, cf, a);
-                qk_step<BITS, 3>(ktab, lo, hi, lanebits, csrow, cf, a);
-                acc[qq] = a;
-            }
-            // half-warp reduction of 8 token partials over the 16 lanes (via shared memory)
-            {
-                float* row = myred + 8 * j + 8 * (j >> 3);
-                const f2 a0 = upk(acc[0]), a1 = upk(acc[1]), a2 = upk(acc[2]), a3 = upk(acc[3]);
-                *reinterpret_cast<float4*>(row) = make_float4(a0.x, a0.y, a1.x, a1.y);
-                *reinterpret_cast<float4*>(row + 4) = make_float4(a2.x, a2.y, a3.x, a3.y);
-                __syncwarp();
-                const int col = j & 7, r0 = 8 * (j >> 3);
-                float sum = 0.0f;
+            for (int d = 0; d < BITS; ++d)
+                w[h][d] = *reinterpret_cast<const uint32_t*>(stage + woff[h] + 4 * d);
+        const float2* bse = base + (ch % 3) * 64;
+        unsigned long long acc[4][HPC];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int r = r0 + k;
-                    sum += myred[8 * r + 8 * (r >> 3) + col];
+        for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+            for (int h = 0; h < HPC; ++h) acc[sl][h] = 0ull;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 B = bse[i + 16 * k];
+#pragma unroll
+            for (int sl = 0; sl < 4; ++sl) {
+                const float2 cs = cmul(B, RS[k][sl]);
+                const unsigned long long Pc = pk(cs.x, cs.y);
+                uint32_t fs[NW];
+#pragma unroll
+                for (int h = 0; h < NW; ++h) {
+                    switch (4 * k + sl) {
+#define KVQ_FS(N) case N: fs[h] = field_to<BITS, N, P>(w[h]); break;
+                        KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5) KVQ_FS(6)
+                        KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11) KVQ_FS(12)
+                        KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
+#undef KVQ_FS
+                    }
                 }
-                sum += __shfl_xor_sync(0xffffffffu, sum, 8);
-                if (j < 8 && active) lg[(2 * u4 + col) * kQKHeads + hh] = sum;
-                __syncwarp();
-            }
-        }
-        __syncthreads();
-        // key outliers of the chunk: logit += (x - zhat) * (rotated query component)
-        {
-            const int m = tc / kChunk;
-            const uint32_t lo = min(chunk[m], kcount), hi = min(chunk[m + 1], kcount);
-            const int khlo = hq0 / g, khhi = (hq0 + nh - 1) / g;
-            for (uint32_t e = lo + tid; e < hi; e += blockDim.x) {
-                const uint32_t p = opos[e];
-                const int tl = (int)(p >> 16);
-                const int jf = (int)(p & 0xffffu);
-                const int kh = jf >> 7, ch = jf & 127;
-                if (tl >= ntok || kh < khlo || kh > khhi) continue;
-                const float x = h2f(oval[e]);
-                const int i = ch & 63;
-                const float4 cs = cs4[(tl >> 1) * 64 + i];
-                const float cc = (tl & 1) ? cs.y : cs.x, ss = (tl & 1) ? cs.w : cs.z;
-                for (int hq2 = max(kh * g, hq0); hq2 < min(kh * g + g, hq0 + nh); ++hq2) {
-                    const int hh2 = hq2 - hq0;
-                    const float d = x - zh[hh2 * kD + ch];
-                    const float qa = qr[hh2 * kD + i], qb = qr[hh2 * kD + i + 64];
-                    const float r = (ch < 64) ? (cc * qa + ss * qb) : (cc * qb - ss * qa);
-                    atomicAdd(&lg[tl * kQKHeads + hh2], d * r);
+#pragma unroll
+                for (int h = 0; h < HPC; ++h) {
+                    const uint32_t off = (fs[SHARE ? 0 : h] & MASK) | lb[h];
+                    acc[sl][h] = fma2(Pc, tld(tab + 128 * k, off), acc[sl][h]);
                 }
             }
         }
-        __syncthreads();
-        // logits out and the split's running softmax statistics (half-warp per head)
-        {
-            float mx = -INFINITY;
-            float v[4];
+        float v[V];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int tl = j + 16 * k;
-                const bool ok = active && tl < ntok;
-                v[k] = ok ? lg[tl * kQKHeads + hh] : -INFINITY;
-                mx = fmaxf(mx, v[k]);
-                if (ok) logits[((size_t)b * Hq + hq) * cfg.T_max + tc + tl] = v[k];
+        for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+            for (int h = 0; h < HPC; ++h) {
+                const f2 a = upk(acc[sl][h]);
+                v[HPC * sl + h] = a.x + a.y;
             }
+        // halve across the half-warp: lane bit 3, 2, ... pairs the upper half of the partials
+        int mk = 8;
 #pragma unroll
-            for (int o = 8; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            const float mn = fmaxf(run_m, mx);
-            float ssum = 0.0f;
+        for (int half = V / 2; half >= 1; half >>= 1, mk >>= 1)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) ssum += (v[k] > -INFINITY) ? expf(v[k] - mn) : 0.0f;
+            for (int t = 0; t < half; ++t) v[t] += __shfl_xor_sync(0xffffffffu, v[t + half], mk);
 #pragma unroll
-            for (int o = 8; o; o >>= 1) ssum += __shfl_xor_sync(0xffffffffu, ssum, o);
-            if (active) {
-                run_l = (run_m > -INFINITY ? run_l * expf(run_m - mn) : 0.0f) + ssum;
-                run_m = mn;
+        for (int m2 = 16 / V / 2; m2 >= 1; m2 >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], m2);
+        {
+            const int t = tc + tq;
+            const float lgt = v[0] + corr[(ch % 3) * 64 * HPC + tq * HPC + hs_out];
+            if (owner && t < t_end) {
+                logits[((size_t)b * Hq + hq0 + hs_out) * cfg.T_max + t] = lgt;
+                if (lgt > run_m) {
+                    run_l = run_l * expf(run_m - lgt) + 1.0f;
+                    run_m = lgt;
+                } else {
+                    run_l += expf(lgt - run_m);
+                }
             }
         }
+        if (ch + 1 < nch) outliers(ch + 1);
+        if (tid < 64 && ch + 2 < nch) {
+            rot64(bc, bs, sc64, ss64);
+            base[((ch + 2) % 3) * 64 + tid] = make_float2((float)bc, (float)bs);
+        }
+        for (int e = tid; e < 64 * HPC; e += kThreads) corr[((ch + 2) % 3) * 64 * HPC + e] = 0.0f;
+        __syncthreads();
+        if (*flag) break;
+        if (tid == 0 && issued < nch) {
+            fence_proxy_async();
+            issue_chunk(ring, L.pitch, bars, src0, quad_stride, row_bytes, t_begin, t_end, issued);
+            ++issued;
+        }
     }
-    if (active && j == 0) stats[((size_t)b * Hq + hq) * S + s] = make_float2(run_m, run_l);
+    if (tid == 0 && *flag) drain_chunks(bars, ch, issued);
+    float2* red = (float2*)(sm + L.red);
+    red[tid] = owner ? make_float2(run_m, run_l) : make_float2(-INFINITY, 0.0f);
+    __syncthreads();
+    if (tid < HPC) {
+        float M = -INFINITY;
+        for (int e = 0; e < kThreads; ++e)
+            if (out_head<HPC>(e & 15) == tid) M = fmaxf(M, red[e].x);
+        float Ls_ = 0.0f;
+        if (M > -INFINITY)
+            for (int e = 0; e < kThreads; ++e)
+                if (out_head<HPC>(e & 15) == tid && red[e].y > 0.0f)
+                    Ls_ += red[e].y * expf(red[e].x - M);
+        stats[((size_t)b * Hq + hq0 + tid) * S + s] = make_float2(M, Ls_);
+    }
 }
 
 // ---------------------------------------------------------------------------------
-// PV: CTA = (split, sequence, group of 16 query heads); 8 lanes per query head, lane j
-// owns the value fields (c, c + 64) for c = j + 8m (m < 8) of every token.
-constexpr int kPVHeads = 16;
-constexpr int kPVThreads = 8 * kPVHeads;
-
-struct PVSmem {  // dynamic part (the pair table is static)
-    static constexpr size_t w2 = 0;                               // [64][16] (w, w)
-    static constexpr size_t pp = w2 + 64 * kPVHeads * 8;          // [64][16] p
-    static constexpr size_t corr = pp + 64 * kPVHeads * 4;        // [16][128]
-    static constexpr size_t vpar = corr + kPVHeads * kD * 4;      // [64] (off, half)
-    static constexpr size_t zv = vpar + 64 * 8;                   // [64]
-    static constexpr size_t vb = zv + 64 * 4;                     // bounds
-    static constexpr size_t total = vb + 16 * 4;
-};
-
-template <int BITS>
-__global__ void __launch_bounds__(kPVThreads, 4) k_pv2(kvq_cfg cfg, kvq_cache c, kvq_codebook cb,
-                                                    const float* __restrict__ logits,
-                                                    const float2* __restrict__ ml, int Ls, int S,
-                                                    int max_len, float* __restrict__ part) {
+// PV.  out_h = sum_t p_t (off_t + half_t L[code]) = sum_t p_t off_t + sum_t (p_t half_t) L[code];
+// per pair (c, c + 64) and token one (La, Lb) lookup (a 16-copy table, copy = lane) and one
+// f32x2 FMA with (w, w), w = p half.  Lane i computes the weight of (token i >> 2 of its quad,
+// head out_head(i)); value outliers of a chunk are applied during the next one.
+template <int BITS, int HPC, bool SHARE>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_pv(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
+         const float2* __restrict__ ml, int Ls, int S, int max_len, int kvb,
+         float* __restrict__ part) {
     using F = Fmt<BITS>;
-    using L = PVSmem;
-    __shared__ __align__(16) unsigned long long vtab[F::NT * 16];
-    extern __shared__ __align__(16) uint8_t sm[];
-    unsigned long long* w2 = (unsigned long long*)(sm + L::w2);
-    float* pp = (float*)(sm + L::pp);
-    float* corr = (float*)(sm + L::corr);
-    float2* vpar = (float2*)(sm + L::vpar);
-    float* zv = (float*)(sm + L::zv);
-    float* vb = (float*)(sm + L::vb);
-    const int s = blockIdx.x, b = blockIdx.y, hq0 = blockIdx.z * kPVHeads;
+    constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << 7;
+    constexpr int NW = SHARE ? 1 : HPC;
+    extern __shared__ __align__(128) uint8_t sm[];
+    const PVPlan L = pv_plan(BITS, HPC, kvb);
+    uint8_t* tab = sm + L.tab;
+    uint8_t* ring = sm + L.ring;
+    unsigned long long* wsm = (unsigned long long*)(sm + L.wsm);
+    float* psm = (float*)(sm + L.psm);
+    float2* vsm = (float2*)(sm + L.vsm);
+    float* corr = (float*)(sm + L.corr);
+    float* pored = (float*)(sm + L.pored);
+    float* posum = (float*)(sm + L.posum);
+    float* vb = (float*)(sm + L.vb);
+    uint64_t* bars = (uint64_t*)(sm + L.bar);
+    int* flag = (int*)(sm + L.flag);
+
+    const int tid = threadIdx.x, i = tid & 15, qd = tid >> 4, x = i >> 2;
+    const int s = blockIdx.x, b = blockIdx.y, hq0 = blockIdx.z * HPC;
     const int Hq = cfg.Hq, Hkv = cfg.Hkv, g = Hq / Hkv;
-    const int nh = min(kPVHeads, Hq - hq0);
-    const int tid = threadIdx.x, hh = tid >> 3, j = tid & 7;
-    const bool active = hh < nh;
-    const int hq = hq0 + (active ? hh : 0);
-    const int h = hq / g;
     const int len = min(c.len[b], max_len);
     const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
+    if (t_begin >= t_end) {
+        for (int e = tid; e < HPC * kD; e += kThreads)
+            part[(((size_t)b * Hq + hq0 + (e >> 7)) * S + s) * kD + (e & 127)] = 0.0f;
+        return;
+    }
+    const int nch = (t_end - t_begin + kChunk - 1) / kChunk;
+    const int kv_first = min(hq0 / g, Hkv - kvb);
+    const size_t NQ = nquads(cfg.T_max);
+    const uint32_t* src0 = c.vcodes + ((size_t)b * NQ * Hkv + kv_first) * F::BW;
+    const size_t quad_stride = (size_t)Hkv * F::BW;
+    const uint32_t row_bytes = (uint32_t)kvb * F::BW * 4;
+    if (tid == 0) {
+        for (int k = 0; k < kStages; ++k) mbar_init(bars + k, 1);
+        *flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    int issued = 0;
+    if (tid == 0) {
+        for (; issued < min(kStages, nch); ++issued)
+            issue_chunk(ring, L.pitch, bars, src0, quad_stride, row_bytes, t_begin, t_end, issued);
+    }
     const int nb = (1 << BITS) - 1;
     if (tid < nb) vb[tid] = cb.bounds[tid];
-    for (int e = tid; e < F::NT * 16; e += blockDim.x) {
+    for (int e = tid; e < F::NT * 16; e += kThreads) {
         const int idx = e >> 4;
-        vtab[e] = pk(cb.levels[idx & ((1 << BITS) - 1)], cb.levels[idx >> BITS]);
+        reinterpret_cast<unsigned long long*>(tab)[e] =
+            pk(cb.levels[idx & nb], cb.levels[idx >> BITS]);
     }
-    for (int e = tid; e < kPVHeads * kD; e += blockDim.x) corr[e] = 0.0f;
-    unsigned long long o[8];
+    for (int e = tid; e < HPC * kD; e += kThreads) corr[e] = 0.0f;
+    const int hs = out_head<HPC>(i);
+    const bool owner = out_owner<HPC>(i);
+    const int tq = 4 * qd + x;
+    const float2 mL = ml[(size_t)b * Hq + hq0 + hs];
+    const float invL = mL.y > 0.0f ? 1.0f / mL.y : 0.0f;
+    const float* lrow = logits + ((size_t)b * Hq + hq0 + hs) * cfg.T_max;
+    const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
+    float lg = -INFINITY;
+    float2 vp = make_float2(0.0f, 0.0f);
+    auto fetch = [&](int cc) {
+        const int t = t_begin + cc * kChunk + tq;
+        const bool ok = t < t_end;
+        lg = (owner && ok) ? lrow[t] : -INFINITY;
+        vp = ok ? vpar[t] : make_float2(0.0f, 0.0f);
+    };
+    fetch(0);
+    uint32_t woff[NW];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) o[m] = 0ull;
-    float poff = 0.0f;
+    for (int h = 0; h < NW; ++h) {
+        const int kvs = SHARE ? 0 : (hq0 + h) / g - kv_first;
+        woff[h] = (uint32_t)(qd * L.pitch + kvs * F::BW * 4 + i * BITS * 4);
+    }
+    const uint32_t lanebits = (uint32_t)i << 3;
+    const int khlo = hq0 / g, khhi = (hq0 + HPC - 1) / g;
     const int nch1 = nchunks(cfg.T_max) + 1;
-    const uint32_t* chunk = c.vchunk + (size_t)b * nch1;
+    const uint32_t* vchunk = c.vchunk + (size_t)b * nch1;
     const uint32_t vcount = c.vcount[b];
     const uint32_t* opos = c.vout_pos + (size_t)b * cfg.out_cap_v;
     const uint16_t* oval = c.vout_val + (size_t)b * cfg.out_cap_v;
-    const size_t row_stride = (size_t)Hkv * F::VRW;
-    int gw_, gsh;
-    group_pos<BITS>(j, gw_, gsh);
-    const uint32_t* vr_lane = c.vcodes + (size_t)b * cfg.T_max * row_stride + (size_t)h * F::VRW + gw_;
-    const uint32_t lanebits = (uint32_t)(tid & 15) << 3;
-    const float2 mL = active ? ml[(size_t)b * Hq + hq] : make_float2(0.0f, 1.0f);
-    for (int tc = t_begin; tc < t_end; tc += kChunk) {
-        const int ntok = min(kChunk, t_end - tc);
-        const uint32_t* rp = vr_lane + (size_t)tc * row_stride;
-        // first four rows of the chunk in flight while the weights are prepared
-        uint32_t nw0[4], nw1[4];
+    // value outliers of chunk cc: out(h, c) += p(t, h) * (x - zhat_t)
+    auto outliers = [&](int cc) {
+        const int m = (t_begin + cc * kChunk) / kChunk;
+        const uint32_t lo = min(vchunk[m], vcount), hi = min(vchunk[m + 1], vcount);
+        const float* pb = psm + (cc & 1) * 64 * HPC;
+        const float2* vv = vsm + (cc & 1) * 64;
+        for (uint32_t e = lo + tid; e < hi; e += kThreads) {
+            const uint32_t pw = opos[e];
+            const int tl = (int)(pw >> 16), jf = (int)(pw & 0xffffu);
+            const int kh = jf >> 7, chn = jf & 127;
+            if (tl >= kChunk || kh < khlo || kh > khhi) continue;
+            const float2 o2 = vv[tl];
+            const float d = h2f(oval[e]) - zero_code_value(o2.x, o2.y, cb.levels, vb, nb);
 #pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-            const bool ok = active && qq < ntok;
-            nw0[qq] = ok ? __ldg(rp + (size_t)qq * row_stride) : 0u;
-            nw1[qq] = (ok && F::GB > 32) ? __ldg(rp + (size_t)qq * row_stride + 1) : 0u;
-        }
-        __syncthreads();
-        if (tid < kChunk) {
-            float2 vp = make_float2(0.0f, 0.0f);
-            float z = 0.0f;
-            if (tid < ntok) {
-                vp = *(const float2*)(c.vparams + ((size_t)b * cfg.T_max + tc + tid) * 2);
-                z = zero_code_value(vp.x, vp.y, cb.levels, vb, nb);
+            for (int h = 0; h < HPC; ++h) {
+                if ((hq0 + h) / g != kh) continue;
+                atomicAdd(&corr[h * kD + chn], pb[tl * HPC + h] * d);
             }
-            vpar[tid] = vp;
-            zv[tid] = z;
         }
-        __syncthreads();
-        // p_t = exp(l_t - M) / L; w = p * half_t; each of the head's 8 lanes takes 8 tokens
+    };
+    __syncthreads();  // tables complete
+    unsigned long long O[4][HPC];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int h = 0; h < HPC; ++h) O[k][h] = 0ull;
+    float po = 0.0f;
+    int ch = 0;
+    for (; ch < nch; ++ch) {
+        const int slot = ch % kStages;
         {
-            float po = 0.0f;
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int dt = j + 8 * k;
-                float p = 0.0f;
-                if (active && dt < ntok)
-                    p = expf(logits[((size_t)b * Hq + hq) * cfg.T_max + tc + dt] - mL.x) / mL.y;
-                pp[dt * kPVHeads + hh] = p;
-                const float w = p * vpar[dt].y;
-                w2[dt * kPVHeads + hh] = pk(w, w);
-                po += p * vpar[dt].x;
+            const float p = (lg > -INFINITY) ? expf(lg - mL.x) * invL : 0.0f;
+            const float wv = p * vp.y;
+            po += p * vp.x;
+            if (owner) {
+                wsm[(qd * 4 + x) * HPC + hs] = pk(wv, wv);
+                psm[(ch & 1) * 64 * HPC + tq * HPC + hs] = p;
+                if (hs == 0) vsm[(ch & 1) * 64 + tq] = vp;
             }
-            po += __shfl_xor_sync(0xffffffffu, po, 1);
-            po += __shfl_xor_sync(0xffffffffu, po, 2);
-            po += __shfl_xor_sync(0xffffffffu, po, 4);
-            poff += po;
         }
+        if (ch + 1 < nch) fetch(ch + 1);
+        __syncwarp();
+        if (!mbar_wait(bars + slot, (uint32_t)(ch / kStages) & 1u)) {
+            atomicOr(flag, 1);
+            set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+        }
+        const uint8_t* stage = ring + (size_t)slot * kQuads * L.pitch;
+        uint32_t w[NW][BITS];
+#pragma unroll
+        for (int h = 0; h < NW; ++h)
+#pragma unroll
+            for (int d = 0; d < BITS; ++d)
+                w[h][d] = *reinterpret_cast<const uint32_t*>(stage + woff[h] + 4 * d);
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) {
+            unsigned long long ww[HPC];
+#pragma unroll
+            for (int h = 0; h < HPC; ++h) ww[h] = wsm[(qd * 4 + (sl ^ x)) * HPC + h];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                for (int h = 0; h < NW; ++h) {
+                    uint32_t fs = 0;
+                    switch (4 * k + sl) {
+#define KVQ_FS(N) case N: fs = field_to<BITS, N, 7>(w[h]); break;
+                        KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5) KVQ_FS(6)
+                        KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11) KVQ_FS(12)
+                        KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
+#undef KVQ_FS
+                    }
+                    const unsigned long long LL = tld(tab, (fs & MASK) | lanebits);
+                    if (SHARE) {
+#pragma unroll
+                        for (int hh = 0; hh < HPC; ++hh) O[k][hh] = fma2(ww[hh], LL, O[k][hh]);
+                    } else {
+                        O[k][h] = fma2(ww[h], LL, O[k][h]);
+                    }
+                }
+            }
+        }
+        if (ch >= 1) outliers(ch - 1);
         __syncthreads();
-        if (active) {
-            for (int d4 = 0; d4 < ntok; d4 += 4) {
-                uint32_t w0[4], w1[4];
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    w0[qq] = nw0[qq];
-                    w1[qq] = nw1[qq];
-                    const int dn = d4 + 4 + qq;
-                    const bool ok = dn < ntok;
-                    nw0[qq] = ok ? __ldg(rp + (size_t)dn * row_stride) : 0u;
-                    nw1[qq] = (ok && F::GB > 32) ? __ldg(rp + (size_t)dn * row_stride + 1) : 0u;
-                }
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    uint32_t lo, hi;
-                    group_align<BITS>(w0[qq], w1[qq], gsh, lo, hi);
-                    const unsigned long long w = w2[(d4 + qq) * kPVHeads + hh];
-                    pv_step<BITS, 0>(vtab, lo, hi, lanebits, w, o);
-                    pv_step<BITS, 1>(vtab, lo, hi, lanebits, w, o);
-                    pv_step<BITS, 2>(vtab, lo, hi, lanebits, w, o);
-                    pv_step<BITS, 3>(vtab, lo, hi, lanebits, w, o);
-                    pv_step<BITS, 4>(vtab, lo, hi, lanebits, w, o);
-                    pv_step<BITS, 5>(vtab, lo, hi, lanebits, w, o);
-                    pv_step<BITS, 6>(vtab, lo, hi, lanebits, w, o);
-                    pv_step<BITS, 7>(vtab, lo, hi, lanebits, w, o);
-                }
-            }
-        }
-        // value outliers: out += p_t * (x - zhat_t) (shared-memory atomics)
-        {
-            const int m = tc / kChunk;
-            const uint32_t lo = min(chunk[m], vcount), hi = min(chunk[m + 1], vcount);
-            const int khlo = hq0 / g, khhi = (hq0 + nh - 1) / g;
-            for (uint32_t e = lo + tid; e < hi; e += blockDim.x) {
-                const uint32_t p = opos[e];
-                const int tl = (int)(p >> 16);
-                const int jf = (int)(p & 0xffffu);
-                const int kh = jf >> 7, ch = jf & 127;
-                if (tl >= ntok || kh < khlo || kh > khhi) continue;
-                const float d = h2f(oval[e]) - zv[tl];
-                for (int hq2 = max(kh * g, hq0); hq2 < min(kh * g + g, hq0 + nh); ++hq2)
-                    atomicAdd(&corr[(hq2 - hq0) * kD + ch], pp[tl * kPVHeads + (hq2 - hq0)] * d);
-            }
+        if (*flag) break;
+        if (tid == 0 && issued < nch) {
+            fence_proxy_async();
+            issue_chunk(ring, L.pitch, bars, src0, quad_stride, row_bytes, t_begin, t_end, issued);
+            ++issued;
         }
     }
+    if (tid == 0 && *flag) drain_chunks(bars, ch, issued);
+    if (!*flag) outliers(nch - 1);
+    pored[tid] = owner ? po : 0.0f;
     __syncthreads();
-    if (active) {
-        float* dst = part + (((size_t)b * Hq + hq) * S + s) * kD;
+    // partial sums of the 16 quads -> the split's output
+    float* red = (float*)ring;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int ch = j + 8 * m;
-            const f2 v = upk(o[m]);
-            dst[ch] = v.x + poff + corr[hh * kD + ch];
-            dst[ch + 64] = v.y + poff + corr[hh * kD + ch + 64];
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int h = 0; h < HPC; ++h) {
+            const f2 o = upk(O[k][h]);
+            red[(qd * HPC + h) * kD + i + 16 * k] = o.x;
+            red[(qd * HPC + h) * kD + i + 16 * k + 64] = o.y;
         }
+    if (tid < HPC) {
+        float a = 0.0f;
+        for (int e = 0; e < kThreads; ++e)
+            if (out_head<HPC>(e & 15) == tid) a += pored[e];
+        posum[tid] = a;
+    }
+    __syncthreads();
+    for (int e = tid; e < HPC * kD; e += kThreads) {
+        const int h = e >> 7, ch2 = e & 127;
+        float a = posum[h] + corr[h * kD + ch2];
+        for (int qq = 0; qq < kQuads; ++qq) a += red[(qq * HPC + h) * kD + ch2];
+        part[(((size_t)b * Hq + hq0 + h) * S + s) * kD + ch2] = a;
     }
 }
 
@@ -748,11 +888,23 @@ __global__ void __launch_bounds__(kF16Threads) k_fp16_attn(kvq_cfg cfg, const ui
 
 using namespace kvq_host;
 
+// Query heads per CTA of the quantized kernels and the number of kv heads they span.
+static int hpc_of(const kvq_cfg* cfg) { return cfg->Hq % 4 == 0 ? 4 : (cfg->Hq % 2 == 0 ? 2 : 1); }
+static int kvb_of(const kvq_cfg* cfg, int hpc) {
+    const int g = cfg->Hq / cfg->Hkv;
+    int m = 1;
+    for (int hq0 = 0; hq0 < cfg->Hq; hq0 += hpc) {
+        const int span = (hq0 + hpc - 1) / g - hq0 / g + 1;
+        m = span > m ? span : m;
+    }
+    return m;
+}
+
 static int auto_splits(const kvq_cfg* cfg, int max_len) {
-    // about four CTAs per SM over (splits x sequences x 16-query-head groups), >= 128 tokens each
-    const int groups = cfg->B * ((cfg->Hq + 15) / 16);
-    int S = (4 * 148 + groups - 1) / groups;
-    const int maxs = (max_len + 127) / 128;
+    // two waves of one CTA per SM over (splits x sequences x head groups), >= 256 tokens each
+    const int groups = cfg->B * (cfg->Hq / hpc_of(cfg));
+    int S = (2 * 148 + groups - 1) / groups;
+    const int maxs = (max_len + 255) / 256;
     if (S > maxs) S = maxs;
     if (S < 1) S = 1;
     if (S > 4096) S = 4096;
@@ -779,17 +931,43 @@ static int check_decode(const kvq_cfg* cfg, int max_len) {
     return KVQ_OK;
 }
 
+typedef void (*QKKernel)(kvq_cfg, kvq_cache, kvq_codebook, const uint16_t*, const int32_t*, int,
+                         int, int, int, float*, float2*);
+typedef void (*PVKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*, int, int,
+                         int, int, float*);
+
 template <int BITS>
+static QKKernel qk_kernel(int hpc, bool share) {
+    if constexpr (BITS == 4) {
+        return k_qk<4, 1, true>;  // one head's 256-entry pair tables already take 128 KB
+    } else {
+        if (hpc == 4) return share ? k_qk<BITS, 4, true> : k_qk<BITS, 4, false>;
+        if (hpc == 2) return share ? k_qk<BITS, 2, true> : k_qk<BITS, 2, false>;
+        return k_qk<BITS, 1, true>;
+    }
+}
+
+template <int BITS>
+static PVKernel pv_kernel(int hpc, bool share) {
+    if (hpc == 4) return share ? k_pv<BITS, 4, true> : k_pv<BITS, 4, false>;
+    if (hpc == 2) return share ? k_pv<BITS, 2, true> : k_pv<BITS, 2, false>;
+    return k_pv<BITS, 1, true>;
+}
+
 static int launch_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
                      const uint16_t* q, const int32_t* qpos, int max_len, float* logits,
                      float* stats, int S, int Ls, cudaStream_t st) {
-    const size_t smem = QKSmem::total;
-    cudaError_t ce = cudaFuncSetAttribute(k_qk2<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)smem);
+    const int hpc = cfg->bits == 4 ? 1 : hpc_of(cfg);
+    const int kvb = kvb_of(cfg, hpc);
+    QKKernel kern = cfg->bits == 2 ? qk_kernel<2>(hpc, kvb == 1)
+                  : cfg->bits == 3 ? qk_kernel<3>(hpc, kvb == 1)
+                                   : qk_kernel<4>(hpc, kvb == 1);
+    const int smem = qk_plan(cfg->bits, hpc, kvb).total;
+    cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (ce) return record_cuda(ce);
-    dim3 grid(S, cfg->B, (cfg->Hq + kQKHeads - 1) / kQKHeads);
-    k_qk2<BITS><<<grid, kQKThreads, smem, st>>>(*cfg, *cache, *cbK, q, qpos, Ls, S, max_len,
-                                                 logits, (float2*)stats);
+    dim3 grid(S, cfg->B, cfg->Hq / hpc);
+    kern<<<grid, kThreads, smem, st>>>(*cfg, *cache, *cbK, q, qpos, Ls, S, max_len, kvb, logits,
+                                       (float2*)stats);
     return record_cuda(cudaGetLastError());
 }
 
@@ -802,12 +980,7 @@ extern "C" int kvq_decode_qk(const kvq_cfg* cfg, const kvq_cache* cache, const k
     if (!q || !qpos || !logits || !stats) return KVQ_ERR_NULL;
     int S, Ls;
     if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
-    cudaStream_t st = (cudaStream_t)stream;
-    switch (cfg->bits) {
-        case 2: return launch_qk<2>(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, st);
-        case 3: return launch_qk<3>(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, st);
-        default: return launch_qk<4>(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, st);
-    }
+    return launch_qk(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, (cudaStream_t)stream);
 }
 
 extern "C" int kvq_softmax_merge(const kvq_cfg* cfg, const float* stats, int32_t splits,
@@ -823,17 +996,20 @@ extern "C" int kvq_softmax_merge(const kvq_cfg* cfg, const float* stats, int32_t
     return record_cuda(cudaGetLastError());
 }
 
-template <int BITS>
 static int launch_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbV,
                      const float* logits, const float* ml, int max_len, float* part, int S,
                      int Ls, cudaStream_t st) {
-    const size_t smem = PVSmem::total;
-    cudaError_t ce = cudaFuncSetAttribute(k_pv2<BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          (int)smem);
+    const int hpc = hpc_of(cfg);
+    const int kvb = kvb_of(cfg, hpc);
+    PVKernel kern = cfg->bits == 2 ? pv_kernel<2>(hpc, kvb == 1)
+                  : cfg->bits == 3 ? pv_kernel<3>(hpc, kvb == 1)
+                                   : pv_kernel<4>(hpc, kvb == 1);
+    const int smem = pv_plan(cfg->bits, hpc, kvb).total;
+    cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (ce) return record_cuda(ce);
-    dim3 grid(S, cfg->B, (cfg->Hq + kPVHeads - 1) / kPVHeads);
-    k_pv2<BITS><<<grid, kPVThreads, smem, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls,
-                                                 S, max_len, part);
+    dim3 grid(S, cfg->B, cfg->Hq / hpc);
+    kern<<<grid, kThreads, smem, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls, S,
+                                       max_len, kvb, part);
     return record_cuda(cudaGetLastError());
 }
 
@@ -847,12 +1023,7 @@ extern "C" int kvq_decode_pv(const kvq_cfg* cfg, const kvq_cache* cache, const k
     int S, Ls;
     if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
     cudaStream_t st = (cudaStream_t)stream;
-    switch (cfg->bits) {
-        case 2: e = launch_pv<2>(cfg, cache, cbV, logits, ml, max_len, part, S, Ls, st); break;
-        case 3: e = launch_pv<3>(cfg, cache, cbV, logits, ml, max_len, part, S, Ls, st); break;
-        default: e = launch_pv<4>(cfg, cache, cbV, logits, ml, max_len, part, S, Ls, st); break;
-    }
-    if (e) return e;
+    if ((e = launch_pv(cfg, cache, cbV, logits, ml, max_len, part, S, Ls, st))) return e;
     k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
     return record_cuda(cudaGetLastError());
 }

@@ -22,13 +22,12 @@ __global__ void k_dequant_dense(kvq_cfg cfg, kvq_cache c, kvq_codebook cbK, kvq_
         vhat[o] = 0;
         return;
     }
-    const int h = j / kD, ch = j % kD, W = row_words(cfg.bits), KW = block_words(cfg.bits);
-    const uint32_t* kblk = c.kcodes + (((size_t)b * npairs(cfg.T_max) + t / 2) * cfg.Hkv + h) * KW;
-    const uint32_t* vrow = c.vcodes + (((size_t)b * cfg.T_max + t) * cfg.Hkv + h) * W;
+    const int h = j / kD, ch = j % kD, BW = block_words(cfg.bits);
+    const size_t blk = (((size_t)b * nquads(cfg.T_max) + t / 4) * cfg.Hkv + h) * BW;
     const float* kp = c.kparams + ((size_t)b * n + j) * 2;
     const float* vp = c.vparams + ((size_t)b * cfg.T_max + t) * 2;
-    const float lk = cbK.levels[k_code(kblk, cfg.bits, ch, t & 1)];
-    const float lv = cbV.levels[v_code(vrow, cfg.bits, ch)];
+    const float lk = cbK.levels[block_code(c.kcodes + blk, cfg.bits, ch, t & 3)];
+    const float lv = cbV.levels[block_code(c.vcodes + blk, cfg.bits, ch, t & 3)];
     khat[o] = __half_as_ushort(__float2half_rn(__fadd_rn(kp[0], __fmul_rn(kp[1], lk))));
     vhat[o] = __half_as_ushort(__float2half_rn(__fadd_rn(vp[0], __fmul_rn(vp[1], lv))));
 }

@@ -398,9 +398,9 @@ __global__ void __launch_bounds__(kScanThreads) k_tok_scan(kvq_cfg cfg, kvq_cach
 }
 
 // ---------------------------------------------------------------------------------
-// Per token pair (2u, 2u+1): encode the tokens of this call in it, write their value
-// rows and outliers, then the pair's key blocks (whole when the even token is new,
-// else only the odd half merged into the existing block).
+// Per token quad (4u .. 4u+3): encode the tokens of this call in it, write their outliers,
+// then the quad's key and value blocks (whole when the call starts at token 4u, else only
+// the fields of this call's tokens merged into the existing block).
 __device__ void compact_outliers(int n, const uint8_t* flag, const uint16_t* x, uint32_t first,
                                  uint32_t tloc, uint32_t* pos, uint16_t* val, uint32_t* sm) {
     const int per = (n + blockDim.x - 1) / blockDim.x;
@@ -419,6 +419,28 @@ __device__ void compact_outliers(int n, const uint8_t* flag, const uint16_t* x, 
     }
 }
 
+// Word `ww` of the block of kv head h from codes [4][n] of the quad's tokens; *wmask gets
+// the bits of the tokens flagged in `present` (bit j = token j of the quad).
+__device__ inline uint32_t block_word(const uint8_t* codes, int n, int h, int bits, int ww,
+                                      uint32_t present, uint32_t* wmask) {
+    const int w2 = 2 * bits, gi = ww / bits, wl = ww % bits;
+    uint32_t word = 0, m = 0;
+    for (int f = max(0, (32 * wl) / w2 - 1); f < 16 && f * w2 < 32 * wl + 32; ++f) {
+        const int o = f * w2 - 32 * wl;
+        if (o + w2 <= 0) continue;
+        const int j = (f & 3) ^ (gi >> 2);   // token of slot f & 3 in lane group gi
+        if (!((present >> j) & 1u)) continue;
+        const int ch = h * kD + gi + 16 * (f >> 2);
+        const uint32_t field =
+            (uint32_t)codes[j * n + ch] | ((uint32_t)codes[j * n + ch + 64] << bits);
+        const uint32_t fm = (1u << w2) - 1u;
+        word |= (o >= 0) ? (field << o) : (field >> (-o));
+        m |= (o >= 0) ? (fm << o) : (fm >> (-o));
+    }
+    *wmask = m;
+    return word;
+}
+
 __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cache c,
                                                            kvq_codebook cbK, kvq_codebook cbV,
                                                            const uint16_t* __restrict__ k,
@@ -427,15 +449,15 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cach
     const int b = blockIdx.y;
     const int nt = ws.ntok[b], t0 = ws.t0[b];
     if (nt == 0) return;
-    const int u = t0 / 2 + blockIdx.x;
-    const int ta = max(2 * u, t0), tb = min(2 * u + 1, t0 + nt - 1);
+    const int u = t0 / 4 + blockIdx.x;
+    const int ta = max(4 * u, t0), tb = min(4 * u + 3, t0 + nt - 1);
     if (ta > tb) return;
     extern __shared__ uint8_t smem[];
     const int n = cfg.Hkv * kD;
-    const int bits = cfg.bits, W = row_words(bits), KW = block_words(bits), nbnd = (1 << bits) - 1;
-    uint8_t* kc = smem;            // [2][n] key codes of tokens 2u, 2u+1 (0 when absent)
-    uint8_t* vc = kc + 2 * n;      // [n]
-    uint8_t* kf = vc + n;          // [n]
+    const int bits = cfg.bits, BW = block_words(bits), nbnd = (1 << bits) - 1;
+    uint8_t* kc = smem;            // [4][n] key codes of tokens 4u .. 4u+3 (0 when absent)
+    uint8_t* vc = kc + 4 * n;      // [4][n] value codes
+    uint8_t* kf = vc + 4 * n;      // [n] outlier flags of the current token
     uint8_t* vf = kf + n;          // [n]
     __shared__ float bK[16], bV[16];
     __shared__ uint32_t sm[32];
@@ -443,7 +465,7 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cach
         bK[threadIdx.x] = cbK.bounds[threadIdx.x];
         bV[threadIdx.x] = cbV.bounds[threadIdx.x];
     }
-    for (int j = threadIdx.x; j < 2 * n; j += blockDim.x) kc[j] = 0;
+    for (int j = threadIdx.x; j < 8 * n; j += blockDim.x) kc[j] = 0;
     __syncthreads();
     const uint16_t* kt = c.kthr + (size_t)b * n * 2;
     const float* kp = c.kparams + (size_t)b * n * 2;
@@ -455,7 +477,8 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cach
         const float vlo = h2f((uint16_t)(vt & 0xffffu)), vhi = h2f((uint16_t)(vt >> 16));
         const float voff = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0];
         const float vhalf = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1];
-        uint8_t* kct = kc + (t & 1) * n;
+        uint8_t* kct = kc + (t & 3) * n;
+        uint8_t* vct = vc + (t & 3) * n;
         for (int j = threadIdx.x; j < n; j += blockDim.x) {
             const float xk = h2f(krow[j]);
             const bool ok_ = xk < h2f(kt[2 * j]) || xk > h2f(kt[2 * j + 1]);
@@ -464,25 +487,9 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cach
             const float xv = h2f(vrow[j]);
             const bool ov = xv < vlo || xv > vhi;
             vf[j] = ov;
-            vc[j] = (uint8_t)encode(normalize(ov ? 0.0f : xv, voff, vhalf), bV, nbnd);
+            vct[j] = (uint8_t)encode(normalize(ov ? 0.0f : xv, voff, vhalf), bV, nbnd);
         }
         __syncthreads();
-        // value rows of token t: field f of head h holds code(c) | code(c+64) << bits
-        const size_t vbase = ((size_t)b * cfg.T_max + t) * cfg.Hkv * W;
-        for (int wi = threadIdx.x; wi < cfg.Hkv * W; wi += blockDim.x) {
-            const int h = wi / W, ww = wi % W;
-            const uint8_t* vh = vc + h * kD;
-            const int w2 = 2 * bits;
-            uint32_t word = 0;
-            for (int f = max(0, (32 * ww) / w2 - 1); f < 64 && f * w2 < 32 * ww + 32; ++f) {
-                const int o = f * w2 - 32 * ww;
-                if (o + w2 <= 0) continue;
-                const int ch = v_field_channel(f);
-                const uint32_t field = (uint32_t)vh[ch] | ((uint32_t)vh[ch + 64] << bits);
-                word |= (o >= 0) ? (field << o) : (field >> (-o));
-            }
-            c.vcodes[vbase + wi] = word;
-        }
         const uint32_t tloc = (uint32_t)(t % kChunk);
         compact_outliers(n, kf, krow, ws.koff[(size_t)b * n_new + i], tloc,
                          c.kout_pos + (size_t)b * cfg.out_cap_k,
@@ -493,34 +500,30 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cach
                          c.vout_val + (size_t)b * cfg.out_cap_v, sm);
         __syncthreads();
     }
-    // key blocks of pair u: whole block if the even token is written here, else odd half only
-    const bool fresh = (ta == 2 * u);
-    const size_t kbase = ((size_t)b * npairs(cfg.T_max) + u) * cfg.Hkv * KW;
-    for (int wi = threadIdx.x; wi < cfg.Hkv * KW; wi += blockDim.x) {
-        const int h = wi / KW, ww = wi % KW;
-        const int w2 = 2 * bits;
-        uint32_t word = 0, oddmask = 0;
-        for (int f = max(0, (32 * ww) / w2 - 1); f < 128 && f * w2 < 32 * ww + 32; ++f) {
-            const int o = f * w2 - 32 * ww;
-            if (o + w2 <= 0) continue;
-            const int ch = h * kD + k_field_channel(f);
-            const uint32_t field = (uint32_t)kc[ch] | ((uint32_t)kc[n + ch] << bits);
-            const uint32_t om = ((1u << bits) - 1u) << bits;
-            word |= (o >= 0) ? (field << o) : (field >> (-o));
-            oddmask |= (o >= 0) ? (om << o) : (om >> (-o));
-        }
-        if (fresh) {
-            c.kcodes[kbase + wi] = word;
-        } else {
-            const uint32_t old = c.kcodes[kbase + wi];
-            c.kcodes[kbase + wi] = (old & ~oddmask) | (word & oddmask);
-        }
+    // key and value blocks of quad u
+    uint32_t present = 0;
+    for (int t = ta; t <= tb; ++t) present |= 1u << (t & 3);
+    const bool fresh = (ta == 4 * u);
+    const size_t base = ((size_t)b * nquads(cfg.T_max) + u) * cfg.Hkv * BW;
+    for (int wi = threadIdx.x; wi < 2 * cfg.Hkv * BW; wi += blockDim.x) {
+        const int which = wi >= cfg.Hkv * BW;
+        const int wv = wi - which * cfg.Hkv * BW;
+        uint32_t m;
+        const uint32_t word = block_word(which ? vc : kc, n, wv / BW, bits, wv % BW, present, &m);
+        uint32_t* dst = (which ? c.vcodes : c.kcodes) + base + wv;
+        *dst = fresh ? word : ((*dst & ~m) | word);
     }
 }
 
 }  // namespace
 
 using namespace kvq_host;
+
+// k_tok_write keeps the codes of a token quad in shared memory: 10 bytes per channel.
+static int tok_write_smem(int n) {
+    return record_cuda(cudaFuncSetAttribute(k_tok_write, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            10 * n));
+}
 
 extern "C" int kvq_quantize_workspace(const kvq_cfg* cfg, int32_t n_new, int32_t calibrate,
                                       size_t* bytes) {
@@ -552,6 +555,7 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
     cudaStream_t st = (cudaStream_t)stream;
     const kvq_cfg C = *cfg;
     const kvq_cache K = *cache;
+    if ((e = tok_write_smem(n))) return e;
     k_begin<<<(C.B + 127) / 128, 128, 0, st>>>(C, K, plen, n_new, calibrate, ws);
     if (calibrate) {
         cudaError_t ce;
@@ -575,8 +579,8 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
     dim3 gt(n_new, C.B);
     k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
     k_tok_scan<<<C.B, kScanThreads, 0, st>>>(C, K, n_new, ws);
-    dim3 gw(n_new / 2 + 1, C.B);
-    k_tok_write<<<gw, kTokThreads, 5 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
+    dim3 gw((n_new + 2) / 4 + 1, C.B);
+    k_tok_write<<<gw, kTokThreads, 10 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
     return record_cuda(cudaGetLastError());
 }
 
@@ -628,11 +632,12 @@ extern "C" int kvq_quantize_append_noalloc(const kvq_cfg* cfg, const kvq_cache* 
     const kvq_cfg C = *cfg;
     const kvq_cache K = *cache;
     const int n = C.Hkv * kD;
+    if ((e = tok_write_smem(n))) return e;
     k_begin<<<(C.B + 127) / 128, 128, 0, st>>>(C, K, plen, n_new, 0, ws);
     dim3 gt(n_new, C.B);
     k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
     k_tok_scan<<<C.B, kScanThreads, 0, st>>>(C, K, n_new, ws);
-    dim3 gw(n_new / 2 + 1, C.B);
-    k_tok_write<<<gw, kTokThreads, 5 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
+    dim3 gw((n_new + 2) / 4 + 1, C.B);
+    k_tok_write<<<gw, kTokThreads, 10 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
     return record_cuda(cudaGetLastError());
 }

@@ -18,6 +18,7 @@ KVQ_OK = 0
 KVQ_STATUS_OUTLIER_OVERFLOW = 1
 KVQ_STATUS_LEN_OVERFLOW = 2
 KVQ_STATUS_NOT_EMPTY = 4
+KVQ_STATUS_WAIT_TIMEOUT = 8
 CHUNK = 64
 NOALLOC_SCRATCH_BYTES = 1 << 20  # KVQ_NOALLOC_SCRATCH_BYTES
 
@@ -154,13 +155,13 @@ class Cache:
         self.cfg = cfg
         sz = kvq_layout(cfg)
         n = cfg.Hkv * cfg.D
-        W = 4 * cfg.bits
+        BW = 16 * cfg.bits                      # words of a 4-token code block
+        nq = (cfg.T_max + 3) // 4
         nch = (cfg.T_max + CHUNK - 1) // CHUNK + 1
         dev = torch.device(device)
         i32, f32, f16 = torch.int32, torch.float32, torch.float16
-        self.kcodes = torch.zeros((cfg.B, (cfg.T_max + 1) // 2, cfg.Hkv, 2 * W), dtype=i32,
-                                  device=dev)
-        self.vcodes = torch.zeros((cfg.B, cfg.T_max, cfg.Hkv, W), dtype=i32, device=dev)
+        self.kcodes = torch.zeros((cfg.B, nq, cfg.Hkv, BW), dtype=i32, device=dev)
+        self.vcodes = torch.zeros((cfg.B, nq, cfg.Hkv, BW), dtype=i32, device=dev)
         self.kthr = torch.zeros((cfg.B, n, 2), dtype=f16, device=dev)
         self.kparams = torch.zeros((cfg.B, n, 2), dtype=f32, device=dev)
         self.vparams = torch.zeros((cfg.B, cfg.T_max, 2), dtype=f32, device=dev)

@@ -38,7 +38,8 @@ listed in the design doc with its ID):
      assignment repeats or after 100 iterations); levels are then rounded to
      the nearest "DB16" binary32 value (bit pattern (u << 16) | u) and
      bounds[j] = binary32((L_j + L_{j+1})/2).
-  R8 packing: see pack_k_block / pack_v_row (a layout of this implementation).
+  R8 packing: see pack_block (a layout of this implementation, shared by keys
+     and values: 4-token blocks per kv head).
   R9 RoPE: rotate-half pairs (i, i + D/2), theta_i = base^(-2i/D), 0-based
      positions; the query is rotated at its own position.
   R10 scale 1/sqrt(D); every cached token is visible; kv head = hq // (Hq/Hkv).
@@ -219,38 +220,22 @@ def fit_codebook(samples16, f, bits, weights=None, max_iter=100):
 # ----------------------------------------------------------------------------------------
 
 
-def row_words(bits: int, D: int = 128) -> int:
-    """Words of one value row (one token, one kv head)."""
-    return D * bits // 32
-
-
 def block_words(bits: int, D: int = 128) -> int:
-    """Words of one key block (two tokens, one kv head)."""
-    return 2 * D * bits // 32
+    """Words of one code block (four tokens, one kv head)."""
+    return 4 * D * bits // 32
 
 
-def _k_field_offsets(bits):
-    """Key block: (channel, bit offset of its 2*bits field) for the 128 channels.
+def _field_offsets(bits):
+    """Code block: (channel c < 64, token j of the quad, bit offset of its 2*bits field).
 
-    Pair-group j in [0, 16) holds rotate-half pairs p = j + 16m (m in [0, 4)); the
-    field of channel c = p + 64s (s = 0, 1) sits at bit 16*bits*j + 2*bits*(2m + s)
-    and holds code(token 2u, c) | code(token 2u+1, c) << bits.
+    Lane group i in [0, 16) owns words [bits*i, bits*i + bits) and the rotate-half
+    pairs (c, c + 64) for c = i + 16k (k in [0, 4)).  In the group's bit string, slot
+    f = 4k + s sits at bit 2*bits*f and holds the field code(4u + j, c) | code(4u + j,
+    c + 64) << bits of token j = s XOR (i >> 2) (the token order within a slot row is
+    rotated per lane group).  Keys and values use the same block.
     """
-    out = []
-    for j in range(16):
-        for m in range(4):
-            for sh in range(2):
-                out.append((j + 16 * m + 64 * sh, 16 * bits * j + 2 * bits * (2 * m + sh)))
-    return out
-
-
-def _v_field_offsets(bits):
-    """Value row: (channel c < 64, bit offset) of the field code(c) | code(c+64) << bits.
-
-    Pair-group j in [0, 8) holds channels c = j + 8m (m in [0, 8)); the field sits at
-    bit 16*bits*j + 2*bits*m.
-    """
-    return [(j + 8 * m, 16 * bits * j + 2 * bits * m) for j in range(8) for m in range(8)]
+    return [(i + 16 * k, s ^ (i >> 2), 32 * bits * i + 2 * bits * (4 * k + s))
+            for i in range(16) for k in range(4) for s in range(4)]
 
 
 def _put_field(out, field, off, width):
@@ -268,47 +253,26 @@ def _get_field(words, off, width):
     return v & np.uint64((1 << width) - 1)
 
 
-def pack_k_block(codes_even, codes_odd, bits):
-    """Key block of a token pair: codes_even/odd [..., 128] -> [..., 8*bits] words."""
-    ce = np.asarray(codes_even, dtype=np.uint64)
-    co = np.asarray(codes_odd, dtype=np.uint64)
-    assert ce.shape[-1] == 128 and co.shape == ce.shape
-    out = np.zeros(ce.shape[:-1] + (block_words(bits),), dtype=np.uint64)
-    for c, off in _k_field_offsets(bits):
-        _put_field(out, ce[..., c] | (co[..., c] << np.uint64(bits)), off, 2 * bits)
+def pack_block(codes, bits):
+    """Code block of a token quad: codes [4, ..., 128] (token j of the quad first) ->
+    [..., 16*bits] words."""
+    cs = [np.asarray(c, dtype=np.uint64) for c in codes]
+    assert len(cs) == 4 and all(c.shape == cs[0].shape for c in cs) and cs[0].shape[-1] == 128
+    out = np.zeros(cs[0].shape[:-1] + (block_words(bits),), dtype=np.uint64)
+    for c, j, off in _field_offsets(bits):
+        _put_field(out, cs[j][..., c] | (cs[j][..., c + 64] << np.uint64(bits)), off, 2 * bits)
     return out.astype(np.uint32)
 
 
-def unpack_k_block(words, bits):
+def unpack_block(words, bits):
+    """Inverse of pack_block: words [..., 16*bits] -> codes [4, ..., 128] (uint8)."""
     words = np.asarray(words, dtype=np.uint64)
-    ce = np.zeros(words.shape[:-1] + (128,), dtype=np.uint8)
-    co = np.zeros_like(ce)
+    codes = np.zeros((4,) + words.shape[:-1] + (128,), dtype=np.uint8)
     mask = np.uint64((1 << bits) - 1)
-    for c, off in _k_field_offsets(bits):
+    for c, j, off in _field_offsets(bits):
         f = _get_field(words, off, 2 * bits)
-        ce[..., c] = (f & mask).astype(np.uint8)
-        co[..., c] = ((f >> np.uint64(bits)) & mask).astype(np.uint8)
-    return ce, co
-
-
-def pack_v_row(codes, bits):
-    """Value row of one token: codes [..., 128] -> [..., 4*bits] words."""
-    codes = np.asarray(codes, dtype=np.uint64)
-    assert codes.shape[-1] == 128
-    out = np.zeros(codes.shape[:-1] + (row_words(bits),), dtype=np.uint64)
-    for c, off in _v_field_offsets(bits):
-        _put_field(out, codes[..., c] | (codes[..., c + 64] << np.uint64(bits)), off, 2 * bits)
-    return out.astype(np.uint32)
-
-
-def unpack_v_row(words, bits):
-    words = np.asarray(words, dtype=np.uint64)
-    codes = np.zeros(words.shape[:-1] + (128,), dtype=np.uint8)
-    mask = np.uint64((1 << bits) - 1)
-    for c, off in _v_field_offsets(bits):
-        f = _get_field(words, off, 2 * bits)
-        codes[..., c] = (f & mask).astype(np.uint8)
-        codes[..., c + 64] = ((f >> np.uint64(bits)) & mask).astype(np.uint8)
+        codes[j][..., c] = (f & mask).astype(np.uint8)
+        codes[j][..., c + 64] = ((f >> np.uint64(bits)) & mask).astype(np.uint8)
     return codes
 
 
@@ -334,10 +298,10 @@ class QuantizedCache:
         assert D == 128
         self.B, self.Hkv, self.D, self.bits, self.T_max, self.f = B, Hkv, D, bits, T_max, f
         self.n = Hkv * D
-        W = row_words(bits, D)
         self.nchunk = (T_max + CHUNK - 1) // CHUNK
-        self.kcodes = np.zeros((B, (T_max + 1) // 2, Hkv, block_words(bits, D)), dtype=np.uint32)
-        self.vcodes = np.zeros((B, T_max, Hkv, W), dtype=np.uint32)
+        nq = (T_max + 3) // 4
+        self.kcodes = np.zeros((B, nq, Hkv, block_words(bits, D)), dtype=np.uint32)
+        self.vcodes = np.zeros((B, nq, Hkv, block_words(bits, D)), dtype=np.uint32)
         self.kthr = np.zeros((B, self.n, 2), dtype=np.uint16)
         self.kparams = np.zeros((B, self.n, 2), dtype=np.float32)
         self.vparams = np.zeros((B, T_max, 2), dtype=np.float32)
@@ -391,13 +355,13 @@ class QuantizedCache:
         self.vparams[b, ts, 1] = vhalf
         self.kc[b, ts] = kc
         self.vc[b, ts] = vc
-        self.vcodes[b, ts] = pack_v_row(vc.reshape(ntok, self.Hkv, self.D), self.bits)
-        # key blocks of every token pair touched; a token not yet written has code 0
-        for u in sorted(set(int(t) // 2 for t in ts)):
-            even = self.kc[b, 2 * u].reshape(self.Hkv, self.D)
-            odd = (self.kc[b, 2 * u + 1] if 2 * u + 1 < self.T_max
-                   else np.zeros(self.n, dtype=np.uint8)).reshape(self.Hkv, self.D)
-            self.kcodes[b, u] = pack_k_block(even, odd, self.bits)
+        # code blocks of every token quad touched; a token not yet written has code 0
+        zero = np.zeros((self.Hkv, self.D), dtype=np.uint8)
+        for u in sorted(set(int(t) // 4 for t in ts)):
+            for arr, cc in ((self.kcodes, self.kc), (self.vcodes, self.vc)):
+                quad = [cc[b, 4 * u + j].reshape(self.Hkv, self.D) if 4 * u + j < self.T_max
+                        else zero for j in range(4)]
+                arr[b, u] = pack_block(quad, self.bits)
         for s, mask, X in (("k", kout, K), ("v", vout, V)):
             per_tok = mask.sum(axis=1)
             start = int(self.out_count[s][b])

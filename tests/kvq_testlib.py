@@ -67,7 +67,7 @@ def compare_cache(g, o, B, hard=True):
         errs.append(f"len {glen} vs {o.len}")
     for b in range(B):
         L = int(o.len[b])
-        for name, n_rows in (("kcodes", (L + 1) // 2), ("vcodes", L)):
+        for name, n_rows in (("kcodes", (L + 3) // 4), ("vcodes", (L + 3) // 4)):
             gv = u32(getattr(g, name)[b, :n_rows])
             ov = getattr(o, name)[b, :n_rows]
             if not np.array_equal(gv, ov):

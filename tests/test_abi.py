@@ -45,7 +45,10 @@ def test_cfg_validation():
 def test_layout_sizes():
     cfg = K.make_cfg(2, 8, 4, 3, 1000, 0.01, 1e4, 50, 70)
     s = K.kvq_layout(cfg)
-    assert s["kcodes"] == 2 * 1000 * 4 * 12 * 4
+    assert s["kcodes"] == 2 * 1000 * 4 * 12 * 4 and s["vcodes"] == s["kcodes"]
+    # code blocks hold four tokens: T_max is rounded up to a multiple of 4
+    s2 = K.kvq_layout(K.make_cfg(2, 8, 4, 3, 1001, 0.01, 1e4, 50, 70))
+    assert s2["kcodes"] == s2["vcodes"] == 2 * 251 * 4 * 48 * 4
     assert s["vparams"] == 2 * 1000 * 2 * 4
     assert s["kout_pos"] == 2 * 50 * 4 and s["vout_val"] == 2 * 70 * 2
     assert s["kchunk"] == 2 * (16 + 1) * 4

@@ -22,6 +22,11 @@ CASES = [
     ("batched_8x8k", dict(B=2, Hq=4, Hkv=4, bits=4), 200, [200, 150], 0),
     ("llama3_8b_gqa_128k", dict(B=2, Hq=16, Hkv=4), 517, [517, 300], 0),
     ("llama7b_layer_32k", dict(Hq=32, Hkv=32), 260, None, 1),
+    # four query heads over two kv heads per CTA; two query heads per CTA (shared / not)
+    ("llama7b_layer_32k", dict(Hq=8, Hkv=4), 301, None, 1),
+    ("llama3_8b_gqa_128k", dict(B=1, Hq=6, Hkv=3), 250, None, 0),
+    ("llama3_8b_gqa_128k", dict(B=1, Hq=6, Hkv=6, bits=2), 190, None, 0),
+    ("llama3_8b_gqa_128k", dict(B=2, Hq=8, Hkv=2, bits=4), 330, [330, 97], 1),
 ]
 
 

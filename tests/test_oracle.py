@@ -197,54 +197,44 @@ def _golden_rows():
                 continue
             lhs, rhs = line.split("|")
             kind, bits, spec = lhs.split(None, 2)
+            assert kind == "b"
             words = [int(x, 16) if x.startswith("0x") else int(x) for x in rhs.split()]
-            if kind == "k":
-                ev, od = spec.split("/")
-                codes = (_spec(ev.strip()), _spec(od.strip()))
-            else:
-                codes = _spec(spec.strip())
-            rows.append((kind, int(bits), codes, np.array(words, dtype=np.uint32)))
+            toks = [_spec(x.strip()) for x in spec.split("/")]
+            assert len(toks) == 4
+            rows.append((int(bits), toks, np.array(words, dtype=np.uint32)))
     return rows
 
 
 def test_pack_golden_rows():
     rows = _golden_rows()
-    assert len(rows) >= 6
-    for kind, bits, codes, words in rows:
-        if kind == "k":
-            got = O.pack_k_block(codes[0], codes[1], bits)
-            assert got.shape == (8 * bits,)
-        else:
-            got = O.pack_v_row(codes, bits)
-            assert got.shape == (4 * bits,)
-        assert np.array_equal(got, words), (kind, bits, [hex(x) for x in got])
+    assert sorted(r[0] for r in rows) == [2, 3, 4]
+    for bits, toks, words in rows:
+        got = O.pack_block(toks, bits)
+        assert got.shape == (16 * bits,)
+        assert np.array_equal(got, words), (bits, [hex(x) for x in got])
 
 
 @pytest.mark.parametrize("bits", [2, 3, 4])
 def test_pack_roundtrip_and_bit_budget(bits):
     rng = np.random.default_rng(bits)
-    ce = rng.integers(0, 1 << bits, size=(50, 128)).astype(np.uint8)
-    co = rng.integers(0, 1 << bits, size=(50, 128)).astype(np.uint8)
-    assert np.array_equal(O.unpack_v_row(O.pack_v_row(ce, bits), bits), ce)
-    e2, o2 = O.unpack_k_block(O.pack_k_block(ce, co, bits), bits)
-    assert np.array_equal(e2, ce) and np.array_equal(o2, co)
+    codes = rng.integers(0, 1 << bits, size=(4, 50, 128)).astype(np.uint8)
+    assert np.array_equal(O.unpack_block(O.pack_block(codes, bits), bits), codes)
     full = np.full(128, (1 << bits) - 1, dtype=np.uint8)
-    assert np.all(O.pack_v_row(full, bits) == 0xFFFFFFFF)
-    assert np.all(O.pack_k_block(full, full, bits) == 0xFFFFFFFF)
-    # single codes touch disjoint bits (each bit of a row/block is used exactly once)
+    assert np.all(O.pack_block([full] * 4, bits) == 0xFFFFFFFF)
+    # single codes touch disjoint bits (each bit of a block is used exactly once)
     zero = np.zeros(128, dtype=np.uint8)
-    acc_v = np.zeros(4 * bits, dtype=np.uint64)
-    acc_k = np.zeros(8 * bits, dtype=np.uint64)
+    acc = np.zeros(16 * bits, dtype=np.uint64)
     for ch in range(128):
-        one = zero.copy()
-        one[ch] = (1 << bits) - 1
-        wv = O.pack_v_row(one, bits).astype(np.uint64)
-        assert not np.any(acc_v & wv)
-        acc_v |= wv
-        for ev, od in ((one, zero), (zero, one)):
-            wk = O.pack_k_block(ev, od, bits).astype(np.uint64)
-            assert not np.any(acc_k & wk)
-            acc_k |= wk
+        for j in range(4):
+            one = zero.copy()
+            one[ch] = (1 << bits) - 1
+            quad = [one if jj == j else zero for jj in range(4)]
+            w = O.pack_block(quad, bits).astype(np.uint64)
+            assert not np.any(acc & w)
+            acc |= w
+            # channel c lives in the words of lane group c % 16 only
+            nz = np.nonzero(w)[0]
+            assert np.all(nz // bits == (ch % 64) % 16)
 
 
 # ---------------------------------------------------------------- quantizer invariants
@@ -381,7 +371,9 @@ def test_append_reuses_key_calibration_and_chunks():
     c2 = O.QuantizedCache(w.B, w.Hkv, w.bits, T + 8, w.f, 1 << 20, 1 << 20)
     c2.calibrate_keys(0, K[0, :T])
     c2.quantize_tokens(0, 0, K[0, : T + 3], V[0, : T + 3], cbK, cbV)
-    assert np.array_equal(c2.kcodes[0, : T + 3], c.kcodes[0, : T + 3])
+    nq = (T + 3 + 3) // 4
+    assert np.array_equal(c2.kcodes[0, :nq], c.kcodes[0, :nq])
+    assert np.array_equal(c2.vcodes[0, :nq], c.vcodes[0, :nq])
     for s in ("k", "v"):
         assert np.array_equal(c2.out_pos[s][0], c.out_pos[s][0])
         assert np.array_equal(c2.chunk_ptr[s][0, : nch + 1], c.chunk_ptr[s][0, : nch + 1])
