@@ -140,15 +140,15 @@ def traffic_for(kernel, units):
 def bytes_model(w, T, kcount, vcount, path):
     """Algorithmic bytes of one layer's decode (attention part) over T tokens.
 
-    Key side (QK): packed key codes, key-outlier entries (4 B position + 2 B value),
-    key chunk pointers; value side (PV): packed value codes, value-outlier entries,
-    value token params (8 B/token), value chunk pointers.  The split path also
+    Key side (QK): packed key codes, key-outlier entries (4 B each: position and value),
+    key chunk pointers (one list per kv head); value side (PV): packed value codes,
+    value-outlier entries, value token params (8 B/token), value chunk pointers.  The split path also
     writes and reads fp32 logits (4 B per token per query head, each way).
     """
     code_row = w.Hkv * w.D * w.bits // 8
     nch = (T + 63) // 64 + 1
-    k_bytes = T * code_row + 6 * kcount + 4 * nch
-    v_bytes = T * code_row + 6 * vcount + 8 * T + 4 * nch
+    k_bytes = T * code_row + 4 * kcount + 4 * nch * w.Hkv
+    v_bytes = T * code_row + 4 * vcount + 8 * T + 4 * nch * w.Hkv
     logit = 4 * w.Hq * T
     if path == "split":
         return {"qk": k_bytes + logit, "pv": v_bytes + logit, "total": k_bytes + v_bytes + 2 * logit}
@@ -249,8 +249,11 @@ def run_kvq(args, rank, world):
     T0 = w.T
     e2e_steps = min(args.steps, 10)
     T_max = T0 + steps_total + e2e_steps + 64
-    kout_cap = int(T_max * max(w.f * w.n * 1.5, 4) + 4096)
-    vout_cap = int(T_max * (2 * math.floor(w.f * w.n / 2 + 0.5) + 2) + 4096)
+    # outlier lists are per (sequence, kv head): a key channel keeps ~f*T outliers, a token's
+    # 2k value outliers spread over the Hkv heads; capacities are multiples of 8
+    ceil8 = lambda x: (int(x) + 7) // 8 * 8  # noqa: E731
+    kout_cap = ceil8(T_max * w.f * w.D * 1.25 + 4096)
+    vout_cap = ceil8(T_max * 2 * math.floor(w.f * w.n / 2 + 0.5) / w.Hkv * 1.5 + 4096)
     cfg = K.make_cfg(w.B, w.Hq, w.Hkv, w.bits, T_max, w.f, w.rope_theta, kout_cap, vout_cap)
     # a different synthetic sequence per rank (weak scaling): layer key offset by rank
     layer_key = lambda l: l + 4096 * rank  # noqa: E731
@@ -296,8 +299,8 @@ def run_kvq(args, rank, world):
             caches.append(c)
             cbs.append(cb)
     setup_s = time.time() - t_setup
-    kcount = int(caches[0].kcount.cpu()[0])
-    vcount = int(caches[0].vcount.cpu()[0])
+    kcount = int(caches[0].kcount.cpu()[0].sum())
+    vcount = int(caches[0].vcount.cpu()[0].sum())
 
     # per-step inputs: appended token K/V and queries, per layer (device and pinned host)
     nL = layers * R
@@ -322,6 +325,7 @@ def run_kvq(args, rank, world):
     BH = w.B * w.Hq
     logits = torch.empty((w.B, w.Hq, T_max), dtype=torch.float32, device=dev)
     stats = torch.empty((w.B, w.Hq, S, 2), dtype=torch.float32, device=dev)
+    qkws = torch.empty(K.kvq_decode_qk_workspace(cfg, T_max), dtype=torch.uint8, device=dev)
     mlb = torch.empty((w.B, w.Hq, 2), dtype=torch.float32, device=dev)
     part = torch.empty((w.B, w.Hq, S, w.D), dtype=torch.float32, device=dev)
     outs = torch.empty((nL, w.B, w.Hq, w.D), dtype=torch.float32, device=dev)
@@ -345,7 +349,7 @@ def run_kvq(args, rank, world):
         if timing:
             marks[1].record()
         if args.path == "split":
-            K.kvq_decode_qk(c, cbK, qall[i, s], qpos[s], max_len, logits, stats, S)
+            K.kvq_decode_qk(c, cbK, qall[i, s], qpos[s], max_len, logits, stats, S, qkws)
             if timing:
                 marks[2].record()
             K.kvq_softmax_merge(cfg, stats, S, mlb)
@@ -436,7 +440,7 @@ def run_kvq(args, rank, world):
             c = caches[i]
             K.kvq_quantize_append(c, cbs[i][0], cbs[i][1], d_k[i], d_v[i], 1, None, 0, aws)
             if args.path == "split":
-                K.kvq_decode_qk(c, cbs[i][0], d_q[i], qpos_e2e[j], ml_len, logits, stats, S)
+                K.kvq_decode_qk(c, cbs[i][0], d_q[i], qpos_e2e[j], ml_len, logits, stats, S, qkws)
                 K.kvq_softmax_merge(cfg, stats, S, mlb)
                 K.kvq_decode_pv(c, cbs[i][1], logits, mlb, ml_len, outs[i], part, S)
             else:
@@ -485,7 +489,9 @@ def run_kvq(args, rank, world):
 
     if rank != 0:
         return 0
-    launches_per_layer_step = 8 if args.path == "split" else 6
+    # append: begin, stats, scan, write; qk: tables, qk, key outliers, split stats; merge;
+    # pv: pv, split sum, value outliers (the fused call launches the same kernels)
+    launches_per_layer_step = 12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,

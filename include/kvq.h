@@ -71,8 +71,8 @@ typedef struct kvq_cfg {
     int32_t D;          /* head dimension; must be 128 */
     int32_t bits;       /* NUQ code width: 2, 3 or 4 */
     int32_t T_max;      /* token capacity per sequence, 1 .. 16,777,216 */
-    int32_t out_cap_k;  /* key-outlier list capacity per sequence (entries) */
-    int32_t out_cap_v;  /* value-outlier list capacity per sequence (entries) */
+    int32_t out_cap_k;  /* key-outlier list capacity per (sequence, kv head); multiple of 8 */
+    int32_t out_cap_v;  /* value-outlier list capacity per (sequence, kv head); multiple of 8 */
     double outlier_frac;/* f: per vector, k = floor(f*N/2 + 1/2) outliers per side */
     double rope_theta;  /* RoPE base; theta_i = rope_theta^(-2i/D) */
 } kvq_cfg;
@@ -80,22 +80,22 @@ typedef struct kvq_cfg {
 /*
  * Device arrays of one layer's cache (all caller-allocated; sizes from kvq_layout).
  * Layouts (codes are little-endian bit strings over consecutive uint32 words):
- *  kcodes  uint32 [B][ceil(T_max/2)][Hkv][8*bits]  key block of the token pair
- *          (2u, 2u+1) of one kv head: channel c = j + 16m + 64s (j < 16, m < 4,
- *          s in {0,1}) is the 2*bits-wide field code(2u, c) | code(2u+1, c) << bits
- *          at bit 16*bits*j + 2*bits*(2m + s).  A block whose odd token is not yet
- *          written holds 0 in the odd half of every field.
- *  vcodes  uint32 [B][T_max][Hkv][4*bits]  value row of one token and kv head:
- *          channels c and c + 64 (c = j + 8m < 64, j < 8, m < 8) share the field
- *          code(c) | code(c + 64) << bits at bit 16*bits*j + 2*bits*m.
+ *  kcodes, vcodes  uint32 [B][Hkv][ceil(T_max/4)][16*bits]  one code block per (sequence,
+ *          kv head, token quad 4u .. 4u+3), keys and values alike.  Lane group i in [0,16)
+ *          owns words [bits*i, bits*i + bits) of the block and the rotate-half pairs
+ *          (c, c + 64), c = i + 16k (k in [0,4)).  Token j of the quad sits in slot
+ *          s = j ^ (i >> 2): the 2*bits-wide field at bit 2*bits*(4k + s) of the group's
+ *          bit string holds code(4u + j, c) | code(4u + j, c + 64) << bits.  Fields of
+ *          tokens not yet written are 0.
  *  kthr    uint16 [B][n][2]  fp16 key thresholds (t_lo, t_hi) per channel
  *  kparams float  [B][n][2]  key channel (off, half)
  *  vparams float  [B][T_max][2] value token (off, half)
- *  k/vout_pos uint32 [B][cap]  outlier entry ((t % 64) << 16) | (h*D + c),
- *          sorted by (t, h*D + c); k/vout_val uint16 [B][cap] its fp16 bits
- *  k/vchunk uint32 [B][ceil(T_max/64)+1]  entries of tokens [64m, 64m+64) are
+ *  kout, vout uint32 [B][Hkv][cap]  one outlier list per (sequence, kv head): entry
+ *          (fp16 bits << 16) | ((t % 64) << 7) | c (c the channel within the head),
+ *          sorted by (t, c)
+ *  k/vchunk uint32 [B][Hkv][ceil(T_max/64)+1]  entries of tokens [64m, 64m+64) are
  *          [chunk[m], chunk[m+1])
- *  k/vcount uint32 [B]  entries in use;  len int32 [B]  tokens in the cache
+ *  k/vcount uint32 [B][Hkv]  entries in use;  len int32 [B]  tokens in the cache
  *  status  int32 [1]  sticky KVQ_STATUS_* bits
  */
 typedef struct kvq_cache {
@@ -104,10 +104,8 @@ typedef struct kvq_cache {
     uint16_t* kthr;
     float* kparams;
     float* vparams;
-    uint32_t* kout_pos;
-    uint16_t* kout_val;
-    uint32_t* vout_pos;
-    uint16_t* vout_val;
+    uint32_t* kout;
+    uint32_t* vout;
     uint32_t* kchunk;
     uint32_t* vchunk;
     uint32_t* kcount;
@@ -127,7 +125,7 @@ typedef struct kvq_codebook {
 /* Byte size of every cache array of kvq_cache, same field names. */
 typedef struct kvq_sizes {
     size_t kcodes, vcodes, kthr, kparams, vparams;
-    size_t kout_pos, kout_val, vout_pos, vout_val;
+    size_t kout, vout;
     size_t kchunk, vchunk, kcount, vcount, len, status;
 } kvq_sizes;
 
@@ -164,9 +162,9 @@ int kvq_quantize_workspace(const kvq_cfg* cfg, int32_t n_new, int32_t calibrate,
  *   Per token: value thresholds/scales over its n values as above; an entry is
  *   an outlier iff x < t_lo or x > t_hi; outliers go to the lists unchanged and
  *   are encoded as 0; xn = (x - off)/half (0 if half == 0); code = #{j: xn >
- *   bounds[j]}.  Tokens whose outliers would exceed the list capacity (counting
- *   from the start of this call, in token order) drop their outliers and set
- *   KVQ_STATUS_OUTLIER_OVERFLOW.
+ *   bounds[j]}.  Per list (sequence, kv head): a token whose outliers in that head
+ *   would exceed the list capacity (counting from the start of this call, in token
+ *   order) drops them there and sets KVQ_STATUS_OUTLIER_OVERFLOW.
  *   workspace: device scratch of kvq_quantize_workspace bytes, 16-byte aligned.
  */
 int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
@@ -188,10 +186,17 @@ int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_co
  *           clipped and sets KVQ_STATUS_LEN_OVERFLOW
  *   logits  float [B][Hq][T_max];  stats float2 [B][Hq][splits]
  *   splits  1 .. 4096, or 0 to let the library choose (kvq_decode_splits)
+ *   workspace  device scratch of kvq_decode_qk_workspace bytes (per-call tables: the
+ *           rotated query, RoPE angle tables, the dense key value at outliers), 16-byte
+ *           aligned
  */
 int kvq_decode_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
                   const uint16_t* q, const int32_t* qpos, int32_t max_len, float* logits,
-                  float* stats, int32_t splits, void* stream);
+                  float* stats, int32_t splits, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* Workspace bytes of kvq_decode_qk for max_len. */
+int kvq_decode_qk_workspace(const kvq_cfg* cfg, int32_t max_len, size_t* bytes);
 
 /* The split count the library uses for `splits = 0`. */
 int kvq_decode_splits(const kvq_cfg* cfg, int32_t max_len);
@@ -280,10 +285,10 @@ int kvq_fit_codebook(const uint16_t* samples, int32_t n_vec, int32_t vec_len, do
  * file-scope device array of KVQ_NOALLOC_SCRATCH_BYTES that the library owns; every GPU
  * that loads libkvq.so holds that array until the process exits.
  *   - Limit: the scratch that kvq_quantize_workspace(cfg, n_new, 0) reports must fit in
- *     KVQ_NOALLOC_SCRATCH_BYTES (1 MiB, about 20 bytes per (sequence, new token): some
- *     52,000 of them, e.g. B = 256 sequences appending up to 200 tokens each); larger
- *     requests return KVQ_ERR_SCRATCH_LIMIT and launch nothing.  Use
- *     kvq_quantize_append with a caller workspace for prefills.
+ *     KVQ_NOALLOC_SCRATCH_BYTES (1 MiB).  A call needs about 4 + 16*Hkv bytes per
+ *     (sequence, new token), 516 bytes at Hkv = 32: some 2,000 of them, e.g. 256 sequences
+ *     appending up to 7 tokens each; larger requests return KVQ_ERR_SCRATCH_LIMIT and launch
+ *     nothing.  Use kvq_quantize_append with a caller workspace for prefills.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any
  *     stream capture begins.

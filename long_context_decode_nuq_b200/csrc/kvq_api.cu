@@ -24,6 +24,7 @@ int check_cfg(const kvq_cfg* cfg) {
     if (cfg->Hq < cfg->Hkv || cfg->Hq % cfg->Hkv != 0 || cfg->Hq / cfg->Hkv > 16) return KVQ_ERR_SHAPE;
     if (cfg->T_max < 1 || cfg->T_max > (1 << 24)) return KVQ_ERR_SHAPE;
     if (cfg->out_cap_k < 0 || cfg->out_cap_v < 0) return KVQ_ERR_SHAPE;
+    if ((cfg->out_cap_k | cfg->out_cap_v) & 7) return KVQ_ERR_SHAPE;  // lists stay 16-byte aligned
     if (!(cfg->outlier_frac >= 0.0 && cfg->outlier_frac <= 1.0)) return KVQ_ERR_SHAPE;
     if (!(cfg->rope_theta > 1.0)) return KVQ_ERR_SHAPE;
     return KVQ_OK;
@@ -37,9 +38,9 @@ int check_cache(const kvq_cfg* cfg, const kvq_cache* c) {
         if (!p) return KVQ_ERR_NULL;
         if (!aligned16(p)) return KVQ_ERR_ALIGN;
     }
-    if (cfg->out_cap_k > 0 && (!c->kout_pos || !c->kout_val)) return KVQ_ERR_NULL;
-    if (cfg->out_cap_v > 0 && (!c->vout_pos || !c->vout_val)) return KVQ_ERR_NULL;
-    const void* opt[] = {c->kout_pos, c->kout_val, c->vout_pos, c->vout_val};
+    if (cfg->out_cap_k > 0 && !c->kout) return KVQ_ERR_NULL;
+    if (cfg->out_cap_v > 0 && !c->vout) return KVQ_ERR_NULL;
+    const void* opt[] = {c->kout, c->vout};
     for (const void* p : opt)
         if (p && !aligned16(p)) return KVQ_ERR_ALIGN;
     return KVQ_OK;
@@ -89,14 +90,13 @@ int kvq_layout(const kvq_cfg* cfg, kvq_sizes* out) {
     out->kthr = B * n * 2 * 2;
     out->kparams = B * n * 2 * 4;
     out->vparams = B * T * 2 * 4;
-    out->kout_pos = B * (size_t)cfg->out_cap_k * 4;
-    out->kout_val = B * (size_t)cfg->out_cap_k * 2;
-    out->vout_pos = B * (size_t)cfg->out_cap_v * 4;
-    out->vout_val = B * (size_t)cfg->out_cap_v * 2;
-    out->kchunk = B * nch * 4;
-    out->vchunk = B * nch * 4;
-    out->kcount = B * 4;
-    out->vcount = B * 4;
+    const size_t BH = B * (size_t)cfg->Hkv;  // one outlier list per (sequence, kv head)
+    out->kout = BH * cfg->out_cap_k * 4;
+    out->vout = BH * cfg->out_cap_v * 4;
+    out->kchunk = BH * nch * 4;
+    out->vchunk = BH * nch * 4;
+    out->kcount = BH * 4;
+    out->vcount = BH * 4;
     out->len = B * 4;
     out->status = 4;
     return KVQ_OK;

@@ -1,16 +1,20 @@
 // Decode attention over the quantized cache (read side of techniques (i)-(iv)):
-// QK with NUQ lookup + on-the-fly RoPE + key-outlier correction, split-K softmax
-// statistics and merge, and the probability-weighted value sum with value-outlier
-// replacement.  Also the uncompressed fp16 comparison kernel.
+// QK with NUQ lookup + on-the-fly RoPE, key-outlier correction, split-K softmax
+// statistics and merge, the probability-weighted value sum and the value-outlier
+// correction.  Also the uncompressed fp16 comparison kernel.
 //
-// The two quantized kernels share one shape.  A CTA covers HPC query heads over one split
-// of the tokens and walks it in 64-token chunks.  The chunk's 4-token code blocks (for the
-// kv heads of those query heads) arrive in a ring of shared-memory stages filled by bulk
-// copies (cp.async.bulk, completion counted on an mbarrier; no multicast).  Half-warp qd
-// of the CTA takes token quad qd of the chunk and lane i of the half-warp the rotate-half
-// pairs (c, c + 64), c = i + 16k: exactly the lane group i of the code block, whose token
-// slot s holds token s ^ (i >> 2) (the rotation that lets QK reduce its 16 partials per
-// lane across the half-warp with plain shuffles).
+// The two streaming kernels share one shape.  A CTA covers HPC query heads over one split of
+// the tokens and walks it in 64-token chunks.  The chunk's code blocks (one contiguous run of
+// 16 blocks per kv head) arrive in a ring of shared-memory stages filled by bulk copies
+// (cp.async.bulk, completion counted on an mbarrier; no multicast) that the last warp issues.
+// Half-warp qd of a consumer warp takes token quad qd of the chunk and lane i of the
+// half-warp the rotate-half pairs (c, c + 64), c = i + 16k: exactly the lane group i of the
+// code block, whose token slot s holds token s ^ (i >> 2) (the rotation that lets QK reduce
+// its partials per lane across the half-warp with plain shuffles).  Consumer warps meet only
+// the stage barriers.  The sparse outliers are applied by separate kernels that walk the
+// outlier lists chunk by chunk: key outliers add (x - zhat) times the rotated query component
+// to the logits before the softmax statistics are taken, value outliers add
+// p (x - zhat) to the output after the merge.
 #include "kvq_common.cuh"
 
 using namespace kvq;
@@ -22,8 +26,8 @@ constexpr int kMaxG = 16;                          // query heads per kv head
 constexpr int kThreads = 256;                      // 8 warps = 16 half-warps
 constexpr int kQuads = kThreads / 16;              // token quads per chunk (64 tokens)
 constexpr int kStages = 4;                         // chunks in the bulk-copy ring
-constexpr int kPitchPad = 64;                      // bytes after each quad row of a stage
 constexpr uint32_t kWaitLimit = 1u << 24;          // mbarrier polls before giving up
+constexpr int kTrigLo = 256;                       // trig tables: t = 256 * hi + lo
 
 __device__ inline float warp_sum(float v) {
 #pragma unroll
@@ -108,13 +112,6 @@ __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigne
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
     return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
 }
-// (c, s) <- (c, s) rotated by the angle whose (cos, sin) is (rc, rs), in binary64.
-__device__ __forceinline__ void rot64(double& c, double& s, double rc, double rs) {
-    const double nc = c * rc - s * rs, ns = s * rc + c * rs;
-    c = nc;
-    s = ns;
-}
-
 template <int BITS>
 struct Fmt {
     static constexpr int FW = 2 * BITS;  // field width (codes of c and c + 64)
@@ -152,122 +149,175 @@ __device__ __forceinline__ float zero_code_value(float off, float half, const fl
     return off + half * levels[encode(xn, bounds, nb)];
 }
 
-// Head slot of lane i's result after the half-warp reduction, and whether lane i is the
-// one lane (of the lanes holding that result) that writes it.
 template <int HPC>
+__host__ __device__ constexpr int heads_per_warp() { return HPC == 4 ? 2 : HPC; }
+template <int HW>
 __device__ __forceinline__ int out_head(int i) {
-    return HPC == 4 ? (i & 3) : (HPC == 2 ? ((i >> 1) & 1) : 0);
+    return HW == 4 ? (i & 3) : (HW == 2 ? ((i >> 1) & 1) : 0);
 }
-template <int HPC>
+template <int HW>
 __device__ __forceinline__ bool out_owner(int i) {
-    return HPC == 4 ? true : (HPC == 2 ? !(i & 1) : !(i & 3));
+    return HW == 4 ? true : (HW == 2 ? !(i & 1) : !(i & 3));
 }
 
-// ---------------------------------------------------------------------------------
-// Shared-memory plans (host and device).
-struct QKPlan {
-    int tab, ring, pitch, base, r8, r1, qr, zh, corr, red, kb, bar, flag, total;
-};
-__host__ __device__ inline QKPlan qk_plan(int bits, int hpc, int kvb) {
-    QKPlan p;
-    int o = 0;
-    p.tab = o;  o += hpc * 64 * (1 << (2 * bits)) * 8;       // [entry][head][pair] (X, Y)
-    p.pitch = kvb * 16 * bits * 4 + kPitchPad;
-    p.ring = o; o += kStages * kQuads * p.pitch;
-    p.base = o; o += 3 * 64 * 8;                              // [3][64] (cos, sin) at chunk start
-    p.r8 = o;   o += 8 * 64 * 8;                              // [8][64] rotation by 8a tokens
-    p.r1 = o;   o += 8 * 64 * 8;                              // [8][64] rotation by a tokens
-    p.qr = o;   o += hpc * 128 * 4;                           // rotated, scaled queries
-    p.zh = o;   o += hpc * 128 * 4;                           // dense value at a key outlier
-    p.corr = o; o += 3 * 64 * hpc * 4;                        // [3][64][hpc] outlier corrections
-    p.red = o;  o += kThreads * 8;
-    p.kb = o;   o += 16 * 4;
-    p.bar = o;  o += kStages * 8;
-    p.flag = o; o += 16;
-    p.total = o;
-    return p;
-}
+// Consumer warps of a CTA: with four query heads per CTA two warps share a quad pair (two
+// heads each), so that a thread's accumulators stay small; one more warp streams the input.
+__host__ __device__ constexpr int consumer_warps(int hpc) { return hpc == 4 ? 16 : 8; }
 
-struct PVPlan {
-    int tab, ring, pitch, wsm, psm, vsm, corr, pored, posum, vb, bar, flag, total;
-};
-__host__ __device__ inline PVPlan pv_plan(int bits, int hpc, int kvb) {
-    PVPlan p;
-    int o = 0;
-    p.tab = o;  o += (1 << (2 * bits)) * 16 * 8;              // [entry][16 lane copies] (La, Lb)
-    p.pitch = kvb * 16 * bits * 4 + kPitchPad;
-    p.ring = o;
-    {
-        const int ring = kStages * kQuads * p.pitch, red = kQuads * hpc * 128 * 4;
-        o += ring > red ? ring : red;                         // reused by the final reduction
-    }
-    p.wsm = o;  o += kQuads * 4 * hpc * 8;                    // [quad][token][head] (w, w)
-    p.psm = o;  o += 2 * 64 * hpc * 4;                        // [2][64][hpc] probabilities
-    p.vsm = o;  o += 2 * 64 * 8;                              // [2][64] value (off, half)
-    p.corr = o; o += hpc * 128 * 4;                           // value-outlier corrections
-    p.pored = o; o += kThreads * 4;
-    p.posum = o; o += 16 * 4;
-    p.vb = o;   o += 16 * 4;
-    p.bar = o;  o += kStages * 8;
-    p.flag = o; o += 16;
-    p.total = o;
-    return p;
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-
-// Issue the bulk copies of chunk `cc` (quads of [tc, min(tc + 64, t_end)) for the CTA's kv
-// heads) into its ring stage.  One thread.
-__device__ inline void issue_chunk(uint8_t* ring, int pitch, uint64_t* bars, const uint32_t* src0,
-                                   size_t quad_stride, uint32_t row_bytes, int t_begin, int t_end,
-                                   int cc) {
-    const int tc = t_begin + cc * kChunk;
-    const int q0 = tc >> 2, q1 = (min(tc + kChunk, t_end) + 3) >> 2;
-    uint64_t* bar = bars + cc % kStages;
-    uint8_t* dst = ring + (size_t)(cc % kStages) * kQuads * pitch;
-    mbar_arrive_expect_tx(bar, (uint32_t)(q1 - q0) * row_bytes);
-    for (int qq = q0; qq < q1; ++qq)
-        bulk_load(dst + (size_t)(qq - q0) * pitch, src0 + (size_t)qq * quad_stride, row_bytes, bar);
-}
-
 // After an abandoned wait: let every copy still in flight land before the CTA exits.
 __device__ inline void drain_chunks(uint64_t* bars, int from, int to) {
     for (int cc = from; cc < to; ++cc) mbar_wait(bars + cc % kStages, (cc / kStages) & 1);
 }
 
 // ---------------------------------------------------------------------------------
-// QK.  Per head slot and pair p the CTA tabulates, for every code pair e = (xa, xb),
+// Shared-memory plans (host and device).
+struct QKPlan {
+    int tab, ring, pitch, stage, base, rs, qr, bar, flag, total;
+};
+__host__ __device__ inline QKPlan qk_plan(int bits, int hpc, int kvb) {
+    QKPlan p;
+    int o = 0;
+    p.tab = o;  o += hpc * 64 * (1 << (2 * bits)) * 8;       // [entry][head][pair] (X, Y)
+    p.pitch = kQuads * 16 * bits * 4;                         // code blocks of one kv head
+    p.stage = kvb * p.pitch;
+    p.ring = o; o += kStages * p.stage;
+    p.base = o; o += kStages * 64 * 8;                        // [stage][64] (cos, sin) at chunk start
+    p.rs = o;   o += 64 * 64 * 8;                             // [token of chunk][pair] rotation
+    p.qr = o;   o += hpc * 128 * 4;                           // rotated, scaled queries
+    p.bar = o;  o += 2 * kStages * 8;                         // full, empty
+    p.flag = o; o += 16;
+    p.total = o;
+    return p;
+}
+
+struct PVPlan {
+    int tab, ring, pitch, stage, wsm, bar, flag, total;
+};
+__host__ __device__ inline PVPlan pv_plan(int bits, int hpc, int kvb) {
+    PVPlan p;
+    int o = 0;
+    p.tab = o;  o += (1 << (2 * bits)) * 16 * 8;              // [entry][16 lane copies] (La, Lb)
+    p.pitch = kQuads * 16 * bits * 4;
+    p.stage = kvb * p.pitch;
+    p.ring = o;
+    {
+        const int ring = kStages * p.stage, red = kQuads * hpc * 128 * 4;
+        o += ring > red ? ring : red;                         // reused by the final reduction
+    }
+    p.wsm = o;  o += kQuads * 4 * hpc * 8;                    // [quad][token][head] (w, w)
+    p.bar = o;  o += 2 * kStages * 8;                         // full, empty
+    p.flag = o; o += 16;
+    p.total = o;
+    return p;
+}
+
+// Thread 0 of the streaming warp: bulk copies of the chunk's code blocks, one contiguous run
+// of 16 blocks per kv head of the CTA, into the chunk's stage (kv head k at k * pitch).
+struct Streamer {
+    uint8_t* ring;
+    uint64_t* full;
+    int pitch, stage, kvb, t_begin, t_end;
+    const uint32_t* src0;  // code blocks of (sequence, first kv head), quad 0
+    size_t head_stride;    // words between the blocks of consecutive kv heads
+    uint32_t quad_bytes;   // bytes of one code block
+
+    __device__ void issue(int cc) {
+        const int tc = t_begin + cc * kChunk;
+        const int q0 = tc >> 2, q1 = (min(tc + kChunk, t_end) + 3) >> 2;
+        uint64_t* bar = full + cc % kStages;
+        uint8_t* dst = ring + (size_t)(cc % kStages) * stage;
+        const uint32_t bytes = (uint32_t)(q1 - q0) * quad_bytes;
+        mbar_arrive_expect_tx(bar, (uint32_t)kvb * bytes);
+        for (int k = 0; k < kvb; ++k)
+            bulk_load(dst + k * pitch, src0 + (size_t)k * head_stride + (size_t)q0 * (quad_bytes / 4),
+                      bytes, bar);
+    }
+};
+
+// (cos, sin) of t * theta_p from the per-call tables: hi[t / 256] rotated by lo[t % 256].
+__device__ __forceinline__ float2 trig_at(const float2* thi, const float2* tlo, int t, int p) {
+    return cmul(thi[(t / kTrigLo) * 64 + p], tlo[(t % kTrigLo) * 64 + p]);
+}
+
+// ---------------------------------------------------------------------------------
+// Per-call tables: rotated, scaled queries qr [B][Hq][128]; trig tables hi [nhi][64] =
+// (cos, sin)(256 j theta_p), lo [256][64] = (cos, sin)(tau theta_p), all from binary64; the
+// dense key value at an outlier zk [B][Hkv][128] = off + half * L[encode(normalize(0))].
+__global__ void k_decode_prep(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const uint16_t* q,
+                              const int32_t* qpos, int nhi, float* qr, float2* thi, float2* tlo,
+                              float* zk) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int nq = cfg.B * cfg.Hq * 64, nh = nhi * 64, nl = kTrigLo * 64, nz = cfg.B * cfg.Hkv * kD;
+    if (e < nq) {
+        const int p = e & 63, bh = e >> 6, b = bh / cfg.Hq;
+        const double th = rope_freq(cfg.rope_theta, p);
+        double cq, sq;
+        rope_cs64((double)qpos[b], th, &cq, &sq);
+        const uint16_t* qv = q + (size_t)bh * kD;
+        const double qa = (double)h2f(qv[p]), qb = (double)h2f(qv[p + 64]);
+        qr[(size_t)bh * kD + p] = (float)((qa * cq - qb * sq) * (double)kInvSqrtD);
+        qr[(size_t)bh * kD + p + 64] = (float)((qa * sq + qb * cq) * (double)kInvSqrtD);
+    } else if (e < nq + nh) {
+        const int f = e - nq, p = f & 63, j = f >> 6;
+        double cc, ss;
+        rope_cs64((double)j * kTrigLo, rope_freq(cfg.rope_theta, p), &cc, &ss);
+        thi[f] = make_float2((float)cc, (float)ss);
+    } else if (e < nq + nh + nl) {
+        const int f = e - nq - nh, p = f & 63, j = f >> 6;
+        double cc, ss;
+        rope_cs64((double)j, rope_freq(cfg.rope_theta, p), &cc, &ss);
+        tlo[f] = make_float2((float)cc, (float)ss);
+    } else if (e < nq + nh + nl + nz) {
+        const int f = e - nq - nh - nl;
+        const int nb = (1 << cfg.bits) - 1;
+        const float* kp = c.kparams + (size_t)f * 2;  // [B][Hkv*128] channels, in order
+        const float xn = normalize(0.0f, kp[0], kp[1]);
+        zk[f] = kp[0] + kp[1] * cb.levels[encode(xn, cb.bounds, nb)];
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// QK.  Per query head and pair p the CTA tabulates, for every code pair e = (xa, xb),
 //   X = qa (off_a + half_a L[xa]) + qb (off_b + half_b L[xb]),
 //   Y = qb (off_a + half_a L[xa]) - qa (off_b + half_b L[xb])
-// (q the query rotated to its own position and scaled by 1/sqrt(D)); the logit of token t
-// is then sum_p cos(t theta_p) X + sin(t theta_p) Y, one f32x2 FMA per pair and token.
-// The (cos, sin) of a lane's tokens come from the chunk's binary64-derived base times fixed
-// per-lane rotations.  Lane i's accumulator slot (token s, head h) holds token s ^ (i >> 2),
-// head h ^ hperm(i), so the 16 (or 8, 4) partials reduce across the half-warp by halving.
+// (q the query rotated to its own position and scaled by 1/sqrt(D)); the dense part of the
+// logit of token t is then sum_p cos(t theta_p) X + sin(t theta_p) Y, one f32x2 FMA per pair
+// and token.  The (cos, sin) of a lane's tokens are the chunk's base times fixed rotations.
+// A consumer warp takes two token quads and HW of the CTA's heads; lane i's accumulator slot
+// (token s, head h) holds token s ^ (i >> 2) and head h ^ hperm(i), so the 4*HW partials
+// reduce across the half-warp by halving.  The last warp streams the chunks and the chunk
+// base angles.
 template <int BITS, int HPC, bool SHARE>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_qk(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const uint16_t* __restrict__ q,
-         const int32_t* __restrict__ qpos, int Ls, int S, int max_len, int kvb,
-         float* __restrict__ logits, float2* __restrict__ stats) {
+__global__ void __launch_bounds__(consumer_warps(HPC) * 32 + 32, 1)
+    k_qk(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ qr_all,
+         const float2* __restrict__ thi, const float2* __restrict__ tlo, int Ls, int max_len,
+         int kvb, float* __restrict__ logits) {
     using F = Fmt<BITS>;
+    constexpr int CW = consumer_warps(HPC), NC = CW * 32;
+    constexpr int HW = heads_per_warp<HPC>();
     constexpr int LH = HPC == 4 ? 2 : (HPC == 2 ? 1 : 0);
     constexpr int P = 9 + LH;  // bit of the entry index in a table byte offset
     constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << P;
-    constexpr int NW = SHARE ? 1 : HPC;
-    constexpr int V = 4 * HPC;  // partials per lane
+    constexpr int NW = SHARE ? 1 : HW;
+    constexpr int V = 4 * HW;  // partials per lane
     extern __shared__ __align__(128) uint8_t sm[];
     const QKPlan L = qk_plan(BITS, HPC, kvb);
     uint8_t* tab = sm + L.tab;
     uint8_t* ring = sm + L.ring;
     float2* base = (float2*)(sm + L.base);
-    float2* r8 = (float2*)(sm + L.r8);
-    float2* r1 = (float2*)(sm + L.r1);
+    float2* rs = (float2*)(sm + L.rs);
     float* qr = (float*)(sm + L.qr);
-    float* zh = (float*)(sm + L.zh);
-    float* corr = (float*)(sm + L.corr);
-    float* kb = (float*)(sm + L.kb);
-    uint64_t* bars = (uint64_t*)(sm + L.bar);
+    uint64_t* full = (uint64_t*)(sm + L.bar);
+    uint64_t* empty = full + kStages;
     int* flag = (int*)(sm + L.flag);
 
-    const int tid = threadIdx.x, i = tid & 15, qd = tid >> 4, x = i >> 2;
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int i = tid & 15, x = i >> 2, lane = tid & 31, warp = tid >> 5;
+    const int qd = 2 * (warp & 7) + ((tid >> 4) & 1);  // token quad of the chunk
+    const int hg = (warp >> 3) * HW;                     // first CTA head of the warp
     const int s = blockIdx.x, b = blockIdx.y, hq0 = blockIdx.z * HPC;
     const int Hq = cfg.Hq, Hkv = cfg.Hkv, g = Hq / Hkv;
     int len = c.len[b];
@@ -276,63 +326,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         len = max_len;
     }
     const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
-    if (t_begin >= t_end) {
-        if (tid < HPC) stats[((size_t)b * Hq + hq0 + tid) * S + s] = make_float2(-INFINITY, 0.0f);
-        return;
-    }
+    if (t_begin >= t_end) return;
     const int nch = (t_end - t_begin + kChunk - 1) / kChunk;
     const int kv_first = min(hq0 / g, Hkv - kvb);
-    const size_t NQ = nquads(cfg.T_max);
-    const uint32_t* src0 = c.kcodes + ((size_t)b * NQ * Hkv + kv_first) * F::BW;
-    const size_t quad_stride = (size_t)Hkv * F::BW;
-    const uint32_t row_bytes = (uint32_t)kvb * F::BW * 4;
     if (tid == 0) {
-        for (int k = 0; k < kStages; ++k) mbar_init(bars + k, 1);
-        *flag = 0;
+        for (int k = 0; k < kStages; ++k) {
+            mbar_init(full + k, 1);
+            mbar_init(empty + k, CW);
+        }
+        flag[0] = 0;
+        flag[1] = 0;
         fence_mbar_init();
     }
-    __syncthreads();
-    int issued = 0;
-    if (tid == 0) {
-        for (; issued < min(kStages, nch); ++issued)
-            issue_chunk(ring, L.pitch, bars, src0, quad_stride, row_bytes, t_begin, t_end, issued);
-    }
     // ---- per-CTA tables
-    const int nb = (1 << BITS) - 1;
-    if (tid < nb) kb[tid] = cb.bounds[tid];
-    double bc = 0.0, bs = 0.0, sc64 = 1.0, ss64 = 0.0;  // threads < 64: next chunk base
-    if (tid < 64) {
-        const double th = rope_freq(cfg.rope_theta, tid);
-        double cq, sq;
-        rope_cs64((double)qpos[b], th, &cq, &sq);
-        for (int h = 0; h < HPC; ++h) {
-            const uint16_t* qv = q + ((size_t)b * Hq + hq0 + h) * kD;
-            const double qa = (double)h2f(qv[tid]), qb = (double)h2f(qv[tid + 64]);
-            qr[h * kD + tid] = (float)((qa * cq - qb * sq) * (double)kInvSqrtD);
-            qr[h * kD + tid + 64] = (float)((qa * sq + qb * cq) * (double)kInvSqrtD);
-        }
-        for (int a = 0; a < 8; ++a) {
-            double cc, ss;
-            rope_cs64((double)(8 * a), th, &cc, &ss);
-            r8[a * 64 + tid] = make_float2((float)cc, (float)ss);
-            rope_cs64((double)a, th, &cc, &ss);
-            r1[a * 64 + tid] = make_float2((float)cc, (float)ss);
-        }
-        rope_cs64((double)kChunk, th, &sc64, &ss64);
-        rope_cs64((double)t_begin, th, &bc, &bs);
-        base[tid] = make_float2((float)bc, (float)bs);
-        rot64(bc, bs, sc64, ss64);
-        base[64 + tid] = make_float2((float)bc, (float)bs);
-    }
-    for (int e = tid; e < 3 * 64 * HPC; e += kThreads) corr[e] = 0.0f;
+    for (int e = tid; e < HPC * kD; e += nthr) qr[e] = qr_all[((size_t)b * Hq + hq0) * kD + e];
+    for (int e = tid; e < 64 * 64; e += nthr) rs[e] = tlo[e];  // rotations by 0 .. 63 tokens
     __syncthreads();
+    const int nb = (1 << BITS) - 1;
     const float* kp = c.kparams + (size_t)b * Hkv * kD * 2;
-    for (int e = tid; e < HPC * kD; e += kThreads) {
-        const int h = e >> 7, ch = e & 127;
-        const float* pp = kp + ((size_t)((hq0 + h) / g) * kD + ch) * 2;
-        zh[e] = zero_code_value(pp[0], pp[1], cb.levels, kb, nb);
-    }
-    for (int e = tid; e < HPC * 64 * F::NT; e += kThreads) {
+    for (int e = tid; e < HPC * 64 * F::NT; e += nthr) {
         const int p = e & 63, h = (e >> 6) & (HPC - 1), idx = e >> (6 + LH);
         const int kvh = (hq0 + h) / g;
         const float* pa = kp + ((size_t)kvh * kD + p) * 2;
@@ -346,374 +358,466 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float Y = fmaf(B2, Lb, fmaf(A2, La, C2));
         reinterpret_cast<unsigned long long*>(tab)[e] = pk(X, Y);
     }
-    // ---- per-lane constants
-    const int hperm = out_head<HPC>(i);
-    uint32_t lb[HPC];
-#pragma unroll
-    for (int h = 0; h < HPC; ++h) lb[h] = ((uint32_t)(h ^ hperm) << 9) | ((uint32_t)i << 3);
-    uint32_t woff[NW];
-#pragma unroll
-    for (int h = 0; h < NW; ++h) {
-        const int kvs = SHARE ? 0 : (hq0 + (h ^ hperm)) / g - kv_first;
-        woff[h] = (uint32_t)(qd * L.pitch + kvs * F::BW * 4 + i * BITS * 4);
-    }
-    const int khlo = hq0 / g, khhi = (hq0 + HPC - 1) / g;
-    const int nch1 = nchunks(cfg.T_max) + 1;
-    const uint32_t* kchunk = c.kchunk + (size_t)b * nch1;
-    const uint32_t kcount = c.kcount[b];
-    const uint32_t* opos = c.kout_pos + (size_t)b * cfg.out_cap_k;
-    const uint16_t* oval = c.kout_val + (size_t)b * cfg.out_cap_k;
-    // key outliers of chunk cc: logit(t, h) += (x - zhat) * (component of q rotated to t)
-    auto outliers = [&](int cc) {
-        const int m = (t_begin + cc * kChunk) / kChunk;
-        const uint32_t lo = min(kchunk[m], kcount), hi = min(kchunk[m + 1], kcount);
-        const float2* bse = base + (cc % 3) * 64;
-        float* cr = corr + (cc % 3) * 64 * HPC;
-        for (uint32_t e = lo + tid; e < hi; e += kThreads) {
-            const uint32_t pw = opos[e];
-            const int tl = (int)(pw >> 16), jf = (int)(pw & 0xffffu);
-            const int kh = jf >> 7, chn = jf & 127;
-            if (tl >= kChunk || kh < khlo || kh > khhi) continue;
-            const int pp = chn & 63;
-            const float2 cs = cmul(cmul(bse[pp], r8[(tl >> 3) * 64 + pp]), r1[(tl & 7) * 64 + pp]);
-            const float xv = h2f(oval[e]);
-#pragma unroll
-            for (int h = 0; h < HPC; ++h) {
-                if ((hq0 + h) / g != kh) continue;
-                const float d = xv - zh[h * kD + chn];
-                const float qa = qr[h * kD + pp], qb = qr[h * kD + pp + 64];
-                const float r = (chn < 64) ? (cs.x * qa + cs.y * qb) : (cs.x * qb - cs.y * qa);
-                atomicAdd(&cr[tl * HPC + h], d * r);
+    __syncthreads();  // tables complete, barriers initialised
+
+    if (tid >= NC) {
+        // ================= streaming warp
+        const int pl = tid - NC;
+        Streamer sr;
+        sr.ring = ring;
+        sr.full = full;
+        sr.pitch = L.pitch;
+        sr.stage = L.stage;
+        sr.kvb = kvb;
+        sr.t_begin = t_begin;
+        sr.t_end = t_end;
+        sr.src0 = c.kcodes + ((size_t)b * Hkv + kv_first) * nquads(cfg.T_max) * F::BW;
+        sr.head_stride = (size_t)nquads(cfg.T_max) * F::BW;
+        sr.quad_bytes = (uint32_t)F::BW * 4;
+        int cc = 0;
+        for (; cc < nch; ++cc) {
+            const int slot = cc % kStages;
+            if (cc >= kStages && !mbar_wait(empty + slot, (uint32_t)(cc / kStages - 1) & 1u)) {
+                if (pl == 0) {
+                    atomicOr(flag, 1);
+                    set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+                }
+                break;
             }
+            if (*flag) break;
+            const int tc = t_begin + cc * kChunk;
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                base[slot * 64 + pl + 32 * u] = trig_at(thi, tlo, tc, pl + 32 * u);
+            __syncwarp();
+            __threadfence_block();
+            if (pl == 0) {
+                fence_proxy_async();
+                sr.issue(cc);
+            }
+            __syncwarp();
         }
-    };
-    __syncthreads();  // tables complete
-    float2 RS[4][4];  // rotation from the chunk start to token 4 qd + (s ^ x), pair i + 16k
+        if (pl == 0) flag[1] = cc;  // chunks issued
+    } else {
+        // ================= consumer warps
+        const int hperm = out_head<HW>(i);
+        uint32_t lb[HW];
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
+        for (int h = 0; h < HW; ++h)
+            lb[h] = ((uint32_t)(hg + (h ^ hperm)) << 9) | ((uint32_t)i << 3);
+        uint32_t woff[NW];
 #pragma unroll
-        for (int sl = 0; sl < 4; ++sl) {
-            const int tau = 4 * qd + (sl ^ x), p = i + 16 * k;
-            RS[k][sl] = cmul(r8[(tau >> 3) * 64 + p], r1[(tau & 7) * 64 + p]);
+        for (int h = 0; h < NW; ++h) {
+            const int kvs = SHARE ? 0 : (hq0 + hg + (h ^ hperm)) / g - kv_first;
+            woff[h] = (uint32_t)(kvs * L.pitch + qd * F::BW * 4 + i * BITS * 4);
         }
-    outliers(0);
-    __syncthreads();
-    const int hs_out = out_head<HPC>(i);
-    const bool owner = out_owner<HPC>(i);
-    const int tq = 4 * qd + x;
-    float run_m = -INFINITY, run_l = 0.0f;
-    int ch = 0;
-    for (; ch < nch; ++ch) {
-        const int tc = t_begin + ch * kChunk;
-        const int slot = ch % kStages;
-        if (!mbar_wait(bars + slot, (uint32_t)(ch / kStages) & 1u)) {
-            atomicOr(flag, 1);
-            set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
-        }
-        const uint8_t* stage = ring + (size_t)slot * kQuads * L.pitch;
-        uint32_t w[NW][BITS];
+        float2 RS[4][4];  // rotation from the chunk start to token 4 qd + (s ^ x), pair i + 16k
 #pragma unroll
-        for (int h = 0; h < NW; ++h)
+        for (int k = 0; k < 4; ++k)
 #pragma unroll
-            for (int d = 0; d < BITS; ++d)
-                w[h][d] = *reinterpret_cast<const uint32_t*>(stage + woff[h] + 4 * d);
-        const float2* bse = base + (ch % 3) * 64;
-        unsigned long long acc[4][HPC];
+            for (int sl = 0; sl < 4; ++sl) RS[k][sl] = rs[(4 * qd + (sl ^ x)) * 64 + i + 16 * k];
+        const int hs_out = hg + hperm;  // CTA head of this lane's logit
+        const bool owner = out_owner<HW>(i);
+        const int tq = 4 * qd + x;
+        float* lrow = logits + ((size_t)b * Hq + hq0 + hs_out) * cfg.T_max;
+        for (int ch = 0; ch < nch; ++ch) {
+            const int slot = ch % kStages;
+            if (!mbar_wait(full + slot, (uint32_t)(ch / kStages) & 1u)) {
+                atomicOr(flag, 1);
+                set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+            }
+            if (*flag) break;
+            const uint8_t* stage = ring + (size_t)slot * L.stage;
+            uint32_t w[NW][BITS];
 #pragma unroll
-        for (int sl = 0; sl < 4; ++sl)
+            for (int h = 0; h < NW; ++h)
 #pragma unroll
-            for (int h = 0; h < HPC; ++h) acc[sl][h] = 0ull;
+                for (int d = 0; d < BITS; ++d)
+                    w[h][d] = *reinterpret_cast<const uint32_t*>(stage + woff[h] + 4 * d);
+            float2 B[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 B = bse[i + 16 * k];
+            for (int k = 0; k < 4; ++k) B[k] = base[slot * 64 + i + 16 * k];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
+            unsigned long long acc[4][HW];
 #pragma unroll
-            for (int sl = 0; sl < 4; ++sl) {
-                const float2 cs = cmul(B, RS[k][sl]);
-                const unsigned long long Pc = pk(cs.x, cs.y);
-                uint32_t fs[NW];
+            for (int sl = 0; sl < 4; ++sl)
 #pragma unroll
-                for (int h = 0; h < NW; ++h) {
-                    switch (4 * k + sl) {
+                for (int h = 0; h < HW; ++h) acc[sl][h] = 0ull;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl) {
+                    const float2 cs = cmul(B[k], RS[k][sl]);
+                    const unsigned long long Pc = pk(cs.x, cs.y);
+                    uint32_t fs[NW];
+#pragma unroll
+                    for (int h = 0; h < NW; ++h) {
+                        switch (4 * k + sl) {
 #define KVQ_FS(N) case N: fs[h] = field_to<BITS, N, P>(w[h]); break;
-                        KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5) KVQ_FS(6)
-                        KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11) KVQ_FS(12)
-                        KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
+                            KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5)
+                            KVQ_FS(6) KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11)
+                            KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
 #undef KVQ_FS
+                        }
+                    }
+#pragma unroll
+                    for (int h = 0; h < HW; ++h) {
+                        const uint32_t off = (fs[SHARE ? 0 : h] & MASK) | lb[h];
+                        acc[sl][h] = fma2(Pc, tld(tab + 128 * k, off), acc[sl][h]);
                     }
                 }
+            }
+            float v[V];
 #pragma unroll
-                for (int h = 0; h < HPC; ++h) {
-                    const uint32_t off = (fs[SHARE ? 0 : h] & MASK) | lb[h];
-                    acc[sl][h] = fma2(Pc, tld(tab + 128 * k, off), acc[sl][h]);
+            for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+                for (int h = 0; h < HW; ++h) {
+                    const f2 a = upk(acc[sl][h]);
+                    v[HW * sl + h] = a.x + a.y;
                 }
-            }
-        }
-        float v[V];
+            // halve across the half-warp: lane bit 3, 2, ... pairs the upper half of the partials
+            int mk = 8;
 #pragma unroll
-        for (int sl = 0; sl < 4; ++sl)
+            for (int half = V / 2; half >= 1; half >>= 1, mk >>= 1)
 #pragma unroll
-            for (int h = 0; h < HPC; ++h) {
-                const f2 a = upk(acc[sl][h]);
-                v[HPC * sl + h] = a.x + a.y;
-            }
-        // halve across the half-warp: lane bit 3, 2, ... pairs the upper half of the partials
-        int mk = 8;
+                for (int t = 0; t < half; ++t)
+                    v[t] += __shfl_xor_sync(0xffffffffu, v[t + half], mk);
 #pragma unroll
-        for (int half = V / 2; half >= 1; half >>= 1, mk >>= 1)
-#pragma unroll
-            for (int t = 0; t < half; ++t) v[t] += __shfl_xor_sync(0xffffffffu, v[t + half], mk);
-#pragma unroll
-        for (int m2 = 16 / V / 2; m2 >= 1; m2 >>= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], m2);
-        {
-            const int t = tc + tq;
-            const float lgt = v[0] + corr[(ch % 3) * 64 * HPC + tq * HPC + hs_out];
-            if (owner && t < t_end) {
-                logits[((size_t)b * Hq + hq0 + hs_out) * cfg.T_max + t] = lgt;
-                if (lgt > run_m) {
-                    run_l = run_l * expf(run_m - lgt) + 1.0f;
-                    run_m = lgt;
-                } else {
-                    run_l += expf(lgt - run_m);
-                }
-            }
-        }
-        if (ch + 1 < nch) outliers(ch + 1);
-        if (tid < 64 && ch + 2 < nch) {
-            rot64(bc, bs, sc64, ss64);
-            base[((ch + 2) % 3) * 64 + tid] = make_float2((float)bc, (float)bs);
-        }
-        for (int e = tid; e < 64 * HPC; e += kThreads) corr[((ch + 2) % 3) * 64 * HPC + e] = 0.0f;
-        __syncthreads();
-        if (*flag) break;
-        if (tid == 0 && issued < nch) {
-            fence_proxy_async();
-            issue_chunk(ring, L.pitch, bars, src0, quad_stride, row_bytes, t_begin, t_end, issued);
-            ++issued;
+            for (int m2 = 16 / V / 2; m2 >= 1; m2 >>= 1)
+                v[0] += __shfl_xor_sync(0xffffffffu, v[0], m2);
+            const int t = t_begin + ch * kChunk + tq;
+            if (owner && t < t_end) lrow[t] = v[0];
         }
     }
-    if (tid == 0 && *flag) drain_chunks(bars, ch, issued);
-    float2* red = (float2*)(sm + L.red);
-    red[tid] = owner ? make_float2(run_m, run_l) : make_float2(-INFINITY, 0.0f);
     __syncthreads();
-    if (tid < HPC) {
-        float M = -INFINITY;
-        for (int e = 0; e < kThreads; ++e)
-            if (out_head<HPC>(e & 15) == tid) M = fmaxf(M, red[e].x);
-        float Ls_ = 0.0f;
-        if (M > -INFINITY)
-            for (int e = 0; e < kThreads; ++e)
-                if (out_head<HPC>(e & 15) == tid && red[e].y > 0.0f)
-                    Ls_ += red[e].y * expf(red[e].x - M);
-        stats[((size_t)b * Hq + hq0 + tid) * S + s] = make_float2(M, Ls_);
+    // after an abandoned wait, copies of the last stages issued may still be in flight
+    if (*flag && tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1]);
+}
+
+// ---------------------------------------------------------------------------------
+// Key outliers: logit(t, hq) += (x - zhat) * r, r the component of the rotated query that
+// meets the outlier's channel after the key is rotated to t.  A warp walks the entries of one
+// 64-token chunk of one (sequence, kv head) list.
+constexpr int kOutWarps = 8;      // warps per block of the outlier kernels
+constexpr int kOutChunks = 64;    // chunks per block
+
+__global__ void __launch_bounds__(kOutWarps * 32) k_key_outliers(
+    kvq_cfg cfg, kvq_cache c, const float* __restrict__ qr, const float2* __restrict__ thi,
+    const float2* __restrict__ tlo, const float* __restrict__ zk, int max_len,
+    float* __restrict__ logits) {
+    const int li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
+    const int g = cfg.Hq / cfg.Hkv;
+    const int len = min(c.len[b], max_len);
+    const int nch1 = nchunks(cfg.T_max) + 1;
+    const uint32_t* cp = c.kchunk + (size_t)li * nch1;
+    const uint32_t cnt = c.kcount[li];
+    const uint32_t* ent = c.kout + (size_t)li * cfg.out_cap_k;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int mend = min((len + kChunk - 1) / kChunk, (int)(blockIdx.x + 1) * kOutChunks);
+    for (int m = blockIdx.x * kOutChunks + warp; m < mend; m += kOutWarps) {
+        const uint32_t lo = min(cp[m], cnt), hi = min(cp[m + 1], cnt);
+        for (uint32_t e = lo + lane; e < hi; e += 32) {
+            const uint32_t w = ent[e];
+            const int t = m * kChunk + (int)((w >> 7) & 63u), ch = (int)(w & 127u);
+            if (t >= len) continue;
+            const int p = ch & 63;
+            const float2 cs = trig_at(thi, tlo, t, p);
+            const float d = h2f((uint16_t)(w >> 16)) - zk[(size_t)li * kD + ch];
+            for (int a = 0; a < g; ++a) {
+                const int hq = h * g + a;
+                const float* qv = qr + ((size_t)b * cfg.Hq + hq) * kD;
+                const float qa = qv[p], qb = qv[p + 64];
+                const float r = (ch < 64) ? (cs.x * qa + cs.y * qb) : (cs.x * qb - cs.y * qa);
+                atomicAdd(&logits[((size_t)b * cfg.Hq + hq) * cfg.T_max + t], d * r);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Softmax statistics of each split from the (corrected) logits: stats = (m_s, l_s).
+__global__ void __launch_bounds__(256) k_logit_stats(kvq_cfg cfg, const int32_t* __restrict__ lens,
+                                                     const float* __restrict__ logits, int Ls,
+                                                     int S, int max_len, float2* __restrict__ stats) {
+    const int s = blockIdx.x, bh = blockIdx.y, b = bh / cfg.Hq;
+    const int len = min(lens[b], max_len);
+    const int t0 = s * Ls, t1 = min(len, t0 + Ls);
+    const float* row = logits + (size_t)bh * cfg.T_max;
+    __shared__ float red[32];
+    float m = -INFINITY;
+    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) m = fmaxf(m, row[t]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    m = -INFINITY;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    __syncthreads();
+    float l = 0.0f;
+    if (m > -INFINITY)
+        for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) l += expf(row[t] - m);
+    l = warp_sum(l);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = l;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float a = 0.0f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) a += red[w];
+        stats[(size_t)bh * S + s] = make_float2(m, a);
     }
 }
 
 // ---------------------------------------------------------------------------------
 // PV.  out_h = sum_t p_t (off_t + half_t L[code]) = sum_t p_t off_t + sum_t (p_t half_t) L[code];
 // per pair (c, c + 64) and token one (La, Lb) lookup (a 16-copy table, copy = lane) and one
-// f32x2 FMA with (w, w), w = p half.  Lane i computes the weight of (token i >> 2 of its quad,
-// head out_head(i)); value outliers of a chunk are applied during the next one.
+// f32x2 FMA with (w, w), w = p half.  A consumer warp takes two token quads and HW heads;
+// lane i computes the weight of (token i >> 2 of its quad, head out_head(i) of the warp).  The
+// last warp streams the chunks.
 template <int BITS, int HPC, bool SHARE>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(consumer_warps(HPC) * 32 + 32, 1)
     k_pv(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
          const float2* __restrict__ ml, int Ls, int S, int max_len, int kvb,
          float* __restrict__ part) {
     using F = Fmt<BITS>;
+    constexpr int CW = consumer_warps(HPC), NC = CW * 32;
+    constexpr int HW = heads_per_warp<HPC>();
     constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << 7;
-    constexpr int NW = SHARE ? 1 : HPC;
+    constexpr int NW = SHARE ? 1 : HW;
     extern __shared__ __align__(128) uint8_t sm[];
     const PVPlan L = pv_plan(BITS, HPC, kvb);
     uint8_t* tab = sm + L.tab;
     uint8_t* ring = sm + L.ring;
     unsigned long long* wsm = (unsigned long long*)(sm + L.wsm);
-    float* psm = (float*)(sm + L.psm);
-    float2* vsm = (float2*)(sm + L.vsm);
-    float* corr = (float*)(sm + L.corr);
-    float* pored = (float*)(sm + L.pored);
-    float* posum = (float*)(sm + L.posum);
-    float* vb = (float*)(sm + L.vb);
-    uint64_t* bars = (uint64_t*)(sm + L.bar);
+    uint64_t* full = (uint64_t*)(sm + L.bar);
+    uint64_t* empty = full + kStages;
     int* flag = (int*)(sm + L.flag);
 
-    const int tid = threadIdx.x, i = tid & 15, qd = tid >> 4, x = i >> 2;
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int i = tid & 15, x = i >> 2, lane = tid & 31, warp = tid >> 5;
+    const int qd = 2 * (warp & 7) + ((tid >> 4) & 1);  // token quad of the chunk
+    const int hg = (warp >> 3) * HW;                     // first CTA head of the warp
     const int s = blockIdx.x, b = blockIdx.y, hq0 = blockIdx.z * HPC;
     const int Hq = cfg.Hq, Hkv = cfg.Hkv, g = Hq / Hkv;
     const int len = min(c.len[b], max_len);
     const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
     if (t_begin >= t_end) {
-        for (int e = tid; e < HPC * kD; e += kThreads)
+        for (int e = tid; e < HPC * kD; e += nthr)
             part[(((size_t)b * Hq + hq0 + (e >> 7)) * S + s) * kD + (e & 127)] = 0.0f;
         return;
     }
     const int nch = (t_end - t_begin + kChunk - 1) / kChunk;
     const int kv_first = min(hq0 / g, Hkv - kvb);
-    const size_t NQ = nquads(cfg.T_max);
-    const uint32_t* src0 = c.vcodes + ((size_t)b * NQ * Hkv + kv_first) * F::BW;
-    const size_t quad_stride = (size_t)Hkv * F::BW;
-    const uint32_t row_bytes = (uint32_t)kvb * F::BW * 4;
     if (tid == 0) {
-        for (int k = 0; k < kStages; ++k) mbar_init(bars + k, 1);
-        *flag = 0;
+        for (int k = 0; k < kStages; ++k) {
+            mbar_init(full + k, 1);
+            mbar_init(empty + k, CW);
+        }
+        flag[0] = 0;
+        flag[1] = 0;
         fence_mbar_init();
     }
-    __syncthreads();
-    int issued = 0;
-    if (tid == 0) {
-        for (; issued < min(kStages, nch); ++issued)
-            issue_chunk(ring, L.pitch, bars, src0, quad_stride, row_bytes, t_begin, t_end, issued);
-    }
     const int nb = (1 << BITS) - 1;
-    if (tid < nb) vb[tid] = cb.bounds[tid];
-    for (int e = tid; e < F::NT * 16; e += kThreads) {
+    for (int e = tid; e < F::NT * 16; e += nthr) {
         const int idx = e >> 4;
         reinterpret_cast<unsigned long long*>(tab)[e] =
             pk(cb.levels[idx & nb], cb.levels[idx >> BITS]);
     }
-    for (int e = tid; e < HPC * kD; e += kThreads) corr[e] = 0.0f;
-    const int hs = out_head<HPC>(i);
-    const bool owner = out_owner<HPC>(i);
-    const int tq = 4 * qd + x;
-    const float2 mL = ml[(size_t)b * Hq + hq0 + hs];
-    const float invL = mL.y > 0.0f ? 1.0f / mL.y : 0.0f;
-    const float* lrow = logits + ((size_t)b * Hq + hq0 + hs) * cfg.T_max;
-    const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
-    float lg = -INFINITY;
-    float2 vp = make_float2(0.0f, 0.0f);
-    auto fetch = [&](int cc) {
-        const int t = t_begin + cc * kChunk + tq;
-        const bool ok = t < t_end;
-        lg = (owner && ok) ? lrow[t] : -INFINITY;
-        vp = ok ? vpar[t] : make_float2(0.0f, 0.0f);
-    };
-    fetch(0);
-    uint32_t woff[NW];
-#pragma unroll
-    for (int h = 0; h < NW; ++h) {
-        const int kvs = SHARE ? 0 : (hq0 + h) / g - kv_first;
-        woff[h] = (uint32_t)(qd * L.pitch + kvs * F::BW * 4 + i * BITS * 4);
-    }
-    const uint32_t lanebits = (uint32_t)i << 3;
-    const int khlo = hq0 / g, khhi = (hq0 + HPC - 1) / g;
-    const int nch1 = nchunks(cfg.T_max) + 1;
-    const uint32_t* vchunk = c.vchunk + (size_t)b * nch1;
-    const uint32_t vcount = c.vcount[b];
-    const uint32_t* opos = c.vout_pos + (size_t)b * cfg.out_cap_v;
-    const uint16_t* oval = c.vout_val + (size_t)b * cfg.out_cap_v;
-    // value outliers of chunk cc: out(h, c) += p(t, h) * (x - zhat_t)
-    auto outliers = [&](int cc) {
-        const int m = (t_begin + cc * kChunk) / kChunk;
-        const uint32_t lo = min(vchunk[m], vcount), hi = min(vchunk[m + 1], vcount);
-        const float* pb = psm + (cc & 1) * 64 * HPC;
-        const float2* vv = vsm + (cc & 1) * 64;
-        for (uint32_t e = lo + tid; e < hi; e += kThreads) {
-            const uint32_t pw = opos[e];
-            const int tl = (int)(pw >> 16), jf = (int)(pw & 0xffffu);
-            const int kh = jf >> 7, chn = jf & 127;
-            if (tl >= kChunk || kh < khlo || kh > khhi) continue;
-            const float2 o2 = vv[tl];
-            const float d = h2f(oval[e]) - zero_code_value(o2.x, o2.y, cb.levels, vb, nb);
-#pragma unroll
-            for (int h = 0; h < HPC; ++h) {
-                if ((hq0 + h) / g != kh) continue;
-                atomicAdd(&corr[h * kD + chn], pb[tl * HPC + h] * d);
-            }
-        }
-    };
-    __syncthreads();  // tables complete
-    unsigned long long O[4][HPC];
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-#pragma unroll
-        for (int h = 0; h < HPC; ++h) O[k][h] = 0ull;
+    __syncthreads();  // tables complete, barriers initialised
+
+    unsigned long long O[4][HW];
     float po = 0.0f;
-    int ch = 0;
-    for (; ch < nch; ++ch) {
-        const int slot = ch % kStages;
-        {
-            const float p = (lg > -INFINITY) ? expf(lg - mL.x) * invL : 0.0f;
-            const float wv = p * vp.y;
-            po += p * vp.x;
-            if (owner) {
-                wsm[(qd * 4 + x) * HPC + hs] = pk(wv, wv);
-                psm[(ch & 1) * 64 * HPC + tq * HPC + hs] = p;
-                if (hs == 0) vsm[(ch & 1) * 64 + tq] = vp;
+    const int hs = hg + out_head<HW>(i);  // CTA head of this lane's weight
+    const bool owner = out_owner<HW>(i);
+    if (tid >= NC) {
+        // ================= streaming warp
+        const int pl = tid - NC;
+        Streamer sr;
+        sr.ring = ring;
+        sr.full = full;
+        sr.pitch = L.pitch;
+        sr.stage = L.stage;
+        sr.kvb = kvb;
+        sr.t_begin = t_begin;
+        sr.t_end = t_end;
+        sr.src0 = c.vcodes + ((size_t)b * Hkv + kv_first) * nquads(cfg.T_max) * F::BW;
+        sr.head_stride = (size_t)nquads(cfg.T_max) * F::BW;
+        sr.quad_bytes = (uint32_t)F::BW * 4;
+        int cc = 0;
+        for (; cc < nch; ++cc) {
+            const int slot = cc % kStages;
+            if (cc >= kStages && !mbar_wait(empty + slot, (uint32_t)(cc / kStages - 1) & 1u)) {
+                if (pl == 0) {
+                    atomicOr(flag, 1);
+                    set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+                }
+                break;
             }
+            if (*flag) break;
+            if (pl == 0) {
+                fence_proxy_async();
+                sr.issue(cc);
+            }
+            __syncwarp();
         }
-        if (ch + 1 < nch) fetch(ch + 1);
-        __syncwarp();
-        if (!mbar_wait(bars + slot, (uint32_t)(ch / kStages) & 1u)) {
-            atomicOr(flag, 1);
-            set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+        if (pl == 0) flag[1] = cc;  // chunks issued
+    } else {
+        // ================= consumer warps
+        const int tq = 4 * qd + x;
+        const float2 mL = ml[(size_t)b * Hq + hq0 + hs];
+        const float invL = mL.y > 0.0f ? 1.0f / mL.y : 0.0f;
+        const float* lrow = logits + ((size_t)b * Hq + hq0 + hs) * cfg.T_max;
+        const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
+        float lg = -INFINITY;
+        float2 vp = make_float2(0.0f, 0.0f);
+        auto fetch = [&](int cc) {
+            const int t = t_begin + cc * kChunk + tq;
+            const bool ok = owner && t < t_end;
+            lg = ok ? lrow[t] : -INFINITY;
+            vp = ok ? vpar[t] : make_float2(0.0f, 0.0f);
+        };
+        fetch(0);
+        uint32_t woff[NW];
+#pragma unroll
+        for (int h = 0; h < NW; ++h) {
+            const int kvs = SHARE ? 0 : (hq0 + hg + h) / g - kv_first;
+            woff[h] = (uint32_t)(kvs * L.pitch + qd * F::BW * 4 + i * BITS * 4);
         }
-        const uint8_t* stage = ring + (size_t)slot * kQuads * L.pitch;
-        uint32_t w[NW][BITS];
+        const uint32_t lanebits = (uint32_t)i << 3;
 #pragma unroll
-        for (int h = 0; h < NW; ++h)
+        for (int k = 0; k < 4; ++k)
 #pragma unroll
-            for (int d = 0; d < BITS; ++d)
-                w[h][d] = *reinterpret_cast<const uint32_t*>(stage + woff[h] + 4 * d);
+            for (int h = 0; h < HW; ++h) O[k][h] = 0ull;
+        for (int ch = 0; ch < nch; ++ch) {
+            const int slot = ch % kStages;
+            {
+                const float p = (lg > -INFINITY) ? expf(lg - mL.x) * invL : 0.0f;
+                const float wv = p * vp.y;
+                po = fmaf(p, vp.x, po);
+                if (owner) wsm[(qd * 4 + x) * HPC + hs] = pk(wv, wv);
+            }
+            __syncwarp();
+            if (ch + 1 < nch) fetch(ch + 1);
+            if (!mbar_wait(full + slot, (uint32_t)(ch / kStages) & 1u)) {
+                atomicOr(flag, 1);
+                set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+            }
+            if (*flag) break;
+            const uint8_t* stage = ring + (size_t)slot * L.stage;
+            uint32_t w[NW][BITS];
 #pragma unroll
-        for (int sl = 0; sl < 4; ++sl) {
-            unsigned long long ww[HPC];
+            for (int h = 0; h < NW; ++h)
 #pragma unroll
-            for (int h = 0; h < HPC; ++h) ww[h] = wsm[(qd * 4 + (sl ^ x)) * HPC + h];
+                for (int d = 0; d < BITS; ++d)
+                    w[h][d] = *reinterpret_cast<const uint32_t*>(stage + woff[h] + 4 * d);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
+            for (int sl = 0; sl < 4; ++sl) {
+                unsigned long long ww[HW];
 #pragma unroll
-                for (int h = 0; h < NW; ++h) {
-                    uint32_t fs = 0;
-                    switch (4 * k + sl) {
+                for (int h = 0; h < HW; ++h) ww[h] = wsm[(qd * 4 + (sl ^ x)) * HPC + hg + h];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                    for (int h = 0; h < NW; ++h) {
+                        uint32_t fs = 0;
+                        switch (4 * k + sl) {
 #define KVQ_FS(N) case N: fs = field_to<BITS, N, 7>(w[h]); break;
-                        KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5) KVQ_FS(6)
-                        KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11) KVQ_FS(12)
-                        KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
+                            KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5)
+                            KVQ_FS(6) KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11)
+                            KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
 #undef KVQ_FS
-                    }
-                    const unsigned long long LL = tld(tab, (fs & MASK) | lanebits);
-                    if (SHARE) {
+                        }
+                        const unsigned long long LL = tld(tab, (fs & MASK) | lanebits);
+                        if (SHARE) {
 #pragma unroll
-                        for (int hh = 0; hh < HPC; ++hh) O[k][hh] = fma2(ww[hh], LL, O[k][hh]);
-                    } else {
-                        O[k][h] = fma2(ww[h], LL, O[k][h]);
+                            for (int hh = 0; hh < HW; ++hh) O[k][hh] = fma2(ww[hh], LL, O[k][hh]);
+                        } else {
+                            O[k][h] = fma2(ww[h], LL, O[k][h]);
+                        }
                     }
                 }
             }
-        }
-        if (ch >= 1) outliers(ch - 1);
-        __syncthreads();
-        if (*flag) break;
-        if (tid == 0 && issued < nch) {
-            fence_proxy_async();
-            issue_chunk(ring, L.pitch, bars, src0, quad_stride, row_bytes, t_begin, t_end, issued);
-            ++issued;
+            __syncwarp();  // wsm is rewritten for the next chunk
         }
     }
-    if (tid == 0 && *flag) drain_chunks(bars, ch, issued);
-    if (!*flag) outliers(nch - 1);
-    pored[tid] = owner ? po : 0.0f;
     __syncthreads();
-    // partial sums of the 16 quads -> the split's output
+    if (*flag) {
+        if (tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1]);
+        return;
+    }
+    // partial sums of the 16 quads -> the split's output (the ring is idle now)
     float* red = (float*)ring;
+    if (tid < NC) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
+        for (int k = 0; k < 4; ++k)
 #pragma unroll
-        for (int h = 0; h < HPC; ++h) {
-            const f2 o = upk(O[k][h]);
-            red[(qd * HPC + h) * kD + i + 16 * k] = o.x;
-            red[(qd * HPC + h) * kD + i + 16 * k + 64] = o.y;
-        }
-    if (tid < HPC) {
-        float a = 0.0f;
-        for (int e = 0; e < kThreads; ++e)
-            if (out_head<HPC>(e & 15) == tid) a += pored[e];
-        posum[tid] = a;
+            for (int h = 0; h < HW; ++h) {
+                const f2 o = upk(O[k][h]);
+                red[(qd * HPC + hg + h) * kD + i + 16 * k] = o.x;
+                red[(qd * HPC + hg + h) * kD + i + 16 * k + 64] = o.y;
+            }
     }
+    // sum_t p_t off_t per head: the owners' shares, reduced through the ring's tail region
+    float* pored = red + kQuads * HPC * kD;
+    if (tid < NC) pored[tid] = owner ? po : 0.0f;
     __syncthreads();
-    for (int e = tid; e < HPC * kD; e += kThreads) {
+    for (int e = tid; e < HPC * kD; e += nthr) {
         const int h = e >> 7, ch2 = e & 127;
-        float a = posum[h] + corr[h * kD + ch2];
+        float a = 0.0f;
         for (int qq = 0; qq < kQuads; ++qq) a += red[(qq * HPC + h) * kD + ch2];
-        part[(((size_t)b * Hq + hq0 + h) * S + s) * kD + ch2] = a;
+        float o = 0.0f;
+        for (int t2 = 0; t2 < NC; ++t2)
+            if (((t2 >> 8) * HW + out_head<HW>(t2 & 15)) == h) o += pored[t2];
+        part[(((size_t)b * Hq + hq0 + h) * S + s) * kD + ch2] = a + o;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Value outliers: out(hq, c) += p(t, hq) (x - zhat_t), p = exp(l - M) / L from the merged
+// statistics, zhat_t = off_t + half_t L[encode(normalize(0))].  A warp walks one chunk of one
+// (sequence, kv head) list; a block adds its sums to the output once.
+__global__ void __launch_bounds__(kOutWarps * 32) k_value_outliers(
+    kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
+    const float2* __restrict__ ml, int max_len, float* __restrict__ out) {
+    const int li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
+    const int g = cfg.Hq / cfg.Hkv;
+    const int len = min(c.len[b], max_len);
+    const int nch1 = nchunks(cfg.T_max) + 1;
+    const uint32_t* cp = c.vchunk + (size_t)li * nch1;
+    const uint32_t cnt = c.vcount[li];
+    const uint32_t* ent = c.vout + (size_t)li * cfg.out_cap_v;
+    __shared__ float acc[kMaxG * kD];
+    __shared__ float bnd[16];
+    const int nb = (1 << cfg.bits) - 1;
+    if (threadIdx.x < nb) bnd[threadIdx.x] = cb.bounds[threadIdx.x];
+    for (int e = threadIdx.x; e < g * kD; e += blockDim.x) acc[e] = 0.0f;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int mend = min((len + kChunk - 1) / kChunk, (int)(blockIdx.x + 1) * kOutChunks);
+    bool any = false;
+    for (int m = blockIdx.x * kOutChunks + warp; m < mend; m += kOutWarps) {
+        const uint32_t lo = min(cp[m], cnt), hi = min(cp[m + 1], cnt);
+        for (uint32_t e = lo + lane; e < hi; e += 32) {
+            const uint32_t w = ent[e];
+            const int t = m * kChunk + (int)((w >> 7) & 63u), ch = (int)(w & 127u);
+            if (t >= len) continue;
+            const float* vp = c.vparams + ((size_t)b * cfg.T_max + t) * 2;
+            const float d = h2f((uint16_t)(w >> 16)) - zero_code_value(vp[0], vp[1], cb.levels, bnd, nb);
+            for (int a = 0; a < g; ++a) {
+                const size_t bh = (size_t)b * cfg.Hq + h * g + a;
+                const float2 mLs = ml[bh];
+                const float p = mLs.y > 0.0f ? expf(logits[bh * cfg.T_max + t] - mLs.x) / mLs.y : 0.0f;
+                atomicAdd(&acc[a * kD + ch], p * d);
+            }
+            any = true;
+        }
+    }
+    any = __syncthreads_or(any);
+    if (!any) return;
+    for (int e = threadIdx.x; e < g * kD; e += blockDim.x) {
+        const float v = acc[e];
+        if (v != 0.0f) atomicAdd(&out[((size_t)b * cfg.Hq + h * g + e / kD) * kD + e % kD], v);
     }
 }
 
@@ -888,7 +992,7 @@ __global__ void __launch_bounds__(kF16Threads) k_fp16_attn(kvq_cfg cfg, const ui
 
 using namespace kvq_host;
 
-// Query heads per CTA of the quantized kernels and the number of kv heads they span.
+// Query heads per CTA of the streaming kernels and the number of kv heads they span.
 static int hpc_of(const kvq_cfg* cfg) { return cfg->Hq % 4 == 0 ? 4 : (cfg->Hq % 2 == 0 ? 2 : 1); }
 static int kvb_of(const kvq_cfg* cfg, int hpc) {
     const int g = cfg->Hq / cfg->Hkv;
@@ -931,8 +1035,33 @@ static int check_decode(const kvq_cfg* cfg, int max_len) {
     return KVQ_OK;
 }
 
-typedef void (*QKKernel)(kvq_cfg, kvq_cache, kvq_codebook, const uint16_t*, const int32_t*, int,
-                         int, int, int, float*, float2*);
+// Per-call tables of the QK path (kvq_decode_qk's workspace).
+struct QKTables {
+    float* qr;     // [B][Hq][128]
+    float2* thi;   // [nhi][64]
+    float2* tlo;   // [256][64]
+    float* zk;     // [B][Hkv][128]
+    int nhi;
+    size_t bytes;
+};
+static QKTables qk_tables(const kvq_cfg* cfg, int max_len, void* ws) {
+    QKTables t;
+    t.nhi = (max_len + kTrigLo - 1) / kTrigLo;
+    const size_t sq = align_up((size_t)cfg->B * cfg->Hq * kD * 4);
+    const size_t sh = align_up((size_t)t.nhi * 64 * 8);
+    const size_t sl = align_up((size_t)kTrigLo * 64 * 8);
+    const size_t sz = align_up((size_t)cfg->B * cfg->Hkv * kD * 4);
+    char* w = (char*)ws;
+    t.qr = (float*)w;
+    t.thi = (float2*)(w + sq);
+    t.tlo = (float2*)(w + sq + sh);
+    t.zk = (float*)(w + sq + sh + sl);
+    t.bytes = sq + sh + sl + sz;
+    return t;
+}
+
+typedef void (*QKKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*,
+                         const float2*, int, int, int, float*);
 typedef void (*PVKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*, int, int,
                          int, int, float*);
 
@@ -954,9 +1083,15 @@ static PVKernel pv_kernel(int hpc, bool share) {
     return k_pv<BITS, 1, true>;
 }
 
-static int launch_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
-                     const uint16_t* q, const int32_t* qpos, int max_len, float* logits,
-                     float* stats, int S, int Ls, cudaStream_t st) {
+// QK over the quantized cache into logits, key-outlier corrections, split statistics.
+static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
+                  const uint16_t* q, const int32_t* qpos, int max_len, float* logits,
+                  float* stats, int S, int Ls, const QKTables& T, cudaStream_t st) {
+    {
+        const int n = cfg->B * cfg->Hq * 64 + T.nhi * 64 + kTrigLo * 64 + cfg->B * cfg->Hkv * kD;
+        k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi, T.qr,
+                                                        T.thi, T.tlo, T.zk);
+    }
     const int hpc = cfg->bits == 4 ? 1 : hpc_of(cfg);
     const int kvb = kvb_of(cfg, hpc);
     QKKernel kern = cfg->bits == 2 ? qk_kernel<2>(hpc, kvb == 1)
@@ -966,21 +1101,39 @@ static int launch_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codeb
     cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (ce) return record_cuda(ce);
     dim3 grid(S, cfg->B, cfg->Hq / hpc);
-    kern<<<grid, kThreads, smem, st>>>(*cfg, *cache, *cbK, q, qpos, Ls, S, max_len, kvb, logits,
-                                       (float2*)stats);
+    kern<<<grid, consumer_warps(hpc) * 32 + 32, smem, st>>>(*cfg, *cache, *cbK, T.qr, T.thi, T.tlo,
+                                                            Ls, max_len, kvb, logits);
+    const int nch = (max_len + kChunk - 1) / kChunk;
+    dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
+    k_key_outliers<<<go, kOutWarps * 32, 0, st>>>(*cfg, *cache, T.qr, T.thi, T.tlo, T.zk, max_len,
+                                                   logits);
+    dim3 gs(S, cfg->B * cfg->Hq);
+    k_logit_stats<<<gs, 256, 0, st>>>(*cfg, cache->len, logits, Ls, S, max_len, (float2*)stats);
     return record_cuda(cudaGetLastError());
+}
+
+extern "C" int kvq_decode_qk_workspace(const kvq_cfg* cfg, int32_t max_len, size_t* bytes) {
+    int e = check_decode(cfg, max_len);
+    if (e) return e;
+    if (!bytes) return KVQ_ERR_NULL;
+    *bytes = qk_tables(cfg, max_len, nullptr).bytes;
+    return KVQ_OK;
 }
 
 extern "C" int kvq_decode_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
                              const uint16_t* q, const int32_t* qpos, int32_t max_len,
-                             float* logits, float* stats, int32_t splits, void* stream) {
+                             float* logits, float* stats, int32_t splits, void* workspace,
+                             size_t workspace_bytes, void* stream) {
     int e = check_decode(cfg, max_len);
     if (e) return e;
     if ((e = check_cache(cfg, cache)) || (e = check_codebook(cbK))) return e;
-    if (!q || !qpos || !logits || !stats) return KVQ_ERR_NULL;
+    if (!q || !qpos || !logits || !stats || !workspace) return KVQ_ERR_NULL;
+    if (!aligned16(workspace)) return KVQ_ERR_ALIGN;
     int S, Ls;
     if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
-    return launch_qk(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, (cudaStream_t)stream);
+    const QKTables T = qk_tables(cfg, max_len, workspace);
+    if (workspace_bytes < T.bytes) return KVQ_ERR_WORKSPACE;
+    return run_qk(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, T, (cudaStream_t)stream);
 }
 
 extern "C" int kvq_softmax_merge(const kvq_cfg* cfg, const float* stats, int32_t splits,
@@ -996,9 +1149,10 @@ extern "C" int kvq_softmax_merge(const kvq_cfg* cfg, const float* stats, int32_t
     return record_cuda(cudaGetLastError());
 }
 
-static int launch_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbV,
-                     const float* logits, const float* ml, int max_len, float* part, int S,
-                     int Ls, cudaStream_t st) {
+// PV over the quantized cache into per-split partials, their sum, value-outlier corrections.
+static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbV,
+                  const float* logits, const float* ml, int max_len, float* out, float* part,
+                  int S, int Ls, cudaStream_t st) {
     const int hpc = hpc_of(cfg);
     const int kvb = kvb_of(cfg, hpc);
     PVKernel kern = cfg->bits == 2 ? pv_kernel<2>(hpc, kvb == 1)
@@ -1008,8 +1162,14 @@ static int launch_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codeb
     cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (ce) return record_cuda(ce);
     dim3 grid(S, cfg->B, cfg->Hq / hpc);
-    kern<<<grid, kThreads, smem, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls, S,
-                                       max_len, kvb, part);
+    kern<<<grid, consumer_warps(hpc) * 32 + 32, smem, st>>>(*cfg, *cache, *cbV, logits,
+                                                            (const float2*)ml, Ls, S, max_len,
+                                                            kvb, part);
+    k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
+    const int nch = (max_len + kChunk - 1) / kChunk;
+    dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
+    k_value_outliers<<<go, kOutWarps * 32, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml,
+                                                     max_len, out);
     return record_cuda(cudaGetLastError());
 }
 
@@ -1022,10 +1182,7 @@ extern "C" int kvq_decode_pv(const kvq_cfg* cfg, const kvq_cache* cache, const k
     if (!logits || !ml || !out || !part) return KVQ_ERR_NULL;
     int S, Ls;
     if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
-    cudaStream_t st = (cudaStream_t)stream;
-    if ((e = launch_pv(cfg, cache, cbV, logits, ml, max_len, part, S, Ls, st))) return e;
-    k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
-    return record_cuda(cudaGetLastError());
+    return run_pv(cfg, cache, cbV, logits, ml, max_len, out, part, S, Ls, (cudaStream_t)stream);
 }
 
 static size_t split_ws_bytes(const kvq_cfg* cfg, int S, int max_len) {
@@ -1033,7 +1190,8 @@ static size_t split_ws_bytes(const kvq_cfg* cfg, int S, int max_len) {
     return align_up(BH * (size_t)cfg->T_max * 4)   // logits
            + align_up(BH * S * 8)                  // stats
            + align_up(BH * 8)                      // ml
-           + align_up(BH * S * kD * 4);            // partials
+           + align_up(BH * S * kD * 4)             // partials
+           + qk_tables(cfg, max_len, nullptr).bytes;
 }
 
 extern "C" int kvq_decode_workspace(const kvq_cfg* cfg, int32_t max_len, int32_t splits,
@@ -1054,7 +1212,9 @@ extern "C" int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache,
                                     int32_t splits, void* stream) {
     int e = check_decode(cfg, max_len);
     if (e) return e;
-    if (!workspace || !out) return KVQ_ERR_NULL;
+    if ((e = check_cache(cfg, cache)) || (e = check_codebook(cbK)) || (e = check_codebook(cbV)))
+        return e;
+    if (!workspace || !out || !q || !qpos) return KVQ_ERR_NULL;
     if (!aligned16(workspace)) return KVQ_ERR_ALIGN;
     int S, Ls;
     if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
@@ -1068,9 +1228,12 @@ extern "C" int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache,
     float* ml = (float*)w;
     w += align_up(BH * 8);
     float* part = (float*)w;
-    if ((e = kvq_decode_qk(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, stream))) return e;
+    w += align_up(BH * S * kD * 4);
+    const QKTables T = qk_tables(cfg, max_len, w);
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((e = run_qk(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, T, st))) return e;
     if ((e = kvq_softmax_merge(cfg, stats, S, ml, stream))) return e;
-    return kvq_decode_pv(cfg, cache, cbV, logits, ml, max_len, out, part, S, stream);
+    return run_pv(cfg, cache, cbV, logits, ml, max_len, out, part, S, Ls, st);
 }
 
 extern "C" int kvq_fp16_decode_attention(const kvq_cfg* cfg, const uint16_t* K, const uint16_t* V,

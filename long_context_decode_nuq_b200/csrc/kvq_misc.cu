@@ -23,7 +23,7 @@ __global__ void k_dequant_dense(kvq_cfg cfg, kvq_cache c, kvq_codebook cbK, kvq_
         return;
     }
     const int h = j / kD, ch = j % kD, BW = block_words(cfg.bits);
-    const size_t blk = (((size_t)b * nquads(cfg.T_max) + t / 4) * cfg.Hkv + h) * BW;
+    const size_t blk = (((size_t)b * cfg.Hkv + h) * nquads(cfg.T_max) + t / 4) * BW;
     const float* kp = c.kparams + ((size_t)b * n + j) * 2;
     const float* vp = c.vparams + ((size_t)b * cfg.T_max + t) * 2;
     const float lk = cbK.levels[block_code(c.kcodes + blk, cfg.bits, ch, t & 3)];
@@ -33,16 +33,16 @@ __global__ void k_dequant_dense(kvq_cfg cfg, kvq_cache c, kvq_codebook cbK, kvq_
 }
 
 // Outlier replacement: entries of tokens in [t0, t0 + nt).
+// Outlier replacement: entries of tokens in [t0, t0 + nt) of list (b, h) = blockIdx.y.
 __global__ void k_dequant_outliers(kvq_cfg cfg, kvq_cache c, int t0, int nt, uint16_t* khat,
                                    uint16_t* vhat, int which) {
-    const int b = blockIdx.y;
+    const int li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
     const int n = cfg.Hkv * kD;
     const int nch1 = nchunks(cfg.T_max) + 1;
-    const uint32_t* chunk = (which ? c.vchunk : c.kchunk) + (size_t)b * nch1;
-    const uint32_t cnt = (which ? c.vcount : c.kcount)[b];
+    const uint32_t* chunk = (which ? c.vchunk : c.kchunk) + (size_t)li * nch1;
+    const uint32_t cnt = (which ? c.vcount : c.kcount)[li];
     const int cap = which ? cfg.out_cap_v : cfg.out_cap_k;
-    const uint32_t* pos = (which ? c.vout_pos : c.kout_pos) + (size_t)b * cap;
-    const uint16_t* val = (which ? c.vout_val : c.kout_val) + (size_t)b * cap;
+    const uint32_t* ent = (which ? c.vout : c.kout) + (size_t)li * cap;
     uint16_t* dst = which ? vhat : khat;
     const int len = c.len[b];
     const int tend = min(t0 + nt, len);
@@ -58,11 +58,11 @@ __global__ void k_dequant_outliers(kvq_cfg cfg, kvq_cache c, int t0, int nt, uin
             const int mid = (a + z + 1) >> 1;
             if (chunk[mid] <= e) a = mid; else z = mid - 1;
         }
-        const uint32_t p = pos[e];
-        const int t = a * kChunk + (int)(p >> 16);
-        const int j = (int)(p & 0xffffu);
-        if (t < t0 || t >= tend || j >= n) continue;
-        dst[((size_t)b * nt + (t - t0)) * n + j] = val[e];
+        const uint32_t p = ent[e];
+        const int t = a * kChunk + (int)((p >> 7) & 63u);
+        const int ch = (int)(p & 127u);
+        if (t < t0 || t >= tend) continue;
+        dst[((size_t)b * nt + (t - t0)) * n + h * kD + ch] = (uint16_t)(p >> 16);
     }
 }
 
@@ -335,7 +335,7 @@ extern "C" int kvq_dequantize(const kvq_cfg* cfg, const kvq_cache* cache, const 
     const int n = cfg->Hkv * kD;
     dim3 g((n + 127) / 128, nt, cfg->B);
     k_dequant_dense<<<g, 128, 0, st>>>(*cfg, *cache, *cbK, *cbV, t0, nt, khat, vhat);
-    dim3 go(64, cfg->B);
+    dim3 go(16, cfg->B * cfg->Hkv);
     k_dequant_outliers<<<go, 256, 0, st>>>(*cfg, *cache, t0, nt, khat, vhat, 0);
     k_dequant_outliers<<<go, 256, 0, st>>>(*cfg, *cache, t0, nt, khat, vhat, 1);
     return record_cuda(cudaGetLastError());

@@ -27,9 +27,9 @@ struct QuantWs {
     uint32_t* sel1;   // [B][n][4]  bin_lo, rem_lo, bin_hi, rem_hi
     uint32_t* hist2;  // [B][n][512]
     uint32_t* vthr;   // [B][n_new] fp16 t_lo | t_hi << 16
-    uint32_t* kcnt;   // [B][n_new]
+    uint32_t* kcnt;   // [B][Hkv][n_new] outliers of token i in head h
     uint32_t* vcnt;
-    uint32_t* koff;   // [B][n_new] first entry of the token, 0xffffffff if dropped
+    uint32_t* koff;   // [B][Hkv][n_new] its first entry in list (b, h), 0xffffffff if dropped
     uint32_t* voff;
 };
 
@@ -45,7 +45,8 @@ WsPlan plan_ws(const kvq_cfg& cfg, int n_new, int calibrate) {
                         calibrate ? B * n * 256 * 4 : 0,
                         calibrate ? B * n * 4 * 4 : 0,
                         calibrate ? B * n * 512 * 4 : 0,
-                        B * T * 4, B * T * 4, B * T * 4, B * T * 4, B * T * 4};
+                        B * T * 4, B * T * cfg.Hkv * 4, B * T * cfg.Hkv * 4,
+                        B * T * cfg.Hkv * 4, B * T * cfg.Hkv * 4};
     WsPlan p;
     size_t o = 0;
     for (int i = 0; i < 11; ++i) {
@@ -262,7 +263,6 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_stats(kvq_cfg cfg, kvq_cach
     const int n = cfg.Hkv * kD;
     __shared__ uint32_t hist[512];
     __shared__ uint32_t sel[4];
-    __shared__ uint32_t red[2][32];
     const uint16_t* vrow = v + ((size_t)b * n_new + i) * n;
     const uint16_t* krow = k + ((size_t)b * n_new + i) * n;
     for (int q = threadIdx.x; q < 512; q += blockDim.x) hist[q] = 0;
@@ -300,26 +300,31 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_stats(kvq_cfg cfg, kvq_cach
         c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1] = __fmul_rn(__fsub_rn(vhi, vlo), 0.5f);
         ws.vthr[(size_t)b * n_new + i] = lo_bits | (hi_bits << 16);
     }
-    uint32_t kc = 0, vc = 0;
-    const uint16_t* kt = c.kthr + (size_t)b * n * 2;
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-        const float xv = h2f(vrow[j]);
-        vc += (xv < vlo || xv > vhi) ? 1u : 0u;
-        const float xk = h2f(krow[j]);
-        kc += (xk < h2f(kt[2 * j]) || xk > h2f(kt[2 * j + 1])) ? 1u : 0u;
-    }
-    for (int o = 16; o; o >>= 1) {
-        kc += __shfl_xor_sync(0xffffffffu, kc, o);
-        vc += __shfl_xor_sync(0xffffffffu, vc, o);
-    }
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (lane == 0) { red[0][warp] = kc; red[1][warp] = vc; }
+    // outliers per kv head: the 32 channels of a warp's pass lie in one head
+    __shared__ uint32_t hk[64], hv[64];
+    for (int h = threadIdx.x; h < cfg.Hkv; h += blockDim.x) hk[h] = hv[h] = 0u;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t sk = 0, sv = 0;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) { sk += red[0][w]; sv += red[1][w]; }
-        ws.kcnt[(size_t)b * n_new + i] = sk;
-        ws.vcnt[(size_t)b * n_new + i] = sv;
+    const uint16_t* kt = c.kthr + (size_t)b * n * 2;
+    for (int base = 0; base < n; base += blockDim.x) {
+        const int j = base + threadIdx.x;
+        bool fk = false, fv = false;
+        if (j < n) {
+            const float xv = h2f(vrow[j]);
+            fv = xv < vlo || xv > vhi;
+            const float xk = h2f(krow[j]);
+            fk = xk < h2f(kt[2 * j]) || xk > h2f(kt[2 * j + 1]);
+        }
+        const uint32_t bk = __ballot_sync(0xffffffffu, fk), bv = __ballot_sync(0xffffffffu, fv);
+        if ((threadIdx.x & 31) == 0 && j < n) {
+            if (bk) atomicAdd(&hk[j >> 7], (uint32_t)__popc(bk));
+            if (bv) atomicAdd(&hv[j >> 7], (uint32_t)__popc(bv));
+        }
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < cfg.Hkv; h += blockDim.x) {
+        const size_t li = ((size_t)b * cfg.Hkv + h) * n_new + i;
+        ws.kcnt[li] = hk[h];
+        ws.vcnt[li] = hv[h];
     }
 }
 
@@ -328,14 +333,14 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_stats(kvq_cfg cfg, kvq_cach
 constexpr int kScanThreads = 1024;
 constexpr int kScanItems = 4;
 
-__device__ void scan_list(int b, int nt, int t0, int n_new, const uint32_t* cnt, uint32_t* off,
+__device__ void scan_list(int li, int nt, int t0, int n_new, const uint32_t* cnt, uint32_t* off,
                           uint32_t cap, uint32_t* count, uint32_t* chunk, int nch1,
                           int32_t* status) {
     __shared__ uint32_t sm[32];
     __shared__ unsigned long long s_acc;
-    const uint32_t* cb = cnt + (size_t)b * n_new;
-    uint32_t* ob = off + (size_t)b * n_new;
-    const uint32_t start = count[b];
+    const uint32_t* cb = cnt + (size_t)li * n_new;
+    uint32_t* ob = off + (size_t)li * n_new;
+    const uint32_t start = count[li];
     const unsigned long long room = cap >= start ? (unsigned long long)(cap - start) : 0ull;
     if (threadIdx.x == 0) s_acc = 0;
     unsigned long long running = 0;
@@ -374,48 +379,59 @@ __device__ void scan_list(int b, int nt, int t0, int n_new, const uint32_t* cnt,
         const int t = t0 + i;
         if (((t % kChunk) == kChunk - 1) || i == nt - 1) {
             const unsigned long long v = incl < acc ? incl : acc;
-            chunk[(size_t)b * nch1 + t / kChunk + 1] = start + (uint32_t)v;
+            chunk[(size_t)li * nch1 + t / kChunk + 1] = start + (uint32_t)v;
         }
         ob[i] = ok ? start + (uint32_t)ex : 0xffffffffu;
     }
     if (threadIdx.x == 0) {
-        count[b] = start + (uint32_t)acc;
+        count[li] = start + (uint32_t)acc;
         if (acc < running) set_status(status, KVQ_STATUS_OUTLIER_OVERFLOW);
     }
     __syncthreads();
 }
 
+// One block per outlier list (sequence b, kv head h).
 __global__ void __launch_bounds__(kScanThreads) k_tok_scan(kvq_cfg cfg, kvq_cache c, int n_new,
                                                            QuantWs ws) {
-    const int b = blockIdx.x;
+    const int li = blockIdx.x, b = li / cfg.Hkv;
     const int nt = ws.ntok[b], t0 = ws.t0[b];
     const int nch1 = nchunks(cfg.T_max) + 1;
-    scan_list(b, nt, t0, n_new, ws.kcnt, ws.koff, (uint32_t)cfg.out_cap_k, c.kcount, c.kchunk,
+    scan_list(li, nt, t0, n_new, ws.kcnt, ws.koff, (uint32_t)cfg.out_cap_k, c.kcount, c.kchunk,
               nch1, c.status);
-    scan_list(b, nt, t0, n_new, ws.vcnt, ws.voff, (uint32_t)cfg.out_cap_v, c.vcount, c.vchunk,
+    scan_list(li, nt, t0, n_new, ws.vcnt, ws.voff, (uint32_t)cfg.out_cap_v, c.vcount, c.vchunk,
               nch1, c.status);
-    if (threadIdx.x == 0 && nt > 0) c.len[b] = t0 + nt;
+    if (threadIdx.x == 0 && nt > 0 && li % cfg.Hkv == 0) c.len[b] = t0 + nt;
 }
 
 // ---------------------------------------------------------------------------------
 // Per token quad (4u .. 4u+3): encode the tokens of this call in it, write their outliers,
 // then the quad's key and value blocks (whole when the call starts at token 4u, else only
 // the fields of this call's tokens merged into the existing block).
-__device__ void compact_outliers(int n, const uint8_t* flag, const uint16_t* x, uint32_t first,
-                                 uint32_t tloc, uint32_t* pos, uint16_t* val, uint32_t* sm) {
-    const int per = (n + blockDim.x - 1) / blockDim.x;
-    const int j0 = threadIdx.x * per;
-    uint32_t cnt = 0;
-    for (int j = j0; j < j0 + per && j < n; ++j) cnt += flag[j];
-    uint32_t total;
-    uint32_t r = block_excl_scan(cnt, sm, &total);
-    if (first == 0xffffffffu) return;
-    for (int j = j0; j < j0 + per && j < n; ++j) {
-        if (flag[j]) {
-            pos[first + r] = (tloc << 16) | (uint32_t)j;
-            val[first + r] = x[j];
-            ++r;
+// Outliers of one token into the lists of its kv heads: flag/x over the n = Hkv*128 channels,
+// first[h] = the token's first entry in list h (0xffffffff: dropped by the capacity rule);
+// an entry is (fp16 bits << 16) | (tloc << 7) | c.  A 256-thread pass covers two heads, the
+// 32 channels of a warp one quarter of a head.
+__device__ void compact_outliers(int n, const uint8_t* flag, const uint16_t* x,
+                                 const uint32_t* first, size_t first_stride, uint32_t tloc,
+                                 uint32_t* out, size_t cap, uint32_t* sm) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int base = 0; base < n; base += blockDim.x) {
+        const int j = base + threadIdx.x;
+        const bool f = j < n && flag[j];
+        const uint32_t bal = __ballot_sync(0xffffffffu, f);
+        if (lane == 0) sm[warp] = __popc(bal);
+        __syncthreads();
+        if (f) {
+            const int h = j >> 7;
+            const uint32_t f0 = first[(size_t)h * first_stride];
+            if (f0 != 0xffffffffu) {
+                uint32_t r = __popc(bal & ((1u << lane) - 1u));
+                for (int w2 = warp & ~3; w2 < warp; ++w2) r += sm[w2];
+                out[(size_t)h * cap + f0 + r] =
+                    ((uint32_t)x[j] << 16) | (tloc << 7) | (uint32_t)(j & 127);
+            }
         }
+        __syncthreads();
     }
 }
 
@@ -491,26 +507,25 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cach
         }
         __syncthreads();
         const uint32_t tloc = (uint32_t)(t % kChunk);
-        compact_outliers(n, kf, krow, ws.koff[(size_t)b * n_new + i], tloc,
-                         c.kout_pos + (size_t)b * cfg.out_cap_k,
-                         c.kout_val + (size_t)b * cfg.out_cap_k, sm);
-        __syncthreads();
-        compact_outliers(n, vf, vrow, ws.voff[(size_t)b * n_new + i], tloc,
-                         c.vout_pos + (size_t)b * cfg.out_cap_v,
-                         c.vout_val + (size_t)b * cfg.out_cap_v, sm);
-        __syncthreads();
+        const size_t li0 = (size_t)b * cfg.Hkv * n_new + i;  // list (b, 0), token i
+        compact_outliers(n, kf, krow, ws.koff + li0, (size_t)n_new, tloc,
+                         c.kout + (size_t)b * cfg.Hkv * cfg.out_cap_k, (size_t)cfg.out_cap_k, sm);
+        compact_outliers(n, vf, vrow, ws.voff + li0, (size_t)n_new, tloc,
+                         c.vout + (size_t)b * cfg.Hkv * cfg.out_cap_v, (size_t)cfg.out_cap_v, sm);
     }
     // key and value blocks of quad u
     uint32_t present = 0;
     for (int t = ta; t <= tb; ++t) present |= 1u << (t & 3);
     const bool fresh = (ta == 4 * u);
-    const size_t base = ((size_t)b * nquads(cfg.T_max) + u) * cfg.Hkv * BW;
+    const size_t NQ = nquads(cfg.T_max);
     for (int wi = threadIdx.x; wi < 2 * cfg.Hkv * BW; wi += blockDim.x) {
         const int which = wi >= cfg.Hkv * BW;
         const int wv = wi - which * cfg.Hkv * BW;
+        const int h = wv / BW;
         uint32_t m;
-        const uint32_t word = block_word(which ? vc : kc, n, wv / BW, bits, wv % BW, present, &m);
-        uint32_t* dst = (which ? c.vcodes : c.kcodes) + base + wv;
+        const uint32_t word = block_word(which ? vc : kc, n, h, bits, wv % BW, present, &m);
+        uint32_t* dst = (which ? c.vcodes : c.kcodes) + (((size_t)b * cfg.Hkv + h) * NQ + u) * BW +
+                        wv % BW;
         *dst = fresh ? word : ((*dst & ~m) | word);
     }
 }
@@ -578,7 +593,7 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
     }
     dim3 gt(n_new, C.B);
     k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
-    k_tok_scan<<<C.B, kScanThreads, 0, st>>>(C, K, n_new, ws);
+    k_tok_scan<<<C.B * C.Hkv, kScanThreads, 0, st>>>(C, K, n_new, ws);
     dim3 gw((n_new + 2) / 4 + 1, C.B);
     k_tok_write<<<gw, kTokThreads, 10 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
     return record_cuda(cudaGetLastError());
@@ -636,7 +651,7 @@ extern "C" int kvq_quantize_append_noalloc(const kvq_cfg* cfg, const kvq_cache* 
     k_begin<<<(C.B + 127) / 128, 128, 0, st>>>(C, K, plen, n_new, 0, ws);
     dim3 gt(n_new, C.B);
     k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
-    k_tok_scan<<<C.B, kScanThreads, 0, st>>>(C, K, n_new, ws);
+    k_tok_scan<<<C.B * C.Hkv, kScanThreads, 0, st>>>(C, K, n_new, ws);
     dim3 gw((n_new + 2) / 4 + 1, C.B);
     k_tok_write<<<gw, kTokThreads, 10 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
     return record_cuda(cudaGetLastError());

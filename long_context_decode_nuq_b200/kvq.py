@@ -24,7 +24,8 @@ NOALLOC_SCRATCH_BYTES = 1 << 20  # KVQ_NOALLOC_SCRATCH_BYTES
 
 EXPORTS = (
     "kvq_abi_version", "kvq_strerror", "kvq_validate_cfg", "kvq_layout", "kvq_cache_reset",
-    "kvq_quantize_workspace", "kvq_quantize_append", "kvq_decode_qk", "kvq_decode_splits",
+    "kvq_quantize_workspace", "kvq_quantize_append", "kvq_decode_qk", "kvq_decode_qk_workspace",
+    "kvq_decode_splits",
     "kvq_softmax_merge", "kvq_decode_pv", "kvq_decode_workspace", "kvq_decode_attention",
     "kvq_dequantize", "kvq_fp16_decode_attention", "kvq_fit_workspace", "kvq_fit_codebook",
     "kvq_get_status", "kvq_quantize_append_noalloc",
@@ -44,8 +45,8 @@ class Cfg(ctypes.Structure):
                 ("out_cap_v", c_int32), ("outlier_frac", c_double), ("rope_theta", c_double)]
 
 
-_CACHE_FIELDS = ("kcodes", "vcodes", "kthr", "kparams", "vparams", "kout_pos", "kout_val",
-                 "vout_pos", "vout_val", "kchunk", "vchunk", "kcount", "vcount", "len", "status")
+_CACHE_FIELDS = ("kcodes", "vcodes", "kthr", "kparams", "vparams", "kout", "vout", "kchunk",
+                 "vchunk", "kcount", "vcount", "len", "status")
 
 
 class CacheStruct(ctypes.Structure):
@@ -84,7 +85,8 @@ def load():
                                  POINTER(CodebookStruct), P, P, c_int32, P, c_int32, P, c_size_t,
                                  P], c_int),
         "kvq_decode_qk": ([POINTER(Cfg), POINTER(CacheStruct), POINTER(CodebookStruct), P, P,
-                           c_int32, P, P, c_int32, P], c_int),
+                           c_int32, P, P, c_int32, P, c_size_t, P], c_int),
+        "kvq_decode_qk_workspace": ([POINTER(Cfg), c_int32, POINTER(c_size_t)], c_int),
         "kvq_decode_splits": ([POINTER(Cfg), c_int32], c_int),
         "kvq_softmax_merge": ([POINTER(Cfg), P, c_int32, P, P], c_int),
         "kvq_decode_pv": ([POINTER(Cfg), POINTER(CacheStruct), POINTER(CodebookStruct), P, P,
@@ -160,19 +162,18 @@ class Cache:
         nch = (cfg.T_max + CHUNK - 1) // CHUNK + 1
         dev = torch.device(device)
         i32, f32, f16 = torch.int32, torch.float32, torch.float16
-        self.kcodes = torch.zeros((cfg.B, nq, cfg.Hkv, BW), dtype=i32, device=dev)
-        self.vcodes = torch.zeros((cfg.B, nq, cfg.Hkv, BW), dtype=i32, device=dev)
+        self.kcodes = torch.zeros((cfg.B, cfg.Hkv, nq, BW), dtype=i32, device=dev)
+        self.vcodes = torch.zeros((cfg.B, cfg.Hkv, nq, BW), dtype=i32, device=dev)
         self.kthr = torch.zeros((cfg.B, n, 2), dtype=f16, device=dev)
         self.kparams = torch.zeros((cfg.B, n, 2), dtype=f32, device=dev)
         self.vparams = torch.zeros((cfg.B, cfg.T_max, 2), dtype=f32, device=dev)
-        self.kout_pos = torch.zeros((cfg.B, max(cfg.out_cap_k, 4)), dtype=i32, device=dev)
-        self.kout_val = torch.zeros((cfg.B, max(cfg.out_cap_k, 8)), dtype=f16, device=dev)
-        self.vout_pos = torch.zeros((cfg.B, max(cfg.out_cap_v, 4)), dtype=i32, device=dev)
-        self.vout_val = torch.zeros((cfg.B, max(cfg.out_cap_v, 8)), dtype=f16, device=dev)
-        self.kchunk = torch.zeros((cfg.B, nch), dtype=i32, device=dev)
-        self.vchunk = torch.zeros((cfg.B, nch), dtype=i32, device=dev)
-        self.kcount = torch.zeros((cfg.B,), dtype=i32, device=dev)
-        self.vcount = torch.zeros((cfg.B,), dtype=i32, device=dev)
+        H = cfg.Hkv  # one outlier list per (sequence, kv head)
+        self.kout = torch.zeros((cfg.B, H, max(cfg.out_cap_k, 8)), dtype=i32, device=dev)
+        self.vout = torch.zeros((cfg.B, H, max(cfg.out_cap_v, 8)), dtype=i32, device=dev)
+        self.kchunk = torch.zeros((cfg.B, H, nch), dtype=i32, device=dev)
+        self.vchunk = torch.zeros((cfg.B, H, nch), dtype=i32, device=dev)
+        self.kcount = torch.zeros((cfg.B, H), dtype=i32, device=dev)
+        self.vcount = torch.zeros((cfg.B, H), dtype=i32, device=dev)
         self.len = torch.zeros((cfg.B,), dtype=i32, device=dev)
         self.status = torch.zeros((4,), dtype=i32, device=dev)
         for f in _CACHE_FIELDS:
@@ -218,11 +219,19 @@ def kvq_decode_splits(cfg: Cfg, max_len: int) -> int:
     return load().kvq_decode_splits(ctypes.byref(cfg), max_len)
 
 
+def kvq_decode_qk_workspace(cfg: Cfg, max_len: int) -> int:
+    n = c_size_t()
+    _check(load().kvq_decode_qk_workspace(ctypes.byref(cfg), max_len, ctypes.byref(n)),
+           "kvq_decode_qk_workspace")
+    return n.value
+
+
 def kvq_decode_qk(cache: Cache, cbK: Codebook, q, qpos, max_len: int, logits, stats, splits: int,
-                  stream=None) -> None:
+                  workspace, stream=None) -> None:
     _check(load().kvq_decode_qk(ctypes.byref(cache.cfg), ctypes.byref(cache.struct),
                                 ctypes.byref(cbK.struct), _ptr(q), _ptr(qpos), max_len,
-                                _ptr(logits), _ptr(stats), splits, _stream(stream)),
+                                _ptr(logits), _ptr(stats), splits, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream)),
            "kvq_decode_qk")
 
 

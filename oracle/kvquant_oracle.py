@@ -284,14 +284,16 @@ def unpack_block(words, bits):
 class QuantizedCache:
     """Mirror of the device cache arrays, filled by the oracle's quantizer.
 
-    Outlier lists (one for keys, one for values, per sequence) hold entries
-    sorted by (token, flat channel j = h*D + c); an entry's position word is
-    ((t % 64) << 16) | j and its value the fp16 bits of the outlier.
-    chunk_ptr[m] .. chunk_ptr[m+1] delimit the entries of tokens
-    [64m, 64m + 64).  Overflow rule: within one call, token t's outliers are
-    stored iff the count at the start of the call plus the outliers of the
-    call's tokens up to and including t fit the capacity; otherwise they are
-    dropped and the sticky status bit STATUS_OUTLIER_OVERFLOW is set.
+    Code blocks are stored head-major: kcodes[b, h, u] is the block of token quad u
+    of kv head h.  Outliers are kept in one list per (sequence, kv head) for keys
+    and one for values.  A list holds entries sorted by (token, channel c of the
+    head); an entry is the word (fp16 bits << 16) | ((t % 64) << 7) | c.
+    chunk_ptr[b, h, m] .. chunk_ptr[b, h, m+1] delimit the entries of
+    tokens [64m, 64m + 64).  Overflow rule, per list: within one call, token t's
+    outliers in head h are stored iff the list's count at the start of the call
+    plus the call's outliers in head h up to and including token t fit the
+    capacity; otherwise they are dropped and the sticky status bit
+    STATUS_OUTLIER_OVERFLOW is set.
     """
 
     def __init__(self, B, Hkv, bits, T_max, f, cap_k, cap_v, D=128):
@@ -300,16 +302,15 @@ class QuantizedCache:
         self.n = Hkv * D
         self.nchunk = (T_max + CHUNK - 1) // CHUNK
         nq = (T_max + 3) // 4
-        self.kcodes = np.zeros((B, nq, Hkv, block_words(bits, D)), dtype=np.uint32)
-        self.vcodes = np.zeros((B, nq, Hkv, block_words(bits, D)), dtype=np.uint32)
+        self.kcodes = np.zeros((B, Hkv, nq, block_words(bits, D)), dtype=np.uint32)
+        self.vcodes = np.zeros((B, Hkv, nq, block_words(bits, D)), dtype=np.uint32)
         self.kthr = np.zeros((B, self.n, 2), dtype=np.uint16)
         self.kparams = np.zeros((B, self.n, 2), dtype=np.float32)
         self.vparams = np.zeros((B, T_max, 2), dtype=np.float32)
         self.cap = {"k": cap_k, "v": cap_v}
-        self.out_pos = {s: np.zeros((B, cap), dtype=np.uint32) for s, cap in self.cap.items()}
-        self.out_val = {s: np.zeros((B, cap), dtype=np.uint16) for s, cap in self.cap.items()}
-        self.out_count = {s: np.zeros(B, dtype=np.uint32) for s in self.cap}
-        self.chunk_ptr = {s: np.zeros((B, self.nchunk + 1), dtype=np.uint32) for s in self.cap}
+        self.out = {s: np.zeros((B, Hkv, cap), dtype=np.uint32) for s, cap in self.cap.items()}
+        self.out_count = {s: np.zeros((B, Hkv), dtype=np.uint32) for s in self.cap}
+        self.chunk_ptr = {s: np.zeros((B, Hkv, self.nchunk + 1), dtype=np.uint32) for s in self.cap}
         self.len = np.zeros(B, dtype=np.int32)
         self.status = 0
         # unpacked codes, kept for the dequantizer
@@ -361,24 +362,27 @@ class QuantizedCache:
             for arr, cc in ((self.kcodes, self.kc), (self.vcodes, self.vc)):
                 quad = [cc[b, 4 * u + j].reshape(self.Hkv, self.D) if 4 * u + j < self.T_max
                         else zero for j in range(4)]
-                arr[b, u] = pack_block(quad, self.bits)
+                arr[b, :, u] = pack_block(quad, self.bits)
+        D = self.D
         for s, mask, X in (("k", kout, K), ("v", vout, V)):
-            per_tok = mask.sum(axis=1)
-            start = int(self.out_count[s][b])
-            incl = start + np.cumsum(per_tok)
-            ok = incl <= self.cap[s]
-            if not ok.all():
-                self.status |= STATUS_OUTLIER_OVERFLOW
-            cnt = start
-            for i in range(ntok):
-                if ok[i] and per_tok[i]:
-                    j = np.nonzero(mask[i])[0].astype(np.uint32)
-                    self.out_pos[s][b, cnt:cnt + j.size] = (
-                        (np.uint32(ts[i] % CHUNK) << np.uint32(16)) | j)
-                    self.out_val[s][b, cnt:cnt + j.size] = X[i, j].view(np.uint16)
-                    cnt += j.size
-                self.chunk_ptr[s][b, ts[i] // CHUNK + 1] = cnt
-            self.out_count[s][b] = cnt
+            for h in range(self.Hkv):
+                mh = mask[:, h * D:(h + 1) * D]
+                per_tok = mh.sum(axis=1)
+                start = int(self.out_count[s][b, h])
+                incl = start + np.cumsum(per_tok)
+                ok = incl <= self.cap[s]
+                if not ok.all():
+                    self.status |= STATUS_OUTLIER_OVERFLOW
+                cnt = start
+                for i in range(ntok):
+                    if ok[i] and per_tok[i]:
+                        ch = np.nonzero(mh[i])[0].astype(np.uint32)
+                        xb = X[i, h * D + ch].view(np.uint16).astype(np.uint32)
+                        self.out[s][b, h, cnt:cnt + ch.size] = (
+                            (xb << np.uint32(16)) | (np.uint32(ts[i] % CHUNK) << np.uint32(7)) | ch)
+                        cnt += ch.size
+                    self.chunk_ptr[s][b, h, ts[i] // CHUNK + 1] = cnt
+                self.out_count[s][b, h] = cnt
         if ntok:
             self.len[b] = max(int(self.len[b]), int(ts[-1]) + 1)
 
@@ -397,15 +401,17 @@ class QuantizedCache:
 
     # -- reconstruction (R5) ---------------------------------------------------------------
     def outlier_entries(self, s, b):
-        """List of (t, j, fp16 bits) of list s ('k' or 'v') of sequence b, in stored order."""
+        """List of (t, j = h*D + c, fp16 bits) of the lists s ('k' or 'v') of sequence b,
+        head by head in stored order."""
         out = []
-        cnt = int(self.out_count[s][b])
-        cp = self.chunk_ptr[s][b]
         nch = (int(self.len[b]) + CHUNK - 1) // CHUNK
-        for m in range(nch):
-            for i in range(int(cp[m]), min(int(cp[m + 1]), cnt)):
-                p = int(self.out_pos[s][b, i])
-                out.append((m * CHUNK + (p >> 16), p & 0xFFFF, int(self.out_val[s][b, i])))
+        for h in range(self.Hkv):
+            cnt = int(self.out_count[s][b, h])
+            cp = self.chunk_ptr[s][b, h]
+            for m in range(nch):
+                for i in range(int(cp[m]), min(int(cp[m + 1]), cnt)):
+                    e = int(self.out[s][b, h, i])
+                    out.append((m * CHUNK + ((e >> 7) & 63), h * self.D + (e & 127), e >> 16))
         return out
 
     def reconstruct(self, b, cbK, cbV):

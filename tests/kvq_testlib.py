@@ -68,8 +68,8 @@ def compare_cache(g, o, B, hard=True):
     for b in range(B):
         L = int(o.len[b])
         for name, n_rows in (("kcodes", (L + 3) // 4), ("vcodes", (L + 3) // 4)):
-            gv = u32(getattr(g, name)[b, :n_rows])
-            ov = getattr(o, name)[b, :n_rows]
+            gv = u32(getattr(g, name)[b, :, :n_rows])
+            ov = getattr(o, name)[b, :, :n_rows]
             if not np.array_equal(gv, ov):
                 bad = np.argwhere(gv != ov)
                 errs.append(f"{name}[b={b}] {len(bad)} words differ, first {bad[:3].tolist()}")
@@ -81,20 +81,18 @@ def compare_cache(g, o, B, hard=True):
         if not np.array_equal(g.vparams[b, :L].cpu().numpy(), o.vparams[b, :L]):
             errs.append(f"vparams[b={b}]")
         for s in ("k", "v"):
-            cnt = int(o.out_count[s][b])
-            gcnt = int(u32(getattr(g, f"{s}count"))[b])
-            if gcnt != cnt:
-                errs.append(f"{s}count[b={b}] {gcnt} vs {cnt}")
-                continue
-            if not np.array_equal(u32(getattr(g, f"{s}out_pos")[b, :cnt]), o.out_pos[s][b, :cnt]):
-                errs.append(f"{s}out_pos[b={b}]")
-            if not np.array_equal(u16(getattr(g, f"{s}out_val")[b, :cnt]), o.out_val[s][b, :cnt]):
-                errs.append(f"{s}out_val[b={b}]")
             nch = (L + 63) // 64
-            if not np.array_equal(u32(getattr(g, f"{s}chunk")[b, : nch + 1]),
-                                  o.chunk_ptr[s][b, : nch + 1]):
-                errs.append(f"{s}chunk[b={b}] {u32(getattr(g, f'{s}chunk')[b, :nch+1])[:8]} vs "
-                            f"{o.chunk_ptr[s][b, :nch+1][:8]}")
+            for h in range(o.Hkv):
+                cnt = int(o.out_count[s][b, h])
+                gcnt = int(u32(getattr(g, f"{s}count"))[b, h])
+                if gcnt != cnt:
+                    errs.append(f"{s}count[b={b},h={h}] {gcnt} vs {cnt}")
+                    continue
+                if not np.array_equal(u32(getattr(g, f"{s}out")[b, h, :cnt]), o.out[s][b, h, :cnt]):
+                    errs.append(f"{s}out[b={b},h={h}]")
+                gch = u32(getattr(g, f"{s}chunk")[b, h, : nch + 1])
+                if not np.array_equal(gch, o.chunk_ptr[s][b, h, : nch + 1]):
+                    errs.append(f"{s}chunk[b={b},h={h}] {gch[:8]} vs {o.chunk_ptr[s][b, h, :nch+1][:8]}")
     st = int(g.status.cpu().numpy()[0])
     if st != o.status:
         errs.append(f"status {st} vs {o.status}")

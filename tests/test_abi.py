@@ -28,30 +28,31 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_cfg_validation():
-    ok = K.make_cfg(1, 32, 32, 3, 4096, 0.01, 1e4, 100, 100)
+    ok = K.make_cfg(1, 32, 32, 3, 4096, 0.01, 1e4, 104, 104)
     assert K.kvq_validate_cfg(ok) == 0
     bad = [
         dict(bits=5), dict(bits=1), dict(D=64), dict(Hq=30), dict(B=0), dict(T_max=0),
-        dict(outlier_frac=1.5), dict(rope_theta=0.5), dict(out_cap_k=-1),
+        dict(outlier_frac=1.5), dict(rope_theta=0.5), dict(out_cap_k=-1), dict(out_cap_v=12),
     ]
     for kw in bad:
         args = dict(B=1, Hq=32, Hkv=32, bits=3, T_max=4096, outlier_frac=0.01, rope_theta=1e4,
-                    out_cap_k=100, out_cap_v=100, D=128)
+                    out_cap_k=104, out_cap_v=104, D=128)
         args.update(kw)
         assert K.kvq_validate_cfg(K.make_cfg(**args)) < 0, kw
     assert K.load().kvq_validate_cfg(None) == -1
 
 
 def test_layout_sizes():
-    cfg = K.make_cfg(2, 8, 4, 3, 1000, 0.01, 1e4, 50, 70)
+    cfg = K.make_cfg(2, 8, 4, 3, 1000, 0.01, 1e4, 48, 72)
     s = K.kvq_layout(cfg)
     assert s["kcodes"] == 2 * 1000 * 4 * 12 * 4 and s["vcodes"] == s["kcodes"]
     # code blocks hold four tokens: T_max is rounded up to a multiple of 4
-    s2 = K.kvq_layout(K.make_cfg(2, 8, 4, 3, 1001, 0.01, 1e4, 50, 70))
+    s2 = K.kvq_layout(K.make_cfg(2, 8, 4, 3, 1001, 0.01, 1e4, 48, 72))
     assert s2["kcodes"] == s2["vcodes"] == 2 * 251 * 4 * 48 * 4
     assert s["vparams"] == 2 * 1000 * 2 * 4
-    assert s["kout_pos"] == 2 * 50 * 4 and s["vout_val"] == 2 * 70 * 2
-    assert s["kchunk"] == 2 * (16 + 1) * 4
+    # one outlier list per (sequence, kv head)
+    assert s["kout"] == 2 * 4 * 48 * 4 and s["vout"] == 2 * 4 * 72 * 4
+    assert s["kchunk"] == 2 * 4 * (16 + 1) * 4 and s["kcount"] == 2 * 4 * 4
     assert K.kvq_quantize_workspace(cfg, 100, 1) > K.kvq_quantize_workspace(cfg, 100, 0)
     assert K.kvq_decode_splits(cfg, 1000) >= 1
 
@@ -67,7 +68,7 @@ def test_argument_errors_without_gpu():
                                  ctypes.byref(cb), null, null, 1, null, 0, null, 0, null)
     assert rc == -1
     # misaligned (never dereferenced) pointers are rejected
-    fake = K.CacheStruct(*([0x1000] * 15))
+    fake = K.CacheStruct(*([0x1000] * 13))
     fake.kcodes = 0x1001
     rc = lib.kvq_cache_reset(ctypes.byref(cfg), ctypes.byref(fake), null)
     assert rc == -2
@@ -78,7 +79,7 @@ def test_argument_errors_without_gpu():
     fake.kcodes = 0x1000
     cbf = K.CodebookStruct(0x1000, 0x1000)
     rc = lib.kvq_decode_qk(ctypes.byref(cfg), ctypes.byref(fake), ctypes.byref(cbf), 0x1000,
-                           0x1000, 100, 0x1000, 0x1000, 5000, null)
+                           0x1000, 100, 0x1000, 0x1000, 5000, 0x1000, 1 << 20, null)
     assert rc == -5
     # fit: too many samples
     assert lib.kvq_fit_workspace(5, 5000, ctypes.byref(ctypes.c_size_t())) == -3
@@ -97,7 +98,7 @@ def test_noalloc_append_argument_errors_without_gpu():
     # a request whose scratch exceeds the fixed array is refused before any device work
     big = K.make_cfg(64, 32, 32, 3, 8192, 0.01, 1e4, 64, 64)
     assert K.kvq_quantize_workspace(big, 4096, 0) > K.NOALLOC_SCRATCH_BYTES
-    fake = K.CacheStruct(*([0x1000] * 15))
+    fake = K.CacheStruct(*([0x1000] * 13))
     rc = lib.kvq_quantize_append_noalloc(ctypes.byref(big), ctypes.byref(fake), ctypes.byref(cb),
                                          ctypes.byref(cb), 0x1000, 0x1000, 4096, null, null)
     assert rc == -8

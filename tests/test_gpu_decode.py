@@ -85,7 +85,8 @@ def test_split_path(name, over, T, plen, appends, splits):
     ml = torch.empty((w.B, w.Hq, 2), device="cuda")
     out = torch.empty((w.B, w.Hq, w.D), device="cuda")
     part = torch.empty((w.B, w.Hq, S, w.D), device="cuda")
-    K.kvq_decode_qk(g, dK, dq, dpos, max_len, logits, stats, S)
+    qws = torch.empty(K.kvq_decode_qk_workspace(g.cfg, max_len), dtype=torch.uint8, device="cuda")
+    K.kvq_decode_qk(g, dK, dq, dpos, max_len, logits, stats, S, qws)
     K.kvq_softmax_merge(g.cfg, stats, S, ml)
     K.kvq_decode_pv(g, dV, logits, ml, max_len, out, part, S)
     torch.cuda.synchronize()
@@ -136,7 +137,7 @@ def test_fp16_comparison_kernel(name, over, T, plen):
     pl = np.array(plen if plen is not None else [T] * w.B, dtype=np.int32)
     q16 = synth.gen_q(w)
     qpos = pl.copy()
-    cfg = K.make_cfg(w.B, w.Hq, w.Hkv, w.bits, T, w.f, w.rope_theta, 1, 1)
+    cfg = K.make_cfg(w.B, w.Hq, w.Hkv, w.bits, T, w.f, w.rope_theta, 0, 0)
     ws = torch.empty(K.kvq_decode_workspace(cfg, T, 0), dtype=torch.uint8, device="cuda")
     out = torch.empty((w.B, w.Hq, w.D), device="cuda")
     K.kvq_fp16_decode_attention(cfg, torch.from_numpy(K16).cuda(), torch.from_numpy(V16).cuda(),

@@ -61,7 +61,7 @@ def test_append_bit_exact(name, over, T, plen):
 
 def test_outlier_capacity_overflow():
     w, K16, V16, cbK, cbV, o, g, dK, dV = _build("llama7b_layer_32k", dict(Hq=4, Hkv=4), 150,
-                                                  None, cap=700)
+                                                  None, cap=200)
     import long_context_decode_nuq_b200 as K
     assert o.status & O.STATUS_OUTLIER_OVERFLOW
     compare_cache(g, o, w.B)

@@ -262,7 +262,7 @@ def test_outliers_roundtrip_and_lie_outside():
     lo = c.kthr[0, :, 0].view(np.float16)
     hi = c.kthr[0, :, 1].view(np.float16)
     ent = c.outlier_entries("k", 0)
-    assert len(ent) == int(c.out_count["k"][0]) > 0
+    assert len(ent) == int(c.out_count["k"][0].sum()) > 0
     for t, j, bits in ent:
         x = K[0, t].reshape(-1)[j]
         assert x.view(np.uint16) == bits                       # stored fp16 unchanged
@@ -288,7 +288,7 @@ def test_outliers_roundtrip_and_lie_outside():
 def test_zero_outlier_fraction_stores_none():
     w = synth.workload("tiny_single_head", f=0.0)
     c, K, V, cbK, cbV = _small_cache(w, 200)
-    assert c.out_count["k"][0] == 0 and c.out_count["v"][0] == 0
+    assert c.out_count["k"][0].sum() == 0 and c.out_count["v"][0].sum() == 0
     lo = c.kthr[0, :, 0].view(np.float16)
     assert np.array_equal(lo, K[0, :200, 0].min(axis=0))
 
@@ -363,10 +363,11 @@ def test_append_reuses_key_calibration_and_chunks():
     assert np.array_equal(before, c.kparams)
     assert c.len[0] == T + 3
     # chunk pointers are monotone and end at the count
-    cp = c.chunk_ptr["k"][0]
     nch = (T + 3 + 63) // 64
-    assert np.all(np.diff(cp[: nch + 1].astype(np.int64)) >= 0)
-    assert cp[nch] == c.out_count["k"][0]
+    for h in range(w.Hkv):
+        cp = c.chunk_ptr["k"][0, h]
+        assert np.all(np.diff(cp[: nch + 1].astype(np.int64)) >= 0)
+        assert cp[nch] == c.out_count["k"][0, h]
     # appending token by token equals prefill-then-quantize of the same tokens
     c2 = O.QuantizedCache(w.B, w.Hkv, w.bits, T + 8, w.f, 1 << 20, 1 << 20)
     c2.calibrate_keys(0, K[0, :T])
@@ -375,21 +376,28 @@ def test_append_reuses_key_calibration_and_chunks():
     assert np.array_equal(c2.kcodes[0, :nq], c.kcodes[0, :nq])
     assert np.array_equal(c2.vcodes[0, :nq], c.vcodes[0, :nq])
     for s in ("k", "v"):
-        assert np.array_equal(c2.out_pos[s][0], c.out_pos[s][0])
-        assert np.array_equal(c2.chunk_ptr[s][0, : nch + 1], c.chunk_ptr[s][0, : nch + 1])
+        assert np.array_equal(c2.out[s][0], c.out[s][0])
+        assert np.array_equal(c2.chunk_ptr[s][0, :, : nch + 1], c.chunk_ptr[s][0, :, : nch + 1])
 
 
 def test_overflow_rule_prefix():
+    """Per (sequence, head) list: a token's outliers are kept iff the prefix fits."""
     w = synth.workload("llama7b_layer_32k", Hq=2, Hkv=2)
     T = 100
-    c, K, V, cbK, cbV = _small_cache(w, T, cap=300)
+    cap = 152
+    c, K, V, cbK, cbV = _small_cache(w, T, cap=cap)
     assert c.status & O.STATUS_OUTLIER_OVERFLOW
     full, _, _, _, _ = _small_cache(w, T)
-    per_tok = np.bincount([t for t, _, _ in full.outlier_entries("v", 0)], minlength=T)
-    stop = int(np.searchsorted(np.cumsum(per_tok), 300, side="right"))
-    assert c.out_count["v"][0] == per_tok[:stop].sum()
-    assert np.array_equal(c.out_pos["v"][0, : c.out_count["v"][0]],
-                          full.out_pos["v"][0, : c.out_count["v"][0]])
+    for s in ("k", "v"):
+        ent = full.outlier_entries(s, 0)
+        for h in range(w.Hkv):
+            per_tok = np.bincount([t for t, j, _ in ent if j // w.D == h], minlength=T)
+            stop = int(np.searchsorted(np.cumsum(per_tok), cap, side="right"))
+            n_kept = int(per_tok[:stop].sum())
+            assert c.out_count[s][0, h] == n_kept
+            assert np.array_equal(c.out[s][0, h, :n_kept], full.out[s][0, h, :n_kept])
+    # the cap binds on at least one list, and a list under the cap is unaffected
+    assert any(full.out_count[s][0, h] > cap for s in ("k", "v") for h in range(w.Hkv))
 
 
 # ---------------------------------------------------------------- RoPE (R9)

@@ -15,11 +15,11 @@ pytestmark = pytest.mark.gpu
 
 def _arrays(c, B):
     out = {}
-    for name in ("kcodes", "vcodes", "kparams", "vparams", "kout_pos", "vout_pos", "kchunk",
+    for name in ("kcodes", "vcodes", "kparams", "vparams", "kout", "vout", "kchunk",
                  "vchunk", "kcount", "vcount", "len", "status"):
         t = getattr(c, name)
         out[name] = t.cpu().numpy().copy()
-    for name in ("kthr", "kout_val", "vout_val"):
+    for name in ("kthr",):
         out[name] = u16(getattr(c, name)).copy()
     return out
 
