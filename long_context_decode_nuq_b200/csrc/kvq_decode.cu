@@ -149,8 +149,14 @@ __device__ __forceinline__ float zero_code_value(float off, float half, const fl
     return off + half * levels[encode(xn, bounds, nb)];
 }
 
-template <int HPC>
-__host__ __device__ constexpr int heads_per_warp() { return HPC == 4 ? 2 : HPC; }
+// Consumer warps of a CTA (one more warp streams the input) and heads per consumer warp.
+// With four query heads per CTA two warps share each quad pair (two heads each): twice the
+// warps to hide latency, at the price of computing a lane's RoPE phases for two heads instead
+// of four.
+__host__ __device__ constexpr int qk_warps(int hpc) { return hpc == 4 ? 16 : 8; }
+__host__ __device__ constexpr int pv_warps(int hpc) { return hpc == 4 ? 16 : 8; }
+template <int HPC, int CW>
+__host__ __device__ constexpr int heads_per_warp() { return HPC * 8 / CW; }
 template <int HW>
 __device__ __forceinline__ int out_head(int i) {
     return HW == 4 ? (i & 3) : (HW == 2 ? ((i >> 1) & 1) : 0);
@@ -160,9 +166,6 @@ __device__ __forceinline__ bool out_owner(int i) {
     return HW == 4 ? true : (HW == 2 ? !(i & 1) : !(i & 3));
 }
 
-// Consumer warps of a CTA: with four query heads per CTA two warps share a quad pair (two
-// heads each), so that a thread's accumulators stay small; one more warp streams the input.
-__host__ __device__ constexpr int consumer_warps(int hpc) { return hpc == 4 ? 16 : 8; }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -291,13 +294,13 @@ __global__ void k_decode_prep(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const u
 // reduce across the half-warp by halving.  The last warp streams the chunks and the chunk
 // base angles.
 template <int BITS, int HPC, bool SHARE>
-__global__ void __launch_bounds__(consumer_warps(HPC) * 32 + 32, 1)
+__global__ void __launch_bounds__(qk_warps(HPC) * 32 + 32, 1)
     k_qk(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ qr_all,
          const float2* __restrict__ thi, const float2* __restrict__ tlo, int Ls, int max_len,
          int kvb, float* __restrict__ logits) {
     using F = Fmt<BITS>;
-    constexpr int CW = consumer_warps(HPC), NC = CW * 32;
-    constexpr int HW = heads_per_warp<HPC>();
+    constexpr int CW = qk_warps(HPC), NC = CW * 32;
+    constexpr int HW = heads_per_warp<HPC, CW>();
     constexpr int LH = HPC == 4 ? 2 : (HPC == 2 ? 1 : 0);
     constexpr int P = 9 + LH;  // bit of the entry index in a table byte offset
     constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << P;
@@ -574,13 +577,13 @@ __global__ void __launch_bounds__(256) k_logit_stats(kvq_cfg cfg, const int32_t*
 // lane i computes the weight of (token i >> 2 of its quad, head out_head(i) of the warp).  The
 // last warp streams the chunks.
 template <int BITS, int HPC, bool SHARE>
-__global__ void __launch_bounds__(consumer_warps(HPC) * 32 + 32, 1)
+__global__ void __launch_bounds__(pv_warps(HPC) * 32 + 32, 1)
     k_pv(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
          const float2* __restrict__ ml, int Ls, int S, int max_len, int kvb,
          float* __restrict__ part) {
     using F = Fmt<BITS>;
-    constexpr int CW = consumer_warps(HPC), NC = CW * 32;
-    constexpr int HW = heads_per_warp<HPC>();
+    constexpr int CW = pv_warps(HPC), NC = CW * 32;
+    constexpr int HW = heads_per_warp<HPC, CW>();
     constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << 7;
     constexpr int NW = SHARE ? 1 : HW;
     extern __shared__ __align__(128) uint8_t sm[];
@@ -1101,7 +1104,7 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (ce) return record_cuda(ce);
     dim3 grid(S, cfg->B, cfg->Hq / hpc);
-    kern<<<grid, consumer_warps(hpc) * 32 + 32, smem, st>>>(*cfg, *cache, *cbK, T.qr, T.thi, T.tlo,
+    kern<<<grid, qk_warps(hpc) * 32 + 32, smem, st>>>(*cfg, *cache, *cbK, T.qr, T.thi, T.tlo,
                                                             Ls, max_len, kvb, logits);
     const int nch = (max_len + kChunk - 1) / kChunk;
     dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
@@ -1162,7 +1165,7 @@ static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     cudaError_t ce = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (ce) return record_cuda(ce);
     dim3 grid(S, cfg->B, cfg->Hq / hpc);
-    kern<<<grid, consumer_warps(hpc) * 32 + 32, smem, st>>>(*cfg, *cache, *cbV, logits,
+    kern<<<grid, pv_warps(hpc) * 32 + 32, smem, st>>>(*cfg, *cache, *cbV, logits,
                                                             (const float2*)ml, Ls, S, max_len,
                                                             kvb, part);
     k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
