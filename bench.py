@@ -51,6 +51,27 @@ def parse():
 
 # ----------------------------------------------------------------------------- helpers
 
+def rank_layer_key(layer: int, rank: int) -> int:
+    """Synthetic-data key of a layer on a rank: every rank holds a different sequence."""
+    return layer + 4096 * rank
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time; every rank calls this at the same point."""
+    if world == 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(tokens_per_rank: float, world: int, ms: float) -> float:
+    """Whole-job KV tokens/s: every rank processed tokens_per_rank in at most ms."""
+    return tokens_per_rank * world / (ms / 1e3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -255,8 +276,8 @@ def run_kvq(args, rank, world):
     kout_cap = ceil8(T_max * w.f * w.D * 1.25 + 4096)
     vout_cap = ceil8(T_max * 2 * math.floor(w.f * w.n / 2 + 0.5) / w.Hkv * 1.5 + 4096)
     cfg = K.make_cfg(w.B, w.Hq, w.Hkv, w.bits, T_max, w.f, w.rope_theta, kout_cap, vout_cap)
-    # a different synthetic sequence per rank (weak scaling): layer key offset by rank
-    layer_key = lambda l: l + 4096 * rank  # noqa: E731
+    # a different synthetic sequence per rank (weak scaling)
+    layer_key = lambda l: rank_layer_key(l, rank)  # noqa: E731
 
     # replicas of the whole cache so that the timed inputs exceed L2 by a wide margin
     one_cache_bytes = sum(K.kvq_layout(cfg).values()) * layers
@@ -383,16 +404,13 @@ def run_kvq(args, rank, world):
                 marks.append(layer_step(i, s, True))
         t_end.record()
         torch.cuda.synchronize()
-    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
         dist.barrier()
     n_layer_steps = len(marks)
     tok_per_layer_step = [T0 + s + 1 for s in range(args.warmup, steps_total) for _ in range(layers)]
     kv_tokens = w.B * sum(tok_per_layer_step) * world
-    value = kv_tokens / (elapsed_ms / 1e3)
+    value = aggregate_rate(w.B * sum(tok_per_layer_step), world, elapsed_ms)
     # per-kernel times
     t_app = sum(m[0].elapsed_time(m[1]) for m in marks)
     t_qk = sum(m[1].elapsed_time(m[2]) for m in marks)
@@ -429,6 +447,9 @@ def run_kvq(args, rank, world):
     torch.cuda.synchronize()
     e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     h2d = d2h = 0
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     e_s.record()
     for j in range(e2e_steps):
         s = args.warmup + j
@@ -451,9 +472,9 @@ def run_kvq(args, rank, world):
         d2h = h_out[:layers].numel() * 4
     e_e.record()
     torch.cuda.synchronize()
-    e2e_ms = e_s.elapsed_time(e_e)
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world, dev)
     e2e_tokens = w.B * sum(T0 + steps_total + j + 1 for j in range(e2e_steps)) * layers
-    e2e_value = e2e_tokens / (e2e_ms / 1e3) * world
+    e2e_value = aggregate_rate(e2e_tokens, world, e2e_ms)
 
     # ---- uncompressed fp16 comparison kernel on one layer (last staged K/V)
     fp16 = None

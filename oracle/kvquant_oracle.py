@@ -369,19 +369,21 @@ class QuantizedCache:
                 mh = mask[:, h * D:(h + 1) * D]
                 per_tok = mh.sum(axis=1)
                 start = int(self.out_count[s][b, h])
-                incl = start + np.cumsum(per_tok)
-                ok = incl <= self.cap[s]
+                # a token's outliers are kept iff the list's prefix up to it fits the capacity
+                ok = start + np.cumsum(per_tok) <= self.cap[s]
                 if not ok.all():
                     self.status |= STATUS_OUTLIER_OVERFLOW
-                cnt = start
-                for i in range(ntok):
-                    if ok[i] and per_tok[i]:
-                        ch = np.nonzero(mh[i])[0].astype(np.uint32)
-                        xb = X[i, h * D + ch].view(np.uint16).astype(np.uint32)
-                        self.out[s][b, h, cnt:cnt + ch.size] = (
-                            (xb << np.uint32(16)) | (np.uint32(ts[i] % CHUNK) << np.uint32(7)) | ch)
-                        cnt += ch.size
-                    self.chunk_ptr[s][b, h, ts[i] // CHUNK + 1] = cnt
+                kept = np.where(ok, per_tok, 0)
+                ti, ch = np.nonzero(mh & ok[:, None])          # (token, channel) order
+                cnt = start + int(kept.sum())
+                ent = ((X[ti, h * D + ch].view(np.uint16).astype(np.uint32) << np.uint32(16))
+                       | ((ts[ti] % CHUNK).astype(np.uint32) << np.uint32(7)) | ch.astype(np.uint32))
+                self.out[s][b, h, start:cnt] = ent
+                # chunk_ptr[m + 1] = entries up to and including the chunk's last token of the call
+                after = start + np.cumsum(kept)
+                m = ts // CHUNK
+                last = np.r_[m[1:] != m[:-1], True] if ntok else np.zeros(0, dtype=bool)
+                self.chunk_ptr[s][b, h, m[last] + 1] = after[last]
                 self.out_count[s][b, h] = cnt
         if ntok:
             self.len[b] = max(int(self.len[b]), int(ts[-1]) + 1)
