@@ -499,74 +499,118 @@ __global__ void __launch_bounds__(qk_warps(HPC) * 32 + 32, 1)
 }
 
 // ---------------------------------------------------------------------------------
-// Key outliers: logit(t, hq) += (x - zhat) * r, r the component of the rotated query that
-// meets the outlier's channel after the key is rotated to t.  A warp walks the entries of one
-// 64-token chunk of one (sequence, kv head) list.
-constexpr int kOutWarps = 8;      // warps per block of the outlier kernels
+// Outlier kernels.  A block takes kOutChunks 64-token chunks of one (sequence, kv head) list:
+// it stages their chunk pointers in shared memory, then its threads walk the entries of the
+// whole range flat, each finding its entry's chunk by a binary search over the staged pointers
+// (the entry itself holds only the token's offset within its chunk).  The per-entry gathers
+// are independent, so a thread has several in flight instead of one chunk's worth of
+// dependent loads after another.
+constexpr int kOutThreads = 256;  // threads per block of the outlier kernels
 constexpr int kOutChunks = 64;    // chunks per block
 
-__global__ void __launch_bounds__(kOutWarps * 32) k_key_outliers(
+struct OutRange {
+    uint32_t lo, hi;  // entries [lo, hi) of the block's chunks
+    int m0, n;        // first chunk and number of chunks
+};
+
+// Stages min(cp[m0 + j], cnt), j <= n, in cps; ends with a block barrier.
+__device__ __forceinline__ OutRange stage_chunks(const uint32_t* __restrict__ cp, uint32_t cnt,
+                                                 int len, uint32_t* cps) {
+    OutRange r;
+    r.m0 = blockIdx.x * kOutChunks;
+    r.n = max(0, min((len + kChunk - 1) / kChunk - r.m0, kOutChunks));
+    if (r.n)
+        for (int j = threadIdx.x; j <= r.n; j += blockDim.x) cps[j] = min(cp[r.m0 + j], cnt);
+    __syncthreads();
+    r.lo = r.n ? cps[0] : 0u;
+    r.hi = r.n ? cps[r.n] : 0u;
+    return r;
+}
+
+// Token of entry e with packed word w: the largest chunk j with cps[j] <= e holds it.
+__device__ __forceinline__ int entry_token(const OutRange& r, const uint32_t* cps, uint32_t e,
+                                           uint32_t w) {
+    int j = 0;
+#pragma unroll
+    for (int step = kOutChunks / 2; step; step >>= 1)
+        if (j + step < r.n && cps[j + step] <= e) j += step;
+    return (r.m0 + j) * kChunk + (int)((w >> 7) & 63u);
+}
+
+// Key outliers: logit(t, hq) += (x - zhat) * r, r the component of the rotated query that
+// meets the outlier's channel after the key is rotated to t.
+__global__ void __launch_bounds__(kOutThreads) k_key_outliers(
     kvq_cfg cfg, kvq_cache c, const float* __restrict__ qr, const float2* __restrict__ thi,
     const float2* __restrict__ tlo, const float* __restrict__ zk, int max_len,
     float* __restrict__ logits) {
     const int li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
     const int g = cfg.Hq / cfg.Hkv;
     const int len = min(c.len[b], max_len);
-    const int nch1 = nchunks(cfg.T_max) + 1;
-    const uint32_t* cp = c.kchunk + (size_t)li * nch1;
-    const uint32_t cnt = c.kcount[li];
+    const uint32_t* cp = c.kchunk + (size_t)li * (nchunks(cfg.T_max) + 1);
     const uint32_t* ent = c.kout + (size_t)li * cfg.out_cap_k;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int mend = min((len + kChunk - 1) / kChunk, (int)(blockIdx.x + 1) * kOutChunks);
-    for (int m = blockIdx.x * kOutChunks + warp; m < mend; m += kOutWarps) {
-        const uint32_t lo = min(cp[m], cnt), hi = min(cp[m + 1], cnt);
-        for (uint32_t e = lo + lane; e < hi; e += 32) {
-            const uint32_t w = ent[e];
-            const int t = m * kChunk + (int)((w >> 7) & 63u), ch = (int)(w & 127u);
-            if (t >= len) continue;
-            const int p = ch & 63;
-            const float2 cs = trig_at(thi, tlo, t, p);
-            const float d = h2f((uint16_t)(w >> 16)) - zk[(size_t)li * kD + ch];
-            for (int a = 0; a < g; ++a) {
-                const int hq = h * g + a;
-                const float* qv = qr + ((size_t)b * cfg.Hq + hq) * kD;
-                const float qa = qv[p], qb = qv[p + 64];
-                const float r = (ch < 64) ? (cs.x * qa + cs.y * qb) : (cs.x * qb - cs.y * qa);
-                atomicAdd(&logits[((size_t)b * cfg.Hq + hq) * cfg.T_max + t], d * r);
-            }
+    __shared__ uint32_t cps[kOutChunks + 1];
+    const OutRange r = stage_chunks(cp, c.kcount[li], len, cps);
+    for (uint32_t e = r.lo + threadIdx.x; e < r.hi; e += blockDim.x) {
+        const uint32_t w = ent[e];
+        const int t = entry_token(r, cps, e, w), ch = (int)(w & 127u);
+        if (t >= len) continue;
+        const int p = ch & 63;
+        const float2 cs = trig_at(thi, tlo, t, p);
+        const float d = h2f((uint16_t)(w >> 16)) - zk[(size_t)li * kD + ch];
+        for (int a = 0; a < g; ++a) {
+            const int hq = h * g + a;
+            const float* qv = qr + ((size_t)b * cfg.Hq + hq) * kD;
+            const float qa = qv[p], qb = qv[p + 64];
+            const float rr = (ch < 64) ? (cs.x * qa + cs.y * qb) : (cs.x * qb - cs.y * qa);
+            atomicAdd(&logits[((size_t)b * cfg.Hq + hq) * cfg.T_max + t], d * rr);
         }
     }
 }
 
 // ---------------------------------------------------------------------------------
-// Softmax statistics of each split from the (corrected) logits: stats = (m_s, l_s).
+// Softmax statistics of each split from the (corrected) logits: stats = (m_s, l_s), one pass
+// with a running (max, sum) per thread, merged across the block.
+__device__ __forceinline__ void online_add(float& m, float& l, float x) {
+    const float mn = fmaxf(m, x);
+    l = (m > -INFINITY ? l * __expf(m - mn) : 0.0f) + __expf(x - mn);
+    m = mn;
+}
+__device__ __forceinline__ void online_merge(float& m, float& l, float m2, float l2) {
+    const float mn = fmaxf(m, m2);
+    if (mn == -INFINITY) return;
+    l = (m > -INFINITY ? l * __expf(m - mn) : 0.0f) + (m2 > -INFINITY ? l2 * __expf(m2 - mn) : 0.0f);
+    m = mn;
+}
+
 __global__ void __launch_bounds__(256) k_logit_stats(kvq_cfg cfg, const int32_t* __restrict__ lens,
                                                      const float* __restrict__ logits, int Ls,
                                                      int S, int max_len, float2* __restrict__ stats) {
     const int s = blockIdx.x, bh = blockIdx.y, b = bh / cfg.Hq;
     const int len = min(lens[b], max_len);
-    const int t0 = s * Ls, t1 = min(len, t0 + Ls);
+    const int t0 = s * Ls, t1 = max(t0, min(len, t0 + Ls));  // empty split: t1 == t0
     const float* row = logits + (size_t)bh * cfg.T_max;
-    __shared__ float red[32];
-    float m = -INFINITY;
-    for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) m = fmaxf(m, row[t]);
+    float m = -INFINITY, l = 0.0f;
+    // t0 is a multiple of 64; whole float4s while the row's address allows, the rest singly
+    const bool vec = ((reinterpret_cast<uintptr_t>(row + t0) & 15u) == 0);
+    const int tv = vec ? t0 + ((t1 - t0) & ~3) : t0;
+    for (int t = t0 + 4 * (int)threadIdx.x; t < tv; t += 4 * blockDim.x) {
+        const float4 x = *reinterpret_cast<const float4*>(row + t);
+        online_add(m, l, x.x);
+        online_add(m, l, x.y);
+        online_add(m, l, x.z);
+        online_add(m, l, x.w);
+    }
+    for (int t = tv + threadIdx.x; t < t1; t += blockDim.x) online_add(m, l, row[t]);
 #pragma unroll
-    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
-    __syncthreads();
-    m = -INFINITY;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
-    __syncthreads();
-    float l = 0.0f;
-    if (m > -INFINITY)
-        for (int t = t0 + threadIdx.x; t < t1; t += blockDim.x) l += expf(row[t] - m);
-    l = warp_sum(l);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = l;
+    for (int o = 16; o; o >>= 1)
+        online_merge(m, l, __shfl_xor_sync(0xffffffffu, m, o), __shfl_xor_sync(0xffffffffu, l, o));
+    __shared__ float2 red[8];
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = make_float2(m, l);
     __syncthreads();
     if (threadIdx.x == 0) {
-        float a = 0.0f;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) a += red[w];
-        stats[(size_t)bh * S + s] = make_float2(m, a);
+        float M = -INFINITY, Lsum = 0.0f;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) online_merge(M, Lsum, red[w].x, red[w].y);
+        stats[(size_t)bh * S + s] = make_float2(M, Lsum);
     }
 }
 
@@ -778,46 +822,42 @@ __global__ void __launch_bounds__(pv_warps(HPC) * 32 + 32, 1)
 
 // ---------------------------------------------------------------------------------
 // Value outliers: out(hq, c) += p(t, hq) (x - zhat_t), p = exp(l - M) / L from the merged
-// statistics, zhat_t = off_t + half_t L[encode(normalize(0))].  A warp walks one chunk of one
-// (sequence, kv head) list; a block adds its sums to the output once.
-__global__ void __launch_bounds__(kOutWarps * 32) k_value_outliers(
+// statistics, zhat_t = off_t + half_t L[encode(normalize(0))]; sums gather in shared memory
+// and a block adds them to the output once.
+__global__ void __launch_bounds__(kOutThreads) k_value_outliers(
     kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
     const float2* __restrict__ ml, int max_len, float* __restrict__ out) {
     const int li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
     const int g = cfg.Hq / cfg.Hkv;
     const int len = min(c.len[b], max_len);
-    const int nch1 = nchunks(cfg.T_max) + 1;
-    const uint32_t* cp = c.vchunk + (size_t)li * nch1;
-    const uint32_t cnt = c.vcount[li];
+    const uint32_t* cp = c.vchunk + (size_t)li * (nchunks(cfg.T_max) + 1);
     const uint32_t* ent = c.vout + (size_t)li * cfg.out_cap_v;
     __shared__ float acc[kMaxG * kD];
     __shared__ float bnd[16];
+    __shared__ float2 mls[kMaxG];
+    __shared__ uint32_t cps[kOutChunks + 1];
     const int nb = (1 << cfg.bits) - 1;
     if (threadIdx.x < nb) bnd[threadIdx.x] = cb.bounds[threadIdx.x];
+    if (threadIdx.x < g) mls[threadIdx.x] = ml[(size_t)b * cfg.Hq + h * g + threadIdx.x];
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x) acc[e] = 0.0f;
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int mend = min((len + kChunk - 1) / kChunk, (int)(blockIdx.x + 1) * kOutChunks);
-    bool any = false;
-    for (int m = blockIdx.x * kOutChunks + warp; m < mend; m += kOutWarps) {
-        const uint32_t lo = min(cp[m], cnt), hi = min(cp[m + 1], cnt);
-        for (uint32_t e = lo + lane; e < hi; e += 32) {
-            const uint32_t w = ent[e];
-            const int t = m * kChunk + (int)((w >> 7) & 63u), ch = (int)(w & 127u);
-            if (t >= len) continue;
-            const float* vp = c.vparams + ((size_t)b * cfg.T_max + t) * 2;
-            const float d = h2f((uint16_t)(w >> 16)) - zero_code_value(vp[0], vp[1], cb.levels, bnd, nb);
-            for (int a = 0; a < g; ++a) {
-                const size_t bh = (size_t)b * cfg.Hq + h * g + a;
-                const float2 mLs = ml[bh];
-                const float p = mLs.y > 0.0f ? expf(logits[bh * cfg.T_max + t] - mLs.x) / mLs.y : 0.0f;
-                atomicAdd(&acc[a * kD + ch], p * d);
-            }
-            any = true;
+    const OutRange r = stage_chunks(cp, c.vcount[li], len, cps);  // barrier covers the above
+    if (r.lo >= r.hi) return;
+    const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
+    const float* lrow = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
+    for (uint32_t e = r.lo + threadIdx.x; e < r.hi; e += blockDim.x) {
+        const uint32_t w = ent[e];
+        const int t = entry_token(r, cps, e, w), ch = (int)(w & 127u);
+        if (t >= len) continue;
+        const float2 vp = vpar[t];
+        const float d = h2f((uint16_t)(w >> 16)) - zero_code_value(vp.x, vp.y, cb.levels, bnd, nb);
+        for (int a = 0; a < g; ++a) {
+            const float2 mL = mls[a];
+            if (mL.y > 0.0f)
+                atomicAdd(&acc[a * kD + ch],
+                          expf(lrow[(size_t)a * cfg.T_max + t] - mL.x) / mL.y * d);
         }
     }
-    any = __syncthreads_or(any);
-    if (!any) return;
+    __syncthreads();
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x) {
         const float v = acc[e];
         if (v != 0.0f) atomicAdd(&out[((size_t)b * cfg.Hq + h * g + e / kD) * kD + e % kD], v);
@@ -1108,7 +1148,7 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
                                                             Ls, max_len, kvb, logits);
     const int nch = (max_len + kChunk - 1) / kChunk;
     dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
-    k_key_outliers<<<go, kOutWarps * 32, 0, st>>>(*cfg, *cache, T.qr, T.thi, T.tlo, T.zk, max_len,
+    k_key_outliers<<<go, kOutThreads, 0, st>>>(*cfg, *cache, T.qr, T.thi, T.tlo, T.zk, max_len,
                                                    logits);
     dim3 gs(S, cfg->B * cfg->Hq);
     k_logit_stats<<<gs, 256, 0, st>>>(*cfg, cache->len, logits, Ls, S, max_len, (float2*)stats);
@@ -1171,7 +1211,7 @@ static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
     const int nch = (max_len + kChunk - 1) / kChunk;
     dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
-    k_value_outliers<<<go, kOutWarps * 32, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml,
+    k_value_outliers<<<go, kOutThreads, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml,
                                                      max_len, out);
     return record_cuda(cudaGetLastError());
 }

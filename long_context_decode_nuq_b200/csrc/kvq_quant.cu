@@ -252,7 +252,7 @@ __global__ void k_calib_select(kvq_cfg cfg, kvq_cache c, QuantWs ws, int pass) {
 
 // ---------------------------------------------------------------------------------
 // Per token: value thresholds over the whole row, value (off, half), outlier counts.
-constexpr int kTokThreads = 256;
+constexpr int kTokThreads = 512;
 
 __global__ void __launch_bounds__(kTokThreads) k_tok_stats(kvq_cfg cfg, kvq_cache c,
                                                            const uint16_t* __restrict__ k,
@@ -457,75 +457,70 @@ __device__ inline uint32_t block_word(const uint8_t* codes, int n, int h, int bi
     return word;
 }
 
-__global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cache c,
-                                                           kvq_codebook cbK, kvq_codebook cbV,
-                                                           const uint16_t* __restrict__ k,
-                                                           const uint16_t* __restrict__ v,
-                                                           int n_new, QuantWs ws) {
-    const int b = blockIdx.y;
+// One block per (token quad, sequence, kv head): the head's 128 channels of the quad's tokens.
+constexpr int kWrThreads = kD;
+
+__global__ void __launch_bounds__(kWrThreads) k_tok_write(kvq_cfg cfg, kvq_cache c,
+                                                         kvq_codebook cbK, kvq_codebook cbV,
+                                                         const uint16_t* __restrict__ k,
+                                                         const uint16_t* __restrict__ v,
+                                                         int n_new, QuantWs ws) {
+    const int b = blockIdx.y, h = blockIdx.z;
     const int nt = ws.ntok[b], t0 = ws.t0[b];
     if (nt == 0) return;
     const int u = t0 / 4 + blockIdx.x;
     const int ta = max(4 * u, t0), tb = min(4 * u + 3, t0 + nt - 1);
     if (ta > tb) return;
-    extern __shared__ uint8_t smem[];
-    const int n = cfg.Hkv * kD;
+    const int n = cfg.Hkv * kD, j = threadIdx.x, jn = h * kD + j;  // channel of the token row
     const int bits = cfg.bits, BW = block_words(bits), nbnd = (1 << bits) - 1;
-    uint8_t* kc = smem;            // [4][n] key codes of tokens 4u .. 4u+3 (0 when absent)
-    uint8_t* vc = kc + 4 * n;      // [4][n] value codes
-    uint8_t* kf = vc + 4 * n;      // [n] outlier flags of the current token
-    uint8_t* vf = kf + n;          // [n]
+    __shared__ uint8_t kc[4 * kD], vc[4 * kD];  // codes of tokens 4u .. 4u+3 (0 when absent)
+    __shared__ uint8_t kf[kD], vf[kD];          // outlier flags of the current token
     __shared__ float bK[16], bV[16];
     __shared__ uint32_t sm[32];
-    if (threadIdx.x < nbnd) {
-        bK[threadIdx.x] = cbK.bounds[threadIdx.x];
-        bV[threadIdx.x] = cbV.bounds[threadIdx.x];
+    if (j < nbnd) {
+        bK[j] = cbK.bounds[j];
+        bV[j] = cbV.bounds[j];
     }
-    for (int j = threadIdx.x; j < 8 * n; j += blockDim.x) kc[j] = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) kc[q * kD + j] = vc[q * kD + j] = 0;
     __syncthreads();
-    const uint16_t* kt = c.kthr + (size_t)b * n * 2;
-    const float* kp = c.kparams + (size_t)b * n * 2;
+    const uint16_t* kt = c.kthr + ((size_t)b * n + jn) * 2;
+    const float* kp = c.kparams + ((size_t)b * n + jn) * 2;
+    const float klo = h2f(kt[0]), khi = h2f(kt[1]), koff = kp[0], khalf = kp[1];
     for (int t = ta; t <= tb; ++t) {
         const int i = t - t0;
-        const uint16_t* vrow = v + ((size_t)b * n_new + i) * n;
-        const uint16_t* krow = k + ((size_t)b * n_new + i) * n;
+        const uint16_t* vrow = v + ((size_t)b * n_new + i) * n + h * kD;
+        const uint16_t* krow = k + ((size_t)b * n_new + i) * n + h * kD;
         const uint32_t vt = ws.vthr[(size_t)b * n_new + i];
         const float vlo = h2f((uint16_t)(vt & 0xffffu)), vhi = h2f((uint16_t)(vt >> 16));
         const float voff = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0];
         const float vhalf = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1];
-        uint8_t* kct = kc + (t & 3) * n;
-        uint8_t* vct = vc + (t & 3) * n;
-        for (int j = threadIdx.x; j < n; j += blockDim.x) {
-            const float xk = h2f(krow[j]);
-            const bool ok_ = xk < h2f(kt[2 * j]) || xk > h2f(kt[2 * j + 1]);
-            kf[j] = ok_;
-            kct[j] = (uint8_t)encode(normalize(ok_ ? 0.0f : xk, kp[2 * j], kp[2 * j + 1]), bK, nbnd);
-            const float xv = h2f(vrow[j]);
-            const bool ov = xv < vlo || xv > vhi;
-            vf[j] = ov;
-            vct[j] = (uint8_t)encode(normalize(ov ? 0.0f : xv, voff, vhalf), bV, nbnd);
-        }
+        const float xk = h2f(krow[j]);
+        const bool ok_ = xk < klo || xk > khi;
+        kf[j] = ok_;
+        kc[(t & 3) * kD + j] = (uint8_t)encode(normalize(ok_ ? 0.0f : xk, koff, khalf), bK, nbnd);
+        const float xv = h2f(vrow[j]);
+        const bool ov = xv < vlo || xv > vhi;
+        vf[j] = ov;
+        vc[(t & 3) * kD + j] = (uint8_t)encode(normalize(ov ? 0.0f : xv, voff, vhalf), bV, nbnd);
         __syncthreads();
         const uint32_t tloc = (uint32_t)(t % kChunk);
-        const size_t li0 = (size_t)b * cfg.Hkv * n_new + i;  // list (b, 0), token i
-        compact_outliers(n, kf, krow, ws.koff + li0, (size_t)n_new, tloc,
-                         c.kout + (size_t)b * cfg.Hkv * cfg.out_cap_k, (size_t)cfg.out_cap_k, sm);
-        compact_outliers(n, vf, vrow, ws.voff + li0, (size_t)n_new, tloc,
-                         c.vout + (size_t)b * cfg.Hkv * cfg.out_cap_v, (size_t)cfg.out_cap_v, sm);
+        const size_t li = ((size_t)b * cfg.Hkv + h) * n_new + i;  // list (b, h), token i
+        compact_outliers(kD, kf, krow, ws.koff + li, 0, tloc,
+                         c.kout + ((size_t)b * cfg.Hkv + h) * cfg.out_cap_k, 0, sm);
+        compact_outliers(kD, vf, vrow, ws.voff + li, 0, tloc,
+                         c.vout + ((size_t)b * cfg.Hkv + h) * cfg.out_cap_v, 0, sm);
     }
-    // key and value blocks of quad u
+    // the head's key and value blocks of quad u
     uint32_t present = 0;
     for (int t = ta; t <= tb; ++t) present |= 1u << (t & 3);
     const bool fresh = (ta == 4 * u);
-    const size_t NQ = nquads(cfg.T_max);
-    for (int wi = threadIdx.x; wi < 2 * cfg.Hkv * BW; wi += blockDim.x) {
-        const int which = wi >= cfg.Hkv * BW;
-        const int wv = wi - which * cfg.Hkv * BW;
-        const int h = wv / BW;
+    const size_t blk = (((size_t)b * cfg.Hkv + h) * nquads(cfg.T_max) + u) * BW;
+    for (int wi = j; wi < 2 * BW; wi += blockDim.x) {
+        const int which = wi >= BW, ww = wi - which * BW;
         uint32_t m;
-        const uint32_t word = block_word(which ? vc : kc, n, h, bits, wv % BW, present, &m);
-        uint32_t* dst = (which ? c.vcodes : c.kcodes) + (((size_t)b * cfg.Hkv + h) * NQ + u) * BW +
-                        wv % BW;
+        const uint32_t word = block_word(which ? vc : kc, kD, 0, bits, ww, present, &m);
+        uint32_t* dst = (which ? c.vcodes : c.kcodes) + blk + ww;
         *dst = fresh ? word : ((*dst & ~m) | word);
     }
 }
@@ -534,11 +529,6 @@ __global__ void __launch_bounds__(kTokThreads) k_tok_write(kvq_cfg cfg, kvq_cach
 
 using namespace kvq_host;
 
-// k_tok_write keeps the codes of a token quad in shared memory: 10 bytes per channel.
-static int tok_write_smem(int n) {
-    return record_cuda(cudaFuncSetAttribute(k_tok_write, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            10 * n));
-}
 
 extern "C" int kvq_quantize_workspace(const kvq_cfg* cfg, int32_t n_new, int32_t calibrate,
                                       size_t* bytes) {
@@ -570,7 +560,6 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
     cudaStream_t st = (cudaStream_t)stream;
     const kvq_cfg C = *cfg;
     const kvq_cache K = *cache;
-    if ((e = tok_write_smem(n))) return e;
     k_begin<<<(C.B + 127) / 128, 128, 0, st>>>(C, K, plen, n_new, calibrate, ws);
     if (calibrate) {
         cudaError_t ce;
@@ -594,8 +583,8 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
     dim3 gt(n_new, C.B);
     k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
     k_tok_scan<<<C.B * C.Hkv, kScanThreads, 0, st>>>(C, K, n_new, ws);
-    dim3 gw((n_new + 2) / 4 + 1, C.B);
-    k_tok_write<<<gw, kTokThreads, 10 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
+    dim3 gw((n_new + 2) / 4 + 1, C.B, C.Hkv);
+    k_tok_write<<<gw, kWrThreads, 0, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
     return record_cuda(cudaGetLastError());
 }
 
@@ -646,13 +635,11 @@ extern "C" int kvq_quantize_append_noalloc(const kvq_cfg* cfg, const kvq_cache* 
     cudaStream_t st = (cudaStream_t)stream;
     const kvq_cfg C = *cfg;
     const kvq_cache K = *cache;
-    const int n = C.Hkv * kD;
-    if ((e = tok_write_smem(n))) return e;
     k_begin<<<(C.B + 127) / 128, 128, 0, st>>>(C, K, plen, n_new, 0, ws);
     dim3 gt(n_new, C.B);
     k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
     k_tok_scan<<<C.B * C.Hkv, kScanThreads, 0, st>>>(C, K, n_new, ws);
-    dim3 gw((n_new + 2) / 4 + 1, C.B);
-    k_tok_write<<<gw, kTokThreads, 10 * n, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
+    dim3 gw((n_new + 2) / 4 + 1, C.B, C.Hkv);
+    k_tok_write<<<gw, kWrThreads, 0, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
     return record_cuda(cudaGetLastError());
 }
