@@ -109,6 +109,11 @@ __device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigne
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
     return d;
 }
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
 __device__ __forceinline__ float2 cmul(float2 a, float2 b) {
     return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
 }
@@ -490,6 +495,234 @@ __global__ void __launch_bounds__(qk_warps(HPC) * 32 + 32, 1)
             for (int m2 = 16 / V / 2; m2 >= 1; m2 >>= 1)
                 v[0] += __shfl_xor_sync(0xffffffffu, v[0], m2);
             const int t = t_begin + ch * kChunk + tq;
+            if (owner && t < t_end) lrow[t] = v[0];
+        }
+    }
+    __syncthreads();
+    // after an abandoned wait, copies of the last stages issued may still be in flight
+    if (*flag && tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1]);
+}
+
+// ---------------------------------------------------------------------------------
+// QK with the in-quad rotation folded into the tables (one query head per CTA, kv heads of
+// one query head each, codes of 2 or 3 bits).  With t = t_q + j, t_q the start of a token
+// quad and j < 4, the pair term is Re(e^{i t_q theta_p} e^{i j theta_p} Z_p(code)); the
+// table holds e^{i j theta_p} Z_p for each j, so a lane needs one phase per (quad, pair)
+// instead of one per (token, pair).  A stage carries 256 tokens (64 quads) of the head; a
+// consumer lane takes two quads and pairs i + 16 k; the reduction is the one of k_qk with
+// the two quads in place of the two heads of a warp.
+constexpr int kQQuads = 64;                  // token quads per stage
+constexpr int kQTokens = 4 * kQQuads;        // tokens per stage
+constexpr int kQWarps = 16;                  // consumer warps
+
+struct QQPlan {
+    int tab, ring, stage, base, lev, bar, flag, total;
+};
+__host__ __device__ inline QQPlan qq_plan(int bits) {
+    QQPlan p;
+    int o = 0;
+    p.tab = o;   o += 4 * (1 << (2 * bits)) * 64 * 8;        // [j][entry][pair] (X, Y)
+    p.stage = kQQuads * 16 * bits * 4;                       // code blocks of 64 quads
+    p.ring = o;  o += kStages * p.stage;
+    p.base = o;  o += kStages * 64 * 16;                     // [stage][pair] (c, c, s, s) at stage start
+    p.lev = o;   o += 16 * 4;                                // codebook levels
+    p.bar = o;   o += 2 * kStages * 8;
+    p.flag = o;  o += 16;
+    p.total = o;
+    return p;
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
+    k_qk_quad(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ qr_all,
+              const float2* __restrict__ thi, const float2* __restrict__ tlo, int Ls,
+              int max_len, float* __restrict__ logits) {
+    using F = Fmt<BITS>;
+    constexpr int NC = kQWarps * 32;
+    constexpr int P = 9;                         // entry bit of a table byte offset
+    constexpr int JS = P + F::FW;                // j bit of a table byte offset
+    constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << P;
+    extern __shared__ __align__(128) uint8_t sm[];
+    const QQPlan L = qq_plan(BITS);
+    uint8_t* tab = sm + L.tab;
+    uint8_t* ring = sm + L.ring;
+    float4* base = (float4*)(sm + L.base);
+    float* lev = (float*)(sm + L.lev);
+    uint64_t* full = (uint64_t*)(sm + L.bar);
+    uint64_t* empty = full + kStages;
+    int* flag = (int*)(sm + L.flag);
+
+    const int tid = threadIdx.x;
+    const int i = tid & 15, x = i >> 2, lane = tid & 31, warp = tid >> 5;
+    const int s = blockIdx.x, b = blockIdx.y, hq = blockIdx.z;
+    const int Hq = cfg.Hq, Hkv = cfg.Hkv, kvh = hq / (Hq / Hkv);
+    int len = c.len[b];
+    if (len > max_len) {
+        if (tid == 0 && s == 0 && hq == 0) set_status(c.status, KVQ_STATUS_LEN_OVERFLOW);
+        len = max_len;
+    }
+    const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
+    if (t_begin >= t_end) return;
+    const int nst = (t_end - t_begin + kQTokens - 1) / kQTokens;
+    if (tid == 0) {
+        for (int k = 0; k < kStages; ++k) {
+            mbar_init(full + k, 1);
+            mbar_init(empty + k, kQWarps);
+        }
+        flag[0] = 0;
+        flag[1] = 0;
+        fence_mbar_init();
+    }
+    // ---- tables: (X, Y) of Z_p(entry) turned by j theta_p.  Thread (p, r) of the first 512
+    // holds pair p's constants and writes entries r, r + 8, ... for every j.
+    if (tid < (1 << BITS)) lev[tid] = cb.levels[tid];
+    __syncthreads();
+    if (tid < 512) {
+        const int p = tid & 63, r0 = tid >> 6;
+        const float* kp = c.kparams + ((size_t)b * Hkv + kvh) * kD * 2;
+        const float* qv = qr_all + ((size_t)b * Hq + hq) * kD;
+        const float offa = kp[2 * p], halfa = kp[2 * p + 1];
+        const float offb = kp[2 * (p + 64)], halfb = kp[2 * (p + 64) + 1];
+        const float qa = qv[p], qb = qv[p + 64];
+        const float A1 = qa * halfa, B1 = qb * halfb, C1 = qa * offa + qb * offb;
+        const float A2 = qb * halfa, B2 = -qa * halfb, C2 = qb * offa - qa * offb;
+        float2 rj[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) rj[j] = tlo[j * 64 + p];
+        unsigned long long* t64 = reinterpret_cast<unsigned long long*>(tab);
+        for (int idx = r0; idx < F::NT; idx += 8) {
+            const float La = lev[idx & ((1 << BITS) - 1)], Lb = lev[idx >> BITS];
+            const float X = fmaf(B1, Lb, fmaf(A1, La, C1));
+            const float Y = fmaf(B2, Lb, fmaf(A2, La, C2));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                t64[(j * F::NT + idx) * 64 + p] =
+                    pk(fmaf(rj[j].x, X, rj[j].y * Y), fmaf(rj[j].x, Y, -rj[j].y * X));
+        }
+    }
+    __syncthreads();  // tables complete, barriers initialised
+
+    if (tid >= NC) {
+        // ================= streaming warp
+        const int pl = tid - NC;
+        const uint32_t* src = c.kcodes + ((size_t)b * Hkv + kvh) * nquads(cfg.T_max) * F::BW;
+        int cc = 0;
+        for (; cc < nst; ++cc) {
+            const int slot = cc % kStages;
+            if (cc >= kStages && !mbar_wait(empty + slot, (uint32_t)(cc / kStages - 1) & 1u)) {
+                if (pl == 0) {
+                    atomicOr(flag, 1);
+                    set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+                }
+                break;
+            }
+            if (*flag) break;
+            const int tc = t_begin + cc * kQTokens;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const float2 cs = trig_at(thi, tlo, tc, pl + 32 * u);
+                base[slot * 64 + pl + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
+            }
+            __syncwarp();
+            __threadfence_block();
+            if (pl == 0) {
+                fence_proxy_async();
+                const int q0 = tc >> 2, q1 = (min(tc + kQTokens, t_end) + 3) >> 2;
+                const uint32_t bytes = (uint32_t)(q1 - q0) * F::BW * 4;
+                mbar_arrive_expect_tx(full + slot, bytes);
+                bulk_load(ring + (size_t)slot * L.stage, src + (size_t)q0 * F::BW, bytes,
+                          full + slot);
+            }
+            __syncwarp();
+        }
+        if (pl == 0) flag[1] = cc;  // stages issued
+    } else {
+        // ================= consumer warps
+        const int uperm = (i >> 1) & 1;     // partial u of the lane holds quad u ^ uperm
+        const bool owner = !(i & 1);
+        // quads 4 warp + hh and 4 warp + hh + 2 (hh the half-warp): the code words of the two
+        // half-warps then sit 16 banks apart
+        const int qbase = 4 * warp + ((tid >> 4) & 1);
+        uint32_t lb[4], woff[2];
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl) lb[sl] = ((uint32_t)(sl ^ x) << JS) | ((uint32_t)i << 3);
+        // phase from the stage start to the quad, pair i + 16 k, as (c, s) and (-s, c)
+        unsigned long long RQ[2][4], RQp[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int q = qbase + 2 * (u ^ uperm);
+            woff[u] = (uint32_t)(q * F::BW + i * BITS) * 4;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 r = tlo[(4 * q) * 64 + i + 16 * k];
+                RQ[u][k] = pk(r.x, r.y);
+                RQp[u][k] = pk(-r.y, r.x);
+            }
+        }
+        const int tq = 4 * (qbase + 2 * uperm) + x;
+        float* lrow = logits + ((size_t)b * Hq + hq) * cfg.T_max;
+        for (int st = 0; st < nst; ++st) {
+            const int slot = st % kStages;
+            if (!mbar_wait(full + slot, (uint32_t)(st / kStages) & 1u)) {
+                atomicOr(flag, 1);
+                set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+            }
+            if (*flag) break;
+            const uint8_t* stage = ring + (size_t)slot * L.stage;
+            uint32_t w[2][BITS];
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int d = 0; d < BITS; ++d)
+                    w[u][d] = *reinterpret_cast<const uint32_t*>(stage + woff[u] + 4 * d);
+            unsigned long long Bc[4], Bs[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 bq = base[slot * 64 + i + 16 * k];
+                Bc[k] = pk(bq.x, bq.y);
+                Bs[k] = pk(bq.z, bq.w);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
+            unsigned long long acc[4][2];
+#pragma unroll
+            for (int sl = 0; sl < 4; ++sl) acc[sl][0] = acc[sl][1] = 0ull;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    // (c_b c_q - s_b s_q, c_b s_q + s_b c_q) in two packed instructions
+                    const unsigned long long Pc = fma2(Bc[k], RQ[u][k], mul2(Bs[k], RQp[u][k]));
+#pragma unroll
+                    for (int sl = 0; sl < 4; ++sl) {
+                        uint32_t fs;
+                        switch (4 * k + sl) {
+#define KVQ_FS(N) case N: fs = field_to<BITS, N, P>(w[u]); break;
+                            KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5)
+                            KVQ_FS(6) KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11)
+                            KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
+#undef KVQ_FS
+                        }
+                        acc[sl][u] = fma2(Pc, tld(tab + 128 * k, (fs & MASK) | lb[sl]), acc[sl][u]);
+                    }
+                }
+            }
+            float v[8];
+#pragma unroll
+            for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const f2 a = upk(acc[sl][u]);
+                    v[2 * sl + u] = a.x + a.y;
+                }
+            int mk = 8;
+#pragma unroll
+            for (int half = 4; half >= 1; half >>= 1, mk >>= 1)
+#pragma unroll
+                for (int t = 0; t < half; ++t)
+                    v[t] += __shfl_xor_sync(0xffffffffu, v[t + half], mk);
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
+            const int t = t_begin + st * kQTokens + tq;
             if (owner && t < t_end) lrow[t] = v[0];
         }
     }
@@ -1105,6 +1338,8 @@ static QKTables qk_tables(const kvq_cfg* cfg, int max_len, void* ws) {
 
 typedef void (*QKKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*,
                          const float2*, int, int, int, float*);
+typedef void (*QKQKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*,
+                          const float2*, int, int, float*);
 typedef void (*PVKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*, int, int,
                          int, int, float*);
 
@@ -1135,6 +1370,15 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
         k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi, T.qr,
                                                         T.thi, T.tlo, T.zk);
     }
+    if (cfg->bits <= 3 && cfg->Hq == cfg->Hkv) {
+        QKQKernel kq = cfg->bits == 2 ? k_qk_quad<2> : k_qk_quad<3>;
+        const int smem = qq_plan(cfg->bits).total;
+        cudaError_t ce = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (ce) return record_cuda(ce);
+        dim3 grid(S, cfg->B, cfg->Hq);
+        kq<<<grid, kQWarps * 32 + 32, smem, st>>>(*cfg, *cache, *cbK, T.qr, T.thi, T.tlo, Ls,
+                                                    max_len, logits);
+    } else {
     const int hpc = cfg->bits == 4 ? 1 : hpc_of(cfg);
     const int kvb = kvb_of(cfg, hpc);
     QKKernel kern = cfg->bits == 2 ? qk_kernel<2>(hpc, kvb == 1)
@@ -1146,6 +1390,7 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     dim3 grid(S, cfg->B, cfg->Hq / hpc);
     kern<<<grid, qk_warps(hpc) * 32 + 32, smem, st>>>(*cfg, *cache, *cbK, T.qr, T.thi, T.tlo,
                                                             Ls, max_len, kvb, logits);
+    }
     const int nch = (max_len + kChunk - 1) / kChunk;
     dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
     k_key_outliers<<<go, kOutThreads, 0, st>>>(*cfg, *cache, T.qr, T.thi, T.tlo, T.zk, max_len,
