@@ -732,14 +732,15 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 }
 
 // ---------------------------------------------------------------------------------
-// Outlier kernels.  A block takes kOutChunks 64-token chunks of one (sequence, kv head) list:
-// it stages their chunk pointers in shared memory, then its threads walk the entries of the
-// whole range flat, each finding its entry's chunk by a binary search over the staged pointers
-// (the entry itself holds only the token's offset within its chunk).  The per-entry gathers
-// are independent, so a thread has several in flight instead of one chunk's worth of
-// dependent loads after another.
+// Outlier kernels.  A block takes kOutChunks 64-token chunks of one (sequence, kv head) list
+// and stages their chunk pointers in shared memory; each warp walks a contiguous range of the
+// block's entries, 32 kOutBatch at a time.  An entry holds only its token's offset within its
+// chunk: a warp keeps the chunk of its current position and, per window, counts for each of
+// its entries the chunk boundaries that fall inside the window (about three per 128 entries
+// at the densities of interest).  A lane's kOutBatch entries are gathered together.
 constexpr int kOutThreads = 256;  // threads per block of the outlier kernels
 constexpr int kOutChunks = 64;    // chunks per block
+constexpr int kOutBatch = 4;      // entries a lane gathers at once
 
 struct OutRange {
     uint32_t lo, hi;  // entries [lo, hi) of the block's chunks
@@ -760,14 +761,41 @@ __device__ __forceinline__ OutRange stage_chunks(const uint32_t* __restrict__ cp
     return r;
 }
 
-// Token of entry e with packed word w: the largest chunk j with cps[j] <= e holds it.
-__device__ __forceinline__ int entry_token(const OutRange& r, const uint32_t* cps, uint32_t e,
-                                           uint32_t w) {
-    int j = 0;
+// Calls fn(t, w) per window: w[u] the packed entries of the lane, t[u] their tokens (-1 where
+// the lane has no entry).
+template <class Fn>
+__device__ __forceinline__ void walk_entries(const OutRange& r, const uint32_t* cps,
+                                             const uint32_t* __restrict__ ent, Fn&& fn) {
+    constexpr uint32_t W = 32 * kOutBatch;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const uint32_t span = ((r.hi - r.lo + nw - 1) / nw + 31) & ~31u;
+    const uint32_t Eb = r.lo + (uint32_t)warp * span, Ee = min(r.hi, Eb + span);
+    if (Eb >= Ee) return;
+    int cur = 0;  // chunk of entry Eb: the largest j < n with cps[j] <= Eb
 #pragma unroll
     for (int step = kOutChunks / 2; step; step >>= 1)
-        if (j + step < r.n && cps[j + step] <= e) j += step;
-    return (r.m0 + j) * kChunk + (int)((w >> 7) & 63u);
+        if (cur + step < r.n && cps[cur + step] <= Eb) cur += step;
+    for (uint32_t E = Eb; E < Ee; E += W) {
+        uint32_t e[kOutBatch], w[kOutBatch];
+        int j[kOutBatch];
+#pragma unroll
+        for (int u = 0; u < kOutBatch; ++u) {
+            e[u] = E + lane + 32 * u;
+            w[u] = e[u] < Ee ? ent[e[u]] : 0u;
+            j[u] = cur;
+        }
+        // boundaries inside the window (warp-uniform loop)
+        while (cur + 1 < r.n && cps[cur + 1] <= E + W - 1) {
+            const uint32_t bd = cps[++cur];
+#pragma unroll
+            for (int u = 0; u < kOutBatch; ++u) j[u] += e[u] >= bd;
+        }
+        int t[kOutBatch];
+#pragma unroll
+        for (int u = 0; u < kOutBatch; ++u)
+            t[u] = e[u] < Ee ? (r.m0 + j[u]) * kChunk + (int)((w[u] >> 7) & 63u) : -1;
+        fn(t, w);
+    }
 }
 
 // Key outliers: logit(t, hq) += (x - zhat) * r, r the component of the rotated query that
@@ -782,32 +810,39 @@ __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
     const uint32_t* cp = c.kchunk + (size_t)li * (nchunks(cfg.T_max) + 1);
     const uint32_t* ent = c.kout + (size_t)li * cfg.out_cap_k;
     __shared__ uint32_t cps[kOutChunks + 1];
-    const OutRange r = stage_chunks(cp, c.kcount[li], len, cps);
-    for (uint32_t e = r.lo + threadIdx.x; e < r.hi; e += blockDim.x) {
-        const uint32_t w = ent[e];
-        const int t = entry_token(r, cps, e, w), ch = (int)(w & 127u);
-        if (t >= len) continue;
-        const int p = ch & 63;
-        const float2 cs = trig_at(thi, tlo, t, p);
-        const float d = h2f((uint16_t)(w >> 16)) - zk[(size_t)li * kD + ch];
-        for (int a = 0; a < g; ++a) {
-            const int hq = h * g + a;
-            const float* qv = qr + ((size_t)b * cfg.Hq + hq) * kD;
-            const float qa = qv[p], qb = qv[p + 64];
-            const float rr = (ch < 64) ? (cs.x * qa + cs.y * qb) : (cs.x * qb - cs.y * qa);
-            atomicAdd(&logits[((size_t)b * cfg.Hq + hq) * cfg.T_max + t], d * rr);
+    __shared__ float zks[kD];
+    __shared__ float qs[kMaxG * kD];
+    for (int e = threadIdx.x; e < kD; e += blockDim.x) zks[e] = zk[(size_t)li * kD + e];
+    for (int e = threadIdx.x; e < g * kD; e += blockDim.x)
+        qs[e] = qr[((size_t)b * cfg.Hq + h * g) * kD + e];
+    const OutRange r = stage_chunks(cp, c.kcount[li], len, cps);  // barrier covers the above
+    float* lb0 = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
+    walk_entries(r, cps, ent, [&](const int (&t)[kOutBatch], const uint32_t (&w)[kOutBatch]) {
+        float2 cs[kOutBatch];
+#pragma unroll
+        for (int u = 0; u < kOutBatch; ++u)
+            cs[u] = (t[u] >= 0 && t[u] < len) ? trig_at(thi, tlo, t[u], (int)(w[u] & 63u))
+                                              : make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int u = 0; u < kOutBatch; ++u) {
+            if (t[u] < 0 || t[u] >= len) continue;
+            const int ch = (int)(w[u] & 127u), p = ch & 63;
+            const float d = h2f((uint16_t)(w[u] >> 16)) - zks[ch];
+            for (int a = 0; a < g; ++a) {
+                const float qa = qs[a * kD + p], qb = qs[a * kD + p + 64];
+                const float rr = (ch < 64) ? (cs[u].x * qa + cs[u].y * qb)
+                                           : (cs[u].x * qb - cs[u].y * qa);
+                atomicAdd(&lb0[(size_t)a * cfg.T_max + t[u]], d * rr);
+            }
         }
-    }
+    });
 }
 
 // ---------------------------------------------------------------------------------
 // Softmax statistics of each split from the (corrected) logits: stats = (m_s, l_s), one pass
-// with a running (max, sum) per thread, merged across the block.
-__device__ __forceinline__ void online_add(float& m, float& l, float x) {
-    const float mn = fmaxf(m, x);
-    l = (m > -INFINITY ? l * __expf(m - mn) : 0.0f) + __expf(x - mn);
-    m = mn;
-}
+// over the split with a running (max, sum) per thread, merged across the block.
+constexpr int kStatThreads = 256;  // threads of the statistics kernel
+constexpr int kStatVec = 8;        // float4 loads per thread and tile
 __device__ __forceinline__ void online_merge(float& m, float& l, float m2, float l2) {
     const float mn = fmaxf(m, m2);
     if (mn == -INFINITY) return;
@@ -815,34 +850,54 @@ __device__ __forceinline__ void online_merge(float& m, float& l, float m2, float
     m = mn;
 }
 
-__global__ void __launch_bounds__(256) k_logit_stats(kvq_cfg cfg, const int32_t* __restrict__ lens,
+__global__ void __launch_bounds__(kStatThreads) k_logit_stats(kvq_cfg cfg, const int32_t* __restrict__ lens,
                                                      const float* __restrict__ logits, int Ls,
                                                      int S, int max_len, float2* __restrict__ stats) {
     const int s = blockIdx.x, bh = blockIdx.y, b = bh / cfg.Hq;
     const int len = min(lens[b], max_len);
     const int t0 = s * Ls, t1 = max(t0, min(len, t0 + Ls));  // empty split: t1 == t0
     const float* row = logits + (size_t)bh * cfg.T_max;
-    float m = -INFINITY, l = 0.0f;
-    // t0 is a multiple of 64; whole float4s while the row's address allows, the rest singly
+    // t0 is a multiple of 64; float4 loads when the row's address allows
     const bool vec = ((reinterpret_cast<uintptr_t>(row + t0) & 15u) == 0);
-    const int tv = vec ? t0 + ((t1 - t0) & ~3) : t0;
-    for (int t = t0 + 4 * (int)threadIdx.x; t < tv; t += 4 * blockDim.x) {
-        const float4 x = *reinterpret_cast<const float4*>(row + t);
-        online_add(m, l, x.x);
-        online_add(m, l, x.y);
-        online_add(m, l, x.z);
-        online_add(m, l, x.w);
+    float m = -INFINITY, l = 0.0f;
+    // tiles of kStatThreads x kStatVec float4s: all loads of a tile in flight at once, then
+    // its max and its sum of exponentials, merged into the running pair
+    for (int tb = t0; tb < t1; tb += 4 * kStatThreads * kStatVec) {
+        float x[kStatVec][4];
+#pragma unroll
+        for (int u = 0; u < kStatVec; ++u) {
+            const int tt = tb + 4 * (threadIdx.x + kStatThreads * u);
+            if (vec && tt + 3 < t1) {
+                const float4 v = *reinterpret_cast<const float4*>(row + tt);
+                x[u][0] = v.x; x[u][1] = v.y; x[u][2] = v.z; x[u][3] = v.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[u][e] = tt + e < t1 ? row[tt + e] : -INFINITY;
+            }
+        }
+        float mt = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kStatVec; ++u)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) mt = fmaxf(mt, x[u][e]);
+        if (mt > -INFINITY) {
+            float lt = 0.0f;
+#pragma unroll
+            for (int u = 0; u < kStatVec; ++u)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) lt += __expf(x[u][e] - mt);
+            online_merge(m, l, mt, lt);
+        }
     }
-    for (int t = tv + threadIdx.x; t < t1; t += blockDim.x) online_add(m, l, row[t]);
 #pragma unroll
     for (int o = 16; o; o >>= 1)
         online_merge(m, l, __shfl_xor_sync(0xffffffffu, m, o), __shfl_xor_sync(0xffffffffu, l, o));
-    __shared__ float2 red[8];
+    __shared__ float2 red[kStatThreads / 32];
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = make_float2(m, l);
     __syncthreads();
     if (threadIdx.x == 0) {
         float M = -INFINITY, Lsum = 0.0f;
-        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) online_merge(M, Lsum, red[w].x, red[w].y);
+        for (int w = 0; w < kStatThreads / 32; ++w) online_merge(M, Lsum, red[w].x, red[w].y);
         stats[(size_t)bh * S + s] = make_float2(M, Lsum);
     }
 }
@@ -1066,30 +1121,43 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
     const uint32_t* cp = c.vchunk + (size_t)li * (nchunks(cfg.T_max) + 1);
     const uint32_t* ent = c.vout + (size_t)li * cfg.out_cap_v;
     __shared__ float acc[kMaxG * kD];
-    __shared__ float bnd[16];
-    __shared__ float2 mls[kMaxG];
+    __shared__ float bnd[16], lev[16];
+    __shared__ float2 mls[kMaxG];  // (M, 1 / L), 1 / L = 0 for an empty row
     __shared__ uint32_t cps[kOutChunks + 1];
     const int nb = (1 << cfg.bits) - 1;
     if (threadIdx.x < nb) bnd[threadIdx.x] = cb.bounds[threadIdx.x];
-    if (threadIdx.x < g) mls[threadIdx.x] = ml[(size_t)b * cfg.Hq + h * g + threadIdx.x];
+    if (threadIdx.x <= nb) lev[threadIdx.x] = cb.levels[threadIdx.x];
+    if (threadIdx.x < g) {
+        const float2 v = ml[(size_t)b * cfg.Hq + h * g + threadIdx.x];
+        mls[threadIdx.x] = make_float2(v.x, v.y > 0.0f ? 1.0f / v.y : 0.0f);
+    }
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x) acc[e] = 0.0f;
     const OutRange r = stage_chunks(cp, c.vcount[li], len, cps);  // barrier covers the above
     if (r.lo >= r.hi) return;
     const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
     const float* lrow = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
-    for (uint32_t e = r.lo + threadIdx.x; e < r.hi; e += blockDim.x) {
-        const uint32_t w = ent[e];
-        const int t = entry_token(r, cps, e, w), ch = (int)(w & 127u);
-        if (t >= len) continue;
-        const float2 vp = vpar[t];
-        const float d = h2f((uint16_t)(w >> 16)) - zero_code_value(vp.x, vp.y, cb.levels, bnd, nb);
-        for (int a = 0; a < g; ++a) {
-            const float2 mL = mls[a];
-            if (mL.y > 0.0f)
-                atomicAdd(&acc[a * kD + ch],
-                          expf(lrow[(size_t)a * cfg.T_max + t] - mL.x) / mL.y * d);
+    walk_entries(r, cps, ent, [&](const int (&t)[kOutBatch], const uint32_t (&w)[kOutBatch]) {
+        float2 vp[kOutBatch];
+        float l0[kOutBatch];
+#pragma unroll
+        for (int u = 0; u < kOutBatch; ++u) {
+            const bool ok = t[u] >= 0 && t[u] < len;
+            vp[u] = ok ? vpar[t[u]] : make_float2(0.0f, 1.0f);
+            l0[u] = ok ? lrow[t[u]] : 0.0f;
         }
-    }
+#pragma unroll
+        for (int u = 0; u < kOutBatch; ++u) {
+            if (t[u] < 0 || t[u] >= len) continue;
+            const int ch = (int)(w[u] & 127u);
+            const float d = h2f((uint16_t)(w[u] >> 16)) -
+                            zero_code_value(vp[u].x, vp[u].y, lev, bnd, nb);
+            for (int a = 0; a < g; ++a) {
+                const float2 mi = mls[a];
+                const float la = a == 0 ? l0[u] : lrow[(size_t)a * cfg.T_max + t[u]];
+                if (mi.y > 0.0f) atomicAdd(&acc[a * kD + ch], __expf(la - mi.x) * mi.y * d);
+            }
+        }
+    });
     __syncthreads();
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x) {
         const float v = acc[e];
@@ -1396,7 +1464,7 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     k_key_outliers<<<go, kOutThreads, 0, st>>>(*cfg, *cache, T.qr, T.thi, T.tlo, T.zk, max_len,
                                                    logits);
     dim3 gs(S, cfg->B * cfg->Hq);
-    k_logit_stats<<<gs, 256, 0, st>>>(*cfg, cache->len, logits, Ls, S, max_len, (float2*)stats);
+    k_logit_stats<<<gs, kStatThreads, 0, st>>>(*cfg, cache->len, logits, Ls, S, max_len, (float2*)stats);
     return record_cuda(cudaGetLastError());
 }
 
