@@ -147,12 +147,6 @@ __device__ __forceinline__ unsigned long long tld(const uint8_t* tab, uint32_t o
     return *reinterpret_cast<const unsigned long long*>(tab + off);
 }
 
-// zhat = off + half * L[encode((0 - off)/half)]: the dense value stored at an outlier.
-__device__ __forceinline__ float zero_code_value(float off, float half, const float* levels,
-                                                 const float* bounds, int nb) {
-    const float xn = normalize(0.0f, off, half);
-    return off + half * levels[encode(xn, bounds, nb)];
-}
 
 // Consumer warps of a CTA (one more warp streams the input) and heads per consumer warp.
 // With four query heads per CTA two warps share each quad pair (two heads each): twice the
@@ -799,40 +793,44 @@ __device__ __forceinline__ void walk_entries(const OutRange& r, const uint32_t* 
 }
 
 // Key outliers: logit(t, hq) += (x - zhat) * r, r the component of the rotated query that
-// meets the outlier's channel after the key is rotated to t.
+// meets the outlier's channel after the key is rotated to t.  G query heads per kv head (0:
+// read from cfg).
+template <int G>
 __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
     kvq_cfg cfg, kvq_cache c, const float* __restrict__ qr, const float2* __restrict__ thi,
     const float2* __restrict__ tlo, const float* __restrict__ zk, int max_len,
     float* __restrict__ logits) {
     const int li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
-    const int g = cfg.Hq / cfg.Hkv;
+    const int g = G ? G : cfg.Hq / cfg.Hkv;
     const int len = min(c.len[b], max_len);
     const uint32_t* cp = c.kchunk + (size_t)li * (nchunks(cfg.T_max) + 1);
     const uint32_t* ent = c.kout + (size_t)li * cfg.out_cap_k;
     __shared__ uint32_t cps[kOutChunks + 1];
     __shared__ float zks[kD];
-    __shared__ float qs[kMaxG * kD];
+    __shared__ float qs[(G ? G : kMaxG) * kD];
     for (int e = threadIdx.x; e < kD; e += blockDim.x) zks[e] = zk[(size_t)li * kD + e];
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x)
         qs[e] = qr[((size_t)b * cfg.Hq + h * g) * kD + e];
     const OutRange r = stage_chunks(cp, c.kcount[li], len, cps);  // barrier covers the above
     float* lb0 = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
+    const size_t T_max = cfg.T_max;
     walk_entries(r, cps, ent, [&](const int (&t)[kOutBatch], const uint32_t (&w)[kOutBatch]) {
+        bool ok[kOutBatch];
         float2 cs[kOutBatch];
 #pragma unroll
-        for (int u = 0; u < kOutBatch; ++u)
-            cs[u] = (t[u] >= 0 && t[u] < len) ? trig_at(thi, tlo, t[u], (int)(w[u] & 63u))
-                                              : make_float2(0.0f, 0.0f);
+        for (int u = 0; u < kOutBatch; ++u) {
+            ok[u] = (unsigned)t[u] < (unsigned)len;
+            cs[u] = trig_at(thi, tlo, ok[u] ? t[u] : 0, (int)(w[u] & 63u));
+        }
 #pragma unroll
         for (int u = 0; u < kOutBatch; ++u) {
-            if (t[u] < 0 || t[u] >= len) continue;
             const int ch = (int)(w[u] & 127u), p = ch & 63;
             const float d = h2f((uint16_t)(w[u] >> 16)) - zks[ch];
+            // rotate-half: channel c < 64 meets (cos, sin) . (q_p, q_p+64), c >= 64 the other
+            const float sa = ch < 64 ? cs[u].x : -cs[u].y, sb = ch < 64 ? cs[u].y : cs[u].x;
             for (int a = 0; a < g; ++a) {
-                const float qa = qs[a * kD + p], qb = qs[a * kD + p + 64];
-                const float rr = (ch < 64) ? (cs[u].x * qa + cs[u].y * qb)
-                                           : (cs[u].x * qb - cs[u].y * qa);
-                atomicAdd(&lb0[(size_t)a * cfg.T_max + t[u]], d * rr);
+                const float rr = fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
+                if (ok[u]) atomicAdd(&lb0[a * T_max + t[u]], d * rr);
             }
         }
     });
@@ -1111,22 +1109,23 @@ __global__ void __launch_bounds__(pv_warps(HPC) * 32 + 32, 1)
 // ---------------------------------------------------------------------------------
 // Value outliers: out(hq, c) += p(t, hq) (x - zhat_t), p = exp(l - M) / L from the merged
 // statistics, zhat_t = off_t + half_t L[encode(normalize(0))]; sums gather in shared memory
-// and a block adds them to the output once.
+// and a block adds them to the output once.  G as for the key outliers.
+template <int BITS, int G>
 __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
     kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
     const float2* __restrict__ ml, int max_len, float* __restrict__ out) {
+    constexpr int NB = (1 << BITS) - 1;
     const int li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
-    const int g = cfg.Hq / cfg.Hkv;
+    const int g = G ? G : cfg.Hq / cfg.Hkv;
     const int len = min(c.len[b], max_len);
     const uint32_t* cp = c.vchunk + (size_t)li * (nchunks(cfg.T_max) + 1);
     const uint32_t* ent = c.vout + (size_t)li * cfg.out_cap_v;
-    __shared__ float acc[kMaxG * kD];
+    __shared__ float acc[(G ? G : kMaxG) * kD];
     __shared__ float bnd[16], lev[16];
     __shared__ float2 mls[kMaxG];  // (M, 1 / L), 1 / L = 0 for an empty row
     __shared__ uint32_t cps[kOutChunks + 1];
-    const int nb = (1 << cfg.bits) - 1;
-    if (threadIdx.x < nb) bnd[threadIdx.x] = cb.bounds[threadIdx.x];
-    if (threadIdx.x <= nb) lev[threadIdx.x] = cb.levels[threadIdx.x];
+    if (threadIdx.x < NB) bnd[threadIdx.x] = cb.bounds[threadIdx.x];
+    if (threadIdx.x <= NB) lev[threadIdx.x] = cb.levels[threadIdx.x];
     if (threadIdx.x < g) {
         const float2 v = ml[(size_t)b * cfg.Hq + h * g + threadIdx.x];
         mls[threadIdx.x] = make_float2(v.x, v.y > 0.0f ? 1.0f / v.y : 0.0f);
@@ -1134,27 +1133,37 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x) acc[e] = 0.0f;
     const OutRange r = stage_chunks(cp, c.vcount[li], len, cps);  // barrier covers the above
     if (r.lo >= r.hi) return;
+    float bd[NB];
+#pragma unroll
+    for (int j = 0; j < NB; ++j) bd[j] = bnd[j];
     const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
     const float* lrow = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
+    const size_t T_max = cfg.T_max;
     walk_entries(r, cps, ent, [&](const int (&t)[kOutBatch], const uint32_t (&w)[kOutBatch]) {
+        bool ok[kOutBatch];
         float2 vp[kOutBatch];
         float l0[kOutBatch];
 #pragma unroll
         for (int u = 0; u < kOutBatch; ++u) {
-            const bool ok = t[u] >= 0 && t[u] < len;
-            vp[u] = ok ? vpar[t[u]] : make_float2(0.0f, 1.0f);
-            l0[u] = ok ? lrow[t[u]] : 0.0f;
+            ok[u] = (unsigned)t[u] < (unsigned)len;
+            const int tt = ok[u] ? t[u] : 0;
+            vp[u] = vpar[tt];
+            l0[u] = lrow[tt];
         }
 #pragma unroll
         for (int u = 0; u < kOutBatch; ++u) {
-            if (t[u] < 0 || t[u] >= len) continue;
+            // the dense value stored at the outlier: the code of 0 in the token's normalization
+            const float xn = normalize(0.0f, vp[u].x, vp[u].y);
+            int code = 0;
+#pragma unroll
+            for (int j = 0; j < NB; ++j) code += xn > bd[j];
+            const float d = h2f((uint16_t)(w[u] >> 16)) - fmaf(vp[u].y, lev[code], vp[u].x);
             const int ch = (int)(w[u] & 127u);
-            const float d = h2f((uint16_t)(w[u] >> 16)) -
-                            zero_code_value(vp[u].x, vp[u].y, lev, bnd, nb);
             for (int a = 0; a < g; ++a) {
                 const float2 mi = mls[a];
-                const float la = a == 0 ? l0[u] : lrow[(size_t)a * cfg.T_max + t[u]];
-                if (mi.y > 0.0f) atomicAdd(&acc[a * kD + ch], __expf(la - mi.x) * mi.y * d);
+                const float la = a == 0 ? l0[u] : lrow[a * T_max + (ok[u] ? t[u] : 0)];
+                if (ok[u] && mi.y > 0.0f)
+                    atomicAdd(&acc[a * kD + ch], __expf(la - mi.x) * mi.y * d);
             }
         }
     });
@@ -1461,8 +1470,8 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     }
     const int nch = (max_len + kChunk - 1) / kChunk;
     dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
-    k_key_outliers<<<go, kOutThreads, 0, st>>>(*cfg, *cache, T.qr, T.thi, T.tlo, T.zk, max_len,
-                                                   logits);
+    auto ko = cfg->Hq == cfg->Hkv ? k_key_outliers<1> : k_key_outliers<0>;
+    ko<<<go, kOutThreads, 0, st>>>(*cfg, *cache, T.qr, T.thi, T.tlo, T.zk, max_len, logits);
     dim3 gs(S, cfg->B * cfg->Hq);
     k_logit_stats<<<gs, kStatThreads, 0, st>>>(*cfg, cache->len, logits, Ls, S, max_len, (float2*)stats);
     return record_cuda(cudaGetLastError());
@@ -1524,8 +1533,11 @@ static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
     const int nch = (max_len + kChunk - 1) / kChunk;
     dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
-    k_value_outliers<<<go, kOutThreads, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml,
-                                                     max_len, out);
+    const bool mha = cfg->Hq == cfg->Hkv;
+    auto vo = cfg->bits == 2 ? (mha ? k_value_outliers<2, 1> : k_value_outliers<2, 0>)
+            : cfg->bits == 3 ? (mha ? k_value_outliers<3, 1> : k_value_outliers<3, 0>)
+                             : (mha ? k_value_outliers<4, 1> : k_value_outliers<4, 0>);
+    vo<<<go, kOutThreads, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, max_len, out);
     return record_cuda(cudaGetLastError());
 }
 
