@@ -755,22 +755,31 @@ __device__ __forceinline__ OutRange stage_chunks(const uint32_t* __restrict__ cp
     return r;
 }
 
-// Calls fn(t, w) per window: w[u] the packed entries of the lane, t[u] their tokens (-1 where
-// the lane has no entry).
-template <class Fn>
-__device__ __forceinline__ void walk_entries(const OutRange& r, const uint32_t* cps,
-                                             const uint32_t* __restrict__ ent, Fn&& fn) {
-    constexpr uint32_t W = 32 * kOutBatch;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const uint32_t span = ((r.hi - r.lo + nw - 1) / nw + 31) & ~31u;
-    const uint32_t Eb = r.lo + (uint32_t)warp * span, Ee = min(r.hi, Eb + span);
-    if (Eb >= Ee) return;
-    int cur = 0;  // chunk of entry Eb: the largest j < n with cps[j] <= Eb
+// A warp's walk over its entry range.  next() fills, for the lane's kOutBatch entries of the
+// next window, w[u] (packed entry) and t[u] (token; -1 where the lane has no entry).
+struct EntryWalker {
+    static constexpr uint32_t W = 32 * kOutBatch;
+    uint32_t E, Ee;
+    int cur, n, m0;
+    __device__ __forceinline__ EntryWalker(const OutRange& r, const uint32_t* cps) {
+        const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+        const uint32_t span = ((r.hi - r.lo + nw - 1) / nw + 31) & ~31u;
+        E = r.lo + (uint32_t)warp * span;
+        Ee = min(r.hi, E + span);
+        n = r.n;
+        m0 = r.m0;
+        cur = 0;  // chunk of entry E: the largest j < n with cps[j] <= E
+        if (E < Ee) {
 #pragma unroll
-    for (int step = kOutChunks / 2; step; step >>= 1)
-        if (cur + step < r.n && cps[cur + step] <= Eb) cur += step;
-    for (uint32_t E = Eb; E < Ee; E += W) {
-        uint32_t e[kOutBatch], w[kOutBatch];
+            for (int step = kOutChunks / 2; step; step >>= 1)
+                if (cur + step < n && cps[cur + step] <= E) cur += step;
+        }
+    }
+    __device__ __forceinline__ bool next(const uint32_t* cps, const uint32_t* __restrict__ ent,
+                                         int (&t)[kOutBatch], uint32_t (&w)[kOutBatch]) {
+        if (E >= Ee) return false;
+        const uint32_t lane = threadIdx.x & 31;
+        uint32_t e[kOutBatch];
         int j[kOutBatch];
 #pragma unroll
         for (int u = 0; u < kOutBatch; ++u) {
@@ -779,18 +788,18 @@ __device__ __forceinline__ void walk_entries(const OutRange& r, const uint32_t* 
             j[u] = cur;
         }
         // boundaries inside the window (warp-uniform loop)
-        while (cur + 1 < r.n && cps[cur + 1] <= E + W - 1) {
+        while (cur + 1 < n && cps[cur + 1] <= E + W - 1) {
             const uint32_t bd = cps[++cur];
 #pragma unroll
             for (int u = 0; u < kOutBatch; ++u) j[u] += e[u] >= bd;
         }
-        int t[kOutBatch];
 #pragma unroll
         for (int u = 0; u < kOutBatch; ++u)
-            t[u] = e[u] < Ee ? (r.m0 + j[u]) * kChunk + (int)((w[u] >> 7) & 63u) : -1;
-        fn(t, w);
+            t[u] = e[u] < Ee ? (m0 + j[u]) * kChunk + (int)((w[u] >> 7) & 63u) : -1;
+        E += W;
+        return true;
     }
-}
+};
 
 // Key outliers: logit(t, hq) += (x - zhat) * r, r the component of the rotated query that
 // meets the outlier's channel after the key is rotated to t.  G query heads per kv head (0:
@@ -814,7 +823,10 @@ __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
     const OutRange r = stage_chunks(cp, c.kcount[li], len, cps);  // barrier covers the above
     float* lb0 = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
     const size_t T_max = cfg.T_max;
-    walk_entries(r, cps, ent, [&](const int (&t)[kOutBatch], const uint32_t (&w)[kOutBatch]) {
+    EntryWalker wk(r, cps);
+    int t[kOutBatch];
+    uint32_t w[kOutBatch];
+    while (wk.next(cps, ent, t, w)) {
         bool ok[kOutBatch];
         float2 cs[kOutBatch];
 #pragma unroll
@@ -828,12 +840,17 @@ __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
             const float d = h2f((uint16_t)(w[u] >> 16)) - zks[ch];
             // rotate-half: channel c < 64 meets (cos, sin) . (q_p, q_p+64), c >= 64 the other
             const float sa = ch < 64 ? cs[u].x : -cs[u].y, sb = ch < 64 ? cs[u].y : cs[u].x;
-            for (int a = 0; a < g; ++a) {
+#pragma unroll
+            for (int a = 0; a < (G ? G : 1); ++a) {
+                const float rr = fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
+                if (ok[u]) atomicAdd(&lb0[a * T_max + t[u]], d * rr);
+            }
+            for (int a = 1; !G && a < g; ++a) {
                 const float rr = fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
                 if (ok[u]) atomicAdd(&lb0[a * T_max + t[u]], d * rr);
             }
         }
-    });
+    }
 }
 
 // ---------------------------------------------------------------------------------
@@ -1139,7 +1156,10 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
     const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
     const float* lrow = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
     const size_t T_max = cfg.T_max;
-    walk_entries(r, cps, ent, [&](const int (&t)[kOutBatch], const uint32_t (&w)[kOutBatch]) {
+    EntryWalker wk(r, cps);
+    int t[kOutBatch];
+    uint32_t w[kOutBatch];
+    while (wk.next(cps, ent, t, w)) {
         bool ok[kOutBatch];
         float2 vp[kOutBatch];
         float l0[kOutBatch];
@@ -1159,14 +1179,19 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
             for (int j = 0; j < NB; ++j) code += xn > bd[j];
             const float d = h2f((uint16_t)(w[u] >> 16)) - fmaf(vp[u].y, lev[code], vp[u].x);
             const int ch = (int)(w[u] & 127u);
-            for (int a = 0; a < g; ++a) {
+#pragma unroll
+            for (int a = 0; a < (G ? G : 1); ++a) {
                 const float2 mi = mls[a];
-                const float la = a == 0 ? l0[u] : lrow[a * T_max + (ok[u] ? t[u] : 0)];
                 if (ok[u] && mi.y > 0.0f)
-                    atomicAdd(&acc[a * kD + ch], __expf(la - mi.x) * mi.y * d);
+                    atomicAdd(&acc[a * kD + ch], __expf(l0[u] - mi.x) * mi.y * d);
+            }
+            for (int a = 1; !G && a < g; ++a) {
+                const float2 mi = mls[a];
+                const float la = lrow[a * T_max + (ok[u] ? t[u] : 0)];
+                if (ok[u] && mi.y > 0.0f) atomicAdd(&acc[a * kD + ch], __expf(la - mi.x) * mi.y * d);
             }
         }
-    });
+    }
     __syncthreads();
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x) {
         const float v = acc[e];
