@@ -1124,6 +1124,204 @@ __global__ void __launch_bounds__(pv_warps(HPC) * 32 + 32, 1)
 }
 
 // ---------------------------------------------------------------------------------
+// PV when every kv head serves one query head: one query head per CTA, 512-token stages of its
+// value codes; half-warp hh of warp w takes the quads 8 w + 2 u + hh (u < 4), so a lane makes
+// 64 (pair, token) steps per stage against one weight computation, one barrier wait and one
+// stage's bookkeeping.  Lane l of warp w computes the weight of token 32 w + l of the stage;
+// the warp's 32 weights sit in its own slice of shared memory.  The code words of the two
+// half-warps are 16 banks apart.
+constexpr int kPQuads = 128;                 // token quads per stage
+constexpr int kPTokens = 4 * kPQuads;        // tokens per stage
+
+struct PQPlan {
+    int tab, ring, stage, wsm, bar, flag, total;
+};
+__host__ __device__ inline PQPlan pq_plan(int bits) {
+    PQPlan p;
+    int o = 0;
+    p.tab = o;   o += (1 << (2 * bits)) * 16 * 8;            // [entry][16 lane copies] (La, Lb)
+    p.stage = kPQuads * 16 * bits * 4;
+    p.ring = o;  o += kStages * p.stage;                     // reused by the final reduction
+    p.wsm = o;   o += kQWarps * 32 * 8;                      // [warp][token] (w, w)
+    p.bar = o;   o += 2 * kStages * 8;
+    p.flag = o;  o += 16;
+    p.total = o;
+    return p;
+}
+
+template <int BITS>
+__global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
+    k_pv_quad(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
+              const float2* __restrict__ ml, int Ls, int S, int max_len,
+              float* __restrict__ part) {
+    using F = Fmt<BITS>;
+    constexpr int NC = kQWarps * 32;
+    constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << 7;
+    extern __shared__ __align__(128) uint8_t sm[];
+    const PQPlan L = pq_plan(BITS);
+    uint8_t* tab = sm + L.tab;
+    uint8_t* ring = sm + L.ring;
+    unsigned long long* wsm = (unsigned long long*)(sm + L.wsm);
+    uint64_t* full = (uint64_t*)(sm + L.bar);
+    uint64_t* empty = full + kStages;
+    int* flag = (int*)(sm + L.flag);
+
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int i = tid & 15, x = i >> 2, lane = tid & 31, warp = tid >> 5, hh = (tid >> 4) & 1;
+    const int s = blockIdx.x, b = blockIdx.y, hq = blockIdx.z;
+    const int Hq = cfg.Hq, Hkv = cfg.Hkv, kvh = hq / (Hq / Hkv);
+    float* po_out = part + (((size_t)b * Hq + hq) * S + s) * kD;
+    const int len = min(c.len[b], max_len);
+    const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
+    if (t_begin >= t_end) {
+        for (int e = tid; e < kD; e += nthr) po_out[e] = 0.0f;
+        return;
+    }
+    const int nst = (t_end - t_begin + kPTokens - 1) / kPTokens;
+    if (tid == 0) {
+        for (int k = 0; k < kStages; ++k) {
+            mbar_init(full + k, 1);
+            mbar_init(empty + k, kQWarps);
+        }
+        flag[0] = 0;
+        flag[1] = 0;
+        fence_mbar_init();
+    }
+    const int nb = (1 << BITS) - 1;
+    for (int e = tid; e < F::NT * 16; e += nthr) {
+        const int idx = e >> 4;
+        reinterpret_cast<unsigned long long*>(tab)[e] =
+            pk(cb.levels[idx & nb], cb.levels[idx >> BITS]);
+    }
+    __syncthreads();  // tables complete, barriers initialised
+
+    unsigned long long O[4] = {0ull, 0ull, 0ull, 0ull};
+    float po = 0.0f;
+    if (tid >= NC) {
+        // ================= streaming warp
+        const int pl = tid - NC;
+        const uint32_t* src = c.vcodes + ((size_t)b * Hkv + kvh) * nquads(cfg.T_max) * F::BW;
+        int cc = 0;
+        for (; cc < nst; ++cc) {
+            const int slot = cc % kStages;
+            if (cc >= kStages && !mbar_wait(empty + slot, (uint32_t)(cc / kStages - 1) & 1u)) {
+                if (pl == 0) {
+                    atomicOr(flag, 1);
+                    set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+                }
+                break;
+            }
+            if (*flag) break;
+            if (pl == 0) {
+                fence_proxy_async();
+                const int tc = t_begin + cc * kPTokens;
+                const int q0 = tc >> 2, q1 = (min(tc + kPTokens, t_end) + 3) >> 2;
+                const uint32_t bytes = (uint32_t)(q1 - q0) * F::BW * 4;
+                mbar_arrive_expect_tx(full + slot, bytes);
+                bulk_load(ring + (size_t)slot * L.stage, src + (size_t)q0 * F::BW, bytes,
+                          full + slot);
+            }
+            __syncwarp();
+        }
+        if (pl == 0) flag[1] = cc;  // stages issued
+    } else {
+        // ================= consumer warps
+        const float2 mL = ml[(size_t)b * Hq + hq];
+        const float invL = mL.y > 0.0f ? 1.0f / mL.y : 0.0f;
+        const float* lrow = logits + ((size_t)b * Hq + hq) * cfg.T_max;
+        const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
+        float lg = -INFINITY;
+        float2 vp = make_float2(0.0f, 0.0f);
+        auto fetch = [&](int st) {
+            const int t = t_begin + st * kPTokens + 32 * warp + lane;
+            const bool ok = t < t_end;
+            lg = ok ? lrow[t] : -INFINITY;
+            vp = ok ? vpar[t] : make_float2(0.0f, 0.0f);
+        };
+        fetch(0);
+        uint32_t woff[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            woff[u] = (uint32_t)((8 * warp + 2 * u + hh) * F::BW + i * BITS) * 4;
+        const uint32_t lanebits = (uint32_t)i << 3;
+        unsigned long long* wsw = wsm + 32 * warp;
+        for (int st = 0; st < nst; ++st) {
+            const int slot = st % kStages;
+            {
+                const float p = (lg > -INFINITY) ? __expf(lg - mL.x) * invL : 0.0f;
+                const float wv = p * vp.y;
+                po = fmaf(p, vp.x, po);
+                wsw[lane] = pk(wv, wv);
+            }
+            __syncwarp();
+            if (st + 1 < nst) fetch(st + 1);
+            if (!mbar_wait(full + slot, (uint32_t)(st / kStages) & 1u)) {
+                atomicOr(flag, 1);
+                set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+            }
+            if (*flag) break;
+            const uint8_t* stage = ring + (size_t)slot * L.stage;
+            uint32_t w[4][BITS];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int d = 0; d < BITS; ++d)
+                    w[u][d] = *reinterpret_cast<const uint32_t*>(stage + woff[u] + 4 * d);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl) {
+                    // token 4 (2 u + hh) + (sl ^ x) of the warp's 32
+                    const unsigned long long ww = wsw[8 * u + 4 * hh + (sl ^ x)];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t fs = 0;
+                        switch (4 * k + sl) {
+#define KVQ_FS(N) case N: fs = field_to<BITS, N, 7>(w[u]); break;
+                            KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5)
+                            KVQ_FS(6) KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11)
+                            KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
+#undef KVQ_FS
+                        }
+                        O[k] = fma2(ww, tld(tab, (fs & MASK) | lanebits), O[k]);
+                    }
+                }
+            }
+            __syncwarp();  // wsw is rewritten for the next stage
+        }
+    }
+    __syncthreads();
+    if (*flag) {
+        if (tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1]);
+        return;
+    }
+    // partial sums of the 32 half-warps -> the split's output (the ring is idle now)
+    float* red = (float*)ring;
+    float* pored = red + 2 * kQWarps * kD;
+    if (tid < NC) {
+        const int row = 2 * warp + hh;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const f2 o = upk(O[k]);
+            red[row * kD + i + 16 * k] = o.x;
+            red[row * kD + i + 16 * k + 64] = o.y;
+        }
+        po = warp_sum(po);  // sum_t p_t off_t over the warp's tokens
+        if (lane == 0) pored[warp] = po;
+    }
+    __syncthreads();
+    for (int e = tid; e < kD; e += nthr) {
+        float a = 0.0f;
+        for (int r = 0; r < 2 * kQWarps; ++r) a += red[r * kD + e];
+        float o = 0.0f;
+        for (int w2 = 0; w2 < kQWarps; ++w2) o += pored[w2];
+        po_out[e] = a + o;
+    }
+}
+
+// ---------------------------------------------------------------------------------
 // Value outliers: out(hq, c) += p(t, hq) (x - zhat_t), p = exp(l - M) / L from the merged
 // statistics, zhat_t = off_t + half_t L[encode(normalize(0))]; sums gather in shared memory
 // and a block adds them to the output once.  G as for the key outliers.
@@ -1442,6 +1640,8 @@ typedef void (*QKKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const f
                          const float2*, int, int, int, float*);
 typedef void (*QKQKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*,
                           const float2*, int, int, float*);
+typedef void (*PVQKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*, int,
+                          int, int, float*);
 typedef void (*PVKernel)(kvq_cfg, kvq_cache, kvq_codebook, const float*, const float2*, int, int,
                          int, int, float*);
 
@@ -1543,6 +1743,15 @@ extern "C" int kvq_softmax_merge(const kvq_cfg* cfg, const float* stats, int32_t
 static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbV,
                   const float* logits, const float* ml, int max_len, float* out, float* part,
                   int S, int Ls, cudaStream_t st) {
+    if (cfg->Hq == cfg->Hkv) {
+        PVQKernel kq = cfg->bits == 2 ? k_pv_quad<2> : cfg->bits == 3 ? k_pv_quad<3> : k_pv_quad<4>;
+        const int smem = pq_plan(cfg->bits).total;
+        cudaError_t ce = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (ce) return record_cuda(ce);
+        dim3 grid(S, cfg->B, cfg->Hq);
+        kq<<<grid, kQWarps * 32 + 32, smem, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls,
+                                                    S, max_len, part);
+    } else {
     const int hpc = hpc_of(cfg);
     const int kvb = kvb_of(cfg, hpc);
     PVKernel kern = cfg->bits == 2 ? pv_kernel<2>(hpc, kvb == 1)
@@ -1555,6 +1764,7 @@ static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     kern<<<grid, pv_warps(hpc) * 32 + 32, smem, st>>>(*cfg, *cache, *cbV, logits,
                                                             (const float2*)ml, Ls, S, max_len,
                                                             kvb, part);
+    }
     k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
     const int nch = (max_len + kChunk - 1) / kChunk;
     dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
