@@ -142,6 +142,14 @@ __device__ __forceinline__ uint32_t field_to(const uint32_t (&w)[BITS]) {
     }
 }
 
+// Shared-memory load at a 32-bit shared-window address plus an immediate byte offset.
+template <int IMM>
+__device__ __forceinline__ unsigned long long lds64(uint32_t addr) {
+    unsigned long long d;
+    asm("ld.shared.b64 %0, [%1+%2];" : "=l"(d) : "r"(addr), "n"(IMM));
+    return d;
+}
+
 // Shared-memory table load at a byte offset.
 __device__ __forceinline__ unsigned long long tld(const uint8_t* tab, uint32_t off) {
     return *reinterpret_cast<const unsigned long long*>(tab + off);
@@ -509,20 +517,24 @@ constexpr int kQQuads = 64;                  // token quads per stage
 constexpr int kQTokens = 4 * kQQuads;        // tokens per stage
 constexpr int kQWarps = 16;                  // consumer warps
 
+// The table goes last, at the first shared-window address past `pre` that is a multiple of
+// its j-slice (64 pairs x NT entries x 8 bytes): a lookup address is then one OR of the
+// entry, the slice and the lane's pair, with no add of the table base.
 struct QQPlan {
-    int tab, ring, stage, base, lev, bar, flag, total;
+    int ring, stage, base, lev, bar, flag, pre, jslice, total;
 };
 __host__ __device__ inline QQPlan qq_plan(int bits) {
     QQPlan p;
     int o = 0;
-    p.tab = o;   o += 4 * (1 << (2 * bits)) * 64 * 8;        // [j][entry][pair] (X, Y)
     p.stage = kQQuads * 16 * bits * 4;                       // code blocks of 64 quads
     p.ring = o;  o += kStages * p.stage;
     p.base = o;  o += kStages * 64 * 16;                     // [stage][pair] (c, c, s, s) at stage start
     p.lev = o;   o += 16 * 4;                                // codebook levels
     p.bar = o;   o += 2 * kStages * 8;
     p.flag = o;  o += 16;
-    p.total = o;
+    p.pre = o;
+    p.jslice = (1 << (2 * bits)) * 64 * 8;
+    p.total = o + p.jslice + 4 * p.jslice;                   // alignment slack + [j][entry][pair]
     return p;
 }
 
@@ -538,7 +550,9 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
     constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << P;
     extern __shared__ __align__(128) uint8_t sm[];
     const QQPlan L = qq_plan(BITS);
-    uint8_t* tab = sm + L.tab;
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t tpos = (sbase + L.pre + L.jslice - 1) & ~(uint32_t)(L.jslice - 1);
+    uint8_t* tab = sm + (tpos - sbase);
     uint8_t* ring = sm + L.ring;
     float4* base = (float4*)(sm + L.base);
     float* lev = (float*)(sm + L.lev);
@@ -639,7 +653,8 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
         const int qbase = 4 * warp + ((tid >> 4) & 1);
         uint32_t lb[4], woff[2];
 #pragma unroll
-        for (int sl = 0; sl < 4; ++sl) lb[sl] = ((uint32_t)(sl ^ x) << JS) | ((uint32_t)i << 3);
+        for (int sl = 0; sl < 4; ++sl)
+            lb[sl] = tpos + ((uint32_t)(sl ^ x) << JS) + ((uint32_t)i << 3);
         // phase from the stage start to the quad, pair i + 16 k, as (c, s) and (-s, c)
         unsigned long long RQ[2][4], RQp[2][4];
 #pragma unroll
@@ -697,7 +712,11 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
                             KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
 #undef KVQ_FS
                         }
-                        acc[sl][u] = fma2(Pc, tld(tab + 128 * k, (fs & MASK) | lb[sl]), acc[sl][u]);
+                        const uint32_t a = (fs & MASK) | lb[sl];
+                        const unsigned long long T = k == 0 ? lds64<0>(a)
+                                                   : k == 1 ? lds64<128>(a)
+                                                   : k == 2 ? lds64<256>(a) : lds64<384>(a);
+                        acc[sl][u] = fma2(Pc, T, acc[sl][u]);
                     }
                 }
             }
@@ -1133,19 +1152,22 @@ __global__ void __launch_bounds__(pv_warps(HPC) * 32 + 32, 1)
 constexpr int kPQuads = 128;                 // token quads per stage
 constexpr int kPTokens = 4 * kPQuads;        // tokens per stage
 
+// The (La, Lb) table goes last, at a shared-window address that is a multiple of its size, so
+// a lookup address is one OR of the entry and the lane's copy.
 struct PQPlan {
-    int tab, ring, stage, wsm, bar, flag, total;
+    int ring, stage, wsm, bar, flag, pre, tsize, total;
 };
 __host__ __device__ inline PQPlan pq_plan(int bits) {
     PQPlan p;
     int o = 0;
-    p.tab = o;   o += (1 << (2 * bits)) * 16 * 8;            // [entry][16 lane copies] (La, Lb)
     p.stage = kPQuads * 16 * bits * 4;
     p.ring = o;  o += kStages * p.stage;                     // reused by the final reduction
     p.wsm = o;   o += kQWarps * 32 * 8;                      // [warp][token] (w, w)
     p.bar = o;   o += 2 * kStages * 8;
     p.flag = o;  o += 16;
-    p.total = o;
+    p.pre = o;
+    p.tsize = (1 << (2 * bits)) * 16 * 8;                    // [entry][16 lane copies] (La, Lb)
+    p.total = o + 2 * p.tsize;                               // alignment slack + table
     return p;
 }
 
@@ -1159,7 +1181,9 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
     constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << 7;
     extern __shared__ __align__(128) uint8_t sm[];
     const PQPlan L = pq_plan(BITS);
-    uint8_t* tab = sm + L.tab;
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t tpos = (sbase + L.pre + L.tsize - 1) & ~(uint32_t)(L.tsize - 1);
+    uint8_t* tab = sm + (tpos - sbase);
     uint8_t* ring = sm + L.ring;
     unsigned long long* wsm = (unsigned long long*)(sm + L.wsm);
     uint64_t* full = (uint64_t*)(sm + L.bar);
@@ -1243,7 +1267,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             woff[u] = (uint32_t)((8 * warp + 2 * u + hh) * F::BW + i * BITS) * 4;
-        const uint32_t lanebits = (uint32_t)i << 3;
+        const uint32_t lanebits = tpos | ((uint32_t)i << 3);
         unsigned long long* wsw = wsm + 32 * warp;
         for (int st = 0; st < nst; ++st) {
             const int slot = st % kStages;
@@ -1285,7 +1309,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
                             KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
 #undef KVQ_FS
                         }
-                        O[k] = fma2(ww, tld(tab, (fs & MASK) | lanebits), O[k]);
+                        O[k] = fma2(ww, lds64<0>((fs & MASK) | lanebits), O[k]);
                     }
                 }
             }
