@@ -41,7 +41,8 @@ def parse():
     p.add_argument("--workload", default="llama7b_1m_32layers")
     p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     p.add_argument("--splits", type=int, default=0)
-    p.add_argument("--path", default="split", choices=["split", "fused"])
+    p.add_argument("--path", default="split", choices=["split", "one-call"],
+                   help="split: kvq_decode_qk + kvq_softmax_merge + kvq_decode_pv; one-call: kvq_decode_attention")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-fp16", action="store_true")
     p.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
@@ -163,8 +164,9 @@ def bytes_model(w, T, kcount, vcount, path):
 
     Key side (QK): packed key codes, key-outlier entries (4 B each: position and value),
     key chunk pointers (one list per kv head); value side (PV): packed value codes,
-    value-outlier entries, value token params (8 B/token), value chunk pointers.  The split path also
-    writes and reads fp32 logits (4 B per token per query head, each way).
+    value-outlier entries, value token params (8 B/token), value chunk pointers.  Both paths
+    (the three calls, or kvq_decode_attention, which makes the same three internally) also
+    write and read fp32 logits (4 B per token per query head, each way).
     """
     code_row = w.Hkv * w.D * w.bits // 8
     nch = (T + 63) // 64 + 1
@@ -173,7 +175,7 @@ def bytes_model(w, T, kcount, vcount, path):
     logit = 4 * w.Hq * T
     if path == "split":
         return {"qk": k_bytes + logit, "pv": v_bytes + logit, "total": k_bytes + v_bytes + 2 * logit}
-    return {"attn": k_bytes + v_bytes, "total": k_bytes + v_bytes}
+    return {"attn": k_bytes + v_bytes + 2 * logit, "total": k_bytes + v_bytes + 2 * logit}
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -511,7 +513,7 @@ def run_kvq(args, rank, world):
     if rank != 0:
         return 0
     # append: begin, stats, scan, write; qk: tables, qk, key outliers, split stats; merge;
-    # pv: pv, split sum, value outliers (the fused call launches the same kernels)
+    # pv: pv, split sum, value outliers (the one-call path launches the same kernels)
     launches_per_layer_step = 12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -221,10 +221,11 @@ int kvq_decode_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
 int kvq_decode_workspace(const kvq_cfg* cfg, int32_t max_len, int32_t splits, size_t* bytes);
 
 /*
- * Fused single-pass decode attention: the same result as kvq_decode_qk +
- * kvq_softmax_merge + kvq_decode_pv, computed with an online softmax per split
- * (no logits written) and one merge; out float [B][Hq][D].
- *   workspace  device scratch of kvq_decode_workspace bytes
+ * Decode attention in one call: kvq_decode_qk, kvq_softmax_merge and kvq_decode_pv
+ * on `stream`, with their buffers (logits [B][Hq][T_max], split statistics, (M, L),
+ * split partials, per-call tables) carved from `workspace`; the same result as the
+ * three calls; out float [B][Hq][D].
+ *   workspace  device scratch of kvq_decode_workspace bytes, 16-byte aligned
  */
 int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
                          const kvq_codebook* cbV, const uint16_t* q, const int32_t* qpos,

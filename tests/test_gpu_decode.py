@@ -109,7 +109,7 @@ def test_split_path(name, over, T, plen, appends, splits):
 
 
 @pytest.mark.parametrize("name,over,T,plen,appends", CASES)
-def test_fused_path(name, over, T, plen, appends):
+def test_one_call_path(name, over, T, plen, appends):
     import torch
     import long_context_decode_nuq_b200 as K
     w, o, g, dK, dV, dq, dpos, refs, _, _ = _setup(name, over, T, plen, appends)

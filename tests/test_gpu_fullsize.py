@@ -49,7 +49,7 @@ def _quantize(cache, dK, dV, k, v, calibrate):
 
 
 def _attend(cache, dK, dV, q, qpos, max_len):
-    """Both decode paths as bench.py runs them: the fused call and the split calls."""
+    """Both decode paths as bench.py runs them: the one-call kvq_decode_attention and the split calls."""
     import torch
     import long_context_decode_nuq_b200 as K
     cfg = cache.cfg
