@@ -212,6 +212,7 @@ int kvq_softmax_merge(const kvq_cfg* cfg, const float* stats, int32_t splits, fl
  *   logits, ml from the two calls above; out float [B][Hq][D]
  *   part   float scratch [B][Hq][splits][D] (per-split partial sums, summed in
  *          split order)
+ * A sequence with no cached token (len 0) gets out = 0.
  */
 int kvq_decode_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbV,
                   const float* logits, const float* ml, int32_t max_len, float* out, float* part,
