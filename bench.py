@@ -159,23 +159,47 @@ def traffic_for(kernel, units):
 
 # ----------------------------------------------------------------------------- algorithmic bytes
 
-def bytes_model(w, T, kcount, vcount, path):
+OUTLIER_ENTRY_BYTES = 4  # one packed uint32 per outlier: (fp16 bits << 16) | (t % 64) << 7 | c
+
+
+def expected_outliers_per_token(w):
+    """Expected outlier entries per cached token of one layer (all kv heads).
+
+    Keys: a channel keeps 2k of its N calibration values as outliers, k = floor(f*N/2 + 1/2),
+    i.e. about f*n per token over the n = Hkv*D channels; values: each token row keeps 2k_v,
+    k_v = floor(f*n/2 + 1/2).
+    """
+    kv = math.floor(w.f * w.n / 2 + 0.5)
+    return w.f * w.n, 2 * kv
+
+
+def cache_bytes_per_token(w, outlier_bytes=OUTLIER_ENTRY_BYTES, params=True):
+    """Stored bytes per token of one layer: K and V codes, outlier entries, value (off, half).
+
+    The per-channel key scales and the chunk pointers are per sequence, not per token.
+    """
+    k_out, v_out = expected_outliers_per_token(w)
+    codes = 2 * w.n * w.bits / 8
+    return codes + outlier_bytes * (k_out + v_out) + (8 if params else 0)
+
+
+def bytes_model(w, T, kcount, vcount, path, outlier_bytes=OUTLIER_ENTRY_BYTES, logits=True):
     """Algorithmic bytes of one layer's decode (attention part) over T tokens.
 
-    Key side (QK): packed key codes, key-outlier entries (4 B each: position and value),
-    key chunk pointers (one list per kv head); value side (PV): packed value codes,
-    value-outlier entries, value token params (8 B/token), value chunk pointers.  Both paths
-    (the three calls, or kvq_decode_attention, which makes the same three internally) also
-    write and read fp32 logits (4 B per token per query head, each way).
+    Key side (QK): packed key codes, key-outlier entries (outlier_bytes each: position and
+    value), key chunk pointers (one list per kv head); value side (PV): packed value codes,
+    value-outlier entries, value token params (8 B/token), value chunk pointers.  The split
+    path (kvq_decode_qk / kvq_softmax_merge / kvq_decode_pv) also writes and reads fp32 logits
+    (4 B per token per query head, each way); the fused one-call path moves no logits.
     """
     code_row = w.Hkv * w.D * w.bits // 8
     nch = (T + 63) // 64 + 1
-    k_bytes = T * code_row + 4 * kcount + 4 * nch * w.Hkv
-    v_bytes = T * code_row + 4 * vcount + 8 * T + 4 * nch * w.Hkv
-    logit = 4 * w.Hq * T
+    k_bytes = T * code_row + outlier_bytes * kcount + 4 * nch * w.Hkv
+    v_bytes = T * code_row + outlier_bytes * vcount + 8 * T + 4 * nch * w.Hkv
+    logit = 4 * w.Hq * T if logits else 0
     if path == "split":
         return {"qk": k_bytes + logit, "pv": v_bytes + logit, "total": k_bytes + v_bytes + 2 * logit}
-    return {"attn": k_bytes + v_bytes + 2 * logit, "total": k_bytes + v_bytes + 2 * logit}
+    return {"attn": k_bytes + v_bytes, "total": k_bytes + v_bytes}
 
 
 # ----------------------------------------------------------------------------- CPU oracle

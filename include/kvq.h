@@ -201,14 +201,29 @@ int kvq_decode_qk_workspace(const kvq_cfg* cfg, int32_t max_len, size_t* bytes);
 /* The split count the library uses for `splits = 0`. */
 int kvq_decode_splits(const kvq_cfg* cfg, int32_t max_len);
 
-/* Split-K softmax merge: ml[b][hq] = (M, L), M = max_s m_s, L = sum_s l_s e^(m_s - M).
- * stats float2 [B][Hq][splits] from kvq_decode_qk; ml float2 [B][Hq]. */
+/*
+ * Split-K softmax merge (the softmax of decode attention, done by the custom decode
+ * kernels that read the quantized cache directly: study.space summary, custom CUDA
+ * kernels for memory- and bandwidth-bound long-context decode).  The pages fix the
+ * softmax, not how it is split; the split into token ranges is this library's, and the
+ * merge is the exact identity softmax(l) over the union of the ranges:
+ *   ml[b][hq] = (M, L), M = max_s m_s, L = sum_s l_s e^(m_s - M)   (binary32).
+ *   stats float2 [B][Hq][splits] from kvq_decode_qk (device); ml float2 [B][Hq] (device)
+ * An empty split (m_s = -inf, l_s = 0) contributes nothing; all splits empty gives
+ * (-inf, 0).  Errors: KVQ_ERR_NULL, KVQ_ERR_RANGE (splits outside 1 .. 4096).
+ */
 int kvq_softmax_merge(const kvq_cfg* cfg, const float* stats, int32_t splits, float* ml,
                       void* stream);
 
 /*
- * Decode PV: out[b][hq][:] = sum_t p_t * vhat_t,h with p_t = exp(logits - M)/L and
- * vhat the dequantized value (off_t + half_t*L[code], outliers replaced).
+ * Decode PV (the value half of the custom decode kernels, study.space summary; the
+ * read side of per-token value quantization onto the NUQ datatype, technique (iii),
+ * with per-vector dense-and-sparse outliers, technique (iv); phantomic12 research
+ * note, components (3) and (4)):
+ *   out[b][hq][:] = sum_t p_t * vhat_t,h with p_t = exp(logits - M)/L and
+ * vhat the dequantized value (off_t + half_t*L[code], outliers replaced).  The sum over
+ * the outlier entries of each output is taken in a fixed order, so two calls on the same
+ * inputs return the same bits.
  *   logits, ml from the two calls above; out float [B][Hq][D]
  *   part   float scratch [B][Hq][splits][D] (per-split partial sums, summed in
  *          split order)
@@ -244,7 +259,10 @@ int kvq_dequantize(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codeboo
                    uint16_t* vhat, void* stream);
 
 /*
- * Uncompressed comparison kernel: decode attention over an fp16 cache.
+ * Uncompressed comparison kernel: decode attention over an fp16 cache.  The pages
+ * measure the KVQuant kernels against fp16 matrix-vector multiplication (study.space
+ * summary, "~1.7x" over the fp16 baseline); this is that baseline, written for the
+ * same layouts and the same RoPE reading, so the two can be timed side by side.
  *   K, V fp16 [B][T_stride][Hkv][D] (keys pre-RoPE, RoPE applied on the fly);
  *   len int32 [B]; q, qpos as kvq_decode_qk; out float [B][Hq][D];
  *   workspace of kvq_decode_workspace bytes for the same cfg/max_len/splits.

@@ -16,8 +16,8 @@ Sources (pages on KVQuant, arXiv 2401.18079):
     non-uniform datatype, with outliers isolated per vector rather than
     globally; 3-bit vs fp16 is a ~5.3x cache reduction.
 
-Where the pages leave a step open the plain reading below is used (each is
-listed in the design doc with its ID):
+Where the pages leave a step open the plain reading below is used; each has an
+ID (R1-R10) by which the CUDA library's notes refer to it:
   R1 vector: a key vector is one channel (b, h, c) over the calibration tokens;
      a value vector is one token's full row over all kv heads (n = Hkv*D).
   R2 outlier count: k = floor(f*N/2 + 1/2) per side (capped at (N-1)//2);
