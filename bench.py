@@ -536,9 +536,11 @@ def run_kvq(args, rank, world):
 
     if rank != 0:
         return 0
-    # append: begin, stats, scan, write; qk: tables, qk, key outliers, split stats; merge;
-    # pv: pv, split sum, value outliers (the one-call path launches the same kernels)
-    launches_per_layer_step = 12
+    # append: begin, stats, scan, write; split path: qk (tables, qk, key outliers, split
+    # stats), merge, pv (pv, value outliers, split sum); one-call path for kv heads of one
+    # query head with 2/3-bit codes: tables, the fused kernel, split merge
+    fused = w.Hq == w.Hkv and w.bits <= 3
+    launches_per_layer_step = 4 + (8 if args.path == "split" else (3 if fused else 8))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,

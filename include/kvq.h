@@ -60,6 +60,11 @@ enum {
 #define KVQ_STATUS_NOT_EMPTY 4        /* a calibrating prefill met a non-empty sequence; skipped */
 #define KVQ_STATUS_WAIT_TIMEOUT 8     /* a decode kernel gave up waiting for its bulk copies; its
                                          outputs of that call are invalid */
+#define KVQ_STATUS_SMEM_LAYOUT 16     /* the fused decode kernel found its shared-memory window
+                                         based too high for its table layout; its outputs of that
+                                         call are invalid */
+#define KVQ_STATUS_CODEBOOK 32        /* the fused decode kernel met value levels that are not of
+                                         the (u << 16) | u form; its outputs are invalid */
 
 #define KVQ_CHUNK 64 /* tokens per outlier chunk */
 

@@ -97,4 +97,10 @@ int check_cfg(const kvq_cfg* cfg);
 int check_cache(const kvq_cfg* cfg, const kvq_cache* c);
 int check_codebook(const kvq_codebook* cb);
 size_t align_up(size_t x);
+// Fused single-pass decode (kvq_fused.cu): shapes it covers, and its launch.
+int fused_supported(const kvq_cfg* cfg);
+int run_fused(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
+              const kvq_codebook* cbV, const float* qr, const float2* thi, const float2* tlo,
+              const float* zk, int max_len, int S, int Ls, float2* st, float* po,
+              cudaStream_t stream);
 }  // namespace kvq_host

@@ -16,18 +16,15 @@
 // to the logits before the softmax statistics are taken, value outliers add
 // p (x - zhat) to the output after the merge.
 #include "kvq_common.cuh"
+#include "kvq_device.cuh"
 
 using namespace kvq;
 
 namespace {
 
-constexpr float kInvSqrtD = 0.08838834764831845f;  // 1/sqrt(128)
-constexpr int kMaxG = 16;                          // query heads per kv head
 constexpr int kThreads = 256;                      // 8 warps = 16 half-warps
 constexpr int kQuads = kThreads / 16;              // token quads per chunk (64 tokens)
 constexpr int kStages = 4;                         // chunks in the bulk-copy ring
-constexpr uint32_t kWaitLimit = 1u << 24;          // mbarrier polls before giving up
-constexpr int kTrigLo = 256;                       // trig tables: t = 256 * hi + lo
 
 __device__ inline float warp_sum(float v) {
 #pragma unroll
@@ -41,120 +38,6 @@ __host__ __device__ inline int split_len(int max_len, int S) {
     per = (per + kChunk - 1) / kChunk * kChunk;
     return per < kChunk ? kChunk : per;
 }
-
-// ---------------------------------------------------------------------------------
-// mbarrier + bulk copy (PTX).
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
-                 : "memory");
-}
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-                 "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait for the phase with the given parity; false when the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    for (uint32_t it = 0; it < kWaitLimit; ++it)
-        if (mbar_try_wait(bar, parity)) return true;
-    return false;
-}
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
-// ---------------------------------------------------------------------------------
-// Packed f32x2 helpers (fma.rn.f32x2: two independent binary32 FMAs per instruction).
-struct f2 {
-    float x, y;
-};
-__device__ __forceinline__ unsigned long long pk(float a, float b) {
-    unsigned long long r;
-    asm("mov.b64 %0, {%1,%2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-__device__ __forceinline__ f2 upk(unsigned long long v) {
-    f2 r;
-    asm("mov.b64 {%0,%1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-    return r;
-}
-__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
-                                                   unsigned long long c) {
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
-    return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
-}
-template <int BITS>
-struct Fmt {
-    static constexpr int FW = 2 * BITS;  // field width (codes of c and c + 64)
-    static constexpr int NT = 1 << FW;   // entries of a pair table
-    static constexpr int BW = 16 * BITS; // words of a code block
-};
-
-// A word holding slot F's field (bit FW*F of the lane group's string w[0 .. BITS)) at bit P
-// (the other bits are junk, masked by the caller).
-template <int BITS, int F, int P>
-__device__ __forceinline__ uint32_t field_to(const uint32_t (&w)[BITS]) {
-    constexpr int FW = 2 * BITS;
-    constexpr int O = FW * F;
-    constexpr int wi = O >> 5, sh = O & 31;
-    if constexpr (sh + FW <= 32) {
-        if constexpr (sh >= P)
-            return w[wi] >> (sh - P);
-        else
-            return w[wi] << (P - sh);
-    } else {
-        static_assert(sh >= P, "a field that crosses words starts above bit P");
-        return __funnelshift_r(w[wi], w[wi + 1], sh - P);
-    }
-}
-
-// Shared-memory load at a 32-bit shared-window address plus an immediate byte offset.
-template <int IMM>
-__device__ __forceinline__ unsigned long long lds64(uint32_t addr) {
-    unsigned long long d;
-    asm("ld.shared.b64 %0, [%1+%2];" : "=l"(d) : "r"(addr), "n"(IMM));
-    return d;
-}
-
-// Shared-memory table load at a byte offset.
-__device__ __forceinline__ unsigned long long tld(const uint8_t* tab, uint32_t off) {
-    return *reinterpret_cast<const unsigned long long*>(tab + off);
-}
-
 
 // Consumer warps of a CTA (one more warp streams the input) and heads per consumer warp.
 // With four query heads per CTA two warps share each quad pair (two heads each): twice the
@@ -173,14 +56,6 @@ __device__ __forceinline__ bool out_owner(int i) {
     return HW == 4 ? true : (HW == 2 ? !(i & 1) : !(i & 3));
 }
 
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// After an abandoned wait: let every copy still in flight land before the CTA exits.
-__device__ inline void drain_chunks(uint64_t* bars, int from, int to) {
-    for (int cc = from; cc < to; ++cc) mbar_wait(bars + cc % kStages, (cc / kStages) & 1);
-}
 
 // ---------------------------------------------------------------------------------
 // Shared-memory plans (host and device).
@@ -246,11 +121,6 @@ struct Streamer {
                       bytes, bar);
     }
 };
-
-// (cos, sin) of t * theta_p from the per-call tables: hi[t / 256] rotated by lo[t % 256].
-__device__ __forceinline__ float2 trig_at(const float2* thi, const float2* tlo, int t, int p) {
-    return cmul(thi[(t / kTrigLo) * 64 + p], tlo[(t % kTrigLo) * 64 + p]);
-}
 
 // ---------------------------------------------------------------------------------
 // Per-call tables: rotated, scaled queries qr [B][Hq][128]; trig tables hi [nhi][64] =
@@ -502,7 +372,7 @@ __global__ void __launch_bounds__(qk_warps(HPC) * 32 + 32, 1)
     }
     __syncthreads();
     // after an abandoned wait, copies of the last stages issued may still be in flight
-    if (*flag && tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1]);
+    if (*flag && tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1], kStages);
 }
 
 // ---------------------------------------------------------------------------------
@@ -741,33 +611,45 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
     }
     __syncthreads();
     // after an abandoned wait, copies of the last stages issued may still be in flight
-    if (*flag && tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1]);
+    if (*flag && tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1], kStages);
 }
 
 // ---------------------------------------------------------------------------------
-// Outlier kernels.  A block takes kOutChunks 64-token chunks of one (sequence, kv head) list
-// and stages their chunk pointers in shared memory; each warp walks a contiguous range of the
-// block's entries, 32 kOutBatch at a time.  An entry holds only its token's offset within its
-// chunk: a warp keeps the chunk of its current position and, per window, counts for each of
-// its entries the chunk boundaries that fall inside the window (about three per 128 entries
-// at the densities of interest).  A lane's kOutBatch entries are gathered together.
+// Outlier kernels.  A block takes up to kOutChunks 64-token chunks of one (sequence, kv head)
+// list and stages their chunk pointers in shared memory; a warp walks a contiguous range of
+// the block's entries, 32 kOutBatch at a time.  An entry holds only its token's offset within
+// its chunk: a warp keeps the chunk of its current position and, per window, counts for each
+// of its entries the chunk boundaries that fall inside the window.  A lane's kOutBatch entries
+// are gathered together; lane l's u-th entry is entry E + 32u + l of the window, so slice u
+// of a window is 32 consecutive entries in list order.
+//
+// Both kernels give the same bits on every run.  The key side gives each warp whole chunks
+// (a token's entries never straddle two warps), sums each token's corrections in list order
+// with a segmented scan across the lanes (a token's entries are contiguous: the list is
+// sorted by token) and lets one lane add the sum to the logit.  The value side adds each
+// entry's term into 2^-40 fixed-point block sums with integer atomics (integer addition is
+// associative, so their order does not matter), then adds each block sum once into its
+// split's PV partial before the partials are summed in split order.
 constexpr int kOutThreads = 256;  // threads per block of the outlier kernels
-constexpr int kOutChunks = 64;    // chunks per block
+constexpr int kOutChunks = 64;    // chunks per staged window of chunk pointers
 constexpr int kOutBatch = 4;      // entries a lane gathers at once
+constexpr float kFixScale = 1099511627776.0f;      // 2^40
+constexpr double kFixInv = 1.0 / 1099511627776.0;  // 2^-40
 
 struct OutRange {
-    uint32_t lo, hi;  // entries [lo, hi) of the block's chunks
+    uint32_t lo, hi;  // entries [lo, hi) of the staged chunks
     int m0, n;        // first chunk and number of chunks
 };
 
-// Stages min(cp[m0 + j], cnt), j <= n, in cps; ends with a block barrier.
+// Stages min(cp[m0 + j], cnt), j <= n, n = chunks of [m0, m_end) below len (at most
+// kOutChunks), in cps; ends with a block barrier.
 __device__ __forceinline__ OutRange stage_chunks(const uint32_t* __restrict__ cp, uint32_t cnt,
-                                                 int len, uint32_t* cps) {
+                                                 int len, int m0, int m_end, uint32_t* cps) {
     OutRange r;
-    r.m0 = blockIdx.x * kOutChunks;
-    r.n = max(0, min((len + kChunk - 1) / kChunk - r.m0, kOutChunks));
+    r.m0 = m0;
+    r.n = max(0, min(min((len + kChunk - 1) / kChunk, m_end) - m0, kOutChunks));
     if (r.n)
-        for (int j = threadIdx.x; j <= r.n; j += blockDim.x) cps[j] = min(cp[r.m0 + j], cnt);
+        for (int j = threadIdx.x; j <= r.n; j += blockDim.x) cps[j] = min(cp[m0 + j], cnt);
     __syncthreads();
     r.lo = r.n ? cps[0] : 0u;
     r.hi = r.n ? cps[r.n] : 0u;
@@ -780,19 +662,31 @@ struct EntryWalker {
     static constexpr uint32_t W = 32 * kOutBatch;
     uint32_t E, Ee;
     int cur, n, m0;
-    __device__ __forceinline__ EntryWalker(const OutRange& r, const uint32_t* cps) {
+    // chunk_aligned: warp w takes whole chunks [w*n/nw, (w+1)*n/nw); otherwise an even share
+    // of the entries
+    __device__ __forceinline__ EntryWalker(const OutRange& r, const uint32_t* cps,
+                                           bool chunk_aligned) {
         const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-        const uint32_t span = ((r.hi - r.lo + nw - 1) / nw + 31) & ~31u;
-        E = r.lo + (uint32_t)warp * span;
-        Ee = min(r.hi, E + span);
         n = r.n;
         m0 = r.m0;
-        cur = 0;  // chunk of entry E: the largest j < n with cps[j] <= E
-        if (E < Ee) {
+        if (chunk_aligned) {
+            const int ca = warp * n / nw, cb = (warp + 1) * n / nw;
+            E = n ? cps[ca] : 0u;
+            Ee = n ? cps[cb] : 0u;
+            cur = ca;
+        } else {
+            const uint32_t span = ((r.hi - r.lo + nw - 1) / nw + 31) & ~31u;
+            E = r.lo + (uint32_t)warp * span;
+            Ee = min(r.hi, E + span);
+            cur = 0;  // chunk of entry E: the largest j < n with cps[j] <= E
+            if (E < Ee) {
 #pragma unroll
-            for (int step = kOutChunks / 2; step; step >>= 1)
-                if (cur + step < n && cps[cur + step] <= E) cur += step;
+                for (int step = kOutChunks / 2; step; step >>= 1)
+                    if (cur + step < n && cps[cur + step] <= E) cur += step;
+            }
         }
+        // entries before E in the first chunk belong to an earlier warp; skip empty chunks
+        while (cur + 1 < n && cps[cur + 1] <= E) ++cur;
     }
     __device__ __forceinline__ bool next(const uint32_t* cps, const uint32_t* __restrict__ ent,
                                          int (&t)[kOutBatch], uint32_t (&w)[kOutBatch]) {
@@ -820,9 +714,21 @@ struct EntryWalker {
     }
 };
 
-// Key outliers: logit(t, hq) += (x - zhat) * r, r the component of the rotated query that
-// meets the outlier's channel after the key is rotated to t.  G query heads per kv head (0:
-// read from cfg).
+// Inclusive scan of v over the lanes, restarted wherever the key t changes (keys contiguous).
+__device__ __forceinline__ float seg_scan(float v, int t, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const float vv = __shfl_up_sync(0xffffffffu, v, off);
+        const int tt = __shfl_up_sync(0xffffffffu, t, off);
+        if (lane >= off && tt == t) v += vv;
+    }
+    return v;
+}
+
+// Key outliers: logit(t, hq) += sum over the token's entries of (x - zhat) * r, r the
+// component of the rotated query that meets the outlier's channel after the key is rotated to
+// t.  G query heads per kv head (0: read from cfg).  The running sum of a token whose entries
+// continue into the next slice is carried in carry[warp][head].
 template <int G>
 __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
     kvq_cfg cfg, kvq_cache c, const float* __restrict__ qr, const float2* __restrict__ thi,
@@ -836,40 +742,54 @@ __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
     __shared__ uint32_t cps[kOutChunks + 1];
     __shared__ float zks[kD];
     __shared__ float qs[(G ? G : kMaxG) * kD];
+    __shared__ float carry[kOutThreads / 32][G ? G : kMaxG];
     for (int e = threadIdx.x; e < kD; e += blockDim.x) zks[e] = zk[(size_t)li * kD + e];
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x)
         qs[e] = qr[((size_t)b * cfg.Hq + h * g) * kD + e];
-    const OutRange r = stage_chunks(cp, c.kcount[li], len, cps);  // barrier covers the above
+    const int m0 = blockIdx.x * kOutChunks;
+    const OutRange r = stage_chunks(cp, c.kcount[li], len, m0, m0 + kOutChunks, cps);
     float* lb0 = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
     const size_t T_max = cfg.T_max;
-    EntryWalker wk(r, cps);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    EntryWalker wk(r, cps, true);
+    int ct = -1;  // token of the carried sums (warp-uniform)
     int t[kOutBatch];
     uint32_t w[kOutBatch];
     while (wk.next(cps, ent, t, w)) {
-        bool ok[kOutBatch];
         float2 cs[kOutBatch];
 #pragma unroll
         for (int u = 0; u < kOutBatch; ++u) {
-            ok[u] = (unsigned)t[u] < (unsigned)len;
-            cs[u] = trig_at(thi, tlo, ok[u] ? t[u] : 0, (int)(w[u] & 63u));
+            if ((unsigned)t[u] >= (unsigned)len) t[u] = -1;  // past the clipped length
+            cs[u] = trig_at(thi, tlo, t[u] >= 0 ? t[u] : 0, (int)(w[u] & 63u));
         }
 #pragma unroll
         for (int u = 0; u < kOutBatch; ++u) {
+            const int tu = t[u];
             const int ch = (int)(w[u] & 127u), p = ch & 63;
-            const float d = h2f((uint16_t)(w[u] >> 16)) - zks[ch];
+            const float d = tu >= 0 ? h2f((uint16_t)(w[u] >> 16)) - zks[ch] : 0.0f;
             // rotate-half: channel c < 64 meets (cos, sin) . (q_p, q_p+64), c >= 64 the other
             const float sa = ch < 64 ? cs[u].x : -cs[u].y, sb = ch < 64 ? cs[u].y : cs[u].x;
-#pragma unroll
-            for (int a = 0; a < (G ? G : 1); ++a) {
-                const float rr = fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
-                if (ok[u]) atomicAdd(&lb0[a * T_max + t[u]], d * rr);
+            const int t0 = __shfl_sync(0xffffffffu, tu, 0);
+            const int tn = __shfl_down_sync(0xffffffffu, tu, 1);
+            const bool tail = tu >= 0 && lane < 31 && tn != tu;
+            const bool flush = ct >= 0 && t0 != ct;  // the carried token ended with the last slice
+            for (int a = 0; a < g; ++a) {
+                float v = d * fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
+                if (ct >= 0 && lane == 0) {
+                    const float cv = carry[warp][a];
+                    if (flush) lb0[a * T_max + ct] += cv;
+                    else v += cv;
+                }
+                v = seg_scan(v, tu, lane);
+                if (tail) lb0[a * T_max + tu] += v;
+                if (lane == 31) carry[warp][a] = v;
             }
-            for (int a = 1; !G && a < g; ++a) {
-                const float rr = fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
-                if (ok[u]) atomicAdd(&lb0[a * T_max + t[u]], d * rr);
-            }
+            __syncwarp();
+            ct = __shfl_sync(0xffffffffu, tu, 31);
         }
     }
+    if (ct >= 0 && lane == 0)
+        for (int a = 0; a < g; ++a) lb0[a * T_max + ct] += carry[warp][a];
 }
 
 // ---------------------------------------------------------------------------------
@@ -1112,7 +1032,7 @@ __global__ void __launch_bounds__(pv_warps(HPC) * 32 + 32, 1)
     }
     __syncthreads();
     if (*flag) {
-        if (tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1]);
+        if (tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1], kStages);
         return;
     }
     // partial sums of the 16 quads -> the split's output (the ring is idle now)
@@ -1318,7 +1238,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
     }
     __syncthreads();
     if (*flag) {
-        if (tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1]);
+        if (tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1], kStages);
         return;
     }
     // partial sums of the 32 half-warps -> the split's output (the ring is idle now)
@@ -1346,20 +1266,23 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 }
 
 // ---------------------------------------------------------------------------------
-// Value outliers: out(hq, c) += p(t, hq) (x - zhat_t), p = exp(l - M) / L from the merged
-// statistics, zhat_t = off_t + half_t L[encode(normalize(0))]; sums gather in shared memory
-// and a block adds them to the output once.  G as for the key outliers.
+// Value outliers: part(s, hq, c) += sum over the split's entries of p(t, hq) (x - zhat_t),
+// p = exp(l - M) / L from the merged statistics, zhat_t = off_t + half_t L[encode(normalize(0))].
+// One block per (split, sequence, kv head) walks the split's chunks kOutChunks at a time; each
+// term goes into a 2^-40 fixed-point sum per (head, channel) with an integer atomic, and one
+// thread adds each sum to the split's partial.  |p (x - zhat)| < 2^18 and the p of a sequence
+// sum to 1, so a block's sums stay below 2^58.  G as for the key outliers.
 template <int BITS, int G>
 __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
     kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
-    const float2* __restrict__ ml, int max_len, float* __restrict__ out) {
+    const float2* __restrict__ ml, int Ls, int S, int max_len, float* __restrict__ part) {
     constexpr int NB = (1 << BITS) - 1;
-    const int li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
+    const int s = blockIdx.x, li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
     const int g = G ? G : cfg.Hq / cfg.Hkv;
     const int len = min(c.len[b], max_len);
     const uint32_t* cp = c.vchunk + (size_t)li * (nchunks(cfg.T_max) + 1);
     const uint32_t* ent = c.vout + (size_t)li * cfg.out_cap_v;
-    __shared__ float acc[(G ? G : kMaxG) * kD];
+    __shared__ unsigned long long acc[(G ? G : kMaxG) * kD];
     __shared__ float bnd[16], lev[16];
     __shared__ float2 mls[kMaxG];  // (M, 1 / L), 1 / L = 0 for an empty row
     __shared__ uint32_t cps[kOutChunks + 1];
@@ -1369,55 +1292,63 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
         const float2 v = ml[(size_t)b * cfg.Hq + h * g + threadIdx.x];
         mls[threadIdx.x] = make_float2(v.x, v.y > 0.0f ? 1.0f / v.y : 0.0f);
     }
-    for (int e = threadIdx.x; e < g * kD; e += blockDim.x) acc[e] = 0.0f;
-    const OutRange r = stage_chunks(cp, c.vcount[li], len, cps);  // barrier covers the above
-    if (r.lo >= r.hi) return;
-    float bd[NB];
-#pragma unroll
-    for (int j = 0; j < NB; ++j) bd[j] = bnd[j];
+    for (int e = threadIdx.x; e < g * kD; e += blockDim.x) acc[e] = 0ull;
     const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
     const float* lrow = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
     const size_t T_max = cfg.T_max;
-    EntryWalker wk(r, cps);
-    int t[kOutBatch];
-    uint32_t w[kOutBatch];
-    while (wk.next(cps, ent, t, w)) {
-        bool ok[kOutBatch];
-        float2 vp[kOutBatch];
-        float l0[kOutBatch];
+    const int mb = s * (Ls / kChunk), me = min(mb + Ls / kChunk, (len + kChunk - 1) / kChunk);
+    const uint32_t cnt = c.vcount[li];
+    bool any = false;
+    for (int m0 = mb; m0 < me; m0 += kOutChunks) {
+        __syncthreads();  // the previous window's cps are no longer read
+        const OutRange r = stage_chunks(cp, cnt, len, m0, me, cps);  // barrier covers the above
+        if (r.lo >= r.hi) continue;
+        any = true;
+        float bd[NB];
 #pragma unroll
-        for (int u = 0; u < kOutBatch; ++u) {
-            ok[u] = (unsigned)t[u] < (unsigned)len;
-            const int tt = ok[u] ? t[u] : 0;
-            vp[u] = vpar[tt];
-            l0[u] = lrow[tt];
-        }
+        for (int j = 0; j < NB; ++j) bd[j] = bnd[j];
+        EntryWalker wk(r, cps, false);
+        int t[kOutBatch];
+        uint32_t w[kOutBatch];
+        while (wk.next(cps, ent, t, w)) {
+            bool ok[kOutBatch];
+            float2 vp[kOutBatch];
+            float l0[kOutBatch];
 #pragma unroll
-        for (int u = 0; u < kOutBatch; ++u) {
-            // the dense value stored at the outlier: the code of 0 in the token's normalization
-            const float xn = normalize(0.0f, vp[u].x, vp[u].y);
-            int code = 0;
-#pragma unroll
-            for (int j = 0; j < NB; ++j) code += xn > bd[j];
-            const float d = h2f((uint16_t)(w[u] >> 16)) - fmaf(vp[u].y, lev[code], vp[u].x);
-            const int ch = (int)(w[u] & 127u);
-#pragma unroll
-            for (int a = 0; a < (G ? G : 1); ++a) {
-                const float2 mi = mls[a];
-                if (ok[u] && mi.y > 0.0f)
-                    atomicAdd(&acc[a * kD + ch], __expf(l0[u] - mi.x) * mi.y * d);
+            for (int u = 0; u < kOutBatch; ++u) {
+                ok[u] = (unsigned)t[u] < (unsigned)len;
+                const int tt = ok[u] ? t[u] : 0;
+                vp[u] = vpar[tt];
+                l0[u] = lrow[tt];
             }
-            for (int a = 1; !G && a < g; ++a) {
-                const float2 mi = mls[a];
-                const float la = lrow[a * T_max + (ok[u] ? t[u] : 0)];
-                if (ok[u] && mi.y > 0.0f) atomicAdd(&acc[a * kD + ch], __expf(la - mi.x) * mi.y * d);
+#pragma unroll
+            for (int u = 0; u < kOutBatch; ++u) {
+                // the dense value stored at the outlier: the code of 0 in the token's normalization
+                const float xn = normalize(0.0f, vp[u].x, vp[u].y);
+                int code = 0;
+#pragma unroll
+                for (int j = 0; j < NB; ++j) code += xn > bd[j];
+                const float d = h2f((uint16_t)(w[u] >> 16)) - fmaf(vp[u].y, lev[code], vp[u].x);
+                const int ch = (int)(w[u] & 127u);
+                for (int a = 0; a < g; ++a) {
+                    const float2 mi = mls[a];
+                    const float la = a == 0 ? l0[u] : lrow[a * T_max + (ok[u] ? t[u] : 0)];
+                    if (ok[u] && mi.y > 0.0f) {
+                        const float v = __expf(la - mi.x) * mi.y * d;
+                        atomicAdd(&acc[a * kD + ch], (unsigned long long)__float2ll_rn(v * kFixScale));
+                    }
+                }
             }
         }
     }
     __syncthreads();
+    if (!any) return;
     for (int e = threadIdx.x; e < g * kD; e += blockDim.x) {
-        const float v = acc[e];
-        if (v != 0.0f) atomicAdd(&out[((size_t)b * cfg.Hq + h * g + e / kD) * kD + e % kD], v);
+        const long long v = (long long)acc[e];
+        if (v != 0) {
+            float* pp = part + (((size_t)b * cfg.Hq + h * g + e / kD) * S + s) * kD + e % kD;
+            *pp += (float)((double)v * kFixInv);
+        }
     }
 }
 
@@ -1789,14 +1720,14 @@ static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
                                                             (const float2*)ml, Ls, S, max_len,
                                                             kvb, part);
     }
-    k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
-    const int nch = (max_len + kChunk - 1) / kChunk;
-    dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
+    dim3 go(S, cfg->B * cfg->Hkv);
     const bool mha = cfg->Hq == cfg->Hkv;
     auto vo = cfg->bits == 2 ? (mha ? k_value_outliers<2, 1> : k_value_outliers<2, 0>)
             : cfg->bits == 3 ? (mha ? k_value_outliers<3, 1> : k_value_outliers<3, 0>)
                              : (mha ? k_value_outliers<4, 1> : k_value_outliers<4, 0>);
-    vo<<<go, kOutThreads, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, max_len, out);
+    vo<<<go, kOutThreads, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls, S, max_len,
+                                   part);
+    k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
     return record_cuda(cudaGetLastError());
 }
 
@@ -1858,6 +1789,18 @@ extern "C" int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache,
     w += align_up(BH * S * kD * 4);
     const QKTables T = qk_tables(cfg, max_len, w);
     cudaStream_t st = (cudaStream_t)stream;
+    if (fused_supported(cfg)) {
+        // one pass: per-call tables, the fused kernel's per-split (m, l, o), the split merge
+        const int n = cfg->B * cfg->Hq * 64 + T.nhi * 64 + kTrigLo * 64 + cfg->B * cfg->Hkv * kD;
+        k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi, T.qr,
+                                                        T.thi, T.tlo, T.zk);
+        if ((e = record_cuda(cudaGetLastError()))) return e;
+        if ((e = run_fused(cfg, cache, cbK, cbV, T.qr, T.thi, T.tlo, T.zk, max_len, S, Ls,
+                           (float2*)stats, part, st)))
+            return e;
+        k_attn_merge<<<(int)BH, kD, 0, st>>>(S, (const float2*)stats, part, out);
+        return record_cuda(cudaGetLastError());
+    }
     if ((e = run_qk(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, T, st))) return e;
     if ((e = kvq_softmax_merge(cfg, stats, S, ml, stream))) return e;
     return run_pv(cfg, cache, cbV, logits, ml, max_len, out, part, S, Ls, st);

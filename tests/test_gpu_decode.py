@@ -152,3 +152,62 @@ def test_fp16_comparison_kernel(name, over, T, plen):
         _, _, ref = O.decode_attention(q16[b], int(qpos[b]), K16[b, : pl[b]], V16[b, : pl[b]],
                                        w.rope_theta)
         assert np.abs(o[b] - ref).max() <= OUT_ATOL
+
+
+# many outliers (5 %), ragged lengths across several 256-token stages and 64-token chunks
+HEAVY = [
+    ("llama7b_layer_32k", dict(B=3, Hq=4, Hkv=4, f=0.05), 1500, [1500, 777, 3], 1),
+    ("batched_8x8k", dict(B=2, Hq=2, Hkv=2, bits=2, f=0.05), 1300, [1300, 1025], 0),
+]
+
+
+@pytest.mark.parametrize("name,over,T,plen,appends", HEAVY)
+@pytest.mark.parametrize("splits", [0, 1, 4])
+def test_outlier_heavy(name, over, T, plen, appends, splits):
+    import torch
+    import long_context_decode_nuq_b200 as K
+    w, o, g, dK, dV, dq, dpos, refs, _, _ = _setup(name, over, T, plen, appends)
+    max_len = int(o.len.max())
+    ws = torch.empty(K.kvq_decode_workspace(g.cfg, max_len, splits), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty((w.B, w.Hq, w.D), device="cuda")
+    K.kvq_decode_attention(g, dK, dV, dq, dpos, max_len, out, ws, splits)
+    torch.cuda.synchronize()
+    _check_out(w, out.cpu().numpy(), refs)
+    assert K.kvq_get_status(g) == 0
+
+
+@pytest.mark.parametrize("name,over,T,plen,appends", [CASES[1], CASES[4], CASES[5], HEAVY[0]])
+def test_decode_is_deterministic(name, over, T, plen, appends):
+    """Two calls on the same inputs give the same bits: one-call path and the three calls."""
+    import torch
+    import long_context_decode_nuq_b200 as K
+    w, o, g, dK, dV, dq, dpos, refs, _, _ = _setup(name, over, T, plen, appends)
+    max_len = int(o.len.max())
+    ws = torch.empty(K.kvq_decode_workspace(g.cfg, max_len, 0), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(2):
+        out = torch.empty((w.B, w.Hq, w.D), device="cuda")
+        ws.fill_(0x55)
+        K.kvq_decode_attention(g, dK, dV, dq, dpos, max_len, out, ws, 0)
+        torch.cuda.synchronize()
+        outs.append(out.cpu().numpy().view(np.uint32))
+    assert np.array_equal(outs[0], outs[1])
+    S = K.kvq_decode_splits(g.cfg, max_len)
+    res = []
+    for _ in range(2):
+        logits = torch.zeros((w.B, w.Hq, g.cfg.T_max), device="cuda")
+        stats = torch.empty((w.B, w.Hq, S, 2), device="cuda")
+        ml = torch.empty((w.B, w.Hq, 2), device="cuda")
+        out = torch.empty((w.B, w.Hq, w.D), device="cuda")
+        part = torch.empty((w.B, w.Hq, S, w.D), device="cuda")
+        qws = torch.empty(K.kvq_decode_qk_workspace(g.cfg, max_len), dtype=torch.uint8,
+                          device="cuda")
+        K.kvq_decode_qk(g, dK, dq, dpos, max_len, logits, stats, S, qws)
+        K.kvq_softmax_merge(g.cfg, stats, S, ml)
+        K.kvq_decode_pv(g, dV, logits, ml, max_len, out, part, S)
+        torch.cuda.synchronize()
+        res.append((logits.cpu().numpy().view(np.uint32), out.cpu().numpy().view(np.uint32)))
+    assert np.array_equal(res[0][0], res[1][0])
+    assert np.array_equal(res[0][1], res[1][1])
+    assert K.kvq_get_status(g) == 0
