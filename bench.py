@@ -47,6 +47,10 @@ def parse():
     p.add_argument("--no-fp16", action="store_true")
     p.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
     p.add_argument("--tokens", type=int, default=0, help="override the cached token count")
+    p.add_argument("--shard", default="tokens", choices=["tokens", "replicas"],
+                   help="N > 1: tokens = one sequence of N x T tokens, rank r holding tokens "
+                        "[r T, (r+1) T) (partials all-gathered and merged per layer); replicas = "
+                        "an independent sequence per rank")
     return p.parse_args()
 
 
@@ -265,7 +269,9 @@ def run_reference(args, rank, world):
         "config": {"workload": w.name, "layers": w.layers, "B": w.B, "kv_heads": w.Hkv,
                    "head_dim": w.D, "T": w.T, "bits": w.bits, "outlier_frac": w.f},
         "cpu_baseline": {"value": val, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-                         "sample": samples[-1]},
+                         "sample": samples[-1],
+                         "extrapolated": "KV tokens/s of a sampled slice, not a run of the "
+                                         "whole workload"},
         "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -290,11 +296,20 @@ def run_kvq(args, rank, world):
         over["T"] = args.tokens
     w = synth.workload(args.workload, **over)
     steps_total = args.warmup + args.steps
+    e2e_steps = min(args.steps, 10)
+    sharded = world > 1 and args.shard == "tokens"
+    shard_n = world if sharded else 1
     if w.T + steps_total + 16 > w.T_gen:
         w = synth.workload(args.workload, appends=1, steps=steps_total + 16, **over)
     layers = w.layers
-    T0 = w.T
-    e2e_steps = min(args.steps, 10)
+    T0 = w.T  # tokens held by this rank's caches
+    # the generator's token extent: the whole sequence when sharded (rank r holds its tokens
+    # [r T0, (r+1) T0), the last rank appends at positions N T0 + s)
+    w_gen = synth.workload(args.workload, appends=1, steps=steps_total + e2e_steps + 16,
+                           **{**over, "T": shard_n * T0})
+    t_base = rank * T0 if sharded else 0          # position of this rank's first token
+    pos0 = shard_n * T0                            # position of the first appended token
+    appends_here = (not sharded) or rank == world - 1
     T_max = T0 + steps_total + e2e_steps + 64
     # outlier lists are per (sequence, kv head): a key channel keeps ~f*T outliers, a token's
     # 2k value outliers spread over the Hkv heads; capacities are multiples of 8
@@ -302,8 +317,8 @@ def run_kvq(args, rank, world):
     kout_cap = ceil8(T_max * w.f * w.D * 1.25 + 4096)
     vout_cap = ceil8(T_max * 2 * math.floor(w.f * w.n / 2 + 0.5) / w.Hkv * 1.5 + 4096)
     cfg = K.make_cfg(w.B, w.Hq, w.Hkv, w.bits, T_max, w.f, w.rope_theta, kout_cap, vout_cap)
-    # a different synthetic sequence per rank (weak scaling)
-    layer_key = lambda l: rank_layer_key(l, rank)  # noqa: E731
+    # replicas: a different synthetic sequence per rank; sharded: one sequence split across ranks
+    layer_key = lambda l: rank_layer_key(l, 0 if sharded else rank)  # noqa: E731
 
     # replicas of the whole cache so that the timed inputs exceed L2 by a wide margin
     one_cache_bytes = sum(K.kvq_layout(cfg).values()) * layers
@@ -319,9 +334,9 @@ def run_kvq(args, rank, world):
     prefill_ms = []
     for r in range(R):
         for l in range(layers):
-            gen = DeviceGen(w, layer_key(l) + 100000 * r, device=dev)
-            gen.fill_k(kstage, 0, T0)
-            gen.fill_v(vstage, 0, T0)
+            gen = DeviceGen(w_gen, layer_key(l) + 100000 * r, device=dev)
+            gen.fill_k(kstage, t_base, T0)
+            gen.fill_v(vstage, t_base, T0)
             cb = []
             for samples in (synth.codebook_samples_k(w, layer_key(l)),
                             synth.codebook_samples_v(w, layer_key(l))):
@@ -356,16 +371,20 @@ def run_kvq(args, rank, world):
     qall = torch.empty((nL, steps_total, w.B, w.Hq, w.D), dtype=torch.float16, device=dev)
     for i in range(nL):
         r, l = divmod(i, layers)
-        gen = DeviceGen(w, layer_key(l) + 100000 * r, device=dev)
+        gen = DeviceGen(w_gen, layer_key(l) + 100000 * r, device=dev)
         for s in range(steps_total):
             tmp = torch.empty((w.B, 1, w.Hkv, w.D), dtype=torch.float16, device=dev)
-            gen.fill_k(tmp, T0 + s, 1)
+            gen.fill_k(tmp, pos0 + s, 1)
             knew[i, s] = tmp
-            gen.fill_v(tmp, T0 + s, 1)
+            gen.fill_v(tmp, pos0 + s, 1)
             vnew[i, s] = tmp
             gen.fill_q(qall[i, s], step=s)
-    qpos = torch.tensor([[T0 + s] * w.B for s in range(steps_total)], dtype=torch.int32,
+    qpos = torch.tensor([[pos0 + s] * w.B for s in range(steps_total)], dtype=torch.int32,
                         device=dev)
+    sdec = None
+    if sharded:
+        from long_context_decode_nuq_b200.shard import ShardedDecode
+        sdec = ShardedDecode(cfg, world, rank, dev)
     S = args.splits or K.kvq_decode_splits(cfg, T_max)
     aws = torch.empty(K.kvq_quantize_workspace(cfg, 1, 0), dtype=torch.uint8, device=dev)
     dws = torch.empty(K.kvq_decode_workspace(cfg, T_max, S), dtype=torch.uint8, device=dev)
@@ -385,17 +404,26 @@ def run_kvq(args, rank, world):
         ev_pool.append(e)
         return e
 
+    def local_len(s):
+        return T0 + s + 1 if appends_here else T0
+
     def layer_step(i, s, timing):
         c = caches[i]
         cbK, cbV = cbs[i]
-        max_len = T0 + s + 1
+        max_len = local_len(s)
         marks = [ev(), ev(), ev(), ev(), ev()] if timing else None
         if timing:
             marks[0].record()
-        K.kvq_quantize_append(c, cbK, cbV, knew[i, s], vnew[i, s], 1, None, 0, aws)
+        if appends_here:
+            K.kvq_quantize_append(c, cbK, cbV, knew[i, s], vnew[i, s], 1, None, 0, aws)
         if timing:
             marks[1].record()
-        if args.path == "split":
+        if sharded:
+            if timing:
+                marks[2].record()
+                marks[3].record()
+            sdec(c, cbK, cbV, qall[i, s], qpos[s], max_len, t_base, outs[i], dws, S)
+        elif args.path == "split":
             K.kvq_decode_qk(c, cbK, qall[i, s], qpos[s], max_len, logits, stats, S, qkws)
             if timing:
                 marks[2].record()
@@ -434,18 +462,20 @@ def run_kvq(args, rank, world):
     if world > 1:
         dist.barrier()
     n_layer_steps = len(marks)
-    tok_per_layer_step = [T0 + s + 1 for s in range(args.warmup, steps_total) for _ in range(layers)]
-    kv_tokens = w.B * sum(tok_per_layer_step) * world
-    value = aggregate_rate(w.B * sum(tok_per_layer_step), world, elapsed_ms)
+    # KV tokens attended per layer-step over the whole job: replicas, each rank its own
+    # sequence of T0 + s + 1 tokens; sharded, one sequence of N T0 + s + 1 tokens
+    tok_job = [(shard_n * T0 + s + 1) * (1 if sharded else world)
+               for s in range(args.warmup, steps_total) for _ in range(layers)]
+    value = w.B * sum(tok_job) / (elapsed_ms / 1e3)
     # per-kernel times
     t_app = sum(m[0].elapsed_time(m[1]) for m in marks)
     t_qk = sum(m[1].elapsed_time(m[2]) for m in marks)
     t_merge = sum(m[2].elapsed_time(m[3]) for m in marks)
     t_pv = sum(m[3].elapsed_time(m[4]) for m in marks)
-    Tmid = T0 + args.warmup + args.steps // 2 + 1
-    bm = bytes_model(w, Tmid, kcount, vcount, args.path)
+    Tmid = T0 + (args.warmup + args.steps // 2 + 1 if appends_here else 0)
+    bm = bytes_model(w, Tmid, kcount, vcount, "one-call" if sharded else args.path)
     hbm, peak_kind = peaks()
-    if args.path == "split":
+    if args.path == "split" and not sharded:
         kernels = {"k_qk": (t_qk, bm["qk"], "kvq_decode.cu"), "k_pv": (t_pv, bm["pv"], "kvq_decode.cu")}
     else:
         kernels = {"k_attn": (t_pv, bm["attn"], "kvq_decode.cu")}
@@ -468,7 +498,7 @@ def run_kvq(args, rank, world):
     d_k = torch.empty((nL, w.B, 1, w.Hkv, w.D), dtype=torch.float16, device=dev)
     d_v = torch.empty_like(d_k)
     # the e2e leg appends at fresh positions after the timed steps (replica 0)
-    qpos_e2e = torch.tensor([[T0 + steps_total + j] * w.B for j in range(e2e_steps)],
+    qpos_e2e = torch.tensor([[pos0 + steps_total + j] * w.B for j in range(e2e_steps)],
                             dtype=torch.int32, device=dev)
     torch.cuda.synchronize()
     e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -479,14 +509,17 @@ def run_kvq(args, rank, world):
     e_s.record()
     for j in range(e2e_steps):
         s = args.warmup + j
-        ml_len = T0 + steps_total + j + 1
+        ml_len = T0 + steps_total + j + 1 if appends_here else T0
         d_q.copy_(h_q[:, s], non_blocking=True)
         d_k.copy_(h_k[:, s], non_blocking=True)
         d_v.copy_(h_v[:, s], non_blocking=True)
         for i in range(layers):
             c = caches[i]
-            K.kvq_quantize_append(c, cbs[i][0], cbs[i][1], d_k[i], d_v[i], 1, None, 0, aws)
-            if args.path == "split":
+            if appends_here:
+                K.kvq_quantize_append(c, cbs[i][0], cbs[i][1], d_k[i], d_v[i], 1, None, 0, aws)
+            if sharded:
+                sdec(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j], ml_len, t_base, outs[i], dws, S)
+            elif args.path == "split":
                 K.kvq_decode_qk(c, cbs[i][0], d_q[i], qpos_e2e[j], ml_len, logits, stats, S, qkws)
                 K.kvq_softmax_merge(cfg, stats, S, mlb)
                 K.kvq_decode_pv(c, cbs[i][1], logits, mlb, ml_len, outs[i], part, S)
@@ -499,8 +532,9 @@ def run_kvq(args, rank, world):
     e_e.record()
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world, dev)
-    e2e_tokens = w.B * sum(T0 + steps_total + j + 1 for j in range(e2e_steps)) * layers
-    e2e_value = aggregate_rate(e2e_tokens, world, e2e_ms)
+    e2e_tokens = w.B * sum((shard_n * T0 + steps_total + j + 1) * (1 if sharded else world)
+                           for j in range(e2e_steps)) * layers
+    e2e_value = e2e_tokens / (e2e_ms / 1e3)
 
     # ---- uncompressed fp16 comparison kernel on one layer (last staged K/V)
     fp16 = None
@@ -522,17 +556,24 @@ def run_kvq(args, rank, world):
         torch.cuda.synchronize()
         fms = f0.elapsed_time(f1) / nrep
         fbytes = 2 * w.B * T0 * w.Hkv * w.D * 2
-        fp16 = {"ms_per_layer": fms, "GB/s": fbytes / (fms / 1e3) / 1e9,
+        f_gbs = fbytes / (fms / 1e3) / 1e9
+        hbm_peak = peaks()[0]
+        # the ratio is quoted only next to the fp16 kernel's own fraction of peak: a slow fp16
+        # kernel would inflate it; the fp16 cache's time at peak bandwidth bounds it honestly
+        fp16 = {"ms_per_layer": fms, "GB/s": f_gbs, "frac_of_peak": f_gbs / hbm_peak,
                 "kv_tokens_per_s": w.B * T0 / (fms / 1e3),
                 "quantized_ms_per_layer": step_attn_ms,
-                "speedup_quantized_vs_fp16": fms / step_attn_ms}
+                "speedup_quantized_vs_fp16": fms / step_attn_ms,
+                "speedup_vs_fp16_at_peak": (fbytes / (hbm_peak * 1e9) * 1e3) / step_attn_ms,
+                "layers_timed": 1}
 
     # ---- CPU oracle baseline (rank 0, N = 1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v_cpu, smp = cpu_oracle_sample(w)
         cpu = {"value": v_cpu, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-               "sample": smp}
+               "sample": smp, "extrapolated": "KV tokens/s of a sampled slice (one layer, "
+               "1,024 tokens), not a run of the whole workload"}
 
     if rank != 0:
         return 0
@@ -540,7 +581,8 @@ def run_kvq(args, rank, world):
     # stats), merge, pv (pv, value outliers, split sum); one-call path for kv heads of one
     # query head with 2/3-bit codes: tables, the fused kernel, split merge
     fused = w.Hq == w.Hkv and w.bits <= 3
-    launches_per_layer_step = 4 + (8 if args.path == "split" else (3 if fused else 8))
+    launches_per_layer_step = (4 if appends_here else 0) + (
+        8 if args.path == "split" and not sharded else (3 if fused else 8)) + (1 if sharded else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
@@ -548,8 +590,12 @@ def run_kvq(args, rank, world):
         "data": "synthetic (seeded Philox4x32-10; LLaMA-7B-shaped K/V distributions)",
         "config": {"workload": w.name, "layers": layers, "B": w.B, "q_heads": w.Hq,
                    "kv_heads": w.Hkv, "head_dim": w.D, "T_cached": T0, "bits": w.bits,
-                   "outlier_frac": w.f, "rope_theta": w.rope_theta, "path": args.path,
+                   "outlier_frac": w.f, "rope_theta": w.rope_theta,
+                   "path": "sharded (partial + all-gather + merge)" if sharded else args.path,
                    "splits": S, "cache_replicas": R,
+                   "parallelism": (f"token-sharded x{world}: one sequence of {shard_n * T0} "
+                                   "tokens, rank r holding [r T, (r+1) T)") if sharded
+                                  else (f"replicas x{world}" if world > 1 else "1 GPU"),
                    "l2": f"inputs {one_cache_bytes * R / 1e9:.1f} GB > 126 MB L2, not flushed"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "peak_source": peak_kind,

@@ -40,7 +40,7 @@
 extern "C" {
 #endif
 
-#define KVQ_ABI_VERSION 1
+#define KVQ_ABI_VERSION 2
 
 enum {
     KVQ_OK = 0,
@@ -254,6 +254,35 @@ int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_c
                          int32_t splits, void* stream);
 
 /*
+ * Decode attention over one token range of a longer sequence, as a partial for a merge: the
+ * building block of the token-sharded decode (the pages' "10 million context across 8 GPUs":
+ * study.space summary; phantomic12 research note, the consequence claim).  A device holds
+ * tokens [pos_offset, pos_offset + len[b]) of sequence b in `cache` (row t of the cache sits at
+ * position pos_offset + t; RoPE uses that position) and computes, per (b, hq),
+ *   ml[b][hq] = (M, L), M = max_t l_t, L = sum_t e^(l_t - M),
+ *   o[b][hq][:] = sum_t e^(l_t - M) vhat_t       (not divided by L),
+ * with l_t, vhat_t exactly as kvq_decode_attention; an empty range gives (-inf, 0) and o = 0.
+ *   pos_offset  host int32 >= 0 (the same for every sequence of the batch)
+ *   ml float2 [B][Hq], o float [B][Hq][D] (device); workspace as kvq_decode_workspace
+ * kvq_decode_partial followed by kvq_merge_partials over all ranges equals
+ * kvq_decode_attention over the whole sequence up to rounding.
+ */
+int kvq_decode_partial(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
+                       const kvq_codebook* cbV, const uint16_t* q, const int32_t* qpos,
+                       int32_t max_len, int32_t pos_offset, float* ml, float* o,
+                       void* workspace, size_t workspace_bytes, int32_t splits, void* stream);
+
+/*
+ * Merge of `parts` partials of kvq_decode_partial (the softmax over the union of their token
+ * ranges, an exact identity): out[b][hq][:] = sum_k e^(M_k - M) o_k / sum_k e^(M_k - M) L_k,
+ * M = max_k M_k, taken in part order; 0 when no part has a token.
+ *   ml float2 [parts][B][Hq], o float [parts][B][Hq][D], out float [B][Hq][D] (device)
+ * Errors: KVQ_ERR_NULL, KVQ_ERR_RANGE (parts outside 1 .. 4096).
+ */
+int kvq_merge_partials(const kvq_cfg* cfg, int32_t parts, const float* ml, const float* o,
+                       float* out, void* stream);
+
+/*
  * Dequantize rows [t0, t0 + nt) of every sequence (test support):
  *   khat, vhat fp16 [B][nt][Hkv][D] (keys pre-RoPE): dense fp16(off + half*L[code])
  *   (binary32 multiply, then add, then round to fp16), outliers replaced by their
@@ -271,6 +300,7 @@ int kvq_dequantize(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codeboo
  *   K, V fp16 [B][T_stride][Hkv][D] (keys pre-RoPE, RoPE applied on the fly);
  *   len int32 [B]; q, qpos as kvq_decode_qk; out float [B][Hq][D];
  *   workspace of kvq_decode_workspace bytes for the same cfg/max_len/splits.
+ * Hq/Hkv must be 1, 2, 4 or 8 (KVQ_ERR_UNSUPPORTED otherwise).
  */
 int kvq_fp16_decode_attention(const kvq_cfg* cfg, const uint16_t* K, const uint16_t* V,
                               int32_t T_stride, const int32_t* len, const uint16_t* q,

@@ -124,11 +124,13 @@ struct Streamer {
 
 // ---------------------------------------------------------------------------------
 // Per-call tables: rotated, scaled queries qr [B][Hq][128]; trig tables hi [nhi][64] =
-// (cos, sin)(256 j theta_p), lo [256][64] = (cos, sin)(tau theta_p), all from binary64; the
-// dense key value at an outlier zk [B][Hkv][128] = off + half * L[encode(normalize(0))].
+// (cos, sin)((256 j + pos_off) theta_p), lo [256][64] = (cos, sin)(tau theta_p), all from
+// binary64, so that hi[t / 256] lo[t % 256] is the rotation of cache row t at position
+// t + pos_off; the dense key value at an outlier zk [B][Hkv][128] = off + half * L[encode(
+// normalize(0))].
 __global__ void k_decode_prep(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const uint16_t* q,
-                              const int32_t* qpos, int nhi, float* qr, float2* thi, float2* tlo,
-                              float* zk) {
+                              const int32_t* qpos, int nhi, int pos_off, float* qr, float2* thi,
+                              float2* tlo, float* zk) {
     const int e = blockIdx.x * blockDim.x + threadIdx.x;
     const int nq = cfg.B * cfg.Hq * 64, nh = nhi * 64, nl = kTrigLo * 64, nz = cfg.B * cfg.Hkv * kD;
     if (e < nq) {
@@ -143,7 +145,7 @@ __global__ void k_decode_prep(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const u
     } else if (e < nq + nh) {
         const int f = e - nq, p = f & 63, j = f >> 6;
         double cc, ss;
-        rope_cs64((double)j * kTrigLo, rope_freq(cfg.rope_theta, p), &cc, &ss);
+        rope_cs64((double)j * kTrigLo + (double)pos_off, rope_freq(cfg.rope_theta, p), &cc, &ss);
         thi[f] = make_float2((float)cc, (float)ss);
     } else if (e < nq + nh + nl) {
         const int f = e - nq - nh, p = f & 63, j = f >> 6;
@@ -1068,7 +1070,9 @@ __global__ void __launch_bounds__(pv_warps(HPC) * 32 + 32, 1)
 // 64 (pair, token) steps per stage against one weight computation, one barrier wait and one
 // stage's bookkeeping.  Lane l of warp w computes the weight of token 32 w + l of the stage;
 // the warp's 32 weights sit in its own slice of shared memory.  The code words of the two
-// half-warps are 16 banks apart.
+// half-warps are 16 banks apart.  Each (La, Lb) lookup reads the two levels' 16-bit patterns
+// (the levels are (u << 16) | u binary32 values) from a table with one copy per lane, and two
+// byte permutes rebuild the exact binary32 pair: half the table bytes of a float pair.
 constexpr int kPQuads = 128;                 // token quads per stage
 constexpr int kPTokens = 4 * kPQuads;        // tokens per stage
 
@@ -1086,7 +1090,7 @@ __host__ __device__ inline PQPlan pq_plan(int bits) {
     p.bar = o;   o += 2 * kStages * 8;
     p.flag = o;  o += 16;
     p.pre = o;
-    p.tsize = (1 << (2 * bits)) * 16 * 8;                    // [entry][16 lane copies] (La, Lb)
+    p.tsize = (1 << (2 * bits)) * 32 * 4;                    // [entry][32 lane copies] 16-bit (La, Lb)
     p.total = o + 2 * p.tsize;                               // alignment slack + table
     return p;
 }
@@ -1132,10 +1136,16 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
         fence_mbar_init();
     }
     const int nb = (1 << BITS) - 1;
-    for (int e = tid; e < F::NT * 16; e += nthr) {
-        const int idx = e >> 4;
-        reinterpret_cast<unsigned long long*>(tab)[e] =
-            pk(cb.levels[idx & nb], cb.levels[idx >> BITS]);
+    // (La, Lb) as the 16-bit patterns u of the (u << 16) | u levels, one copy per lane
+    for (int e = tid; e < F::NT * 32; e += nthr) {
+        const int idx = e >> 5;
+        const uint32_t ua = __float_as_uint(cb.levels[idx & nb]);
+        const uint32_t ub = __float_as_uint(cb.levels[idx >> BITS]);
+        reinterpret_cast<uint32_t*>(tab)[e] = (ua & 0xFFFFu) | (ub << 16);
+    }
+    if (tid <= nb) {
+        const uint32_t u = __float_as_uint(cb.levels[tid]);
+        if ((u >> 16) != (u & 0xFFFFu)) set_status(c.status, KVQ_STATUS_CODEBOOK);
     }
     __syncthreads();  // tables complete, barriers initialised
 
@@ -1187,7 +1197,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             woff[u] = (uint32_t)((8 * warp + 2 * u + hh) * F::BW + i * BITS) * 4;
-        const uint32_t lanebits = tpos | ((uint32_t)i << 3);
+        const uint32_t lanebits = tpos | ((uint32_t)lane << 2);
         unsigned long long* wsw = wsm + 32 * warp;
         for (int st = 0; st < nst; ++st) {
             const int slot = st % kStages;
@@ -1229,7 +1239,11 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
                             KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
 #undef KVQ_FS
                         }
-                        O[k] = fma2(ww, lds64<0>((fs & MASK) | lanebits), O[k]);
+                        const uint32_t lv = lds32((fs & MASK) | lanebits);
+                        const unsigned long long LL =
+                            pk(__uint_as_float(__byte_perm(lv, 0u, 0x1010)),
+                               __uint_as_float(__byte_perm(lv, 0u, 0x3232)));
+                        O[k] = fma2(ww, LL, O[k]);
                     }
                 }
             }
@@ -1376,8 +1390,10 @@ __global__ void k_pv_reduce(int S, const float* __restrict__ part, float* __rest
 
 // ---------------------------------------------------------------------------------
 // Merge of per-split (m, l, o) partials: out = sum_s e^(m_s-M) o_s / sum_s e^(m_s-M) l_s.
+// With ml != nullptr the merged partial itself is written instead: ml = (M, L) and
+// out = sum_s e^(m_s-M) o_s (not divided by L).
 __global__ void k_attn_merge(int S, const float2* __restrict__ st, const float* __restrict__ po,
-                             float* __restrict__ out) {
+                             float* __restrict__ out, float2* __restrict__ ml = nullptr) {
     const int r = blockIdx.x, ch = threadIdx.x;
     float M = -INFINITY;
     for (int s = 0; s < S; ++s) M = fmaxf(M, st[(size_t)r * S + s].x);
@@ -1391,129 +1407,239 @@ __global__ void k_attn_merge(int S, const float2* __restrict__ st, const float* 
                 o += po[((size_t)r * S + s) * kD + ch] * w;
             }
         }
-    out[(size_t)r * kD + ch] = Ls > 0.0f ? o / Ls : 0.0f;
+    if (ml) {
+        out[(size_t)r * kD + ch] = o;
+        if (ch == 0) ml[r] = make_float2(M, Ls);
+    } else {
+        out[(size_t)r * kD + ch] = Ls > 0.0f ? o / Ls : 0.0f;
+    }
+}
+
+// A normalized output and its (M, L) turned into a partial: o = out * L (in place).
+__global__ void k_to_partial(const float2* __restrict__ ml_in, float* __restrict__ o,
+                             float2* __restrict__ ml_out) {
+    const int r = blockIdx.x, ch = threadIdx.x;
+    const float2 m = ml_in[r];
+    o[(size_t)r * kD + ch] *= m.y;
+    if (ch == 0) ml_out[r] = m;
+}
+
+// Merge of partials from `parts` sources laid out [part][rows]: out = sum_r e^(M_r-M) o_r /
+// sum_r e^(M_r-M) L_r, taken in part order; 0 where no source has a token.
+__global__ void k_parts_merge(int parts, int rows, const float2* __restrict__ ml,
+                              const float* __restrict__ o, float* __restrict__ out) {
+    const int r = blockIdx.x, ch = threadIdx.x;
+    float M = -INFINITY;
+    for (int k = 0; k < parts; ++k) M = fmaxf(M, ml[(size_t)k * rows + r].x);
+    float Ls = 0.0f, acc = 0.0f;
+    if (M > -INFINITY)
+        for (int k = 0; k < parts; ++k) {
+            const float2 x = ml[(size_t)k * rows + r];
+            if (x.y > 0.0f) {
+                const float w = expf(x.x - M);
+                Ls += x.y * w;
+                acc += o[((size_t)k * rows + r) * kD + ch] * w;
+            }
+        }
+    out[(size_t)r * kD + ch] = Ls > 0.0f ? acc / Ls : 0.0f;
 }
 
 // ---------------------------------------------------------------------------------
-// fp16 comparison kernel: one CTA per (split, sequence, kv head), warps take tokens
-// round-robin; lane l owns channels 2l, 2l+1 (pairs i0, i1) and their partners
-// 2l+64, 2l+65.  Each lane advances its own (cos, sin) by a fixed rotation of
-// 4*theta per step from a binary64 base at every chunk start.
-constexpr int kF16Threads = 128;
-constexpr int kF16Warps = kF16Threads / 32;
+// fp16 comparison kernel (the uncompressed baseline).  CTA = (split, sequence, kv head) with
+// kF16W warps; warp w takes the split's 64-token chunks w, w + kF16W, ... and walks a chunk 4
+// tokens per step with all 32 lanes on each token: lane l holds channels 4 (l & 15) + e of
+// the first (l < 16) or second (l >= 16) half of the rotate-half pairs p = 4 (l & 15) + e,
+// e < 4, loaded 8 bytes per lane (one whole 256-byte row per warp instruction), and the rows
+// of the next step are loaded before the current step is used.  RoPE turns the query instead
+// of the key: the term of channel p (first half) is k (cos qa + sin qb), of channel p + 64
+// k (cos qb - sin qa), with (cos, sin) of t theta_p from the per-call tables at each chunk
+// start and advanced by one token's rotation within the chunk.  Each warp keeps an online
+// softmax per query head; the warps are merged in order at the end.
+constexpr int kF16W = 8;
 
-__global__ void __launch_bounds__(kF16Threads) k_fp16_attn(kvq_cfg cfg, const uint16_t* __restrict__ K,
-                                                           const uint16_t* __restrict__ V, int Tst,
-                                                           const int32_t* __restrict__ lens,
-                                                           const uint16_t* __restrict__ q,
-                                                           const int32_t* __restrict__ qpos, int Ls,
-                                                           int S, int max_len, float2* __restrict__ st,
-                                                           float* __restrict__ po) {
-    __shared__ float wm[kF16Warps][kMaxG], wl[kF16Warps][kMaxG];
-    __shared__ float wo[kF16Warps][kMaxG][kD];
+__global__ void k_fp16_prep(kvq_cfg cfg, const uint16_t* q, const int32_t* qpos, int nhi,
+                            float* qr, float2* thi, float2* tlo) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    const int nq = cfg.B * cfg.Hq * 64, nh = nhi * 64, nl = kTrigLo * 64;
+    if (e < nq) {
+        const int p = e & 63, bh = e >> 6, b = bh / cfg.Hq;
+        double cq, sq;
+        rope_cs64((double)qpos[b], rope_freq(cfg.rope_theta, p), &cq, &sq);
+        const uint16_t* qv = q + (size_t)bh * kD;
+        const double qa = (double)h2f(qv[p]), qb = (double)h2f(qv[p + 64]);
+        qr[(size_t)bh * kD + p] = (float)((qa * cq - qb * sq) * (double)kInvSqrtD);
+        qr[(size_t)bh * kD + p + 64] = (float)((qa * sq + qb * cq) * (double)kInvSqrtD);
+    } else if (e < nq + nh) {
+        const int f = e - nq, p = f & 63, j = f >> 6;
+        double cc, ss;
+        rope_cs64((double)j * kTrigLo, rope_freq(cfg.rope_theta, p), &cc, &ss);
+        thi[f] = make_float2((float)cc, (float)ss);
+    } else if (e < nq + nh + nl) {
+        const int f = e - nq - nh, p = f & 63, j = f >> 6;
+        double cc, ss;
+        rope_cs64((double)j, rope_freq(cfg.rope_theta, p), &cc, &ss);
+        tlo[f] = make_float2((float)cc, (float)ss);
+    }
+}
+
+__device__ __forceinline__ void half4_to_float(uint2 r, float (&f)[4]) {
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&r.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&r.y));
+    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kF16W * 32) k_fp16_attn(
+    kvq_cfg cfg, const uint16_t* __restrict__ K, const uint16_t* __restrict__ V, int Tst,
+    const int32_t* __restrict__ lens, const float* __restrict__ qr, const float2* __restrict__ thi,
+    const float2* __restrict__ tlo, int Ls, int S, int max_len, float2* __restrict__ st,
+    float* __restrict__ po) {
+    __shared__ float wm[kF16W][G], wl[kF16W][G];
+    __shared__ float wo[kF16W][G][kD];
     const int s = blockIdx.x, b = blockIdx.y, h = blockIdx.z;
-    const int Hq = cfg.Hq, Hkv = cfg.Hkv, g = Hq / Hkv;
+    const int Hq = cfg.Hq, Hkv = cfg.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int half = lane >> 4, e0 = 4 * (lane & 15);
     const int len = min(lens[b], max_len);
     const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
-    const int i0 = 2 * lane, i1 = 2 * lane + 1;
-    const double th0 = rope_freq(cfg.rope_theta, i0), th1 = rope_freq(cfg.rope_theta, i1);
-    float qa0[kMaxG], qb0[kMaxG], qa1[kMaxG], qb1[kMaxG];
-    float mst[kMaxG], lst[kMaxG], o[kMaxG][4];
-    {
-        double c0, s0, c1, s1;
-        rope_cs64((double)qpos[b], th0, &c0, &s0);
-        rope_cs64((double)qpos[b], th1, &c1, &s1);
+    float U[G][4], W[G][4];
 #pragma unroll
-        for (int a = 0; a < kMaxG; ++a) {
-            mst[a] = -INFINITY;
-            lst[a] = 0.0f;
-            o[a][0] = o[a][1] = o[a][2] = o[a][3] = 0.0f;
-            qa0[a] = qb0[a] = qa1[a] = qb1[a] = 0.0f;
-            if (a < g) {
-                const uint16_t* qv = q + ((size_t)b * Hq + h * g + a) * kD;
-                const double xa0 = h2f(qv[i0]), xb0 = h2f(qv[i0 + kPairs]);
-                const double xa1 = h2f(qv[i1]), xb1 = h2f(qv[i1 + kPairs]);
-                qa0[a] = (float)((xa0 * c0 - xb0 * s0) * (double)kInvSqrtD);
-                qb0[a] = (float)((xa0 * s0 + xb0 * c0) * (double)kInvSqrtD);
-                qa1[a] = (float)((xa1 * c1 - xb1 * s1) * (double)kInvSqrtD);
-                qb1[a] = (float)((xa1 * s1 + xb1 * c1) * (double)kInvSqrtD);
+    for (int a = 0; a < G; ++a)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float* qv = qr + ((size_t)b * Hq + h * G + a) * kD;
+            const float qa = qv[e0 + e], qb = qv[e0 + e + 64];
+            U[a][e] = half ? qb : qa;
+            W[a][e] = half ? -qa : qb;
+        }
+    float2 R1[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) R1[e] = tlo[64 + e0 + e];  // one token's rotation
+    float m[G], l[G], o[G][4];
+#pragma unroll
+    for (int a = 0; a < G; ++a) {
+        m[a] = -INFINITY;
+        l[a] = 0.0f;
+        o[a][0] = o[a][1] = o[a][2] = o[a][3] = 0.0f;
+    }
+    const size_t rs = (size_t)Hkv * kD;  // elements between consecutive tokens
+    const uint16_t* Kb = K + ((size_t)b * Tst * Hkv + h) * kD + e0 + 64 * half;
+    const uint16_t* Vb = V + ((size_t)b * Tst * Hkv + h) * kD + e0 + 64 * half;
+    const int jt = 2 * half + ((lane >> 3) & 1);  // token of the step this lane's logit ends on
+    for (int cc = warp;; cc += kF16W) {
+        const int tc = t_begin + cc * kChunk;
+        if (tc >= t_end) break;
+        const int n = min(kChunk, t_end - tc);
+        float2 ph[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ph[e] = trig_at(thi, tlo, tc, e0 + e);
+        uint2 kr[4], vr[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const bool ok = j < n;
+            kr[j] = ok ? *reinterpret_cast<const uint2*>(Kb + (size_t)(tc + j) * rs) : make_uint2(0, 0);
+            vr[j] = ok ? *reinterpret_cast<const uint2*>(Vb + (size_t)(tc + j) * rs) : make_uint2(0, 0);
+        }
+        for (int j0 = 0; j0 < n; j0 += 4) {
+            uint2 kn[4], vn[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const bool ok = j0 + 4 + j < n;
+                kn[j] = ok ? *reinterpret_cast<const uint2*>(Kb + (size_t)(tc + j0 + 4 + j) * rs)
+                           : make_uint2(0, 0);
+                vn[j] = ok ? *reinterpret_cast<const uint2*>(Vb + (size_t)(tc + j0 + 4 + j) * rs)
+                           : make_uint2(0, 0);
             }
-        }
-    }
-    float sd0, cd0, sd1, cd1;
-    {
-        double c, s_;
-        rope_cs64((double)kF16Warps, th0, &c, &s_);
-        cd0 = (float)c; sd0 = (float)s_;
-        rope_cs64((double)kF16Warps, th1, &c, &s_);
-        cd1 = (float)c; sd1 = (float)s_;
-    }
-    for (int tc = t_begin; tc < t_end; tc += kChunk) {
-        float c0, s0, c1, s1;
-        {
-            double c, s_;
-            rope_cs64((double)(tc + warp), th0, &c, &s_);
-            c0 = (float)c; s0 = (float)s_;
-            rope_cs64((double)(tc + warp), th1, &c, &s_);
-            c1 = (float)c; s1 = (float)s_;
-        }
-        for (int dt = warp; dt < kChunk; dt += kF16Warps) {
-            const int t = tc + dt;
-            if (t >= t_end) break;
-            const size_t rb = (((size_t)b * Tst + t) * Hkv + h) * kD;
-            const __half2 ka = *(const __half2*)(K + rb + i0);
-            const __half2 kb = *(const __half2*)(K + rb + i0 + kPairs);
-            const __half2 va = *(const __half2*)(V + rb + i0);
-            const __half2 vb = *(const __half2*)(V + rb + i0 + kPairs);
-            const float2 fka = __half22float2(ka), fkb = __half22float2(kb);
-            const float2 fva = __half22float2(va), fvb = __half22float2(vb);
-            const float ra0 = fka.x * c0 - fkb.x * s0, rb0 = fka.x * s0 + fkb.x * c0;
-            const float ra1 = fka.y * c1 - fkb.y * s1, rb1 = fka.y * s1 + fkb.y * c1;
+            float lp[G][4];
 #pragma unroll
-            for (int a = 0; a < kMaxG; ++a) {
-                if (a < g) {
-                    const float lg = warp_sum(qa0[a] * ra0 + qb0[a] * rb0 + qa1[a] * ra1 + qb1[a] * rb1);
-                    const float mn = fmaxf(mst[a], lg);
-                    const float sc = expf(mst[a] - mn);
-                    const float pp = expf(lg - mn);
-                    lst[a] = lst[a] * sc + pp;
-                    o[a][0] = o[a][0] * sc + pp * fva.x;
-                    o[a][1] = o[a][1] * sc + pp * fva.y;
-                    o[a][2] = o[a][2] * sc + pp * fvb.x;
-                    o[a][3] = o[a][3] * sc + pp * fvb.y;
-                    mst[a] = mn;
+            for (int j = 0; j < 4; ++j) {
+                float kf[4];
+                half4_to_float(kr[j], kf);
+#pragma unroll
+                for (int a = 0; a < G; ++a) {
+                    float acc = 0.0f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        acc = fmaf(kf[e], fmaf(ph[e].x, U[a][e], ph[e].y * W[a][e]), acc);
+                    lp[a][j] = acc;
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ph[e] = cmul(ph[e], R1[e]);
             }
-            const float n0 = c0 * cd0 - s0 * sd0, m0 = s0 * cd0 + c0 * sd0;
-            const float n1 = c1 * cd1 - s1 * sd1, m1 = s1 * cd1 + c1 * sd1;
-            c0 = n0; s0 = m0; c1 = n1; s1 = m1;
+            const bool b3 = (lane >> 3) & 1;
+            const bool valid = tc + j0 + jt < t_end;
+            float pj[G][4];
+#pragma unroll
+            for (int a = 0; a < G; ++a) {
+                // transposed reduction over the 32 lanes: lane ends with token jt's logit
+                const float x0 = (half ? lp[a][2] : lp[a][0]) +
+                                 __shfl_xor_sync(0xffffffffu, half ? lp[a][0] : lp[a][2], 16);
+                const float x1 = (half ? lp[a][3] : lp[a][1]) +
+                                 __shfl_xor_sync(0xffffffffu, half ? lp[a][1] : lp[a][3], 16);
+                float y = (b3 ? x1 : x0) + __shfl_xor_sync(0xffffffffu, b3 ? x0 : x1, 8);
+                y += __shfl_xor_sync(0xffffffffu, y, 4);
+                y += __shfl_xor_sync(0xffffffffu, y, 2);
+                y += __shfl_xor_sync(0xffffffffu, y, 1);
+                const float lg = valid ? y : -INFINITY;
+                float mx = lg;
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                if (mx > m[a]) {
+                    const float sc = m[a] == -INFINITY ? 0.0f : __expf(m[a] - mx);
+                    l[a] *= sc;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[a][e] *= sc;
+                    m[a] = mx;
+                }
+                const float p = valid ? __expf(lg - m[a]) : 0.0f;
+                if ((lane & 7) == 0) l[a] += p;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    pj[a][j] = __shfl_sync(0xffffffffu, p, (j >> 1) * 16 + (j & 1) * 8);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float vf[4];
+                half4_to_float(vr[j], vf);
+#pragma unroll
+                for (int a = 0; a < G; ++a)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o[a][e] = fmaf(pj[a][j], vf[e], o[a][e]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                kr[j] = kn[j];
+                vr[j] = vn[j];
+            }
         }
     }
 #pragma unroll
-    for (int a = 0; a < kMaxG; ++a) {
-        if (a < g) {
-            if (lane == 0) { wm[warp][a] = mst[a]; wl[warp][a] = lst[a]; }
-            wo[warp][a][i0] = o[a][0];
-            wo[warp][a][i1] = o[a][1];
-            wo[warp][a][i0 + kPairs] = o[a][2];
-            wo[warp][a][i1 + kPairs] = o[a][3];
+    for (int a = 0; a < G; ++a) {
+        // l: the owner lanes (lane & 7 == 0) summed in lane order
+        float lt = l[a];
+#pragma unroll
+        for (int off = 8; off < 32; off <<= 1) lt += __shfl_xor_sync(0xffffffffu, lt, off);
+        if (lane == 0) {
+            wm[warp][a] = m[a];
+            wl[warp][a] = lt;
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) wo[warp][a][e0 + e + 64 * half] = o[a][e];
     }
     __syncthreads();
-    for (int idx = threadIdx.x; idx < g * kD; idx += blockDim.x) {
+    for (int idx = threadIdx.x; idx < G * kD; idx += blockDim.x) {
         const int a = idx / kD, ch = idx % kD;
         float M = -INFINITY;
-        for (int w = 0; w < kF16Warps; ++w) M = fmaxf(M, wm[w][a]);
+        for (int w2 = 0; w2 < kF16W; ++w2) M = fmaxf(M, wm[w2][a]);
         float Ls_ = 0.0f, oo = 0.0f;
         if (M > -INFINITY)
-            for (int w = 0; w < kF16Warps; ++w)
-                if (wl[w][a] > 0.0f) {
-                    const float sc = expf(wm[w][a] - M);
-                    Ls_ += wl[w][a] * sc;
-                    oo += wo[w][a][ch] * sc;
+            for (int w2 = 0; w2 < kF16W; ++w2)
+                if (wm[w2][a] > -INFINITY) {
+                    const float sc = expf(wm[w2][a] - M);
+                    Ls_ = fmaf(wl[w2][a], sc, Ls_);
+                    oo = fmaf(wo[w2][a][ch], sc, oo);
                 }
-        const size_t r = (size_t)b * Hq + h * g + a;
+        const size_t r = (size_t)b * Hq + h * G + a;
         po[(r * S + s) * kD + ch] = oo;
         if (ch == 0) st[r * S + s] = make_float2(M, Ls_);
     }
@@ -1621,11 +1747,12 @@ static PVKernel pv_kernel(int hpc, bool share) {
 // QK over the quantized cache into logits, key-outlier corrections, split statistics.
 static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
                   const uint16_t* q, const int32_t* qpos, int max_len, float* logits,
-                  float* stats, int S, int Ls, const QKTables& T, cudaStream_t st) {
+                  float* stats, int S, int Ls, const QKTables& T, cudaStream_t st,
+                  int pos_off = 0) {
     {
         const int n = cfg->B * cfg->Hq * 64 + T.nhi * 64 + kTrigLo * 64 + cfg->B * cfg->Hkv * kD;
-        k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi, T.qr,
-                                                        T.thi, T.tlo, T.zk);
+        k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi,
+                                                        pos_off, T.qr, T.thi, T.tlo, T.zk);
     }
     if (cfg->bits <= 3 && cfg->Hq == cfg->Hkv) {
         QKQKernel kq = cfg->bits == 2 ? k_qk_quad<2> : k_qk_quad<3>;
@@ -1763,17 +1890,20 @@ extern "C" int kvq_decode_workspace(const kvq_cfg* cfg, int32_t max_len, int32_t
     return KVQ_OK;
 }
 
-extern "C" int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache,
-                                    const kvq_codebook* cbK, const kvq_codebook* cbV,
-                                    const uint16_t* q, const int32_t* qpos, int32_t max_len,
-                                    float* out, void* workspace, size_t workspace_bytes,
-                                    int32_t splits, void* stream) {
+// Decode over a cache whose row t sits at position t + pos_off.  With ml_part == nullptr,
+// out receives the normalized attention output; otherwise out receives the unnormalized
+// partial o = sum_t e^(l_t - M) vhat_t and ml_part its (M, L).
+static int decode_core(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
+                       const kvq_codebook* cbV, const uint16_t* q, const int32_t* qpos,
+                       int32_t max_len, int32_t pos_off, float* out, float2* ml_part,
+                       void* workspace, size_t workspace_bytes, int32_t splits, void* stream) {
     int e = check_decode(cfg, max_len);
     if (e) return e;
     if ((e = check_cache(cfg, cache)) || (e = check_codebook(cbK)) || (e = check_codebook(cbV)))
         return e;
     if (!workspace || !out || !q || !qpos) return KVQ_ERR_NULL;
     if (!aligned16(workspace)) return KVQ_ERR_ALIGN;
+    if (pos_off < 0 || (int64_t)pos_off + max_len > (int64_t)1 << 30) return KVQ_ERR_RANGE;
     int S, Ls;
     if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
     if (workspace_bytes < split_ws_bytes(cfg, S, max_len)) return KVQ_ERR_WORKSPACE;
@@ -1792,18 +1922,54 @@ extern "C" int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache,
     if (fused_supported(cfg)) {
         // one pass: per-call tables, the fused kernel's per-split (m, l, o), the split merge
         const int n = cfg->B * cfg->Hq * 64 + T.nhi * 64 + kTrigLo * 64 + cfg->B * cfg->Hkv * kD;
-        k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi, T.qr,
-                                                        T.thi, T.tlo, T.zk);
+        k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi,
+                                                        pos_off, T.qr, T.thi, T.tlo, T.zk);
         if ((e = record_cuda(cudaGetLastError()))) return e;
         if ((e = run_fused(cfg, cache, cbK, cbV, T.qr, T.thi, T.tlo, T.zk, max_len, S, Ls,
                            (float2*)stats, part, st)))
             return e;
-        k_attn_merge<<<(int)BH, kD, 0, st>>>(S, (const float2*)stats, part, out);
+        k_attn_merge<<<(int)BH, kD, 0, st>>>(S, (const float2*)stats, part, out, ml_part);
         return record_cuda(cudaGetLastError());
     }
-    if ((e = run_qk(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, T, st))) return e;
+    if ((e = run_qk(cfg, cache, cbK, q, qpos, max_len, logits, stats, S, Ls, T, st, pos_off)))
+        return e;
     if ((e = kvq_softmax_merge(cfg, stats, S, ml, stream))) return e;
-    return run_pv(cfg, cache, cbV, logits, ml, max_len, out, part, S, Ls, st);
+    if ((e = run_pv(cfg, cache, cbV, logits, ml, max_len, out, part, S, Ls, st))) return e;
+    if (ml_part) {
+        k_to_partial<<<(int)BH, kD, 0, st>>>((const float2*)ml, out, ml_part);
+        return record_cuda(cudaGetLastError());
+    }
+    return KVQ_OK;
+}
+
+extern "C" int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache,
+                                    const kvq_codebook* cbK, const kvq_codebook* cbV,
+                                    const uint16_t* q, const int32_t* qpos, int32_t max_len,
+                                    float* out, void* workspace, size_t workspace_bytes,
+                                    int32_t splits, void* stream) {
+    return decode_core(cfg, cache, cbK, cbV, q, qpos, max_len, 0, out, nullptr, workspace,
+                       workspace_bytes, splits, stream);
+}
+
+extern "C" int kvq_decode_partial(const kvq_cfg* cfg, const kvq_cache* cache,
+                                  const kvq_codebook* cbK, const kvq_codebook* cbV,
+                                  const uint16_t* q, const int32_t* qpos, int32_t max_len,
+                                  int32_t pos_offset, float* ml, float* o, void* workspace,
+                                  size_t workspace_bytes, int32_t splits, void* stream) {
+    if (!ml) return KVQ_ERR_NULL;
+    return decode_core(cfg, cache, cbK, cbV, q, qpos, max_len, pos_offset, o, (float2*)ml,
+                       workspace, workspace_bytes, splits, stream);
+}
+
+extern "C" int kvq_merge_partials(const kvq_cfg* cfg, int32_t parts, const float* ml,
+                                  const float* o, float* out, void* stream) {
+    int e = check_cfg(cfg);
+    if (e) return e;
+    if (!ml || !o || !out) return KVQ_ERR_NULL;
+    if (parts < 1 || parts > 4096) return KVQ_ERR_RANGE;
+    const int rows = cfg->B * cfg->Hq;
+    k_parts_merge<<<rows, kD, 0, (cudaStream_t)stream>>>(parts, rows, (const float2*)ml, o, out);
+    return record_cuda(cudaGetLastError());
 }
 
 extern "C" int kvq_fp16_decode_attention(const kvq_cfg* cfg, const uint16_t* K, const uint16_t* V,
@@ -1816,17 +1982,24 @@ extern "C" int kvq_fp16_decode_attention(const kvq_cfg* cfg, const uint16_t* K, 
     if (!K || !V || !len || !q || !qpos || !out || !workspace) return KVQ_ERR_NULL;
     if (!aligned16(K) || !aligned16(V) || !aligned16(workspace)) return KVQ_ERR_ALIGN;
     if (T_stride < max_len) return KVQ_ERR_RANGE;
+    const int g = cfg->Hq / cfg->Hkv;
+    if (g != 1 && g != 2 && g != 4 && g != 8) return KVQ_ERR_UNSUPPORTED;
     int S, Ls;
     if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
     const size_t BH = (size_t)cfg->B * cfg->Hq;
-    const size_t need = align_up(BH * S * 8) + align_up(BH * S * kD * 4);
-    if (workspace_bytes < need) return KVQ_ERR_WORKSPACE;
+    const size_t a0 = align_up(BH * S * 8), a1 = align_up(BH * S * kD * 4);
+    const QKTables T = qk_tables(cfg, max_len, (char*)workspace + a0 + a1);
+    if (workspace_bytes < a0 + a1 + T.bytes) return KVQ_ERR_WORKSPACE;
     float2* st = (float2*)workspace;
-    float* po = (float*)((char*)workspace + align_up(BH * S * 8));
+    float* po = (float*)((char*)workspace + a0);
     cudaStream_t s = (cudaStream_t)stream;
+    const int n = cfg->B * cfg->Hq * 64 + T.nhi * 64 + kTrigLo * 64;
+    k_fp16_prep<<<(n + 255) / 256, 256, 0, s>>>(*cfg, q, qpos, T.nhi, T.qr, T.thi, T.tlo);
     dim3 grid(S, cfg->B, cfg->Hkv);
-    k_fp16_attn<<<grid, kF16Threads, 0, s>>>(*cfg, K, V, T_stride, len, q, qpos, Ls, S, max_len,
-                                             st, po);
+    auto kern = g == 1 ? k_fp16_attn<1> : g == 2 ? k_fp16_attn<2> : g == 4 ? k_fp16_attn<4>
+                       : k_fp16_attn<8>;
+    kern<<<grid, kF16W * 32, 0, s>>>(*cfg, K, V, T_stride, len, T.qr, T.thi, T.tlo, Ls, S, max_len,
+                                     st, po);
     k_attn_merge<<<(int)BH, kD, 0, s>>>(S, st, po, out);
     return record_cuda(cudaGetLastError());
 }

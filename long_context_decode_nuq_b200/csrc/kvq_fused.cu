@@ -5,16 +5,19 @@
 // (i)-(iv): study.space summary, custom kernels for memory- and bandwidth-bound decode;
 // phantomic12 research note, components (1)-(4).)
 //
-// A CTA has 16 consumer warps and two helper warps and walks its split in 256-token stages.
-//  - Streaming warp: per stage, one bulk copy of the key code blocks into a ring slot
-//    (cp.async.bulk, completion counted on an mbarrier; no multicast), the (cos, sin) of the
-//    stage start for the 64 RoPE pairs, and the key-outlier correction of every token of the
-//    stage, kc[tau] = sum over the token's entries of (x - zhat_c) r, r the rotated query
-//    component that meets channel c at token t (entries summed in list order by a segmented
-//    scan, so the result is the same on every run).
-//  - Value helper: per stage, the dense value the cache holds at a value outlier of each
-//    token, zv = off + half L[code of 0], and the first value-outlier entry of each 16-token
-//    slice of the stage.
+// A CTA has 16 consumer warps and two helper warps and walks its split in 256-token stages
+// through a ring of kFSlots shared-memory slots.
+//  - Streaming warp: per stage, bulk copies (cp.async.bulk, completion counted on an
+//    mbarrier; no multicast) of the key code blocks, the tokens' value (off, half), and the
+//    stage's key- and value-outlier entries (up to kFEnt of each; entries past that are read
+//    from global memory), plus the (cos, sin) of the stage start for the 64 RoPE pairs.  One
+//    stage later, once that stage's copies have landed, the key-outlier correction of every
+//    token, kc[tau] = sum over the token's entries of (x - zhat_c) r, r the rotated query
+//    component that meets channel c at the token (entries summed in list order by a
+//    segmented scan, so the result is the same on every run).
+//  - Value helper: per stage, once its copies have landed, the dense value the cache holds at
+//    a value outlier of each token, zv = off + half L[code of 0], and the first value-outlier
+//    entry of each 16-token slice of the stage.
 //  - Consumer warp w owns tokens [16 w, 16 w + 16) of every stage and keeps its own online
 //    softmax state (running max m, sum l, sum of p off, and the value accumulators).  Per
 //    stage: QK over its four quads from the key ring (tables of e^{i j theta_p} Z_p(code) for
@@ -40,6 +43,10 @@ constexpr int kFQuads = 64;               // token quads per stage
 constexpr int kFTok = 4 * kFQuads;        // tokens per stage (the lo trig table spans a stage)
 constexpr int kFSlots = 3;                // stages in flight
 constexpr uint32_t kFAnchor = 32768;      // shared-window address of the QK tables
+constexpr int kFEnt = 512;                // outlier entries of each kind staged per slot
+constexpr int kFSide = 16;                // words of a slot's side record
+constexpr float kKcScale = 4294967296.0f;           // 2^32
+constexpr double kKcInv = 1.0 / 4294967296.0;       // 2^-32
 static_assert(kFTok == kTrigLo, "the in-stage rotation comes from the lo trig table");
 
 // Shared-memory plan.  The small buffers sit from the window base up to the PV table, which
@@ -49,18 +56,19 @@ static_assert(kFTok == kTrigLo, "the in-stage rotation comes from the lo trig ta
 // kernel whose window base leaves too little room below the PV table reports
 // KVQ_STATUS_SMEM_LAYOUT and writes nothing.
 struct FusedPlan {
-    int base, kc, zv, vsl, wsm, wp, scr, zk, qv, levk, levv, bar, flag, small;
+    int base, kc, zv, vsl, side, wsm, wp, scr, zk, qv, levk, levv, bar, flag, small;
     int pv, jslice;
-    int stage, ring, accv, post;
+    int stage, ring, vps, kent, vent, accv, post;
     int total;
 };
 __host__ __device__ inline FusedPlan fused_plan(int bits) {
     FusedPlan p;
     int o = 0;
     p.base = o; o += kFSlots * 64 * 16;   // [slot][pair] (c, c, s, s) at the stage start
-    p.kc = o;   o += kFSlots * kFTok * 4; // [slot][token] key-outlier correction
+    p.kc = o;   o += kFSlots * kFTok * 8; // [slot][token] key-outlier correction, 2^-32 fixed point
     p.zv = o;   o += kFSlots * kFTok * 4; // [slot][token] dense value at a value outlier
     p.vsl = o;  o += kFSlots * 32 * 4;    // [slot][slice] first value entry (17 used)
+    p.side = o; o += kFSlots * kFSide * 4;  // [slot] staged entry ranges and value-param count
     p.wsm = o;  o += kFW * 16 * 8;        // [warp][token] (w, w), w = p half
     p.wp = o;   o += kFW * 16 * 4;        // [warp][token] p
     p.scr = o;  o += kFW * 32 * 4;        // [warp][lane] scratch
@@ -76,6 +84,9 @@ __host__ __device__ inline FusedPlan fused_plan(int bits) {
     o = 0;
     p.stage = kFQuads * 16 * bits * 4;
     p.ring = o; o += kFSlots * p.stage;
+    p.vps = o;  o += kFSlots * kFTok * 8; // [slot][token] value (off, half)
+    p.kent = o; o += kFSlots * kFEnt * 4; // [slot] key-outlier entries of the stage
+    p.vent = o; o += kFSlots * kFEnt * 4; // [slot] value-outlier entries of the stage
     p.accv = o; o += kFW * kD * 4;        // [warp][channel] value-outlier sums
     p.post = o;
     p.total = (int)kFAnchor + 4 * p.jslice + p.post;
@@ -95,17 +106,6 @@ __device__ __forceinline__ void add_ordered(float* acc, float* scr, int ch, floa
         acc[ch] += sum;
     }
     __syncwarp();
-}
-
-// Inclusive scan of v over the lanes, restarted wherever the key t changes (keys contiguous).
-__device__ __forceinline__ float seg_scan_f(float v, int t, int lane) {
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const float vv = __shfl_up_sync(0xffffffffu, v, off);
-        const int tt = __shfl_up_sync(0xffffffffu, t, off);
-        if (lane >= off && tt == t) v += vv;
-    }
-    return v;
 }
 
 // Bounded wait by every lane, made warp-uniform; false (and the abort flag set) on a timeout
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         return;
     }
     float4* base = reinterpret_cast<float4*>(sm + L.base);
-    float* kc = reinterpret_cast<float*>(sm + L.kc);
+    unsigned long long* kc = reinterpret_cast<unsigned long long*>(sm + L.kc);
     float* zv = reinterpret_cast<float*>(sm + L.zv);
     uint32_t* vsl = reinterpret_cast<uint32_t*>(sm + L.vsl);
     unsigned long long* wsm = reinterpret_cast<unsigned long long*>(sm + L.wsm);
@@ -236,84 +236,152 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const int i = lane & 15, hh = lane >> 4;
     unsigned long long O[4] = {0ull, 0ull, 0ull, 0ull};  // consumer lanes: (o[c], o[c + 64]), c = i + 16 k
     const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
+    const uint32_t* kent = c.kout + li * cfg.out_cap_k;
+    const uint32_t* vent = c.vout + li * cfg.out_cap_v;
+    uint32_t* side = reinterpret_cast<uint32_t*>(sm + L.side);  // [slot][kFSide]
+    float2* vps = reinterpret_cast<float2*>(post + L.vps);
+    uint32_t* kents = reinterpret_cast<uint32_t*>(post + L.kent);
+    uint32_t* vents = reinterpret_cast<uint32_t*>(post + L.vent);
+    // side[slot][]: 0 kB, 1 kN (staged key entries [kB, kB + kN)), 2 kE0, 3 kE1 (the stage's key
+    // entries), 4..6 the key chunk boundaries, 7 the stage's chunks, 8 vB, 9 vN, 10 vE0, 11 vE1,
+    // 12..14 the value chunk boundaries, 15 value params staged
     if (warp == kFW) {
-        // ================= streaming warp: key codes, stage phases, key-outlier corrections
+        // ================= streaming warp
         const uint32_t* ksrc = c.kcodes + li * nquads(cfg.T_max) * F::BW;
         const uint32_t* kcp = c.kchunk + li * (nchunks(cfg.T_max) + 1);
-        const uint32_t* kent = c.kout + li * cfg.out_cap_k;
-        const uint32_t kcnt = c.kcount[li];
-        int cc = 0;
-        for (; cc < nst; ++cc) {
-            const int slot = cc % kFSlots;
-            if (cc >= kFSlots &&
-                !warp_wait(empty + slot, (uint32_t)(cc / kFSlots - 1) & 1u, flag, c.status))
-                break;
-            if (__shfl_sync(0xffffffffu, *(volatile int*)flag, 0)) break;
-            const int tc = t_begin + cc * kFTok;
-            if (lane == 0) {
-                fence_proxy_async();
-                const int q0 = tc >> 2, q1 = (min(tc + kFTok, t_end) + 3) >> 2;
-                const uint32_t bytes = (uint32_t)(q1 - q0) * F::BW * 4;
-                mbar_arrive_expect_tx(bcopy + slot, bytes);
-                bulk_load(ring + (size_t)slot * L.stage, ksrc + (size_t)q0 * F::BW, bytes,
-                          bcopy + slot);
-            }
-            float4* bs = base + slot * 64;
+        const uint32_t* vcp = c.vchunk + li * (nchunks(cfg.T_max) + 1);
+        const uint32_t kcnt = c.kcount[li], vcnt = c.vcount[li];
+        uint32_t kcpl = 0, vcpl = 0;  // chunk pointers of the next stage to issue (lanes 0 .. 4)
+        auto load_cp = [&](int st) {
+            const int tc = t_begin + st * kFTok, m0 = tc >> 6;
+            const int nm = min(4, ((t_end + 63) >> 6) - m0);
+            kcpl = lane <= nm ? min(kcp[m0 + lane], kcnt) : 0u;
+            vcpl = lane <= nm ? min(vcp[m0 + lane], vcnt) : 0u;
+        };
+        load_cp(0);
+        int issued = 0;
+        float2 thv[2], tlv[2];  // (cos, sin) tables of the stage being issued
+        for (int cc = 0; cc <= nst; ++cc) {
+            if (cc < nst) {
+                const int slot = cc % kFSlots;
+                if (cc >= kFSlots &&
+                    !warp_wait(empty + slot, (uint32_t)(cc / kFSlots - 1) & 1u, flag, c.status))
+                    break;
+                if (__shfl_sync(0xffffffffu, *(volatile int*)flag, 0)) break;
+                const int tc = t_begin + cc * kFTok, m0 = tc >> 6;
+                const int nm = min(4, ((t_end + 63) >> 6) - m0);
+                const int n = min(kFTok, t_end - tc);
+                // value params: an even count from a 16-byte aligned start, so the copy is a
+                // whole number of 16-byte units; none staged when the row starts mid-unit (the
+                // readers then load them from global memory)
+                const bool va = (((size_t)b * cfg.T_max + tc) & 1) == 0;
+                const int nv = !va ? 0 : !(n & 1) ? n : (tc + n + 1 <= cfg.T_max ? n + 1 : n - 1);
+                uint32_t sv[kFSide];
+                sv[2] = __shfl_sync(0xffffffffu, kcpl, 0);
+                sv[3] = __shfl_sync(0xffffffffu, kcpl, nm);
+                sv[10] = __shfl_sync(0xffffffffu, vcpl, 0);
+                sv[11] = __shfl_sync(0xffffffffu, vcpl, nm);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const float2 cs = trig_at(thi, tlo, tc, lane + 32 * u);
-                bs[lane + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
+                for (int k = 1; k < 4; ++k) {
+                    sv[3 + k] = __shfl_sync(0xffffffffu, kcpl, k);
+                    sv[11 + k] = __shfl_sync(0xffffffffu, vcpl, k);
+                }
+                sv[7] = (uint32_t)nm;
+                sv[15] = (uint32_t)nv;
+                sv[0] = sv[2] & ~3u;
+                sv[1] = min(((sv[3] + 3u) & ~3u) - sv[0], (uint32_t)kFEnt);
+                sv[8] = sv[10] & ~3u;
+                sv[9] = min(((sv[11] + 3u) & ~3u) - sv[8], (uint32_t)kFEnt);
+                if (sv[3] == sv[2]) sv[1] = 0;
+                if (sv[11] == sv[10]) sv[9] = 0;
+                if (lane == 0) {
+#pragma unroll
+                    for (int k = 0; k < kFSide; ++k) side[slot * kFSide + k] = sv[k];
+                }
+                __syncwarp();  // the side record is complete before the copies are announced
+                if (lane == 0) {
+                    fence_proxy_async();
+                    const int q0 = tc >> 2, q1 = (min(tc + kFTok, t_end) + 3) >> 2;
+                    const uint32_t kbytes = (uint32_t)(q1 - q0) * F::BW * 4;
+                    mbar_arrive_expect_tx(bcopy + slot,
+                                          kbytes + 8u * (uint32_t)nv + 4u * (sv[1] + sv[9]));
+                    bulk_load(ring + (size_t)slot * L.stage, ksrc + (size_t)q0 * F::BW, kbytes,
+                              bcopy + slot);
+                    if (nv) bulk_load(vps + slot * kFTok, vpar + tc, 8u * nv, bcopy + slot);
+                    if (sv[1]) bulk_load(kents + slot * kFEnt, kent + sv[0], 4u * sv[1], bcopy + slot);
+                    if (sv[9]) bulk_load(vents + slot * kFEnt, vent + sv[8], 4u * sv[9], bcopy + slot);
+                }
+                // the stage's start phases: requested now, stored after the corrections below
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    thv[u] = thi[(tc / kTrigLo) * 64 + lane + 32 * u];
+                    tlv[u] = tlo[(tc % kTrigLo) * 64 + lane + 32 * u];
+                }
+                issued = cc + 1;
+                if (cc + 1 < nst) load_cp(cc + 1);
             }
-            float* kcs = kc + slot * kFTok;
-            for (int j = lane; j < kFTok; j += 32) kcs[j] = 0.0f;
-            __syncwarp();
-            const int m0 = tc >> 6, nm = min(4, ((t_end + 63) >> 6) - m0);
-            const uint32_t cpl = lane <= nm ? min(kcp[m0 + lane], kcnt) : 0u;
-            const uint32_t E0 = __shfl_sync(0xffffffffu, cpl, 0);
-            const uint32_t E1 = __shfl_sync(0xffffffffu, cpl, nm);
-            const uint32_t bd1 = __shfl_sync(0xffffffffu, cpl, 1);
-            const uint32_t bd2 = __shfl_sync(0xffffffffu, cpl, 2);
-            const uint32_t bd3 = __shfl_sync(0xffffffffu, cpl, 3);
-            int ct = -1;
-            float cv = 0.0f;
-            for (uint32_t E = E0; E < E1; E += 32) {
-                const uint32_t e = E + lane;
-                const uint32_t w = e < E1 ? kent[e] : 0u;
-                const int mc = (nm > 1 && e >= bd1) + (nm > 2 && e >= bd2) + (nm > 3 && e >= bd3);
-                const int tau = mc * kChunk + (int)((w >> 7) & 63u);
-                const int key = (e < E1 && tc + tau < t_end) ? tau : -1;
-                float v = 0.0f;
-                if (key >= 0) {
-                    const int ch = (int)(w & 127u), p = ch & 63;
-                    const float d = h2f((uint16_t)(w >> 16)) - zks[ch];
-                    const float4 bq = bs[p];
-                    const float2 cs = cmul(make_float2(bq.x, bq.z), tlo[tau * 64 + p]);
-                    // rotate-half: channel c < 64 meets (cos, sin) . (q_p, q_p+64), c >= 64 the other
-                    const float sa = ch < 64 ? cs.x : -cs.y, sb = ch < 64 ? cs.y : cs.x;
-                    v = d * fmaf(sa, qs[p], sb * qs[p + 64]);
-                }
-                const int k0 = __shfl_sync(0xffffffffu, key, 0);
-                if (ct >= 0 && lane == 0) {
-                    if (k0 == ct) v += cv;
-                    else kcs[ct] += cv;
-                }
-                v = seg_scan_f(v, key, lane);
-                const int kn = __shfl_down_sync(0xffffffffu, key, 1);
-                if (key >= 0 && lane < 31 && kn != key) kcs[key] += v;
-                ct = __shfl_sync(0xffffffffu, key, 31);
-                cv = __shfl_sync(0xffffffffu, v, 31);
+            if (cc >= 1) {
+                // ---- key-outlier corrections of the previous stage, from its staged entries
+                const int ps = (cc - 1) % kFSlots;
+                if (!warp_wait(bcopy + ps, (uint32_t)((cc - 1) / kFSlots) & 1u, flag, c.status))
+                    break;
+                const uint32_t* sd = side + ps * kFSide;
+                const uint32_t kB = sd[0], kN = sd[1], E0 = sd[2], E1 = sd[3];
+                const uint32_t bd1 = sd[4], bd2 = sd[5], bd3 = sd[6];
+                const int nm = (int)sd[7];
+                const int tc = t_begin + (cc - 1) * kFTok;
+                const float4* bs = base + ps * 64;
+                const uint32_t* se = kents + ps * kFEnt;
+                unsigned long long* kcs = kc + ps * kFTok;
+                for (int j = lane; j < kFTok; j += 32) kcs[j] = 0ull;
                 __syncwarp();
+                // each entry's term in 2^-32 fixed point, added with an integer atomic: the sum
+                // of a token's terms does not depend on their order.  A term is below 2^17 *
+                // |q| in magnitude (|x - zhat| < 2^17), far inside the 2^31 range.
+                constexpr int kKB = 8;
+                for (uint32_t EW = E0; EW < E1; EW += 32 * kKB) {
+                    uint32_t wv[kKB];
+                    int kv[kKB];
+                    float2 rv[kKB];
+#pragma unroll
+                    for (int u = 0; u < kKB; ++u) {
+                        const uint32_t e = EW + 32 * u + lane;
+                        wv[u] = e < E1 ? (e - kB < kN ? se[e - kB] : kent[e]) : 0u;
+                        const int mc =
+                            (nm > 1 && e >= bd1) + (nm > 2 && e >= bd2) + (nm > 3 && e >= bd3);
+                        const int tau = mc * kChunk + (int)((wv[u] >> 7) & 63u);
+                        kv[u] = (e < E1 && tc + tau < t_end) ? tau : -1;
+                        rv[u] = tlo[(kv[u] >= 0 ? kv[u] : 0) * 64 + (int)(wv[u] & 63u)];
+                    }
+#pragma unroll
+                    for (int u = 0; u < kKB; ++u) {
+                        if (kv[u] < 0) continue;
+                        const uint32_t w = wv[u];
+                        const int ch = (int)(w & 127u), p = ch & 63;
+                        const float d = h2f((uint16_t)(w >> 16)) - zks[ch];
+                        const float4 bq = bs[p];
+                        const float2 cs = cmul(make_float2(bq.x, bq.z), rv[u]);
+                        // rotate-half: channel c < 64 meets (cos, sin) . (q_p, q_p+64), c >= 64 the other
+                        const float sa = ch < 64 ? cs.x : -cs.y, sb = ch < 64 ? cs.y : cs.x;
+                        const float v = d * fmaf(sa, qs[p], sb * qs[p + 64]);
+                        atomicAdd(kcs + kv[u], (unsigned long long)__float2ll_rn(v * kKcScale));
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(full + ps);
             }
-            if (ct >= 0 && lane == 0) kcs[ct] += cv;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(full + slot);
+            if (cc < nst) {
+                float4* bs = base + (cc % kFSlots) * 64;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const float2 cs = cmul(thv[u], tlv[u]);
+                    bs[lane + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
+                }
+            }
         }
-        if (lane == 0) flag[1] = cc;  // stages issued
+        if (lane == 0) flag[1] = issued;  // stages whose copies were issued
     } else if (warp == kFW + 1) {
         // ================= value helper: zv per token, first value entry per 16-token slice
-        const uint32_t* vcp = c.vchunk + li * (nchunks(cfg.T_max) + 1);
-        const uint32_t* vent = c.vout + li * cfg.out_cap_v;
-        const uint32_t vcnt = c.vcount[li];
         float bd[NB];
 #pragma unroll
         for (int j = 0; j < NB; ++j) bd[j] = cbV.bounds[j];
@@ -322,15 +390,21 @@ __global__ void __launch_bounds__(kFThreads, 1)
             if (cc >= kFSlots &&
                 !warp_wait(empty + slot, (uint32_t)(cc / kFSlots - 1) & 1u, flag, c.status))
                 break;
-            if (__shfl_sync(0xffffffffu, *(volatile int*)flag, 0)) break;
+            if (!warp_wait(bcopy + slot, (uint32_t)(cc / kFSlots) & 1u, flag, c.status)) break;
+            const uint32_t* sd = side + slot * kFSide;
+            const uint32_t vB = sd[8], vN = sd[9], E0 = sd[10], E1 = sd[11];
+            const uint32_t bd1 = sd[12], bd2 = sd[13], bd3 = sd[14];
+            const int nm = (int)sd[7], nv = (int)sd[15];
             const int tc = t_begin + cc * kFTok;
+            const float2* vs_ = vps + slot * kFTok;
             float* zs = zv + slot * kFTok;
+#pragma unroll
             for (int j = lane; j < kFTok; j += 32) {
                 const int t = tc + j;
                 float z = 0.0f;
                 if (t < t_end) {
                     // the dense value stored at an outlier: the code of 0 in the token's normalization
-                    const float2 vp = vpar[t];
+                    const float2 vp = j < nv ? vs_[j] : vpar[t];
                     const float xn = normalize(0.0f, vp.x, vp.y);
                     int code = 0;
 #pragma unroll
@@ -340,17 +414,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 zs[j] = z;
             }
             uint32_t* vs = vsl + slot * 32;
-            const int m0 = tc >> 6, nm = min(4, ((t_end + 63) >> 6) - m0);
-            const uint32_t cpl = lane <= nm ? min(vcp[m0 + lane], vcnt) : 0u;
-            const uint32_t E0 = __shfl_sync(0xffffffffu, cpl, 0);
-            const uint32_t E1 = __shfl_sync(0xffffffffu, cpl, nm);
-            const uint32_t bd1 = __shfl_sync(0xffffffffu, cpl, 1);
-            const uint32_t bd2 = __shfl_sync(0xffffffffu, cpl, 2);
-            const uint32_t bd3 = __shfl_sync(0xffffffffu, cpl, 3);
+            const uint32_t* se = vents + slot * kFEnt;
             int qprev = -1;  // slice of the entry before the window
             for (uint32_t E = E0; E < E1; E += 32) {
                 const uint32_t e = E + lane;
-                const uint32_t w = e < E1 ? vent[e] : 0u;
+                const uint32_t w = e < E1 ? (e - vB < vN ? se[e - vB] : vent[e]) : 0u;
                 const int mc = (nm > 1 && e >= bd1) + (nm > 2 && e >= bd2) + (nm > 3 && e >= bd3);
                 const int tau = mc * kChunk + (int)((w >> 7) & 63u);
                 const int q = (e < E1 && tc + tau < t_end) ? (tau >> 4) : 16;
@@ -358,7 +426,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 if (lane == 0) qp = qprev;
                 if (e < E1)
                     for (int r = qp + 1; r <= q; ++r) vs[r] = e;
-                qprev = __shfl_sync(0xffffffffu, e < E1 ? q : 16, min(31, (int)(E1 - 1 - E)));
+                qprev = __shfl_sync(0xffffffffu, q, min(31, (int)(E1 - 1 - E)));
             }
             for (int r = qprev + 1 + lane; r <= 16; r += 32) vs[r] = E1;
             __syncwarp();
@@ -389,8 +457,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
         const uint32_t pvlane = (kFAnchor - (uint32_t)L.pv) | ((uint32_t)lane << 2);
         const uint32_t* vsrc = c.vcodes + li * nquads(cfg.T_max) * F::BW + i * BITS;
-        const uint32_t* vent = c.vout + li * cfg.out_cap_v;
-        uint32_t vw[2][BITS];  // value code words of quads qbase + 2u of the current stage
         auto load_v = [&](int st, uint32_t (&dst)[2][BITS]) {
             const int q0 = (t_begin + st * kFTok) >> 2;
 #pragma unroll
@@ -401,32 +467,24 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 for (int d = 0; d < BITS; ++d) dst[u][d] = ok ? vsrc[(size_t)q * F::BW + d] : 0u;
             }
         };
-        auto load_vp = [&](int st) {
-            const int t = t_begin + st * kFTok + 16 * warp + tl;
-            return t < t_end ? vpar[t] : make_float2(0.0f, 0.0f);
-        };
-        load_v(0, vw);
-        float2 vp = load_vp(0);
         float m_w = -INFINITY, l_w = 0.0f, po_w = 0.0f;
         float* accw = accv + warp * kD;
         unsigned long long* wsw = wsm + warp * 16;
         float* wpw = wp + warp * 16;
         float* scw = scr + warp * 32;
-        for (int st = 0; st < nst; ++st) {
+        // one stage: vw holds its value codes; the next stage's go into vwn, first read one
+        // stage later (the two buffers alternate), so their loads are in flight for a stage
+        auto stage_fn = [&](int st, const uint32_t (&vw)[2][BITS], uint32_t (&vwn)[2][BITS]) -> bool {
             const int slot = st % kFSlots;
             const uint32_t par = (uint32_t)(st / kFSlots) & 1u;
-            if (!warp_wait(bcopy + slot, par, flag, c.status)) break;
-            if (!warp_wait(full + slot, par, flag, c.status)) break;
-            // loads for the next stage and this stage's value-outlier entries, in flight
-            // during QK and PV
-            uint32_t vwn[2][BITS];
-            float2 vpn = make_float2(0.0f, 0.0f);
-            if (st + 1 < nst) {
-                load_v(st + 1, vwn);
-                vpn = load_vp(st + 1);
-            }
+            if (!warp_wait(bcopy + slot, par, flag, c.status)) return false;
+            if (!warp_wait(full + slot, par, flag, c.status)) return false;
+            if (st + 1 < nst) load_v(st + 1, vwn);
+            const uint32_t* sd = side + slot * kFSide;
+            const uint32_t vB = sd[8], vN = sd[9];
+            const int nv = (int)sd[15];
             const uint32_t ea = vsl[slot * 32 + warp], eb = vsl[slot * 32 + warp + 1];
-            const uint32_t went = ea + lane < eb ? vent[ea + lane] : 0u;
+            const uint32_t* se = vents + slot * kFEnt;
             // ---- QK over quads qbase + 2 (u ^ uperm)
             const uint8_t* stage = ring + (size_t)slot * L.stage;
             uint32_t w[2][BITS];
@@ -484,8 +542,13 @@ __global__ void __launch_bounds__(kFThreads, 1)
                     v[t] += __shfl_xor_sync(0xffffffffu, v[t + half], mk);
             v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
             // ---- logit, the warp's online softmax
-            const int tabs = t_begin + st * kFTok + 16 * warp + tl;
-            const float lg = tabs < t_end ? v[0] + kc[slot * kFTok + 16 * warp + tl] : -INFINITY;
+            const int tst = 16 * warp + tl;  // token within the stage
+            const int tabs = t_begin + st * kFTok + tst;
+            const float lg =
+                tabs < t_end ? v[0] + (float)((double)(long long)kc[slot * kFTok + tst] * kKcInv)
+                             : -INFINITY;
+            const float2 vp = tabs < t_end ? (tst < nv ? vps[slot * kFTok + tst] : vpar[tabs])
+                                           : make_float2(0.0f, 0.0f);
             float mx = lg;
 #pragma unroll
             for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -536,7 +599,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
             for (uint32_t E = ea; E < eb; E += 32) {
                 const uint32_t e = E + lane;
                 const bool ok = e < eb;
-                const uint32_t we = E == ea ? went : (ok ? vent[e] : 0u);
+                const uint32_t we = ok ? (e - vB < vN ? se[e - vB] : vent[e]) : 0u;
                 const int tau = (int)((we >> 7) & 15u);  // token within the slice
                 const int ch = (int)(we & 127u);
                 float val = 0.0f;
@@ -546,13 +609,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
-#pragma unroll
-            for (int u = 0; u < 2; ++u)
-#pragma unroll
-                for (int d = 0; d < BITS; ++d) vw[u][d] = vwn[u][d];
-            vp = vpn;
+            return true;
+        };
+        uint32_t vA[2][BITS], vB[2][BITS];
+        load_v(0, vA);
+        for (int st = 0; st < nst; st += 2) {
+            if (!stage_fn(st, vA, vB)) break;
+            if (st + 1 < nst && !stage_fn(st + 1, vB, vA)) break;
         }
-        // the warp's state: l and sum p off over the owner lanes, in lane order
+        // the warp's state: l and sum p off over the owner lanes
 #pragma unroll
         for (int o = 16; o; o >>= 1) {
             l_w += __shfl_xor_sync(0xffffffffu, l_w, o);

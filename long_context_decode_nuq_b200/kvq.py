@@ -28,7 +28,7 @@ EXPORTS = (
     "kvq_decode_splits",
     "kvq_softmax_merge", "kvq_decode_pv", "kvq_decode_workspace", "kvq_decode_attention",
     "kvq_dequantize", "kvq_fp16_decode_attention", "kvq_fit_workspace", "kvq_fit_codebook",
-    "kvq_get_status", "kvq_quantize_append_noalloc",
+    "kvq_get_status", "kvq_quantize_append_noalloc", "kvq_decode_partial", "kvq_merge_partials",
 )
 
 
@@ -103,6 +103,10 @@ def load():
         "kvq_fit_codebook": ([P, c_int32, c_int32, c_double, P, c_int32, c_int32, P, P, P,
                               c_size_t, P], c_int),
         "kvq_get_status": ([POINTER(CacheStruct), POINTER(c_int32), P], c_int),
+        "kvq_decode_partial": ([POINTER(Cfg), POINTER(CacheStruct), POINTER(CodebookStruct),
+                                POINTER(CodebookStruct), P, P, c_int32, c_int32, P, P, P,
+                                c_size_t, c_int32, P], c_int),
+        "kvq_merge_partials": ([POINTER(Cfg), c_int32, P, P, P, P], c_int),
         "kvq_quantize_append_noalloc": ([POINTER(Cfg), POINTER(CacheStruct),
                                          POINTER(CodebookStruct), POINTER(CodebookStruct), P, P,
                                          c_int32, P, P], c_int),
@@ -261,6 +265,20 @@ def kvq_decode_attention(cache: Cache, cbK: Codebook, cbV: Codebook, q, qpos, ma
         ctypes.byref(cbV.struct), _ptr(q), _ptr(qpos), max_len, _ptr(out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), splits, _stream(stream)),
         "kvq_decode_attention")
+
+
+def kvq_decode_partial(cache: Cache, cbK: Codebook, cbV: Codebook, q, qpos, max_len: int,
+                       pos_offset: int, ml, o, workspace, splits: int = 0, stream=None) -> None:
+    _check(load().kvq_decode_partial(
+        ctypes.byref(cache.cfg), ctypes.byref(cache.struct), ctypes.byref(cbK.struct),
+        ctypes.byref(cbV.struct), _ptr(q), _ptr(qpos), max_len, pos_offset, _ptr(ml), _ptr(o),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), splits, _stream(stream)),
+        "kvq_decode_partial")
+
+
+def kvq_merge_partials(cfg: Cfg, parts: int, ml, o, out, stream=None) -> None:
+    _check(load().kvq_merge_partials(ctypes.byref(cfg), parts, _ptr(ml), _ptr(o), _ptr(out),
+                                     _stream(stream)), "kvq_merge_partials")
 
 
 def kvq_dequantize(cache: Cache, cbK: Codebook, cbV: Codebook, t0: int, nt: int, khat, vhat,

@@ -471,11 +471,12 @@ def rope_rotate(x, pos, base):
     return np.concatenate([a * c - bb * s, a * s + bb * c], axis=-1)
 
 
-def decode_attention(q16, qpos, Kh, Vh, base):
+def decode_attention(q16, qpos, Kh, Vh, base, kpos=None):
     """One decode step for one sequence, binary64.
 
     q16: [Hq, D] pre-RoPE query; Kh, Vh: [T, Hkv, D] dequantized cache (keys
-    pre-RoPE).  Returns (logits [Hq, T], probs [Hq, T], out [Hq, D]).
+    pre-RoPE) whose row t sits at position kpos[t] (default t, reading R9).
+    Returns (logits [Hq, T], probs [Hq, T], out [Hq, D]).
     """
     Hq, D = q16.shape
     T, Hkv, _ = Kh.shape
@@ -484,7 +485,7 @@ def decode_attention(q16, qpos, Kh, Vh, base):
     logits = np.empty((Hq, T))
     out = np.empty((Hq, D))
     probs = np.empty((Hq, T))
-    tpos = np.arange(T)
+    tpos = np.arange(T) if kpos is None else np.asarray(kpos)
     for h in range(Hkv):
         kr = rope_rotate(np.asarray(Kh[:, h], dtype=np.float64), tpos, base)
         vh = np.asarray(Vh[:, h], dtype=np.float64)
@@ -517,3 +518,27 @@ def merge_splits(logits, V, S):
     L = sum(p[1] * math.exp(p[0] - M) for p in parts if p[1] > 0)
     o = sum(p[2] * math.exp(p[0] - M) for p in parts if p[1] > 0)
     return o / L, M, L
+
+
+def partial_attention(q16, qpos, Kh, Vh, base, kpos):
+    """The attention of one token range as a mergeable partial, binary64:
+    M = max_t l_t, L = sum_t e^(l_t - M), o = sum_t e^(l_t - M) vhat_t (per query head).
+    An empty range gives (-inf, 0, 0)."""
+    Hq, D = q16.shape
+    if Kh.shape[0] == 0:
+        return np.full(Hq, -np.inf), np.zeros(Hq), np.zeros((Hq, D))
+    lg, p, out = decode_attention(q16, qpos, Kh, Vh, base, kpos=kpos)
+    M = lg.max(axis=1)
+    L = np.exp(lg - M[:, None]).sum(axis=1)
+    return M, L, out * L[:, None]
+
+
+def merge_partials(M, L, o):
+    """Softmax over the union of the ranges of partials M [P, Hq], L [P, Hq], o [P, Hq, D]
+    (the same identity as the split-K merge): sum_k e^(M_k - M) o_k / sum_k e^(M_k - M) L_k."""
+    M = np.asarray(M, dtype=np.float64)
+    Mx = M.max(axis=0)
+    w = np.where(np.asarray(L) > 0, np.exp(M - Mx[None]), 0.0)
+    Ls = (w * L).sum(axis=0)
+    return (w[:, :, None] * o).sum(axis=0) / Ls[:, None]
+

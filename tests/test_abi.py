@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
     for name in names:
         assert hasattr(lib, name), name
     assert set(names) == set(K.EXPORTS)
-    assert K.kvq_abi_version() == 1
+    assert K.kvq_abi_version() == 2
 
 
 def test_cfg_validation():

@@ -211,3 +211,51 @@ def test_decode_is_deterministic(name, over, T, plen, appends):
     assert np.array_equal(res[0][0], res[1][0])
     assert np.array_equal(res[0][1], res[1][1])
     assert K.kvq_get_status(g) == 0
+
+
+@pytest.mark.parametrize("name,over,T,cut", [
+    ("llama7b_layer_32k", dict(Hq=4, Hkv=4), 900, 448),          # fused kernel
+    ("llama3_8b_gqa_128k", dict(B=1, Hq=8, Hkv=2), 700, 320),    # split kernels (GQA)
+    ("batched_8x8k", dict(B=1, Hq=4, Hkv=4, bits=4), 500, 500),  # second range empty
+])
+def test_sharded_partials(name, over, T, cut):
+    """Two token ranges of one sequence in two caches (each calibrated on its own range), their
+    partials at absolute positions merged by kvq_merge_partials, against the oracle's attention
+    over the two ranges' reconstructions concatenated."""
+    import torch
+    import long_context_decode_nuq_b200 as K
+    w = synth.workload(name, **over)
+    K16, V16 = host_block(w, T)
+    cbK, cbV = oracle_codebooks(w)
+    dK, dV = to_dev_codebook(cbK), to_dev_codebook(cbV)
+    cap = 1 << 16
+    q16 = synth.gen_q(w)
+    qpos = torch.full((w.B,), T, dtype=torch.int32, device="cuda")
+    dq = torch.from_numpy(q16).cuda()
+    mls, os_, recon = [], [], []
+    for lo, hi in ((0, cut), (cut, T)):
+        n = hi - lo
+        g = gpu_cache(w, max(n, 1) + 16, cap, cap)
+        oc = O.QuantizedCache(w.B, w.Hkv, w.bits, max(n, 1) + 16, w.f, cap, cap)
+        if n:
+            gpu_quantize(g, dK, dV, K16[:, lo:hi], V16[:, lo:hi], calibrate=1)
+            oc.prefill(K16[:, lo:hi], V16[:, lo:hi], [n], cbK, cbV)
+            recon.append(oc.reconstruct(0, cbK, cbV))
+        ml = torch.empty((w.B, w.Hq, 2), device="cuda")
+        o = torch.empty((w.B, w.Hq, w.D), device="cuda")
+        ws = torch.empty(K.kvq_decode_workspace(g.cfg, max(n, 1), 0), dtype=torch.uint8,
+                         device="cuda")
+        K.kvq_decode_partial(g, dK, dV, dq, qpos, max(n, 1), lo, ml, o, ws, 0)
+        torch.cuda.synchronize()
+        assert K.kvq_get_status(g) == 0
+        if not n:
+            assert np.all(ml[..., 0].cpu().numpy() == -np.inf) and not o.cpu().numpy().any()
+        mls.append(ml)
+        os_.append(o)
+    out = torch.empty((w.B, w.Hq, w.D), device="cuda")
+    K.kvq_merge_partials(g.cfg, 2, torch.stack(mls), torch.stack(os_), out)
+    torch.cuda.synchronize()
+    Kx = np.concatenate([r[0] for r in recon])
+    Vx = np.concatenate([r[1] for r in recon])
+    _, _, ref = O.decode_attention(q16[0], T, Kx, Vx, w.rope_theta)
+    assert np.abs(out.cpu().numpy()[0] - ref).max() <= OUT_ATOL

@@ -179,26 +179,60 @@ def _unpack_head(words, bits):
     return np.transpose(q, (1, 0, 2)).reshape(-1, 128)
 
 
-def _head_attention(q16, qpos, kx, vx, base, chunk=1 << 16):
-    """binary64 attention of one query head over one kv head, in token chunks."""
-    qr = O.rope_rotate(np.asarray(q16, dtype=np.float64)[None], qpos, base)[0]
-    T = kx.shape[0]
-    lg = np.empty(T)
-    for a in range(0, T, chunk):
-        kr = O.rope_rotate(kx[a:a + chunk], np.arange(a, min(T, a + chunk)), base)
-        lg[a:a + chunk] = kr @ qr / math.sqrt(128)
-    p = np.exp(lg - lg.max())
-    p /= p.sum()
-    out = np.zeros(128)
-    for a in range(0, T, chunk):
-        out += p[a:a + chunk] @ vx[a:a + chunk]
-    return lg, out
+def _unpack_head3(words):
+    """_unpack_head for 3-bit blocks, vectorised over the 16 lane groups (a test helper for
+    the 1M-token check; checked against the oracle's unpacker on sampled blocks).  Lane group
+    i holds 16 six-bit fields in its three words; field 4k + s is token s ^ (i >> 2), codes of
+    channels i + 16k (low 3 bits) and i + 16k + 64 (high 3 bits)."""
+    nq = words.shape[0]
+    W = words.reshape(nq, 16, 3).astype(np.uint64)
+    A = W[..., 0] | (W[..., 1] << np.uint64(32))
+    B = W[..., 2]
+    F = np.empty((nq, 16, 16), dtype=np.uint8)
+    for f in range(16):
+        o = 6 * f
+        if o + 6 <= 64:
+            v = A >> np.uint64(o)
+        elif o < 64:
+            v = (A >> np.uint64(o)) | (B << np.uint64(64 - o))
+        else:
+            v = B >> np.uint64(o - 64)
+        F[..., f] = (v & np.uint64(63)).astype(np.uint8)
+    i = np.arange(16)[:, None, None]
+    k = np.arange(4)[None, :, None]
+    j = np.arange(4)[None, None, :]
+    ii = np.broadcast_to(i, (16, 4, 4))
+    ff = np.broadcast_to(4 * k + (j ^ (i >> 2)), (16, 4, 4))   # field of token j, channel i+16k
+    src = F[:, ii, ff]                                          # [nq, 16 i, 4 k, 4 j]
+    codes = np.empty((nq, 4, 128), dtype=np.uint8)
+    ch = (np.arange(16)[:, None] + 16 * np.arange(4)[None, :]).reshape(-1)   # i + 16k
+    lo = np.transpose(src, (0, 3, 1, 2)).reshape(nq, 4, 64)
+    codes[:, :, ch] = lo & 7
+    codes[:, :, ch + 64] = lo >> 3
+    sample = np.random.default_rng(nq).integers(0, nq, 64)
+    ref = O.unpack_block(words[sample], 3)                     # [4, 64, 128]
+    assert np.array_equal(np.transpose(ref, (1, 0, 2)), codes[sample])
+    return codes.reshape(-1, 128)
+
+
+def _device_entries(g, s, h, m):
+    """Entries of chunk m in the device list s ('k' or 'v') of (sequence 0, kv head h)."""
+    cp = u32(getattr(g, f"{s}chunk")[0, h, m:m + 2])
+    return u32(getattr(g, f"{s}out")[0, h, int(cp[0]):int(cp[1])])
 
 
 def test_llama7b_1m_layer_sampled():
-    """One layer of the 1M-token workload as bench.py builds it: sampled key channels and
-    tokens against the oracle's quantizer, and one head's attention over all 1,048,576 tokens
-    recomputed in binary64 from the device cache."""
+    """One layer of the 1M-token workload as bench.py builds it.
+
+    Quantizer, against the oracle's own quantizer:
+      * key calibration: thresholds and (off, half) of every channel of two kv heads, from the
+        oracle's order statistics over all 1,048,576 tokens;
+      * sampled 64-token chunks (several past token 131,072): key codes and key-outlier entries
+        of those heads (the oracle's QuantizedCache calibrated on the head's full columns and
+        quantizing the chunk), value (off, half), value codes and value-outlier entries of all
+        32 kv heads (the oracle quantizing the chunk's rows).
+    Attention of all 32 heads over every token, in binary64 from the device cache (whose
+    sampled rows the checks above tie to the oracle), against both decode paths."""
     import torch
     import long_context_decode_nuq_b200 as K
     w = synth.workload("llama7b_1m_32layers", layers=1)
@@ -214,64 +248,90 @@ def test_llama7b_1m_layer_sampled():
     torch.cuda.synchronize()
     assert K.kvq_get_status(g) == 0
     rng = np.random.default_rng(7)
-    # key calibration of sampled channels: exact order statistics over the million tokens
-    chans = [0, 1, 777, 2048, 4095] + rng.integers(0, w.n, 5).tolist()
+    chunks = sorted({0, 1, 2047, 2048, 2049, T // 64 - 1}
+                    | set(int(x) for x in rng.integers(2049, T // 64 - 1, 6)))
     kthr = u16(g.kthr[0])
     kpar = g.kparams[0].cpu().numpy()
-    for j in chans:
-        col = Kd[0, :, j // 128, j % 128].cpu().numpy()
-        lo, hi = O.order_stat_thresholds(col, w.f, axis=0)
-        assert kthr[j, 0] == lo.view(np.uint16) and kthr[j, 1] == hi.view(np.uint16), j
-        off, half = O.affine_params(lo, hi)
-        assert kpar[j, 0] == off and kpar[j, 1] == half, j
-    # sampled tokens: value thresholds, value codes and their outliers, key codes of the
-    # sampled channels
-    toks = [0, 1, 63, 64, T - 1] + rng.integers(0, T, 11).tolist()
+    for h in (7, 30):
+        col = Kd[0, :, h:h + 1].cpu().numpy()               # [T, 1, 128]
+        ok = O.QuantizedCache(1, 1, w.bits, 64, w.f, 64 * 128, 64 * 128)
+        ok.calibrate_keys(0, col)
+        sl = slice(h * 128, (h + 1) * 128)
+        assert np.array_equal(kthr[sl], ok.kthr[0]), h
+        assert np.array_equal(kpar[sl], ok.kparams[0]), h
+        for m in chunks:
+            oc = O.QuantizedCache(1, 1, w.bits, 64, w.f, 64 * 128, 64 * 128)
+            oc.kthr[:], oc.kparams[:] = ok.kthr, ok.kparams
+            rows = slice(64 * m, 64 * m + 64)
+            oc.quantize_tokens(0, 0, col[rows], Vd[0, rows, h:h + 1].cpu().numpy(), cbK, cbV)
+            assert np.array_equal(u32(g.kcodes[0, h, 16 * m:16 * m + 16]), oc.kcodes[0, 0]), (h, m)
+            n = int(oc.out_count["k"][0, 0])
+            assert np.array_equal(_device_entries(g, "k", h, m), oc.out["k"][0, 0, :n]), (h, m)
     vpar = g.vparams[0].cpu().numpy()
-    kc_all = {h: None for h in range(w.Hkv)}
-    for t in toks:
-        row = Vd[0, t].reshape(-1).cpu().numpy()
-        lo, hi = O.order_stat_thresholds(row[None], w.f, axis=1)
-        off, half = O.affine_params(lo[0], hi[0])
-        assert vpar[t, 0] == off and vpar[t, 1] == half, t
-        vout = (row < lo[0]) | (row > hi[0])
-        codes = O.encode(O.normalize(np.where(vout, np.float16(0), row), off, half), cbV[1])
-        blk = u32(g.vcodes[0, :, t // 4])              # [Hkv, 16*bits]
-        got = O.unpack_block(blk, w.bits)[t % 4].reshape(-1)
-        assert np.array_equal(got, codes), t
-        krow = Kd[0, t].reshape(-1).cpu().numpy()
-        kblk = O.unpack_block(u32(g.kcodes[0, :, t // 4]), w.bits)[t % 4].reshape(-1)
-        for j in chans:
-            lo_j = kthr[j, 0].view(np.float16)
-            hi_j = kthr[j, 1].view(np.float16)
-            x = krow[j]
-            xk = np.float16(0) if (x < lo_j or x > hi_j) else x
-            cj = O.encode(O.normalize(np.array([xk]), kpar[j, 0], kpar[j, 1]), cbK[1])[0]
-            assert kblk[j] == cj, (t, j)
-    # one head's attention over every token, from the device cache
-    h = 7
+    for m in chunks:
+        rows = slice(64 * m, 64 * m + 64)
+        ov = O.QuantizedCache(1, w.Hkv, w.bits, 64, w.f, 64 * 128, 64 * 128)
+        ov.prefill(Kd[:, rows].cpu().numpy(), Vd[:, rows].cpu().numpy(), [64], cbK, cbV)
+        assert np.array_equal(vpar[rows], ov.vparams[0]), m
+        assert np.array_equal(u32(g.vcodes[0, :, 16 * m:16 * m + 16]), ov.vcodes[0]), m
+        for h in range(w.Hkv):
+            n = int(ov.out_count["v"][0, h])
+            assert np.array_equal(_device_entries(g, "v", h, m), ov.out["v"][0, h, :n]), (h, m)
+    # attention of every head over every token, from the device cache: the oracle's
+    # decode_attention per head, heads spread over a spawn-started process pool
     q = _device_q(w)
     qpos = torch.full((w.B,), T, dtype=torch.int32, device="cuda")
     out, out2, logits = _attend(g, dK, dV, q, qpos, T)
-    kc = _unpack_head(u32(g.kcodes[0, h]), w.bits)[:T]
-    vc = _unpack_head(u32(g.vcodes[0, h]), w.bits)[:T]
-    levK = np.asarray(cbK[0], dtype=np.float64)
-    levV = np.asarray(cbV[0], dtype=np.float64)
-    kp = kpar[h * 128:(h + 1) * 128].astype(np.float64)
-    vp = vpar[:T].astype(np.float64)
-    kx = kp[:, 0] + kp[:, 1] * levK[kc]
-    vx = vp[:, 0:1] + vp[:, 1:2] * levV[vc]
-    for s, X in (("k", kx), ("v", vx)):
-        n = int(u32(getattr(g, f"{s}count"))[0, h])
-        ent = u32(getattr(g, f"{s}out")[0, h, :n]).astype(np.int64)
-        nch = (T + 63) // 64                                      # chunks of the cached tokens
-        cp = u32(getattr(g, f"{s}chunk")[0, h, :nch + 1]).astype(np.int64)
-        m = np.searchsorted(cp, np.arange(n), side="right") - 1   # chunk of each entry
-        t = m * 64 + ((ent >> 7) & 63)
-        X[t, ent & 127] = (ent >> 16).astype(np.uint16).view(np.float16).astype(np.float64)
-    for hq in (h,):
-        lg_ref, o_ref = _head_attention(q.cpu().numpy()[0, hq], T, kx, vx, w.rope_theta)
-        assert np.abs(out[0, hq] - o_ref).max() <= OUT_ATOL
-        assert np.abs(out2[0, hq] - o_ref).max() <= OUT_ATOL
+    nch = (T + 63) // 64
+    q16 = q.cpu().numpy()[0]
+    jobs = []
+    for h in range(w.Hkv):
+        lists = {}
+        for s_ in ("k", "v"):
+            n = int(u32(getattr(g, f"{s_}count"))[0, h])
+            lists[s_] = (u32(getattr(g, f"{s_}out")[0, h, :n]),
+                         u32(getattr(g, f"{s_}chunk")[0, h, :nch + 1]))
+        jobs.append((q16[h], T, u32(g.kcodes[0, h]), u32(g.vcodes[0, h]),
+                     kpar[h * 128:(h + 1) * 128], vpar[:T], lists, cbK[0], cbV[0], w.rope_theta))
+    for h, (lg_ref, o_ref) in enumerate(_pool_map(_head_reference, jobs)):
+        assert np.abs(out[0, h] - o_ref).max() <= OUT_ATOL, h
+        assert np.abs(out2[0, h] - o_ref).max() <= OUT_ATOL, h
         tol = LOGIT_RTOL * max(1.0, np.abs(lg_ref).max())
-        assert np.abs(logits[0, hq, :T] - lg_ref).max() <= tol
+        assert np.abs(logits[0, h, :T] - lg_ref).max() <= tol, h
+
+
+def _head_reference(job):
+    """One kv head (one query head) of the 1M-token check: rebuild the head's exact K-hat and
+    V-hat from the device codes and outlier lists (off + half L[code], outliers replaced by
+    their stored value) and run the oracle's binary64 decode attention on them."""
+    q16, T, kwords, vwords, kp, vp, lists, levK, levV, base = job
+    kc = _unpack_head3(kwords)[:T]
+    vc = _unpack_head3(vwords)[:T]
+    kp = kp.astype(np.float64)
+    vp = vp.astype(np.float64)
+    kx = kp[:, 0] + kp[:, 1] * np.asarray(levK, dtype=np.float64)[kc]
+    vx = vp[:, 0:1] + vp[:, 1:2] * np.asarray(levV, dtype=np.float64)[vc]
+    del kc, vc
+    for s_, X in (("k", kx), ("v", vx)):
+        ent, cp = lists[s_]
+        ent = ent.astype(np.int64)
+        mm = np.searchsorted(cp.astype(np.int64), np.arange(len(ent)), side="right") - 1
+        t = mm * 64 + ((ent >> 7) & 63)
+        X[t, ent & 127] = (ent >> 16).astype(np.uint16).view(np.float16).astype(np.float64)
+    lg, _, out = O.decode_attention(q16[None], T, kx[:, None], vx[:, None], base)
+    return lg[0], out[0]
+
+
+def _pool_map(fn, jobs):
+    """Map over a process pool started with spawn (safe after CUDA use), sized to the host."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    import os
+    try:
+        import psutil
+        mem_workers = int(psutil.virtual_memory().available // (8 << 30))
+    except Exception:  # pragma: no cover
+        mem_workers = 4
+    n = max(1, min(len(jobs), os.cpu_count() or 1, mem_workers, 16))
+    with cf.ProcessPoolExecutor(max_workers=n, mp_context=mp.get_context("spawn")) as ex:
+        return list(ex.map(fn, jobs))

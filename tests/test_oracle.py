@@ -563,3 +563,37 @@ def test_reconstruct_is_exact_affine_and_rounds_to_dequantize():
         assert np.abs(X - H.astype(np.float64)).max() <= np.abs(X).max() * 2 ** -10
     for t_, j_, bits in c.outlier_entries("v", 0):
         assert Vx.reshape(T, -1)[t_, j_] == float(np.uint16(bits).view(np.float16))
+
+
+# ---------------------------------------------------------------------------------------------
+# Token-range partials and their merge (the token-sharded decode)
+
+
+def test_partials_of_any_split_merge_to_the_whole():
+    rng = np.random.default_rng(11)
+    T, Hkv, Hq, D = 300, 2, 4, 128
+    Kh = rng.standard_normal((T, Hkv, D))
+    Vh = rng.standard_normal((T, Hkv, D))
+    q = rng.standard_normal((Hq, D)).astype(np.float16)
+    _, _, ref = O.decode_attention(q, T, Kh, Vh, 1e4)
+    for cuts in ([0, 300], [0, 64, 300], [0, 0, 100, 250, 300], [0, 299, 300]):
+        parts = [O.partial_attention(q, T, Kh[a:b], Vh[a:b], 1e4, np.arange(a, b))
+                 for a, b in zip(cuts[:-1], cuts[1:])]
+        M, L, o = (np.stack(x) for x in zip(*parts))
+        assert np.abs(O.merge_partials(M, L, o) - ref).max() < 1e-12
+    # an empty range contributes nothing
+    M, L, o = O.partial_attention(q, T, Kh[:0], Vh[:0], 1e4, np.arange(0))
+    assert np.all(M == -np.inf) and not L.any() and not o.any()
+
+
+def test_key_positions_shift_with_the_query():
+    # RoPE logits depend only on (query position - key position)
+    rng = np.random.default_rng(12)
+    T, D = 50, 128
+    Kh = rng.standard_normal((T, 1, D))
+    Vh = rng.standard_normal((T, 1, D))
+    q = rng.standard_normal((1, D)).astype(np.float16)
+    a = O.decode_attention(q, T, Kh, Vh, 1e4)
+    b = O.decode_attention(q, T + 1000, Kh, Vh, 1e4, kpos=np.arange(T) + 1000)
+    assert np.abs(a[0] - b[0]).max() < 1e-9
+    assert np.abs(a[2] - b[2]).max() < 1e-9
