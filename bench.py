@@ -41,8 +41,10 @@ def parse():
     p.add_argument("--workload", default="llama7b_1m_32layers")
     p.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
     p.add_argument("--splits", type=int, default=0)
-    p.add_argument("--path", default="split", choices=["split", "one-call"],
-                   help="split: kvq_decode_qk + kvq_softmax_merge + kvq_decode_pv; one-call: kvq_decode_attention")
+    p.add_argument("--path", default="split", choices=["split", "one-call", "fused"],
+                   help="split: kvq_decode_qk + kvq_softmax_merge + kvq_decode_pv; one-call: "
+                        "kvq_decode_attention (the same kernels); fused: "
+                        "kvq_decode_attention_fused (one kernel per split, no logits)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-fp16", action="store_true")
     p.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
@@ -194,7 +196,8 @@ def bytes_model(w, T, kcount, vcount, path, outlier_bytes=OUTLIER_ENTRY_BYTES, l
     value), key chunk pointers (one list per kv head); value side (PV): packed value codes,
     value-outlier entries, value token params (8 B/token), value chunk pointers.  The split
     path (kvq_decode_qk / kvq_softmax_merge / kvq_decode_pv) also writes and reads fp32 logits
-    (4 B per token per query head, each way); the fused one-call path moves no logits.
+    (4 B per token per query head, each way), and so does kvq_decode_attention, which runs the
+    same kernels; the fused path (kvq_decode_attention_fused) moves no logits.
     """
     code_row = w.Hkv * w.D * w.bits // 8
     nch = (T + 63) // 64 + 1
@@ -203,6 +206,8 @@ def bytes_model(w, T, kcount, vcount, path, outlier_bytes=OUTLIER_ENTRY_BYTES, l
     logit = 4 * w.Hq * T if logits else 0
     if path == "split":
         return {"qk": k_bytes + logit, "pv": v_bytes + logit, "total": k_bytes + v_bytes + 2 * logit}
+    if path == "one-call":
+        return {"attn": k_bytes + v_bytes + 2 * logit, "total": k_bytes + v_bytes + 2 * logit}
     return {"attn": k_bytes + v_bytes, "total": k_bytes + v_bytes}
 
 
@@ -435,7 +440,11 @@ def run_kvq(args, rank, world):
             if timing:
                 marks[2].record()
                 marks[3].record()
-            K.kvq_decode_attention(c, cbK, cbV, qall[i, s], qpos[s], max_len, outs[i], dws, S)
+            if args.path == "fused":
+                K.kvq_decode_attention_fused(c, cbK, cbV, qall[i, s], qpos[s], max_len, outs[i],
+                                             dws, S)
+            else:
+                K.kvq_decode_attention(c, cbK, cbV, qall[i, s], qpos[s], max_len, outs[i], dws, S)
         if timing:
             marks[4].record()
         return marks
@@ -523,6 +532,9 @@ def run_kvq(args, rank, world):
                 K.kvq_decode_qk(c, cbs[i][0], d_q[i], qpos_e2e[j], ml_len, logits, stats, S, qkws)
                 K.kvq_softmax_merge(cfg, stats, S, mlb)
                 K.kvq_decode_pv(c, cbs[i][1], logits, mlb, ml_len, outs[i], part, S)
+            elif args.path == "fused":
+                K.kvq_decode_attention_fused(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j],
+                                             ml_len, outs[i], dws, S)
             else:
                 K.kvq_decode_attention(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j], ml_len,
                                        outs[i], dws, S)
@@ -577,12 +589,13 @@ def run_kvq(args, rank, world):
 
     if rank != 0:
         return 0
-    # append: begin, stats, scan, write; split path: qk (tables, qk, key outliers, split
-    # stats), merge, pv (pv, value outliers, split sum); one-call path for kv heads of one
-    # query head with 2/3-bit codes: tables, the fused kernel, split merge
-    fused = w.Hq == w.Hkv and w.bits <= 3
-    launches_per_layer_step = (4 if appends_here else 0) + (
-        8 if args.path == "split" and not sharded else (3 if fused else 8)) + (1 if sharded else 0)
+    # append: begin, stats, scan, write; split kernels: qk (tables, qk, key outliers, split
+    # stats), merge, pv (pv, value outliers, split sum); fused: tables, fused kernel, merge;
+    # sharded: the split kernels and the conversion to a partial, then one merge of the
+    # gathered partials
+    fused_path = args.path == "fused" and not sharded
+    launches_per_layer_step = (4 if appends_here else 0) + (3 if fused_path else 8) + (
+        2 if sharded else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,

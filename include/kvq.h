@@ -245,7 +245,7 @@ int kvq_decode_workspace(const kvq_cfg* cfg, int32_t max_len, int32_t splits, si
  * Decode attention in one call: kvq_decode_qk, kvq_softmax_merge and kvq_decode_pv
  * on `stream`, with their buffers (logits [B][Hq][T_max], split statistics, (M, L),
  * split partials, per-call tables) carved from `workspace`; the same result as the
- * three calls; out float [B][Hq][D].
+ * three calls, the same bits on every run; out float [B][Hq][D].
  *   workspace  device scratch of kvq_decode_workspace bytes, 16-byte aligned
  */
 int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
@@ -281,6 +281,27 @@ int kvq_decode_partial(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_cod
  */
 int kvq_merge_partials(const kvq_cfg* cfg, int32_t parts, const float* ml, const float* o,
                        float* out, void* stream);
+
+/*
+ * Decode attention in one fused pass per (split, sequence, head): QK with NUQ lookup and RoPE,
+ * the key-outlier correction, an online softmax, PV and the value-outlier correction in one
+ * kernel, then the split merge (the custom decode kernels of the study.space summary, here
+ * without a logits buffer).  The same result as kvq_decode_attention up to rounding, summed in
+ * a fixed order (the same bits on every run).  For kv heads that serve one query head each
+ * (Hq == Hkv) and bits 2 or 3 (KVQ_ERR_UNSUPPORTED otherwise); the value levels must have the
+ * (u << 16) | u form the codebook contract states (else KVQ_STATUS_CODEBOOK is set).
+ *   workspace  kvq_decode_fused_workspace bytes: no [B][Hq][T_max] logits, so far smaller
+ *              than kvq_decode_workspace at long contexts (134 MB less at 2^20 tokens x 32 heads)
+ */
+int kvq_decode_attention_fused(const kvq_cfg* cfg, const kvq_cache* cache,
+                               const kvq_codebook* cbK, const kvq_codebook* cbV,
+                               const uint16_t* q, const int32_t* qpos, int32_t max_len,
+                               float* out, void* workspace, size_t workspace_bytes,
+                               int32_t splits, void* stream);
+
+/* Workspace bytes of kvq_decode_attention_fused (KVQ_ERR_UNSUPPORTED for other shapes). */
+int kvq_decode_fused_workspace(const kvq_cfg* cfg, int32_t max_len, int32_t splits,
+                               size_t* bytes);
 
 /*
  * Dequantize rows [t0, t0 + nt) of every sequence (test support):

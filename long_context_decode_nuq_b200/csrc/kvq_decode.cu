@@ -1870,6 +1870,13 @@ extern "C" int kvq_decode_pv(const kvq_cfg* cfg, const kvq_cache* cache, const k
     return run_pv(cfg, cache, cbV, logits, ml, max_len, out, part, S, Ls, (cudaStream_t)stream);
 }
 
+// The fused path's workspace: the split path's without the [B][Hq][T_max] logits.
+static size_t fused_ws_bytes(const kvq_cfg* cfg, int S, int max_len) {
+    const size_t BH = (size_t)cfg->B * cfg->Hq;
+    return align_up(BH * S * 8) + align_up(BH * 8) + align_up(BH * S * kD * 4) +
+           qk_tables(cfg, max_len, nullptr).bytes;
+}
+
 static size_t split_ws_bytes(const kvq_cfg* cfg, int S, int max_len) {
     const size_t BH = (size_t)cfg->B * cfg->Hq;
     return align_up(BH * (size_t)cfg->T_max * 4)   // logits
@@ -1896,7 +1903,8 @@ extern "C" int kvq_decode_workspace(const kvq_cfg* cfg, int32_t max_len, int32_t
 static int decode_core(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook* cbK,
                        const kvq_codebook* cbV, const uint16_t* q, const int32_t* qpos,
                        int32_t max_len, int32_t pos_off, float* out, float2* ml_part,
-                       void* workspace, size_t workspace_bytes, int32_t splits, void* stream) {
+                       void* workspace, size_t workspace_bytes, int32_t splits, void* stream,
+                       bool fused = false) {
     int e = check_decode(cfg, max_len);
     if (e) return e;
     if ((e = check_cache(cfg, cache)) || (e = check_codebook(cbK)) || (e = check_codebook(cbV)))
@@ -1906,11 +1914,13 @@ static int decode_core(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_cod
     if (pos_off < 0 || (int64_t)pos_off + max_len > (int64_t)1 << 30) return KVQ_ERR_RANGE;
     int S, Ls;
     if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
-    if (workspace_bytes < split_ws_bytes(cfg, S, max_len)) return KVQ_ERR_WORKSPACE;
+    if (fused && !fused_supported(cfg)) return KVQ_ERR_UNSUPPORTED;
+    if (workspace_bytes < (fused ? fused_ws_bytes(cfg, S, max_len) : split_ws_bytes(cfg, S, max_len)))
+        return KVQ_ERR_WORKSPACE;
     const size_t BH = (size_t)cfg->B * cfg->Hq;
     char* w = (char*)workspace;
     float* logits = (float*)w;
-    w += align_up(BH * (size_t)cfg->T_max * 4);
+    if (!fused) w += align_up(BH * (size_t)cfg->T_max * 4);
     float* stats = (float*)w;
     w += align_up(BH * S * 8);
     float* ml = (float*)w;
@@ -1919,7 +1929,7 @@ static int decode_core(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_cod
     w += align_up(BH * S * kD * 4);
     const QKTables T = qk_tables(cfg, max_len, w);
     cudaStream_t st = (cudaStream_t)stream;
-    if (fused_supported(cfg)) {
+    if (fused) {
         // one pass: per-call tables, the fused kernel's per-split (m, l, o), the split merge
         const int n = cfg->B * cfg->Hq * 64 + T.nhi * 64 + kTrigLo * 64 + cfg->B * cfg->Hkv * kD;
         k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi,
@@ -1949,6 +1959,27 @@ extern "C" int kvq_decode_attention(const kvq_cfg* cfg, const kvq_cache* cache,
                                     int32_t splits, void* stream) {
     return decode_core(cfg, cache, cbK, cbV, q, qpos, max_len, 0, out, nullptr, workspace,
                        workspace_bytes, splits, stream);
+}
+
+extern "C" int kvq_decode_fused_workspace(const kvq_cfg* cfg, int32_t max_len, int32_t splits,
+                                          size_t* bytes) {
+    int e = check_decode(cfg, max_len);
+    if (e) return e;
+    if (!bytes) return KVQ_ERR_NULL;
+    if (!fused_supported(cfg)) return KVQ_ERR_UNSUPPORTED;
+    int S, Ls;
+    if ((e = resolve_splits(cfg, max_len, splits, &S, &Ls))) return e;
+    *bytes = fused_ws_bytes(cfg, S, max_len);
+    return KVQ_OK;
+}
+
+extern "C" int kvq_decode_attention_fused(const kvq_cfg* cfg, const kvq_cache* cache,
+                                          const kvq_codebook* cbK, const kvq_codebook* cbV,
+                                          const uint16_t* q, const int32_t* qpos, int32_t max_len,
+                                          float* out, void* workspace, size_t workspace_bytes,
+                                          int32_t splits, void* stream) {
+    return decode_core(cfg, cache, cbK, cbV, q, qpos, max_len, 0, out, nullptr, workspace,
+                       workspace_bytes, splits, stream, true);
 }
 
 extern "C" int kvq_decode_partial(const kvq_cfg* cfg, const kvq_cache* cache,

@@ -5,16 +5,17 @@
 // (i)-(iv): study.space summary, custom kernels for memory- and bandwidth-bound decode;
 // phantomic12 research note, components (1)-(4).)
 //
-// A CTA has 16 consumer warps and two helper warps and walks its split in 256-token stages
+// A CTA has 16 consumer warps and three helper warps and walks its split in 256-token stages
 // through a ring of kFSlots shared-memory slots.
-//  - Streaming warp: per stage, bulk copies (cp.async.bulk, completion counted on an
-//    mbarrier; no multicast) of the key code blocks, the tokens' value (off, half), and the
-//    stage's key- and value-outlier entries (up to kFEnt of each; entries past that are read
-//    from global memory), plus the (cos, sin) of the stage start for the 64 RoPE pairs.  One
-//    stage later, once that stage's copies have landed, the key-outlier correction of every
-//    token, kc[tau] = sum over the token's entries of (x - zhat_c) r, r the rotated query
-//    component that meets channel c at the token (entries summed in list order by a
-//    segmented scan, so the result is the same on every run).
+//  - Issuing warp: per stage, bulk copies (cp.async.bulk, completion counted on an mbarrier;
+//    no multicast) of the key code blocks, the tokens' value (off, half), and the stage's key-
+//    and value-outlier entries (up to kFEnt of each; entries past that are read from global
+//    memory).  It waits only for the slot to be released, so copies run a full ring ahead.
+//  - Key warp: per stage, the (cos, sin) of the stage start for the 64 RoPE pairs and, once
+//    the stage's copies have landed, the key-outlier correction of every token,
+//    kc[tau] = sum over the token's entries of (x - zhat_c) r, r the rotated query component
+//    that meets channel c at the token, each term added in 2^-32 fixed point with an integer
+//    atomic (associative, so the sum is the same on every run).
 //  - Value helper: per stage, once its copies have landed, the dense value the cache holds at
 //    a value outlier of each token, zv = off + half L[code of 0], and the first value-outlier
 //    entry of each 16-token slice of the stage.
@@ -38,7 +39,7 @@ namespace {
 
 constexpr int kFW = 16;                   // consumer warps
 constexpr int kFCons = kFW * 32;          // consumer threads
-constexpr int kFThreads = kFCons + 64;    // + streaming warp + value-helper warp
+constexpr int kFThreads = kFCons + 96;    // + issuing, key and value-helper warps
 constexpr int kFQuads = 64;               // token quads per stage
 constexpr int kFTok = 4 * kFQuads;        // tokens per stage (the lo trig table spans a stage)
 constexpr int kFSlots = 3;                // stages in flight
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     if (tid == 0) {
         for (int k = 0; k < kFSlots; ++k) {
             mbar_init(bcopy + k, 1);
-            mbar_init(full + k, 2);
+            mbar_init(full + k, 2);   // key warp, value helper
             mbar_init(empty + k, kFW);
         }
         flag[0] = 0;
@@ -246,7 +247,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // entries), 4..6 the key chunk boundaries, 7 the stage's chunks, 8 vB, 9 vN, 10 vE0, 11 vE1,
     // 12..14 the value chunk boundaries, 15 value params staged
     if (warp == kFW) {
-        // ================= streaming warp
+        // ================= issuing warp: the stage's side record and its bulk copies
         const uint32_t* ksrc = c.kcodes + li * nquads(cfg.T_max) * F::BW;
         const uint32_t* kcp = c.kchunk + li * (nchunks(cfg.T_max) + 1);
         const uint32_t* vcp = c.vchunk + li * (nchunks(cfg.T_max) + 1);
@@ -260,127 +261,133 @@ __global__ void __launch_bounds__(kFThreads, 1)
         };
         load_cp(0);
         int issued = 0;
-        float2 thv[2], tlv[2];  // (cos, sin) tables of the stage being issued
-        for (int cc = 0; cc <= nst; ++cc) {
-            if (cc < nst) {
-                const int slot = cc % kFSlots;
-                if (cc >= kFSlots &&
-                    !warp_wait(empty + slot, (uint32_t)(cc / kFSlots - 1) & 1u, flag, c.status))
-                    break;
-                if (__shfl_sync(0xffffffffu, *(volatile int*)flag, 0)) break;
-                const int tc = t_begin + cc * kFTok, m0 = tc >> 6;
-                const int nm = min(4, ((t_end + 63) >> 6) - m0);
-                const int n = min(kFTok, t_end - tc);
-                // value params: an even count from a 16-byte aligned start, so the copy is a
-                // whole number of 16-byte units; none staged when the row starts mid-unit (the
-                // readers then load them from global memory)
-                const bool va = (((size_t)b * cfg.T_max + tc) & 1) == 0;
-                const int nv = !va ? 0 : !(n & 1) ? n : (tc + n + 1 <= cfg.T_max ? n + 1 : n - 1);
-                uint32_t sv[kFSide];
-                sv[2] = __shfl_sync(0xffffffffu, kcpl, 0);
-                sv[3] = __shfl_sync(0xffffffffu, kcpl, nm);
-                sv[10] = __shfl_sync(0xffffffffu, vcpl, 0);
-                sv[11] = __shfl_sync(0xffffffffu, vcpl, nm);
+        for (int cc = 0; cc < nst; ++cc) {
+            const int slot = cc % kFSlots;
+            if (cc >= kFSlots &&
+                !warp_wait(empty + slot, (uint32_t)(cc / kFSlots - 1) & 1u, flag, c.status))
+                break;
+            if (__shfl_sync(0xffffffffu, *(volatile int*)flag, 0)) break;
+            const int tc = t_begin + cc * kFTok;
+            const int nm = min(4, ((t_end + 63) >> 6) - (tc >> 6));
+            const int n = min(kFTok, t_end - tc);
+            // value params: an even count from a 16-byte aligned start, so the copy is a
+            // whole number of 16-byte units; none staged when the row starts mid-unit (the
+            // readers then load them from global memory)
+            const bool va = (((size_t)b * cfg.T_max + tc) & 1) == 0;
+            const int nv = !va ? 0 : !(n & 1) ? n : (tc + n + 1 <= cfg.T_max ? n + 1 : n - 1);
+            uint32_t sv[kFSide];
+            sv[2] = __shfl_sync(0xffffffffu, kcpl, 0);
+            sv[3] = __shfl_sync(0xffffffffu, kcpl, nm);
+            sv[10] = __shfl_sync(0xffffffffu, vcpl, 0);
+            sv[11] = __shfl_sync(0xffffffffu, vcpl, nm);
 #pragma unroll
-                for (int k = 1; k < 4; ++k) {
-                    sv[3 + k] = __shfl_sync(0xffffffffu, kcpl, k);
-                    sv[11 + k] = __shfl_sync(0xffffffffu, vcpl, k);
-                }
-                sv[7] = (uint32_t)nm;
-                sv[15] = (uint32_t)nv;
-                sv[0] = sv[2] & ~3u;
-                sv[1] = min(((sv[3] + 3u) & ~3u) - sv[0], (uint32_t)kFEnt);
-                sv[8] = sv[10] & ~3u;
-                sv[9] = min(((sv[11] + 3u) & ~3u) - sv[8], (uint32_t)kFEnt);
-                if (sv[3] == sv[2]) sv[1] = 0;
-                if (sv[11] == sv[10]) sv[9] = 0;
-                if (lane == 0) {
-#pragma unroll
-                    for (int k = 0; k < kFSide; ++k) side[slot * kFSide + k] = sv[k];
-                }
-                __syncwarp();  // the side record is complete before the copies are announced
-                if (lane == 0) {
-                    fence_proxy_async();
-                    const int q0 = tc >> 2, q1 = (min(tc + kFTok, t_end) + 3) >> 2;
-                    const uint32_t kbytes = (uint32_t)(q1 - q0) * F::BW * 4;
-                    mbar_arrive_expect_tx(bcopy + slot,
-                                          kbytes + 8u * (uint32_t)nv + 4u * (sv[1] + sv[9]));
-                    bulk_load(ring + (size_t)slot * L.stage, ksrc + (size_t)q0 * F::BW, kbytes,
-                              bcopy + slot);
-                    if (nv) bulk_load(vps + slot * kFTok, vpar + tc, 8u * nv, bcopy + slot);
-                    if (sv[1]) bulk_load(kents + slot * kFEnt, kent + sv[0], 4u * sv[1], bcopy + slot);
-                    if (sv[9]) bulk_load(vents + slot * kFEnt, vent + sv[8], 4u * sv[9], bcopy + slot);
-                }
-                // the stage's start phases: requested now, stored after the corrections below
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    thv[u] = thi[(tc / kTrigLo) * 64 + lane + 32 * u];
-                    tlv[u] = tlo[(tc % kTrigLo) * 64 + lane + 32 * u];
-                }
-                issued = cc + 1;
-                if (cc + 1 < nst) load_cp(cc + 1);
+            for (int k = 1; k < 4; ++k) {
+                sv[3 + k] = __shfl_sync(0xffffffffu, kcpl, k);
+                sv[11 + k] = __shfl_sync(0xffffffffu, vcpl, k);
             }
-            if (cc >= 1) {
-                // ---- key-outlier corrections of the previous stage, from its staged entries
-                const int ps = (cc - 1) % kFSlots;
-                if (!warp_wait(bcopy + ps, (uint32_t)((cc - 1) / kFSlots) & 1u, flag, c.status))
-                    break;
-                const uint32_t* sd = side + ps * kFSide;
-                const uint32_t kB = sd[0], kN = sd[1], E0 = sd[2], E1 = sd[3];
-                const uint32_t bd1 = sd[4], bd2 = sd[5], bd3 = sd[6];
-                const int nm = (int)sd[7];
-                const int tc = t_begin + (cc - 1) * kFTok;
-                const float4* bs = base + ps * 64;
-                const uint32_t* se = kents + ps * kFEnt;
-                unsigned long long* kcs = kc + ps * kFTok;
-                for (int j = lane; j < kFTok; j += 32) kcs[j] = 0ull;
-                __syncwarp();
-                // each entry's term in 2^-32 fixed point, added with an integer atomic: the sum
-                // of a token's terms does not depend on their order.  A term is below 2^17 *
-                // |q| in magnitude (|x - zhat| < 2^17), far inside the 2^31 range.
-                constexpr int kKB = 8;
-                for (uint32_t EW = E0; EW < E1; EW += 32 * kKB) {
-                    uint32_t wv[kKB];
-                    int kv[kKB];
-                    float2 rv[kKB];
+            sv[7] = (uint32_t)nm;
+            sv[15] = (uint32_t)nv;
+            sv[0] = sv[2] & ~3u;
+            sv[1] = min(((sv[3] + 3u) & ~3u) - sv[0], (uint32_t)kFEnt);
+            sv[8] = sv[10] & ~3u;
+            sv[9] = min(((sv[11] + 3u) & ~3u) - sv[8], (uint32_t)kFEnt);
+            if (sv[3] == sv[2]) sv[1] = 0;
+            if (sv[11] == sv[10]) sv[9] = 0;
+            if (lane == 0) {
 #pragma unroll
-                    for (int u = 0; u < kKB; ++u) {
-                        const uint32_t e = EW + 32 * u + lane;
-                        wv[u] = e < E1 ? (e - kB < kN ? se[e - kB] : kent[e]) : 0u;
-                        const int mc =
-                            (nm > 1 && e >= bd1) + (nm > 2 && e >= bd2) + (nm > 3 && e >= bd3);
-                        const int tau = mc * kChunk + (int)((wv[u] >> 7) & 63u);
-                        kv[u] = (e < E1 && tc + tau < t_end) ? tau : -1;
-                        rv[u] = tlo[(kv[u] >= 0 ? kv[u] : 0) * 64 + (int)(wv[u] & 63u)];
-                    }
-#pragma unroll
-                    for (int u = 0; u < kKB; ++u) {
-                        if (kv[u] < 0) continue;
-                        const uint32_t w = wv[u];
-                        const int ch = (int)(w & 127u), p = ch & 63;
-                        const float d = h2f((uint16_t)(w >> 16)) - zks[ch];
-                        const float4 bq = bs[p];
-                        const float2 cs = cmul(make_float2(bq.x, bq.z), rv[u]);
-                        // rotate-half: channel c < 64 meets (cos, sin) . (q_p, q_p+64), c >= 64 the other
-                        const float sa = ch < 64 ? cs.x : -cs.y, sb = ch < 64 ? cs.y : cs.x;
-                        const float v = d * fmaf(sa, qs[p], sb * qs[p + 64]);
-                        atomicAdd(kcs + kv[u], (unsigned long long)__float2ll_rn(v * kKcScale));
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(full + ps);
+                for (int k = 0; k < kFSide; ++k) side[slot * kFSide + k] = sv[k];
             }
-            if (cc < nst) {
-                float4* bs = base + (cc % kFSlots) * 64;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const float2 cs = cmul(thv[u], tlv[u]);
-                    bs[lane + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
-                }
+            __syncwarp();  // the side record is complete before the copies are announced
+            if (lane == 0) {
+                fence_proxy_async();
+                const int q0 = tc >> 2, q1 = (min(tc + kFTok, t_end) + 3) >> 2;
+                const uint32_t kbytes = (uint32_t)(q1 - q0) * F::BW * 4;
+                mbar_arrive_expect_tx(bcopy + slot,
+                                      kbytes + 8u * (uint32_t)nv + 4u * (sv[1] + sv[9]));
+                bulk_load(ring + (size_t)slot * L.stage, ksrc + (size_t)q0 * F::BW, kbytes,
+                          bcopy + slot);
+                if (nv) bulk_load(vps + slot * kFTok, vpar + tc, 8u * nv, bcopy + slot);
+                if (sv[1]) bulk_load(kents + slot * kFEnt, kent + sv[0], 4u * sv[1], bcopy + slot);
+                if (sv[9]) bulk_load(vents + slot * kFEnt, vent + sv[8], 4u * sv[9], bcopy + slot);
             }
+            issued = cc + 1;
+            if (cc + 1 < nst) load_cp(cc + 1);
         }
         if (lane == 0) flag[1] = issued;  // stages whose copies were issued
     } else if (warp == kFW + 1) {
+        // ================= key warp: the stage's start phases and key-outlier corrections
+        float2 thv[2], tlv[2];  // (cos, sin) tables of the next stage
+        auto load_tr = [&](int st) {
+            const int tc = t_begin + st * kFTok;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                thv[u] = thi[(tc / kTrigLo) * 64 + lane + 32 * u];
+                tlv[u] = tlo[(tc % kTrigLo) * 64 + lane + 32 * u];
+            }
+        };
+        load_tr(0);
+        for (int cc = 0; cc < nst; ++cc) {
+            const int ps = cc % kFSlots;
+            if (cc >= kFSlots &&
+                !warp_wait(empty + ps, (uint32_t)(cc / kFSlots - 1) & 1u, flag, c.status))
+                break;
+            {
+                float4* bsw = base + ps * 64;
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const float2 cs = cmul(thv[u], tlv[u]);
+                    bsw[lane + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
+                }
+            }
+            if (cc + 1 < nst) load_tr(cc + 1);
+            if (!warp_wait(bcopy + ps, (uint32_t)(cc / kFSlots) & 1u, flag, c.status)) break;
+            __syncwarp();
+            const uint32_t* sd = side + ps * kFSide;
+            const uint32_t kB = sd[0], kN = sd[1], E0 = sd[2], E1 = sd[3];
+            const uint32_t bd1 = sd[4], bd2 = sd[5], bd3 = sd[6];
+            const int nm = (int)sd[7];
+            const int tc = t_begin + cc * kFTok;
+            const float4* bs = base + ps * 64;
+            const uint32_t* se = kents + ps * kFEnt;
+            unsigned long long* kcs = kc + ps * kFTok;
+            for (int j = lane; j < kFTok; j += 32) kcs[j] = 0ull;
+            __syncwarp();
+            // each entry's term in 2^-32 fixed point, added with an integer atomic: the sum
+            // of a token's terms does not depend on their order.  A term is below 2^17 *
+            // |q| in magnitude (|x - zhat| < 2^17), far inside the 2^31 range.
+            constexpr int kKB = 8;
+            for (uint32_t EW = E0; EW < E1; EW += 32 * kKB) {
+                uint32_t wv[kKB];
+                int kv[kKB];
+                float2 rv[kKB];
+#pragma unroll
+                for (int u = 0; u < kKB; ++u) {
+                    const uint32_t e = EW + 32 * u + lane;
+                    wv[u] = e < E1 ? (e - kB < kN ? se[e - kB] : kent[e]) : 0u;
+                    const int mc =
+                        (nm > 1 && e >= bd1) + (nm > 2 && e >= bd2) + (nm > 3 && e >= bd3);
+                    const int tau = mc * kChunk + (int)((wv[u] >> 7) & 63u);
+                    kv[u] = (e < E1 && tc + tau < t_end) ? tau : -1;
+                    rv[u] = tlo[(kv[u] >= 0 ? kv[u] : 0) * 64 + (int)(wv[u] & 63u)];
+                }
+#pragma unroll
+                for (int u = 0; u < kKB; ++u) {
+                    if (kv[u] < 0) continue;
+                    const uint32_t w = wv[u];
+                    const int ch = (int)(w & 127u), p = ch & 63;
+                    const float d = h2f((uint16_t)(w >> 16)) - zks[ch];
+                    const float4 bq = bs[p];
+                    const float2 cs = cmul(make_float2(bq.x, bq.z), rv[u]);
+                    // rotate-half: channel c < 64 meets (cos, sin) . (q_p, q_p+64), c >= 64 the other
+                    const float sa = ch < 64 ? cs.x : -cs.y, sb = ch < 64 ? cs.y : cs.x;
+                    const float v = d * fmaf(sa, qs[p], sb * qs[p + 64]);
+                    atomicAdd(kcs + kv[u], (unsigned long long)__float2ll_rn(v * kKcScale));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(full + ps);
+        }
+    } else if (warp == kFW + 2) {
         // ================= value helper: zv per token, first value entry per 16-token slice
         float bd[NB];
 #pragma unroll

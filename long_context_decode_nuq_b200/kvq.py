@@ -29,6 +29,7 @@ EXPORTS = (
     "kvq_softmax_merge", "kvq_decode_pv", "kvq_decode_workspace", "kvq_decode_attention",
     "kvq_dequantize", "kvq_fp16_decode_attention", "kvq_fit_workspace", "kvq_fit_codebook",
     "kvq_get_status", "kvq_quantize_append_noalloc", "kvq_decode_partial", "kvq_merge_partials",
+    "kvq_decode_attention_fused", "kvq_decode_fused_workspace",
 )
 
 
@@ -107,6 +108,11 @@ def load():
                                 POINTER(CodebookStruct), P, P, c_int32, c_int32, P, P, P,
                                 c_size_t, c_int32, P], c_int),
         "kvq_merge_partials": ([POINTER(Cfg), c_int32, P, P, P, P], c_int),
+        "kvq_decode_attention_fused": ([POINTER(Cfg), POINTER(CacheStruct),
+                                        POINTER(CodebookStruct), POINTER(CodebookStruct), P, P,
+                                        c_int32, P, P, c_size_t, c_int32, P], c_int),
+        "kvq_decode_fused_workspace": ([POINTER(Cfg), c_int32, c_int32, POINTER(c_size_t)],
+                                       c_int),
         "kvq_quantize_append_noalloc": ([POINTER(Cfg), POINTER(CacheStruct),
                                          POINTER(CodebookStruct), POINTER(CodebookStruct), P, P,
                                          c_int32, P, P], c_int),
@@ -265,6 +271,22 @@ def kvq_decode_attention(cache: Cache, cbK: Codebook, cbV: Codebook, q, qpos, ma
         ctypes.byref(cbV.struct), _ptr(q), _ptr(qpos), max_len, _ptr(out), _ptr(workspace),
         workspace.numel() * workspace.element_size(), splits, _stream(stream)),
         "kvq_decode_attention")
+
+
+def kvq_decode_fused_workspace(cfg: Cfg, max_len: int, splits: int) -> int:
+    b = c_size_t()
+    _check(load().kvq_decode_fused_workspace(ctypes.byref(cfg), max_len, splits, ctypes.byref(b)),
+           "kvq_decode_fused_workspace")
+    return b.value
+
+
+def kvq_decode_attention_fused(cache: Cache, cbK: Codebook, cbV: Codebook, q, qpos, max_len: int,
+                               out, workspace, splits: int = 0, stream=None) -> None:
+    _check(load().kvq_decode_attention_fused(
+        ctypes.byref(cache.cfg), ctypes.byref(cache.struct), ctypes.byref(cbK.struct),
+        ctypes.byref(cbV.struct), _ptr(q), _ptr(qpos), max_len, _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), splits, _stream(stream)),
+        "kvq_decode_attention_fused")
 
 
 def kvq_decode_partial(cache: Cache, cbK: Codebook, cbV: Codebook, q, qpos, max_len: int,

@@ -64,15 +64,17 @@ def test_closed_form_per_token(name, over, expect):
     assert round(got) == expect
     # the decode traffic per token equals the stored bytes plus the chunk pointers (one uint32
     # per 64 tokens per kv head, K and V) for the fused path, and adds the logits (4 B per
-    # query head, written then read) for the split path
+    # query head, written then read) for the split kernels (three calls or one)
     T = 1 << 16
     k_out, v_out = bench.expected_outliers_per_token(w)
-    fused = bench.bytes_model(w, T, k_out * T, v_out * T, "one-call", outlier_bytes=6)["total"]
+    fused = bench.bytes_model(w, T, k_out * T, v_out * T, "fused", outlier_bytes=6)["total"]
     ptr = 2 * 4 * w.Hkv * ((T + 63) // 64 + 1)
     assert (fused - ptr) / T == pytest.approx(got, rel=1e-12)
     split = bench.bytes_model(w, T, k_out * T, v_out * T, "split", outlier_bytes=6)
     assert split["total"] - fused == 2 * 4 * w.Hq * T
     assert split["qk"] + split["pv"] == split["total"]
+    one = bench.bytes_model(w, T, k_out * T, v_out * T, "one-call", outlier_bytes=6)["total"]
+    assert one == split["total"]
 
 
 def test_default_counts_one_packed_word_per_outlier():

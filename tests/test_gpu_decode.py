@@ -126,6 +126,33 @@ def test_one_call_path(name, over, T, plen, appends):
         _check_out(w, out.cpu().numpy(), refs)
 
 
+def _fused_ok(w):
+    return w.Hq == w.Hkv and w.bits <= 3
+
+
+@pytest.mark.parametrize("name,over,T,plen,appends", CASES)
+def test_fused_path(name, over, T, plen, appends):
+    """kvq_decode_attention_fused (one kernel per split, no logits in memory) where it applies;
+    KVQ_ERR_UNSUPPORTED elsewhere."""
+    import torch
+    import long_context_decode_nuq_b200 as K
+    w, o, g, dK, dV, dq, dpos, refs, _, _ = _setup(name, over, T, plen, appends)
+    max_len = int(o.len.max())
+    if not _fused_ok(w):
+        with pytest.raises(K.KvqError):
+            K.kvq_decode_fused_workspace(g.cfg, max_len, 0)
+        return
+    for splits in (0, 2, 5):
+        ws = torch.empty(K.kvq_decode_fused_workspace(g.cfg, max_len, splits), dtype=torch.uint8,
+                         device="cuda")
+        assert ws.numel() < K.kvq_decode_workspace(g.cfg, max_len, splits)
+        out = torch.empty((w.B, w.Hq, w.D), device="cuda")
+        K.kvq_decode_attention_fused(g, dK, dV, dq, dpos, max_len, out, ws, splits)
+        torch.cuda.synchronize()
+        _check_out(w, out.cpu().numpy(), refs)
+    assert K.kvq_get_status(g) == 0
+
+
 @pytest.mark.parametrize("name,over,T,plen", [("tiny_single_head", {}, 2048, None),
                                               ("llama3_8b_gqa_128k", dict(B=2, Hq=16, Hkv=4),
                                                517, [517, 300]),
@@ -174,6 +201,10 @@ def test_outlier_heavy(name, over, T, plen, appends, splits):
     K.kvq_decode_attention(g, dK, dV, dq, dpos, max_len, out, ws, splits)
     torch.cuda.synchronize()
     _check_out(w, out.cpu().numpy(), refs)
+    if _fused_ok(w):   # many outliers: past the per-stage staging of the fused kernel
+        K.kvq_decode_attention_fused(g, dK, dV, dq, dpos, max_len, out, ws, splits)
+        torch.cuda.synchronize()
+        _check_out(w, out.cpu().numpy(), refs)
     assert K.kvq_get_status(g) == 0
 
 
@@ -193,6 +224,15 @@ def test_decode_is_deterministic(name, over, T, plen, appends):
         torch.cuda.synchronize()
         outs.append(out.cpu().numpy().view(np.uint32))
     assert np.array_equal(outs[0], outs[1])
+    if _fused_ok(w):
+        fo = []
+        for _ in range(2):
+            out = torch.empty((w.B, w.Hq, w.D), device="cuda")
+            ws.fill_(0x33)
+            K.kvq_decode_attention_fused(g, dK, dV, dq, dpos, max_len, out, ws, 0)
+            torch.cuda.synchronize()
+            fo.append(out.cpu().numpy().view(np.uint32))
+        assert np.array_equal(fo[0], fo[1])
     S = K.kvq_decode_splits(g.cfg, max_len)
     res = []
     for _ in range(2):
@@ -214,7 +254,7 @@ def test_decode_is_deterministic(name, over, T, plen, appends):
 
 
 @pytest.mark.parametrize("name,over,T,cut", [
-    ("llama7b_layer_32k", dict(Hq=4, Hkv=4), 900, 448),          # fused kernel
+    ("llama7b_layer_32k", dict(Hq=4, Hkv=4), 900, 448),          # one query head per kv head
     ("llama3_8b_gqa_128k", dict(B=1, Hq=8, Hkv=2), 700, 320),    # split kernels (GQA)
     ("batched_8x8k", dict(B=1, Hq=4, Hkv=4, bits=4), 500, 500),  # second range empty
 ])
