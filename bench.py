@@ -366,6 +366,9 @@ def run_kvq(args, rank, world):
             caches.append(c)
             cbs.append(cb)
     setup_s = time.time() - t_setup
+    if args.no_fp16:  # the staged K/V of the last layer serve only the fp16 comparison
+        del kstage, vstage
+        torch.cuda.empty_cache()
     kcount = int(caches[0].kcount.cpu()[0].sum())
     vcount = int(caches[0].vcount.cpu()[0].sum())
 

@@ -155,7 +155,8 @@ int kvq_quantize_workspace(const kvq_cfg* cfg, int32_t n_new, int32_t calibrate,
 
 /*
  * Quantize and append tokens (technique (i)-(iv) on the write side).
- *   k, v     fp16 [B][n_new][Hkv][D] pre-RoPE keys and values (device)
+ *   k, v     fp16 [B][n_new][Hkv][D] pre-RoPE keys and values (device, 16-byte
+ *            aligned; KVQ_ERR_ALIGN otherwise)
  *   plen     int32 [B] tokens of sequence b to take from the block (<= n_new),
  *            or NULL for n_new each (device)
  *   calibrate 1: prefill -- the sequence must be empty; per key channel the
@@ -361,10 +362,11 @@ int kvq_fit_codebook(const uint16_t* samples, int32_t n_vec, int32_t vec_len, do
  * file-scope device array of KVQ_NOALLOC_SCRATCH_BYTES that the library owns; every GPU
  * that loads libkvq.so holds that array until the process exits.
  *   - Limit: the scratch that kvq_quantize_workspace(cfg, n_new, 0) reports must fit in
- *     KVQ_NOALLOC_SCRATCH_BYTES (1 MiB).  A call needs about 4 + 16*Hkv bytes per
- *     (sequence, new token), 516 bytes at Hkv = 32: some 2,000 of them, e.g. 256 sequences
- *     appending up to 7 tokens each; larger requests return KVQ_ERR_SCRATCH_LIMIT and launch
- *     nothing.  Use kvq_quantize_append with a caller workspace for prefills.
+ *     KVQ_NOALLOC_SCRATCH_BYTES (1 MiB).  A call needs about 36 bytes per (sequence, new
+ *     token) and 16*(n_new/64 + 2) + 32 bytes per (sequence, kv head): 256 sequences with
+ *     32 kv heads fit appending up to 56 tokens each; larger requests return
+ *     KVQ_ERR_SCRATCH_LIMIT and launch nothing.  Use kvq_quantize_append with a caller
+ *     workspace for prefills.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call before any
  *     stream capture begins.

@@ -628,7 +628,9 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 // Both kernels give the same bits on every run.  The key side gives each warp whole chunks
 // (a token's entries never straddle two warps), sums each token's corrections in list order
 // with a segmented scan across the lanes (a token's entries are contiguous: the list is
-// sorted by token) and lets one lane add the sum to the logit.  The value side adds each
+// sorted by token) and lets one lane add the sum to the logit: each logit receives exactly one
+// addition, so the fire-and-forget atomic add gives the same bits as a read-modify-write
+// without waiting on the read.  The value side adds each
 // entry's term into 2^-40 fixed-point block sums with integer atomics (integer addition is
 // associative, so their order does not matter), then adds each block sum once into its
 // split's PV partial before the partials are summed in split order.
@@ -779,11 +781,11 @@ __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
                 float v = d * fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
                 if (ct >= 0 && lane == 0) {
                     const float cv = carry[warp][a];
-                    if (flush) lb0[a * T_max + ct] += cv;
+                    if (flush) atomicAdd(&lb0[a * T_max + ct], cv);
                     else v += cv;
                 }
                 v = seg_scan(v, tu, lane);
-                if (tail) lb0[a * T_max + tu] += v;
+                if (tail) atomicAdd(&lb0[a * T_max + tu], v);
                 if (lane == 31) carry[warp][a] = v;
             }
             __syncwarp();
@@ -791,7 +793,7 @@ __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
         }
     }
     if (ct >= 0 && lane == 0)
-        for (int a = 0; a < g; ++a) lb0[a * T_max + ct] += carry[warp][a];
+        for (int a = 0; a < g; ++a) atomicAdd(&lb0[a * T_max + ct], carry[warp][a]);
 }
 
 // ---------------------------------------------------------------------------------

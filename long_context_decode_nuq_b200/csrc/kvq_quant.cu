@@ -6,11 +6,14 @@
 //   k_begin        per sequence: start position, token count, calibration flag
 //   k_calib_*      (calibrating prefill only) per key channel: two-pass 8-bit radix
 //                  select of t_lo = s[k], t_hi = s[N-1-k] over the block's tokens
-//   k_tok_stats    per token: value thresholds (radix select in shared memory),
-//                  value (off, half), key/value outlier counts
-//   k_tok_scan     per sequence: outlier offsets, the capacity rule, chunk pointers,
+//   k_key_cuts     (calibrating prefill only) per key channel: the cut table of its codes
+//   k_tok_stats    per token: value thresholds (radix select in a warp's histogram), value
+//                  (off, half) and cut table; outlier counts per (64-token chunk, kv head)
+//   k_tok_scan     per outlier list: chunk offsets, the capacity rule, chunk pointers,
 //                  counts and len
-//   k_tok_write    per token: encode, bit-pack both rows, compact the outliers
+//   k_tok_write    per (64-token chunk, kv head): encode, bit-pack both blocks, write the
+//                  outliers
+//   k_tok_final    lists whose room ran out: count and chunk pointers
 #include <mutex>
 
 #include "kvq_common.cuh"
@@ -26,30 +29,41 @@ struct QuantWs {
     uint32_t* hist1;  // [B][n][256]
     uint32_t* sel1;   // [B][n][4]  bin_lo, rem_lo, bin_hi, rem_hi
     uint32_t* hist2;  // [B][n][512]
+    uint32_t* kcut;   // [B][Hkv][64][16] key cut pairs (calibrating calls)
     uint32_t* vthr;   // [B][n_new] fp16 t_lo | t_hi << 16
-    uint32_t* kcnt;   // [B][Hkv][n_new] outliers of token i in head h
-    uint32_t* vcnt;
-    uint32_t* koff;   // [B][Hkv][n_new] its first entry in list (b, h), 0xffffffff if dropped
-    uint32_t* voff;
+    uint16_t* vcut;   // [B][n_new][16] value cuts of each token, slot 15 force-zero flag
+    uint32_t* kcc;    // [B*Hkv][nchc] outliers of this call in chunk cl of list (b, h)
+    uint32_t* vcc;
+    uint32_t* kce;    // [B*Hkv][nchc] their exclusive prefix
+    uint32_t* vce;
+    int32_t* lst;     // [B*Hkv][8] start K/V, first overflowing chunk K/V (-1: none), kept K/V
 };
 
+constexpr int kWsParts = 14;
+
 struct WsPlan {
-    size_t off[11];
+    size_t off[kWsParts];
     size_t total;
 };
+
+// Chunks a call's tokens can touch in one sequence (its first may be partly filled already).
+inline int call_chunks(int n_new) { return n_new / kChunk + 2; }
 
 WsPlan plan_ws(const kvq_cfg& cfg, int n_new, int calibrate) {
     using kvq_host::align_up;
     const size_t B = cfg.B, n = (size_t)cfg.Hkv * kD, T = (size_t)n_new;
-    size_t sizes[11] = {B * 4, B * 4, B * 4,
-                        calibrate ? B * n * 256 * 4 : 0,
-                        calibrate ? B * n * 4 * 4 : 0,
-                        calibrate ? B * n * 512 * 4 : 0,
-                        B * T * 4, B * T * cfg.Hkv * 4, B * T * cfg.Hkv * 4,
-                        B * T * cfg.Hkv * 4, B * T * cfg.Hkv * 4};
+    const size_t L = B * cfg.Hkv, C = (size_t)call_chunks(n_new);
+    size_t sizes[kWsParts] = {B * 4, B * 4, B * 4,
+                              calibrate ? B * n * 256 * 4 : 0,
+                              calibrate ? B * n * 4 * 4 : 0,
+                              calibrate ? B * n * 512 * 4 : 0,
+                              calibrate ? B * n * 32 : 0,
+                              B * T * 4, B * T * 32,
+                              L * C * 4, L * C * 4, L * C * 4, L * C * 4,
+                              L * 8 * 4};
     WsPlan p;
     size_t o = 0;
-    for (int i = 0; i < 11; ++i) {
+    for (int i = 0; i < kWsParts; ++i) {
         p.off[i] = o;
         o += align_up(sizes[i]);
     }
@@ -65,11 +79,14 @@ QuantWs bind_ws(char* base, const WsPlan& p) {
     w.hist1 = (uint32_t*)(base + p.off[3]);
     w.sel1 = (uint32_t*)(base + p.off[4]);
     w.hist2 = (uint32_t*)(base + p.off[5]);
-    w.vthr = (uint32_t*)(base + p.off[6]);
-    w.kcnt = (uint32_t*)(base + p.off[7]);
-    w.vcnt = (uint32_t*)(base + p.off[8]);
-    w.koff = (uint32_t*)(base + p.off[9]);
-    w.voff = (uint32_t*)(base + p.off[10]);
+    w.kcut = (uint32_t*)(base + p.off[6]);
+    w.vthr = (uint32_t*)(base + p.off[7]);
+    w.vcut = (uint16_t*)(base + p.off[8]);
+    w.kcc = (uint32_t*)(base + p.off[9]);
+    w.vcc = (uint32_t*)(base + p.off[10]);
+    w.kce = (uint32_t*)(base + p.off[11]);
+    w.vce = (uint32_t*)(base + p.off[12]);
+    w.lst = (int32_t*)(base + p.off[13]);
     return w;
 }
 
@@ -101,30 +118,6 @@ __device__ uint32_t block_excl_scan(uint32_t v, uint32_t* sm, uint32_t* total) {
     return before + incl - v;
 }
 
-// A full warp finds the bin of 0-based rank r in a 256-bin histogram.
-__device__ void warp_find_rank(const uint32_t* hist, uint32_t r, uint32_t* bin, uint32_t* rem) {
-    const int lane = threadIdx.x & 31;
-    uint32_t loc[8];
-    uint32_t s = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-        loc[q] = hist[lane * 8 + q];
-        s += loc[q];
-    }
-    const uint32_t incl = warp_incl_scan(s);
-    uint32_t cum = incl - s;
-    if (cum <= r && r < incl) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            if (cum <= r && r < cum + loc[q]) {
-                *bin = lane * 8 + q;
-                *rem = r - cum;
-            }
-            cum += loc[q];
-        }
-    }
-}
-
 // ---------------------------------------------------------------------------------
 __global__ void k_begin(kvq_cfg cfg, kvq_cache c, const int32_t* plen, int n_new, int calibrate,
                         QuantWs ws) {
@@ -154,49 +147,73 @@ __global__ void k_begin(kvq_cfg cfg, kvq_cache c, const int32_t* plen, int n_new
 }
 
 // ---------------------------------------------------------------------------------
-// Key channel calibration: per-channel radix select (technique (i), pre-RoPE (ii)).
-constexpr int kCalCols = 32;
+// Key channel calibration: per-channel radix select (technique (i), pre-RoPE (ii)).  A block
+// takes kCalCols adjacent channels over a range of tokens; lane l of each warp reads channels
+// 2l and 2l + 1 of a token row (one 4-byte load, 128 bytes per warp and row), kCalU rows in
+// flight per warp; per-channel histograms in shared memory with a stride of 257 words (the
+// same bin of neighbouring channels falls in different banks), added to the global ones at
+// the end.  Pass 1 counts the high byte of the fp16 order key; pass 2 the low byte of the keys
+// whose high byte is the bin of t_lo (first 256 bins) or of t_hi (next 256).
+constexpr int kCalCols = 64;
+constexpr int kCalThreads = 512;
+constexpr int kCalU = 8;
+constexpr int kCalStride = 257;
 
-__global__ void k_calib_hist(kvq_cfg cfg, const uint16_t* __restrict__ k, int n_new, QuantWs ws,
-                             int pass) {
+__global__ void __launch_bounds__(kCalThreads) k_calib_hist(kvq_cfg cfg,
+                                                            const uint16_t* __restrict__ k,
+                                                            int n_new, QuantWs ws, int pass) {
     extern __shared__ uint32_t sh[];
     const int b = blockIdx.z;
     if (!ws.calib[b]) return;
     const int n = cfg.Hkv * kD;
     const int N = ws.ntok[b];
-    const int nb = pass == 1 ? 256 : 512;
-    for (int i = threadIdx.x; i < kCalCols * nb; i += blockDim.x) sh[i] = 0;
+    const int nh = pass == 1 ? 1 : 2;  // histograms per channel
+    for (int i = threadIdx.x; i < kCalCols * nh * kCalStride; i += blockDim.x) sh[i] = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const int j = blockIdx.x * kCalCols + lane;
+    const int j0 = blockIdx.x * kCalCols + 2 * lane;  // this lane's first channel
     const int per = (N + gridDim.y - 1) / gridDim.y;
     const int i0 = blockIdx.y * per;
     const int i1 = min(N, i0 + per);
-    if (j < n) {
-        uint32_t bl = 0, bh = 0;
+    if (j0 < n) {
+        uint32_t bl0 = 0, bh0 = 0, bl1 = 0, bh1 = 0;
         if (pass == 2) {
-            const uint32_t* s = ws.sel1 + ((size_t)b * n + j) * 4;
-            bl = s[0];
-            bh = s[2];
+            const uint32_t* s0 = ws.sel1 + ((size_t)b * n + j0) * 4;
+            bl0 = s0[0]; bh0 = s0[2]; bl1 = s0[4]; bh1 = s0[6];
         }
-        const uint16_t* src = k + (size_t)b * n_new * n + j;
-        for (int i = i0 + warp; i < i1; i += nw) {
-            const uint32_t key = okey(src[(size_t)i * n]);
-            if (pass == 1) {
-                atomicAdd(&sh[lane * 256 + (key >> 8)], 1u);
-            } else {
-                const uint32_t hb = key >> 8;
-                if (hb == bl) atomicAdd(&sh[lane * 512 + (key & 255u)], 1u);
-                if (hb == bh) atomicAdd(&sh[lane * 512 + 256 + (key & 255u)], 1u);
+        uint32_t* h0 = sh + (2 * lane) * nh * kCalStride;
+        uint32_t* h1 = h0 + nh * kCalStride;
+        const uint16_t* src = k + (size_t)b * n_new * n + j0;
+        for (int ib = i0 + warp; ib < i1; ib += nw * kCalU) {
+            uint32_t v[kCalU];
+#pragma unroll
+            for (int u = 0; u < kCalU; ++u) {
+                const int i = ib + u * nw;
+                v[u] = i < i1 ? *reinterpret_cast<const uint32_t*>(src + (size_t)i * n) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kCalU; ++u) {
+                if (ib + u * nw >= i1) break;
+                const uint32_t k0 = okey(v[u] & 0xFFFFu), k1 = okey(v[u] >> 16);
+                if (pass == 1) {
+                    atomicAdd(&h0[k0 >> 8], 1u);
+                    atomicAdd(&h1[k1 >> 8], 1u);
+                } else {
+                    if ((k0 >> 8) == bl0) atomicAdd(&h0[k0 & 255u], 1u);
+                    if ((k0 >> 8) == bh0) atomicAdd(&h0[kCalStride + (k0 & 255u)], 1u);
+                    if ((k1 >> 8) == bl1) atomicAdd(&h1[k1 & 255u], 1u);
+                    if ((k1 >> 8) == bh1) atomicAdd(&h1[kCalStride + (k1 & 255u)], 1u);
+                }
             }
         }
     }
     __syncthreads();
+    const int nb = 256 * nh;
     uint32_t* gh = (pass == 1 ? ws.hist1 : ws.hist2) + ((size_t)b * n + blockIdx.x * kCalCols) * nb;
     for (int i = threadIdx.x; i < kCalCols * nb; i += blockDim.x) {
-        const int col = i / nb;
+        const int col = i / nb, r = i % nb;
         if (blockIdx.x * kCalCols + col < n) {
-            const uint32_t v = sh[i];
+            const uint32_t v = sh[col * nh * kCalStride + (r >> 8) * kCalStride + (r & 255)];
             if (v) atomicAdd(&gh[i], v);
         }
     }
@@ -251,278 +268,828 @@ __global__ void k_calib_select(kvq_cfg cfg, kvq_cache c, QuantWs ws, int pass) {
 }
 
 // ---------------------------------------------------------------------------------
-// Per token: value thresholds over the whole row, value (off, half), outlier counts.
-constexpr int kTokThreads = 512;
+// Encoding by cut tables.  For a normalization (off, half) and a decision bound b, the set of
+// fp16 inputs x with normalize(x, off, half) > b is an upper range of the fp16 total order:
+// the binary32 subtraction and division round monotonically, half >= 0 always (t_hi >= t_lo),
+// and when off or half is not finite every input maps to NaN and the set is empty.  Its least
+// element is the cut of b, so code(x) = #{j : x >= cut_j}, a comparison of fp16 values that the
+// tensor of inputs supports two at a time (HSET2).  NaN inputs compare false (code 0, as the
+// division gives), a cut that no input reaches is stored as a NaN, and -0 and +0 always land on
+// the same side (normalize gives them equal values), so a cut is never +0.  half == 0 makes
+// every input, NaN included, normalize to 0: such a channel or token is flagged in slot 15 of
+// its record and its inputs are replaced by +0 before the comparison.
 
-__global__ void __launch_bounds__(kTokThreads) k_tok_stats(kvq_cfg cfg, kvq_cache c,
-                                                           const uint16_t* __restrict__ k,
-                                                           const uint16_t* __restrict__ v,
-                                                           int n_new, QuantWs ws) {
-    const int b = blockIdx.y, i = blockIdx.x;
-    if (i >= ws.ntok[b]) return;
-    const int n = cfg.Hkv * kD;
-    __shared__ uint32_t hist[512];
-    __shared__ uint32_t sel[4];
-    const uint16_t* vrow = v + ((size_t)b * n_new + i) * n;
-    const uint16_t* krow = k + ((size_t)b * n_new + i) * n;
-    for (int q = threadIdx.x; q < 512; q += blockDim.x) hist[q] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < n; j += blockDim.x) atomicAdd(&hist[okey(vrow[j]) >> 8], 1u);
-    __syncthreads();
-    const int kk = vector_k(cfg.outlier_frac, n);
-    const uint32_t rl = kk, rh = n - 1 - kk;
-    if (threadIdx.x < 32) {
-        warp_find_rank(hist, rl, &sel[0], &sel[1]);
-        warp_find_rank(hist, rh, &sel[2], &sel[3]);
+// Least fp16 value in the fp16 total order whose normalized value exceeds `bound` (fp16 bits),
+// found by bisection over the order keys of -inf .. +inf; 0x7E00 (NaN) when none does.
+__device__ uint32_t cut_of(float bound, float off, float half) {
+    auto above = [&](uint32_t key) {
+        return normalize(h2f((uint16_t)okey_inv(key)), off, half) > bound;
+    };
+    uint32_t lo = 0x03FFu, hi = 0xFC00u;
+    if (!above(hi)) return 0x7E00u;
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi) >> 1;
+        if (above(mid)) hi = mid;
+        else lo = mid + 1;
     }
-    __syncthreads();
-    const uint32_t bl = sel[0], bh = sel[2];
-    for (int q = threadIdx.x; q < 512; q += blockDim.x) hist[q] = 0;
-    __syncthreads();
-    for (int j = threadIdx.x; j < n; j += blockDim.x) {
-        const uint32_t key = okey(vrow[j]);
-        if ((key >> 8) == bl) atomicAdd(&hist[key & 255u], 1u);
-        if ((key >> 8) == bh) atomicAdd(&hist[256 + (key & 255u)], 1u);
-    }
-    __syncthreads();
-    __shared__ uint32_t lowb[4];
-    if (threadIdx.x < 32) {
-        warp_find_rank(hist, sel[1], &lowb[0], &lowb[1]);
-        warp_find_rank(hist + 256, sel[3], &lowb[2], &lowb[3]);
-    }
-    __syncthreads();
-    const uint32_t lo_bits = okey_inv((bl << 8) | lowb[0]);
-    const uint32_t hi_bits = okey_inv((bh << 8) | lowb[2]);
-    const float vlo = h2f((uint16_t)lo_bits), vhi = h2f((uint16_t)hi_bits);
-    const int t = ws.t0[b] + i;
-    if (threadIdx.x == 0) {
-        c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0] = __fmul_rn(__fadd_rn(vlo, vhi), 0.5f);
-        c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1] = __fmul_rn(__fsub_rn(vhi, vlo), 0.5f);
-        ws.vthr[(size_t)b * n_new + i] = lo_bits | (hi_bits << 16);
-    }
-    // outliers per kv head: the 32 channels of a warp's pass lie in one head
-    __shared__ uint32_t hk[64], hv[64];
-    for (int h = threadIdx.x; h < cfg.Hkv; h += blockDim.x) hk[h] = hv[h] = 0u;
-    __syncthreads();
-    const uint16_t* kt = c.kthr + (size_t)b * n * 2;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int j = base + threadIdx.x;
-        bool fk = false, fv = false;
-        if (j < n) {
-            const float xv = h2f(vrow[j]);
-            fv = xv < vlo || xv > vhi;
-            const float xk = h2f(krow[j]);
-            fk = xk < h2f(kt[2 * j]) || xk > h2f(kt[2 * j + 1]);
+    return okey_inv(lo);
+}
+
+__device__ __forceinline__ __half2 as_h2(uint32_t x) { return *reinterpret_cast<__half2*>(&x); }
+__device__ __forceinline__ uint32_t ge2(uint32_t a, uint32_t b) { return __hge2_mask(as_h2(a), as_h2(b)); }
+__device__ __forceinline__ uint32_t out2(uint32_t x, uint32_t lo, uint32_t hi) {
+    return __hlt2_mask(as_h2(x), as_h2(lo)) | __hgt2_mask(as_h2(x), as_h2(hi));
+}
+
+// Codes of the two fp16 inputs in x (low and high half) against the cut pairs C[0 .. 2^BITS-2]
+// (cut j of each half's row or channel in the same half): a bisection over the sorted cuts in
+// which each level selects the next cut per half with the masks of the levels above.
+template <int BITS>
+__device__ __forceinline__ uint32_t enc_pair(uint32_t x, const uint32_t* C) {
+    uint32_t m[BITS];
+    uint32_t code = 0;
+#pragma unroll
+    for (int L = 0; L < BITS; ++L) {
+        uint32_t cand[1 << (BITS - 1)];
+#pragma unroll
+        for (int nd = 0; nd < (1 << L); ++nd) cand[nd] = C[((2 * nd + 1) << (BITS - 1 - L)) - 1];
+#pragma unroll
+        for (int lv = L - 1; lv >= 0; --lv) {
+#pragma unroll
+            for (int p = 0; p < (1 << lv); ++p)
+                cand[p] = (cand[2 * p + 1] & m[lv]) | (cand[2 * p] & ~m[lv]);
         }
-        const uint32_t bk = __ballot_sync(0xffffffffu, fk), bv = __ballot_sync(0xffffffffu, fv);
-        if ((threadIdx.x & 31) == 0 && j < n) {
-            if (bk) atomicAdd(&hk[j >> 7], (uint32_t)__popc(bk));
-            if (bv) atomicAdd(&hv[j >> 7], (uint32_t)__popc(bv));
-        }
+        m[L] = ge2(x, cand[0]);
+        code |= m[L] & (0x00010001u << (BITS - 1 - L));
     }
-    __syncthreads();
-    for (int h = threadIdx.x; h < cfg.Hkv; h += blockDim.x) {
-        const size_t li = ((size_t)b * cfg.Hkv + h) * n_new + i;
-        ws.kcnt[li] = hk[h];
-        ws.vcnt[li] = hv[h];
+    return code;
+}
+
+// Per key channel pair (c, c + 64) of every kv head, after calibration: record p of head h
+// holds word j = cut_j(c) | cut_j(c + 64) << 16 for c = 128h + p, p < 64; word 15 the
+// force-zero flags (0xFFFF per half whose channel has half == 0).
+__global__ void k_key_cuts(kvq_cfg cfg, kvq_cache c, kvq_codebook cbK, QuantWs ws) {
+    const int n = cfg.Hkv * kD, nb = (1 << cfg.bits) - 1;
+    const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (size_t)cfg.B * (n / 2) * 16) return;
+    const int j = (int)(gid & 15);
+    const size_t rec = gid >> 4;  // (b, h, p)
+    const int b = (int)(rec / (n / 2));
+    if (!ws.calib[b]) return;
+    const int hp = (int)(rec % (n / 2)), h = hp >> 6, p = hp & 63;
+    const float* kp0 = c.kparams + ((size_t)b * n + h * kD + p) * 2;
+    const float* kp1 = kp0 + 64 * 2;
+    uint32_t word;
+    if (j < nb) {
+        const float bd = cbK.bounds[j];
+        word = cut_of(bd, kp0[0], kp0[1]) | (cut_of(bd, kp1[0], kp1[1]) << 16);
+    } else if (j == 15) {
+        word = (kp0[1] == 0.0f ? 0xFFFFu : 0u) | (kp1[1] == 0.0f ? 0xFFFF0000u : 0u);
+    } else {
+        word = 0x7E007E00u;
     }
+    ws.kcut[gid] = word;
 }
 
 // ---------------------------------------------------------------------------------
-// Per sequence: offsets of each token's outliers under the capacity rule.
-constexpr int kScanThreads = 1024;
-constexpr int kScanItems = 4;
+// Per token: value thresholds over the whole row (radix select in a warp's own shared
+// histogram), value (off, half) and cuts, and the outlier counts of each kv head, summed per
+// (64-token chunk, kv head).  One block per (chunk, sequence); warp w takes tokens ta + w,
+// ta + w + 8, ...
+constexpr int kStWarps = 8;
 
-__device__ void scan_list(int li, int nt, int t0, int n_new, const uint32_t* cnt, uint32_t* off,
-                          uint32_t cap, uint32_t* count, uint32_t* chunk, int nch1,
-                          int32_t* status) {
-    __shared__ uint32_t sm[32];
-    __shared__ unsigned long long s_acc;
-    const uint32_t* cb = cnt + (size_t)li * n_new;
-    uint32_t* ob = off + (size_t)li * n_new;
-    const uint32_t start = count[li];
-    const unsigned long long room = cap >= start ? (unsigned long long)(cap - start) : 0ull;
-    if (threadIdx.x == 0) s_acc = 0;
-    unsigned long long running = 0;
-    const int tile = kScanThreads * kScanItems;
-    for (int base = 0; base < nt; base += tile) {
-        const int i0 = base + threadIdx.x * kScanItems;
-        uint32_t loc[kScanItems];
-        uint32_t s = 0;
+// A full warp finds the bin of 0-based rank r in a 256-bin histogram; every lane gets it.
+__device__ inline void warp_rank(const uint32_t* hist, uint32_t r, uint32_t& bin, uint32_t& rem) {
+    const int lane = threadIdx.x & 31;
+    const uint4 a = reinterpret_cast<const uint4*>(hist)[2 * lane];
+    const uint4 bq = reinterpret_cast<const uint4*>(hist)[2 * lane + 1];
+    const uint32_t loc[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+    uint32_t s = 0;
 #pragma unroll
-        for (int q = 0; q < kScanItems; ++q) {
-            loc[q] = (i0 + q < nt) ? cb[i0 + q] : 0u;
-            s += loc[q];
-        }
-        uint32_t total;
-        const uint32_t ex = block_excl_scan(s, sm, &total);
-        unsigned long long incl = running + ex;
-        unsigned long long best = 0;
+    for (int q = 0; q < 8; ++q) s += loc[q];
+    const uint32_t incl = warp_incl_scan(s);
+    uint32_t cum = incl - s, fb = 0, fr = 0;
+    const bool mine = cum <= r && r < incl;
+    if (mine) {
 #pragma unroll
-        for (int q = 0; q < kScanItems; ++q) {
-            if (i0 + q < nt) {
-                incl += loc[q];
-                ob[i0 + q] = incl > 0xffffffffull ? 0xffffffffu : (uint32_t)incl;
-                if (incl <= room && incl > best) best = incl;
+        for (int q = 0; q < 8; ++q) {
+            if (cum <= r && r < cum + loc[q]) {
+                fb = lane * 8 + q;
+                fr = r - cum;
             }
+            cum += loc[q];
         }
-        if (best) atomicMax(&s_acc, best);
-        running += total;
-        __syncthreads();
     }
-    __syncthreads();
-    const unsigned long long acc = s_acc;
-    for (int i = threadIdx.x; i < nt; i += blockDim.x) {
-        const unsigned long long incl = ob[i];
-        const bool ok = incl <= room;
-        const unsigned long long ex = incl - cb[i];
-        const int t = t0 + i;
-        if (((t % kChunk) == kChunk - 1) || i == nt - 1) {
-            const unsigned long long v = incl < acc ? incl : acc;
-            chunk[(size_t)li * nch1 + t / kChunk + 1] = start + (uint32_t)v;
-        }
-        ob[i] = ok ? start + (uint32_t)ex : 0xffffffffu;
-    }
-    if (threadIdx.x == 0) {
-        count[li] = start + (uint32_t)acc;
-        if (acc < running) set_status(status, KVQ_STATUS_OUTLIER_OVERFLOW);
-    }
-    __syncthreads();
+    int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    src = src < 0 ? 0 : src;
+    bin = __shfl_sync(0xffffffffu, fb, src);
+    rem = __shfl_sync(0xffffffffu, fr, src);
 }
 
-// One block per outlier list (sequence b, kv head h).
-__global__ void __launch_bounds__(kScanThreads) k_tok_scan(kvq_cfg cfg, kvq_cache c, int n_new,
-                                                           QuantWs ws) {
-    const int li = blockIdx.x, b = li / cfg.Hkv;
-    const int nt = ws.ntok[b], t0 = ws.t0[b];
-    const int nch1 = nchunks(cfg.T_max) + 1;
-    scan_list(li, nt, t0, n_new, ws.kcnt, ws.koff, (uint32_t)cfg.out_cap_k, c.kcount, c.kchunk,
-              nch1, c.status);
-    scan_list(li, nt, t0, n_new, ws.vcnt, ws.voff, (uint32_t)cfg.out_cap_v, c.vcount, c.vchunk,
-              nch1, c.status);
-    if (threadIdx.x == 0 && nt > 0 && li % cfg.Hkv == 0) c.len[b] = t0 + nt;
-}
-
-// ---------------------------------------------------------------------------------
-// Per token quad (4u .. 4u+3): encode the tokens of this call in it, write their outliers,
-// then the quad's key and value blocks (whole when the call starts at token 4u, else only
-// the fields of this call's tokens merged into the existing block).
-// Outliers of one token into the lists of its kv heads: flag/x over the n = Hkv*128 channels,
-// first[h] = the token's first entry in list h (0xffffffff: dropped by the capacity rule);
-// an entry is (fp16 bits << 16) | (tloc << 7) | c.  A 256-thread pass covers two heads, the
-// 32 channels of a warp one quarter of a head.
-__device__ void compact_outliers(int n, const uint8_t* flag, const uint16_t* x,
-                                 const uint32_t* first, size_t first_stride, uint32_t tloc,
-                                 uint32_t* out, size_t cap, uint32_t* sm) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int j = base + threadIdx.x;
-        const bool f = j < n && flag[j];
-        const uint32_t bal = __ballot_sync(0xffffffffu, f);
-        if (lane == 0) sm[warp] = __popc(bal);
-        __syncthreads();
-        if (f) {
-            const int h = j >> 7;
-            const uint32_t f0 = first[(size_t)h * first_stride];
-            if (f0 != 0xffffffffu) {
-                uint32_t r = __popc(bal & ((1u << lane) - 1u));
-                for (int w2 = warp & ~3; w2 < warp; ++w2) r += sm[w2];
-                out[(size_t)h * cap + f0 + r] =
-                    ((uint32_t)x[j] << 16) | (tloc << 7) | (uint32_t)(j & 127);
-            }
-        }
-        __syncthreads();
-    }
-}
-
-// Word `ww` of the block of kv head h from codes [4][n] of the quad's tokens; *wmask gets
-// the bits of the tokens flagged in `present` (bit j = token j of the quad).
-__device__ inline uint32_t block_word(const uint8_t* codes, int n, int h, int bits, int ww,
-                                      uint32_t present, uint32_t* wmask) {
-    const int w2 = 2 * bits, gi = ww / bits, wl = ww % bits;
-    uint32_t word = 0, m = 0;
-    for (int f = max(0, (32 * wl) / w2 - 1); f < 16 && f * w2 < 32 * wl + 32; ++f) {
-        const int o = f * w2 - 32 * wl;
-        if (o + w2 <= 0) continue;
-        const int j = (f & 3) ^ (gi >> 2);   // token of slot f & 3 in lane group gi
-        if (!((present >> j) & 1u)) continue;
-        const int ch = h * kD + gi + 16 * (f >> 2);
-        const uint32_t field =
-            (uint32_t)codes[j * n + ch] | ((uint32_t)codes[j * n + ch + 64] << bits);
-        const uint32_t fm = (1u << w2) - 1u;
-        word |= (o >= 0) ? (field << o) : (field >> (-o));
-        m |= (o >= 0) ? (fm << o) : (fm >> (-o));
-    }
-    *wmask = m;
-    return word;
-}
-
-// One block per (token quad, sequence, kv head): the head's 128 channels of the quad's tokens.
-constexpr int kWrThreads = kD;
-
-__global__ void __launch_bounds__(kWrThreads) k_tok_write(kvq_cfg cfg, kvq_cache c,
-                                                         kvq_codebook cbK, kvq_codebook cbV,
-                                                         const uint16_t* __restrict__ k,
-                                                         const uint16_t* __restrict__ v,
-                                                         int n_new, QuantWs ws) {
-    const int b = blockIdx.y, h = blockIdx.z;
+__global__ void __launch_bounds__(kStWarps * 32) k_tok_stats(kvq_cfg cfg, kvq_cache c,
+                                                            kvq_codebook cbV,
+                                                            const uint16_t* __restrict__ k,
+                                                            const uint16_t* __restrict__ v,
+                                                            int n_new, int nchc, QuantWs ws) {
+    const int b = blockIdx.y, cl = blockIdx.x;
     const int nt = ws.ntok[b], t0 = ws.t0[b];
     if (nt == 0) return;
-    const int u = t0 / 4 + blockIdx.x;
-    const int ta = max(4 * u, t0), tb = min(4 * u + 3, t0 + nt - 1);
-    if (ta > tb) return;
-    const int n = cfg.Hkv * kD, j = threadIdx.x, jn = h * kD + j;  // channel of the token row
-    const int bits = cfg.bits, BW = block_words(bits), nbnd = (1 << bits) - 1;
-    __shared__ uint8_t kc[4 * kD], vc[4 * kD];  // codes of tokens 4u .. 4u+3 (0 when absent)
-    __shared__ uint8_t kf[kD], vf[kD];          // outlier flags of the current token
-    __shared__ float bK[16], bV[16];
-    __shared__ uint32_t sm[32];
-    if (j < nbnd) {
-        bK[j] = cbK.bounds[j];
-        bV[j] = cbV.bounds[j];
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) kc[q * kD + j] = vc[q * kD + j] = 0;
+    const int chk = t0 / kChunk + cl;
+    const int ta = max(chk * kChunk, t0), tb = min(chk * kChunk + kChunk, t0 + nt);
+    if (ta >= tb) return;
+    __shared__ __align__(16) uint32_t hist[kStWarps][512];
+    __shared__ uint32_t ck[64], cv[64];
+    __shared__ float bnd[16];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int Hkv = cfg.Hkv, n = Hkv * kD, n8 = n / 8;
+    const int nb = (1 << cfg.bits) - 1;
+    for (int h = threadIdx.x; h < 64; h += blockDim.x) ck[h] = cv[h] = 0u;
+    if (threadIdx.x < nb) bnd[threadIdx.x] = cbV.bounds[threadIdx.x];
     __syncthreads();
-    const uint16_t* kt = c.kthr + ((size_t)b * n + jn) * 2;
-    const float* kp = c.kparams + ((size_t)b * n + jn) * 2;
-    const float klo = h2f(kt[0]), khi = h2f(kt[1]), koff = kp[0], khalf = kp[1];
-    for (int t = ta; t <= tb; ++t) {
+    uint32_t* hw = hist[warp];
+    const int kk = vector_k(cfg.outlier_frac, n);
+    const uint32_t rl = kk, rh = n - 1 - kk;
+    const uint4* kt4 = reinterpret_cast<const uint4*>(c.kthr + (size_t)b * n * 2);
+    for (int t = ta + warp; t < tb; t += kStWarps) {
         const int i = t - t0;
-        const uint16_t* vrow = v + ((size_t)b * n_new + i) * n + h * kD;
-        const uint16_t* krow = k + ((size_t)b * n_new + i) * n + h * kD;
-        const uint32_t vt = ws.vthr[(size_t)b * n_new + i];
-        const float vlo = h2f((uint16_t)(vt & 0xffffu)), vhi = h2f((uint16_t)(vt >> 16));
-        const float voff = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0];
-        const float vhalf = c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1];
-        const float xk = h2f(krow[j]);
-        const bool ok_ = xk < klo || xk > khi;
-        kf[j] = ok_;
-        kc[(t & 3) * kD + j] = (uint8_t)encode(normalize(ok_ ? 0.0f : xk, koff, khalf), bK, nbnd);
-        const float xv = h2f(vrow[j]);
-        const bool ov = xv < vlo || xv > vhi;
-        vf[j] = ov;
-        vc[(t & 3) * kD + j] = (uint8_t)encode(normalize(ov ? 0.0f : xv, voff, vhalf), bV, nbnd);
+        const uint4* vr = reinterpret_cast<const uint4*>(v + ((size_t)b * n_new + i) * n);
+        const uint4* kr = reinterpret_cast<const uint4*>(k + ((size_t)b * n_new + i) * n);
+        // pass 1: the high byte of each value's order key
+        for (int q = lane; q < 512; q += 32) hw[q] = 0u;
+        __syncwarp();
+        for (int x = lane; x < n8; x += 32) {
+            const uint4 w = vr[x];
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                atomicAdd(&hw[okey(ww[e] & 0xFFFFu) >> 8], 1u);
+                atomicAdd(&hw[okey(ww[e] >> 16) >> 8], 1u);
+            }
+        }
+        __syncwarp();
+        uint32_t bl, reml, bh, remh;
+        warp_rank(hw, rl, bl, reml);
+        warp_rank(hw, rh, bh, remh);
+        __syncwarp();
+        for (int q = lane; q < 512; q += 32) hw[q] = 0u;
+        __syncwarp();
+        // pass 2: the low byte of the keys in the two selected bins
+        for (int x = lane; x < n8; x += 32) {
+            const uint4 w = vr[x];
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const uint32_t key = okey(hf ? (ww[e] >> 16) : (ww[e] & 0xFFFFu));
+                    if ((key >> 8) == bl) atomicAdd(&hw[key & 255u], 1u);
+                    if ((key >> 8) == bh) atomicAdd(&hw[256 + (key & 255u)], 1u);
+                }
+            }
+        }
+        __syncwarp();
+        uint32_t lb, d0, hb, d1;
+        warp_rank(hw, reml, lb, d0);
+        warp_rank(hw + 256, remh, hb, d1);
+        __syncwarp();
+        const uint32_t lo_bits = okey_inv((bl << 8) | lb);
+        const uint32_t hi_bits = okey_inv((bh << 8) | hb);
+        const float vlo = h2f((uint16_t)lo_bits), vhi = h2f((uint16_t)hi_bits);
+        const float off = __fmul_rn(__fadd_rn(vlo, vhi), 0.5f);
+        const float half = __fmul_rn(__fsub_rn(vhi, vlo), 0.5f);
+        if (lane == 0) {
+            c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0] = off;
+            c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1] = half;
+            ws.vthr[(size_t)b * n_new + i] = lo_bits | (hi_bits << 16);
+        }
+        if (lane < 16) {
+            uint32_t cut = 0x7E00u;
+            if (lane < nb) cut = cut_of(bnd[lane], off, half);
+            else if (lane == 15) cut = half == 0.0f ? 0xFFFFu : 0u;
+            ws.vcut[((size_t)b * n_new + i) * 16 + lane] = (uint16_t)cut;
+        }
+        // outliers per kv head: lanes 0-15 of a pass lie in head x >> 4, lanes 16-31 in the next
+        const uint32_t lo2 = lo_bits | (lo_bits << 16), hi2 = hi_bits | (hi_bits << 16);
+        for (int base = 0; base < n8; base += 32) {
+            const int x = base + lane;
+            uint32_t nv = 0, nk = 0;
+            if (x < n8) {
+                const uint4 w = vr[x];
+                nv = __popc(out2(w.x, lo2, hi2)) + __popc(out2(w.y, lo2, hi2)) +
+                     __popc(out2(w.z, lo2, hi2)) + __popc(out2(w.w, lo2, hi2));
+                const uint4 kw = kr[x];
+                const uint4 p = kt4[2 * x], q = kt4[2 * x + 1];  // (t_lo, t_hi) of 8 channels
+                nk = __popc(out2(kw.x, __byte_perm(p.x, p.y, 0x5410), __byte_perm(p.x, p.y, 0x7632))) +
+                     __popc(out2(kw.y, __byte_perm(p.z, p.w, 0x5410), __byte_perm(p.z, p.w, 0x7632))) +
+                     __popc(out2(kw.z, __byte_perm(q.x, q.y, 0x5410), __byte_perm(q.x, q.y, 0x7632))) +
+                     __popc(out2(kw.w, __byte_perm(q.z, q.w, 0x5410), __byte_perm(q.z, q.w, 0x7632)));
+            }
+#pragma unroll
+            for (int o = 8; o; o >>= 1) {
+                nv += __shfl_xor_sync(0xffffffffu, nv, o);
+                nk += __shfl_xor_sync(0xffffffffu, nk, o);
+            }
+            if ((lane & 15) == 0 && x < n8) {
+                if (nv) atomicAdd(&cv[x >> 4], nv >> 4);
+                if (nk) atomicAdd(&ck[x >> 4], nk >> 4);
+            }
+        }
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < Hkv; h += blockDim.x) {
+        const size_t li = (size_t)b * Hkv + h;
+        ws.kcc[li * nchc + cl] = ck[h];
+        ws.vcc[li * nchc + cl] = cv[h];
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Per outlier list (sequence b, kv head h): exclusive prefix of the chunk counts, the capacity
+// rule at chunk level, the chunk pointers and the count when nothing is dropped, len.  A token
+// keeps its outliers iff the inclusive count of this call's outliers up to it fits in the
+// list's room; the first chunk whose end does not fit (if any) is resolved token by token by
+// k_tok_write and finished by k_tok_final.
+constexpr int kScThreads = 256;
+
+__global__ void __launch_bounds__(kScThreads) k_tok_scan(kvq_cfg cfg, kvq_cache c, int nchc,
+                                                         QuantWs ws) {
+    const int li = blockIdx.x, b = li / cfg.Hkv;
+    const int nt = ws.ntok[b], t0 = ws.t0[b];
+    if (nt == 0) return;
+    const int c0 = t0 / kChunk, nch = (t0 + nt - 1) / kChunk - c0 + 1;
+    const int nch1 = nchunks(cfg.T_max) + 1;
+    __shared__ uint32_t sm[32];
+    __shared__ int s_star;
+    for (int which = 0; which < 2; ++which) {
+        const uint32_t* cnt = (which ? ws.vcc : ws.kcc) + (size_t)li * nchc;
+        uint32_t* ex = (which ? ws.vce : ws.kce) + (size_t)li * nchc;
+        uint32_t* count = which ? c.vcount : c.kcount;
+        uint32_t* chunk = (which ? c.vchunk : c.kchunk) + (size_t)li * nch1;
+        const uint32_t cap = (uint32_t)(which ? cfg.out_cap_v : cfg.out_cap_k);
+        const uint32_t start = count[li];
+        const unsigned long long room = cap >= start ? (unsigned long long)(cap - start) : 0ull;
+        if (threadIdx.x == 0) s_star = 0x7fffffff;
         __syncthreads();
-        const uint32_t tloc = (uint32_t)(t % kChunk);
-        const size_t li = ((size_t)b * cfg.Hkv + h) * n_new + i;  // list (b, h), token i
-        compact_outliers(kD, kf, krow, ws.koff + li, 0, tloc,
-                         c.kout + ((size_t)b * cfg.Hkv + h) * cfg.out_cap_k, 0, sm);
-        compact_outliers(kD, vf, vrow, ws.voff + li, 0, tloc,
-                         c.vout + ((size_t)b * cfg.Hkv + h) * cfg.out_cap_v, 0, sm);
+        unsigned long long running = 0;
+        for (int base = 0; base < nch; base += blockDim.x) {
+            const int q = base + threadIdx.x;
+            const uint32_t v = q < nch ? cnt[q] : 0u;
+            uint32_t tot;
+            const uint32_t e = block_excl_scan(v, sm, &tot);
+            if (q < nch) {
+                const unsigned long long E = running + e, I = E + v;
+                ex[q] = E > 0xffffffffull ? 0xffffffffu : (uint32_t)E;
+                if (I > room) atomicMin(&s_star, q);
+                else chunk[c0 + q + 1] = start + (uint32_t)I;
+            }
+            running += tot;
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) {
+            const int star = s_star;
+            ws.lst[li * 8 + which] = (int32_t)start;
+            ws.lst[li * 8 + 2 + which] = star == 0x7fffffff ? -1 : star;
+            ws.lst[li * 8 + 4 + which] = 0;
+            if (star == 0x7fffffff) count[li] = start + (uint32_t)running;
+            if (which == 0 && li % cfg.Hkv == 0) c.len[b] = t0 + nt;
+        }
+        __syncthreads();
     }
-    // the head's key and value blocks of quad u
-    uint32_t present = 0;
-    for (int t = ta; t <= tb; ++t) present |= 1u << (t & 3);
-    const bool fresh = (ta == 4 * u);
-    const size_t blk = (((size_t)b * cfg.Hkv + h) * nquads(cfg.T_max) + u) * BW;
-    for (int wi = j; wi < 2 * BW; wi += blockDim.x) {
-        const int which = wi >= BW, ww = wi - which * BW;
-        uint32_t m;
-        const uint32_t word = block_word(which ? vc : kc, kD, 0, bits, ww, present, &m);
-        uint32_t* dst = (which ? c.vcodes : c.kcodes) + blk + ww;
-        *dst = fresh ? word : ((*dst & ~m) | word);
+}
+
+// The lists whose room ran out inside a chunk: count and the pointers from that chunk on.
+__global__ void k_tok_final(kvq_cfg cfg, kvq_cache c, QuantWs ws) {
+    const int li = blockIdx.x, b = li / cfg.Hkv;
+    const int nt = ws.ntok[b], t0 = ws.t0[b];
+    if (nt == 0) return;
+    const int c0 = t0 / kChunk, nch = (t0 + nt - 1) / kChunk - c0 + 1;
+    const int nch1 = nchunks(cfg.T_max) + 1;
+    for (int which = 0; which < 2; ++which) {
+        const int star = ws.lst[li * 8 + 2 + which];
+        if (star < 0) continue;
+        const uint32_t start = (uint32_t)ws.lst[li * 8 + which];
+        const uint32_t acc = (uint32_t)ws.lst[li * 8 + 4 + which];
+        uint32_t* chunk = (which ? c.vchunk : c.kchunk) + (size_t)li * nch1;
+        for (int q = star + threadIdx.x; q < nch; q += blockDim.x) chunk[c0 + q + 1] = start + acc;
+        if (threadIdx.x == 0) {
+            (which ? c.vcount : c.kcount)[li] = start + acc;
+            set_status(c.status, KVQ_STATUS_OUTLIER_OVERFLOW);
+        }
     }
+}
+
+// ---------------------------------------------------------------------------------
+// Encode and pack.  One warp per (64-token chunk, kv head) of a sequence, two token quads at a
+// time: half-warp hw takes quad u + hw and lane i = lane & 15 builds the lane group i words
+// of that quad's key and value blocks itself.  Lane group i owns the channel pairs
+// (c, c + 64), c = i + 16kk (kk < 4), and holds token 4u + (s ^ (i >> 2)) in slot s, so every
+// field's bit offset is a constant.  The rows of the two quads (keys and values of one kv
+// head, 256 bytes per token) reach shared memory through a three-stage ring of 16-byte
+// asynchronous copies, a warp's own; quad 1's rows sit 32 bytes further on so that the two
+// half-warps read disjoint banks.  Outliers are written per token in channel order: channel
+// c = i + 16*k2 (k2 < 8) ranks after all flagged channels of the lower k2 and the lower
+// lanes of its own k2.
+constexpr int kWrWarps = 4;
+constexpr int kWrStages = 3;
+constexpr int kQStride = 4 * 256 + 32;
+constexpr int kKVStride = 2 * kQStride;
+constexpr int kStageBytes = 2 * kKVStride;
+constexpr int kWrSmem = kWrWarps * kWrStages * kStageBytes;
+
+__device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ uint32_t lds16(const unsigned char* p) {
+    return (uint32_t)*reinterpret_cast<const uint16_t*>(p);
+}
+
+template <int BITS, bool KCUTS>
+__global__ void __launch_bounds__(kWrWarps * 32) k_tok_write(kvq_cfg cfg, kvq_cache c,
+                                                            kvq_codebook cbK,
+                                                            const uint16_t* __restrict__ k,
+                                                            const uint16_t* __restrict__ v,
+                                                            int n_new, int nchc, QuantWs ws) {
+    constexpr int NB = (1 << BITS) - 1;
+    constexpr int W2 = 2 * BITS;
+    extern __shared__ __align__(16) unsigned char wsm[];
+    const int b = blockIdx.y, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int Hkv = cfg.Hkv;
+    const int task = blockIdx.x * kWrWarps + warp;
+    const int cl = task / Hkv, h = task % Hkv;
+    const int nt = ws.ntok[b], t0 = ws.t0[b];
+    if (nt == 0 || cl >= nchc) return;
+    const int chk = t0 / kChunk + cl;
+    const int ta = max(chk * kChunk, t0), tb = min(chk * kChunk + kChunk, t0 + nt);
+    if (ta >= tb) return;
+    const int n = Hkv * kD, i = lane & 15, hw = lane >> 4;
+    const size_t li = (size_t)b * Hkv + h;
+    unsigned char* ring = wsm + warp * (kWrStages * kStageBytes);
+    const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
+    const int ua = ta >> 2, ub = (tb - 1) >> 2;
+    const int nit = (ub - ua) / 2 + 1;
+    // stage `it`: rows of quads ua + 2it and ua + 2it + 1, keys then values
+    auto issue = [&](int it) {
+        const int u0 = ua + 2 * it;
+        const uint32_t sb = ring_s + (it % kWrStages) * kStageBytes;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int pc = lane + 32 * r;
+            const int which = pc >> 7, hq = (pc >> 6) & 1, j = (pc >> 4) & 3, seg = pc & 15;
+            const int t = 4 * (u0 + hq) + j;
+            if (t >= ta && t < tb) {
+                const uint16_t* src =
+                    (which ? v : k) + ((size_t)b * n_new + (t - t0)) * n + h * kD + seg * 8;
+                cp16(sb + which * kKVStride + hq * kQStride + j * 256 + seg * 16, src);
+            }
+        }
+    };
+#pragma unroll
+    for (int p = 0; p < kWrStages - 1; ++p) {
+        if (p < nit) issue(p);
+        cp_commit();
+    }
+    // key channel data of the lane's four pairs
+    uint32_t klo[4], khi[4], kz[4];
+    uint32_t KC[4][KCUTS ? NB : 1];
+    float kof[4][2], khf[4][2], bK[KCUTS ? 1 : NB];
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        const int p = i + 16 * kk;
+        const uint32_t* th = reinterpret_cast<const uint32_t*>(c.kthr) + (size_t)b * n + h * kD + p;
+        const uint32_t a0 = th[0], a1 = th[64];
+        klo[kk] = __byte_perm(a0, a1, 0x5410);
+        khi[kk] = __byte_perm(a0, a1, 0x7632);
+        if constexpr (KCUTS) {
+            const uint4* rec = reinterpret_cast<const uint4*>(ws.kcut + (li * 64 + p) * 16);
+            const uint4 r0 = rec[0], r1 = rec[1], r2 = rec[2], r3 = rec[3];
+            const uint32_t rw[16] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w,
+                                     r2.x, r2.y, r2.z, r2.w, r3.x, r3.y, r3.z, r3.w};
+#pragma unroll
+            for (int j = 0; j < NB; ++j) KC[kk][j] = rw[j];
+            kz[kk] = rw[15];
+        } else {
+            const float* kp = c.kparams + ((size_t)b * n + h * kD + p) * 2;
+            kof[kk][0] = kp[0];
+            khf[kk][0] = kp[1];
+            kof[kk][1] = kp[128];
+            khf[kk][1] = kp[129];
+            kz[kk] = 0u;
+        }
+    }
+    if constexpr (!KCUTS) {
+#pragma unroll
+        for (int j = 0; j < NB; ++j) bK[j] = cbK.bounds[j];
+    }
+    (void)kof;
+    (void)khf;
+    (void)bK;
+    (void)KC;
+    // outlier lists: this call's outliers before the chunk, start, room
+    uint32_t inc[2] = {ws.kce[li * nchc + cl], ws.vce[li * nchc + cl]};
+    uint32_t room[2], start[2];
+    int star[2];
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        start[w] = (uint32_t)ws.lst[li * 8 + w];
+        star[w] = ws.lst[li * 8 + 2 + w];
+        const uint32_t cap = (uint32_t)(w ? cfg.out_cap_v : cfg.out_cap_k);
+        room[w] = cap >= start[w] ? cap - start[w] : 0u;
+    }
+    uint32_t acc[2] = {inc[0], inc[1]};
+    uint32_t* outl[2] = {c.kout + li * cfg.out_cap_k, c.vout + li * cfg.out_cap_v};
+    const size_t blk0 = li * nquads(cfg.T_max);
+    for (int it = 0; it < nit; ++it) {
+        if (it + kWrStages - 1 < nit) issue(it + kWrStages - 1);
+        cp_commit();
+        cp_wait<kWrStages - 1>();
+        __syncwarp();
+        const unsigned char* sbuf = ring + (it % kWrStages) * kStageBytes;
+        const int u0 = ua + 2 * it, u = u0 + hw;
+        const unsigned char* qk = sbuf + hw * kQStride;  // this half-warp's quad, keys
+        const unsigned char* qv = qk + kKVStride;        // and values
+        uint32_t kw[BITS], vw[BITS], fm[BITS];
+#pragma unroll
+        for (int q = 0; q < BITS; ++q) kw[q] = vw[q] = fm[q] = 0u;
+        uint32_t FK = 0, FV = 0;  // outlier flags, bit 8s + k2
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            const int j = s ^ (i >> 2), t = 4 * u + j;
+            const bool pr = u <= ub && t >= ta && t < tb;
+            const uint32_t pm = pr ? 0xFFFFFFFFu : 0u;
+            uint32_t vlo2, vhi2, VC[NB], vz;
+            {
+                const size_t ti = (size_t)b * n_new + (pr ? t - t0 : 0);
+                const uint32_t vt = ws.vthr[ti];
+                vlo2 = __byte_perm(vt, 0, 0x1010);
+                vhi2 = __byte_perm(vt, 0, 0x3232);
+                const uint4* cr = reinterpret_cast<const uint4*>(ws.vcut + ti * 16);
+                const uint4 c0v = cr[0], c1v = cr[1];
+                const uint32_t cw[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+#pragma unroll
+                for (int jj = 0; jj < NB; ++jj)
+                    VC[jj] = __byte_perm(cw[jj >> 1], 0, (jj & 1) ? 0x3232 : 0x1010);
+                vz = (cw[7] >> 16) ? 0xFFFFFFFFu : 0u;
+            }
+            const unsigned char* rk = qk + j * 256;
+            const unsigned char* rv = qv + j * 256;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const int f = 4 * kk + s, off = f * W2, wd = off >> 5, bt = off & 31;
+                const int cb = 2 * (i + 16 * kk);
+                const uint32_t xk = pr ? (lds16(rk + cb) | (lds16(rk + cb + 128) << 16)) : 0u;
+                const uint32_t xv = pr ? (lds16(rv + cb) | (lds16(rv + cb + 128) << 16)) : 0u;
+                // keys
+                const uint32_t ok = out2(xk, klo[kk], khi[kk]) & pm;
+                FK |= ((ok & 1u) << (8 * s + kk)) | (((ok >> 16) & 1u) << (8 * s + kk + 4));
+                uint32_t cp;
+                if constexpr (KCUTS) {
+                    cp = enc_pair<BITS>(xk & ~(ok | kz[kk]), KC[kk]);
+                } else {
+                    uint32_t c2[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const float xf =
+                            ((ok >> (16 * e)) & 1u) ? 0.0f : h2f((uint16_t)(xk >> (16 * e)));
+                        c2[e] = encode(normalize(xf, kof[kk][e], khf[kk][e]), bK, NB);
+                    }
+                    cp = c2[0] | (c2[1] << 16);
+                }
+                const uint32_t fk = pr ? ((cp & 0xFFFFu) | ((cp >> 16) << BITS)) : 0u;
+                // values
+                const uint32_t ov = out2(xv, vlo2, vhi2) & pm;
+                FV |= ((ov & 1u) << (8 * s + kk)) | (((ov >> 16) & 1u) << (8 * s + kk + 4));
+                const uint32_t cq = enc_pair<BITS>(xv & ~(ov | vz), VC);
+                const uint32_t fv = pr ? ((cq & 0xFFFFu) | ((cq >> 16) << BITS)) : 0u;
+                const uint32_t fmask = pr ? ((1u << W2) - 1u) : 0u;
+                kw[wd] |= fk << bt;
+                vw[wd] |= fv << bt;
+                fm[wd] |= fmask << bt;
+                if (bt + W2 > 32) {
+                    kw[wd + 1] |= fk >> (32 - bt);
+                    vw[wd + 1] |= fv >> (32 - bt);
+                    fm[wd + 1] |= fmask >> (32 - bt);
+                }
+            }
+        }
+        // outlier entries, token by token in order (half 0's quad, then half 1's)
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            const uint32_t F = w ? FV : FK;
+            if (!__ballot_sync(0xffffffffu, F != 0u)) continue;
+            for (int hh = 0; hh < 2; ++hh) {
+                const uint32_t hmask = hh ? 0xFFFF0000u : 0x0000FFFFu;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int s = j ^ (i >> 2);
+                    const uint32_t f8 = (F >> (8 * s)) & 0xFFu;
+                    if (!(__ballot_sync(0xffffffffu, f8 != 0u) & hmask)) continue;
+                    uint32_t bal[8], tot = 0;
+#pragma unroll
+                    for (int k2 = 0; k2 < 8; ++k2) {
+                        bal[k2] = __ballot_sync(0xffffffffu, (f8 >> k2) & 1u) & hmask;
+                        tot += __popc(bal[k2]);
+                    }
+                    const uint32_t incl = inc[w] + tot;
+                    const bool kept = incl <= room[w];
+                    if (kept && hw == hh) {
+                        const uint32_t tloc = (uint32_t)((4 * (u0 + hh) + j) % kChunk);
+                        const unsigned char* row = (w ? qv : qk) + j * 256;
+                        uint32_t before = 0;
+#pragma unroll
+                        for (int k2 = 0; k2 < 8; ++k2) {
+                            if ((f8 >> k2) & 1u) {
+                                const uint32_t r = before + __popc(bal[k2] & ((1u << lane) - 1u));
+                                const uint32_t x16 = lds16(row + 2 * (i + 16 * k2));
+                                outl[w][start[w] + inc[w] + r] =
+                                    (x16 << 16) | (tloc << 7) | (uint32_t)(i + 16 * k2);
+                            }
+                            before += __popc(bal[k2]);
+                        }
+                    }
+                    if (kept) acc[w] = incl;
+                    inc[w] = incl;
+                }
+            }
+        }
+        // the quad's blocks: fresh when the quad starts at or after this call's first token,
+        // else only the fields of this call's tokens replace the stored ones
+        if (u <= ub) {
+            const size_t o = (blk0 + u) * (16 * BITS) + BITS * i;
+            const bool fresh = 4 * u >= t0;
+#pragma unroll
+            for (int q = 0; q < BITS; ++q) {
+                if (fresh) {
+                    c.kcodes[o + q] = kw[q];
+                    c.vcodes[o + q] = vw[q];
+                } else {
+                    c.kcodes[o + q] = (c.kcodes[o + q] & ~fm[q]) | kw[q];
+                    c.vcodes[o + q] = (c.vcodes[o + q] & ~fm[q]) | vw[q];
+                }
+            }
+        }
+        __syncwarp();
+    }
+    cp_wait<0>();
+    if (lane == 0) {
+#pragma unroll
+        for (int w = 0; w < 2; ++w)
+            if (star[w] == cl) ws.lst[li * 8 + 4 + w] = (int32_t)acc[w];
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// Short appends (decode steps): one block per sequence does a call's few tokens one after
+// another -- value statistics over the whole row with a block-wide radix select, encode by
+// division, the quad's fields, outliers appended at the end of each list in channel order,
+// chunk pointers, counts, len -- in a single launch and without scratch.  Half-warp h takes kv
+// head h; lane i = lane & 15 is lane group i of the code block and holds channels i + 16e
+// (e < 8), so the field of pair (c, c + 64), c = i + 16kk, is code(e = kk) | code(e = kk + 4)
+// << bits.  The outcome is the same as the general pipeline's for the same tokens.  Used for
+// appends of at most kSmallAppend tokens per sequence with at most 32 kv heads.
+constexpr int kSmallAppend = 16;
+
+template <int BITS>
+__global__ void __launch_bounds__(512) k_append_small(kvq_cfg cfg, kvq_cache c,
+                                                       kvq_codebook cbK, kvq_codebook cbV,
+                                                       const uint16_t* __restrict__ k,
+                                                       const uint16_t* __restrict__ v,
+                                                       int n_new, const int32_t* plen) {
+    constexpr int NB = (1 << BITS) - 1;
+    constexpr int W2 = 2 * BITS;
+    const int b = blockIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int h = threadIdx.x >> 4, i = threadIdx.x & 15;
+    const int Hkv = cfg.Hkv, n = Hkv * kD;
+    const bool act = h < Hkv;
+    __shared__ __align__(16) uint32_t hist[512];
+    __shared__ uint32_t sel[4];
+    __shared__ float bK[16], bV[16];
+    __shared__ int s_nt, s_t0;
+    if (threadIdx.x < NB) {
+        bK[threadIdx.x] = cbK.bounds[threadIdx.x];
+        bV[threadIdx.x] = cbV.bounds[threadIdx.x];
+    }
+    if (threadIdx.x == 0) {
+        int nt = plen ? plen[b] : n_new;
+        nt = nt < 0 ? 0 : (nt > n_new ? n_new : nt);
+        const int t0 = c.len[b];
+        if ((long long)t0 + nt > cfg.T_max) {
+            set_status(c.status, KVQ_STATUS_LEN_OVERFLOW);
+            nt = 0;
+        }
+        s_nt = nt;
+        s_t0 = t0;
+    }
+    __syncthreads();
+    const int nt = s_nt, t0 = s_t0;
+    if (nt == 0) return;
+    const int hh = act ? h : 0;
+    const size_t li = (size_t)b * Hkv + hh;
+    const int nch1 = nchunks(cfg.T_max) + 1;
+    // the lane's key channels: thresholds and normalization
+    uint32_t kth[8];
+    float kof[8], khf[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const size_t ch = (size_t)b * n + hh * kD + i + 16 * e;
+        kth[e] = reinterpret_cast<const uint32_t*>(c.kthr)[ch];  // t_lo | t_hi << 16
+        kof[e] = c.kparams[ch * 2];
+        khf[e] = c.kparams[ch * 2 + 1];
+    }
+    const uint32_t cap[2] = {(uint32_t)cfg.out_cap_k, (uint32_t)cfg.out_cap_v};
+    const uint32_t start[2] = {c.kcount[li], c.vcount[li]};
+    const uint32_t room[2] = {cap[0] >= start[0] ? cap[0] - start[0] : 0u,
+                              cap[1] >= start[1] ? cap[1] - start[1] : 0u};
+    uint32_t incl[2] = {0u, 0u}, acc[2] = {0u, 0u};
+    uint32_t* outl[2] = {c.kout + li * cfg.out_cap_k, c.vout + li * cfg.out_cap_v};
+    uint32_t* chunk[2] = {c.kchunk + li * nch1, c.vchunk + li * nch1};
+    const int kk_rank = vector_k(cfg.outlier_frac, n);
+    const uint32_t hmask = (lane >> 4) ? 0xFFFF0000u : 0x0000FFFFu;
+    for (int tt = 0; tt < nt; ++tt) {
+        const int t = t0 + tt;
+        uint32_t xk[8], xv[8];
+        const size_t row = ((size_t)b * n_new + tt) * n + hh * kD + i;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            xk[e] = act ? (uint32_t)__ldg(k + row + 16 * e) : 0u;
+            xv[e] = act ? (uint32_t)__ldg(v + row + 16 * e) : 0u;
+        }
+        // value thresholds: two 8-bit passes over the row's order keys
+        for (int q = threadIdx.x; q < 512; q += blockDim.x) hist[q] = 0u;
+        __syncthreads();
+        if (act) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) atomicAdd(&hist[okey(xv[e]) >> 8], 1u);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t b0, r0, b1, r1;
+            warp_rank(hist, (uint32_t)kk_rank, b0, r0);
+            warp_rank(hist, (uint32_t)(n - 1 - kk_rank), b1, r1);
+            if (lane == 0) {
+                sel[0] = b0; sel[1] = r0; sel[2] = b1; sel[3] = r1;
+            }
+        }
+        __syncthreads();
+        const uint32_t bl = sel[0], bh = sel[2], rl = sel[1], rh = sel[3];
+        for (int q = threadIdx.x; q < 512; q += blockDim.x) hist[q] = 0u;
+        __syncthreads();
+        if (act) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t key = okey(xv[e]);
+                if ((key >> 8) == bl) atomicAdd(&hist[key & 255u], 1u);
+                if ((key >> 8) == bh) atomicAdd(&hist[256 + (key & 255u)], 1u);
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            uint32_t lb, d0, hb, d1;
+            warp_rank(hist, rl, lb, d0);
+            warp_rank(hist + 256, rh, hb, d1);
+            if (lane == 0) {
+                sel[0] = lb; sel[2] = hb;
+            }
+        }
+        __syncthreads();
+        const uint32_t lo_bits = okey_inv((bl << 8) | sel[0]);
+        const uint32_t hi_bits = okey_inv((bh << 8) | sel[2]);
+        __syncthreads();  // sel is rewritten by the next token
+        const float vlo = h2f((uint16_t)lo_bits), vhi = h2f((uint16_t)hi_bits);
+        const float voff = __fmul_rn(__fadd_rn(vlo, vhi), 0.5f);
+        const float vhalf = __fmul_rn(__fsub_rn(vhi, vlo), 0.5f);
+        if (threadIdx.x == 0) {
+            c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0] = voff;
+            c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1] = vhalf;
+        }
+        // encode, flags
+        uint32_t ck[8], cv[8], fk = 0, fv = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const float x = h2f((uint16_t)xk[e]);
+            const bool o = act && (x < h2f((uint16_t)(kth[e] & 0xFFFFu)) || x > h2f((uint16_t)(kth[e] >> 16)));
+            fk |= (o ? 1u : 0u) << e;
+            ck[e] = encode(normalize(o ? 0.0f : x, kof[e], khf[e]), bK, NB);
+            const float y = h2f((uint16_t)xv[e]);
+            const bool p = act && (y < vlo || y > vhi);
+            fv |= (p ? 1u : 0u) << e;
+            cv[e] = encode(normalize(p ? 0.0f : y, voff, vhalf), bV, NB);
+        }
+        // the token's fields in the quad block: slot s = (t & 3) ^ (i >> 2)
+        if (act) {
+            const int s = (t & 3) ^ (i >> 2);
+            uint32_t kw[BITS], vw[BITS], fm[BITS];
+#pragma unroll
+            for (int q = 0; q < BITS; ++q) kw[q] = vw[q] = fm[q] = 0u;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+                for (int ss = 0; ss < 4; ++ss) {
+                    if (ss != s) continue;
+                    const int off = (4 * kk + ss) * W2, wd = off >> 5, bt = off & 31;
+                    const uint32_t a = ck[kk] | (ck[kk + 4] << BITS);
+                    const uint32_t d = cv[kk] | (cv[kk + 4] << BITS);
+                    const uint32_t m = (1u << W2) - 1u;
+                    kw[wd] |= a << bt;
+                    vw[wd] |= d << bt;
+                    fm[wd] |= m << bt;
+                    if (bt + W2 > 32) {
+                        kw[wd + 1] |= a >> (32 - bt);
+                        vw[wd + 1] |= d >> (32 - bt);
+                        fm[wd + 1] |= m >> (32 - bt);
+                    }
+                }
+            }
+            const size_t o = (li * nquads(cfg.T_max) + (t >> 2)) * (16 * BITS) + BITS * i;
+            const bool fresh = (t & 3) == 0;
+#pragma unroll
+            for (int q = 0; q < BITS; ++q) {
+                c.kcodes[o + q] = fresh ? kw[q] : ((c.kcodes[o + q] & ~fm[q]) | kw[q]);
+                c.vcodes[o + q] = fresh ? vw[q] : ((c.vcodes[o + q] & ~fm[q]) | vw[q]);
+            }
+        }
+        // outliers in channel order (channel i + 16e ranks by (e, i))
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+            const uint32_t f8 = w ? fv : fk;
+            uint32_t bal[8], tot = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                bal[e] = __ballot_sync(0xffffffffu, (f8 >> e) & 1u) & hmask;
+                tot += __popc(bal[e]);
+            }
+            const uint32_t before = incl[w];
+            incl[w] += tot;
+            const bool kept = incl[w] <= room[w];
+            if (kept && act) {
+                const uint32_t tloc = (uint32_t)(t % kChunk);
+                uint32_t r0 = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    if ((f8 >> e) & 1u) {
+                        const uint32_t r = r0 + __popc(bal[e] & ((1u << lane) - 1u));
+                        const uint32_t x16 = w ? xv[e] : xk[e];
+                        outl[w][start[w] + before + r] =
+                            (x16 << 16) | (tloc << 7) | (uint32_t)(i + 16 * e);
+                    }
+                    r0 += __popc(bal[e]);
+                }
+            }
+            if (kept) acc[w] = incl[w];
+            if (act && i == 0 && ((t % kChunk) == kChunk - 1 || tt == nt - 1))
+                chunk[w][t / kChunk + 1] = start[w] + acc[w];
+        }
+    }
+    if (act && i == 0) {
+        c.kcount[li] = start[0] + acc[0];
+        c.vcount[li] = start[1] + acc[1];
+        if (acc[0] < incl[0] || acc[1] < incl[1]) set_status(c.status, KVQ_STATUS_OUTLIER_OVERFLOW);
+    }
+    if (threadIdx.x == 0) c.len[b] = t0 + nt;
+}
+
+int launch_small(const kvq_cfg& C, const kvq_cache& K, const kvq_codebook& cbK,
+                 const kvq_codebook& cbV, const uint16_t* k, const uint16_t* v, int n_new,
+                 const int32_t* plen, cudaStream_t st) {
+    const int threads = ((16 * C.Hkv + 31) / 32) * 32;
+    switch (C.bits) {
+        case 2: k_append_small<2><<<C.B, threads, 0, st>>>(C, K, cbK, cbV, k, v, n_new, plen); break;
+        case 3: k_append_small<3><<<C.B, threads, 0, st>>>(C, K, cbK, cbV, k, v, n_new, plen); break;
+        default: k_append_small<4><<<C.B, threads, 0, st>>>(C, K, cbK, cbV, k, v, n_new, plen); break;
+    }
+    return 0;
+}
+
+// The per-token kernels of a call (stats, scan, write, final).  kcuts: the key cut tables in
+// the workspace are valid (calibrating calls); otherwise keys are encoded by division.
+template <int BITS>
+void launch_write(const kvq_cfg& C, const kvq_cache& K, const kvq_codebook& cbK,
+                  const uint16_t* k, const uint16_t* v, int n_new, int nchc, bool kcuts,
+                  const QuantWs& ws, cudaStream_t st) {
+    const long long tasks = (long long)nchc * C.Hkv;
+    dim3 gw((unsigned)((tasks + kWrWarps - 1) / kWrWarps), C.B);
+    auto kern = kcuts ? k_tok_write<BITS, true> : k_tok_write<BITS, false>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kWrSmem);
+    kern<<<gw, kWrWarps * 32, kWrSmem, st>>>(C, K, cbK, k, v, n_new, nchc, ws);
+}
+
+void launch_tokens(const kvq_cfg& C, const kvq_cache& K, const kvq_codebook& cbK,
+                   const kvq_codebook& cbV, const uint16_t* k, const uint16_t* v, int n_new,
+                   bool kcuts, const QuantWs& ws, cudaStream_t st) {
+    const int nchc = call_chunks(n_new);
+    dim3 gt(nchc, C.B);
+    k_tok_stats<<<gt, kStWarps * 32, 0, st>>>(C, K, cbV, k, v, n_new, nchc, ws);
+    k_tok_scan<<<C.B * C.Hkv, kScThreads, 0, st>>>(C, K, nchc, ws);
+    switch (C.bits) {
+        case 2: launch_write<2>(C, K, cbK, k, v, n_new, nchc, kcuts, ws, st); break;
+        case 3: launch_write<3>(C, K, cbK, k, v, n_new, nchc, kcuts, ws, st); break;
+        default: launch_write<4>(C, K, cbK, k, v, n_new, nchc, kcuts, ws, st); break;
+    }
+    k_tok_final<<<C.B * C.Hkv, 128, 0, st>>>(C, K, ws);
 }
 
 }  // namespace
@@ -552,7 +1119,7 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
     if (n_new < 0 || n_new > cfg->T_max) return KVQ_ERR_RANGE;
     if (n_new == 0) return KVQ_OK;
     if (!k || !v || !workspace) return KVQ_ERR_NULL;
-    if (!aligned16(workspace)) return KVQ_ERR_ALIGN;
+    if (!aligned16(workspace) || !aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGN;
     const int n = cfg->Hkv * kD;
     const WsPlan p = plan_ws(*cfg, n_new, calibrate);
     if (workspace_bytes < p.total) return KVQ_ERR_WORKSPACE;
@@ -560,31 +1127,34 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
     cudaStream_t st = (cudaStream_t)stream;
     const kvq_cfg C = *cfg;
     const kvq_cache K = *cache;
+    if (!calibrate && n_new <= kSmallAppend && C.Hkv <= 32) {
+        launch_small(C, K, *cbK, *cbV, k, v, n_new, plen, st);
+        return record_cuda(cudaGetLastError());
+    }
     k_begin<<<(C.B + 127) / 128, 128, 0, st>>>(C, K, plen, n_new, calibrate, ws);
     if (calibrate) {
         cudaError_t ce;
         if ((ce = cudaMemsetAsync(ws.hist1, 0, (size_t)C.B * n * 256 * 4, st))) return record_cuda(ce);
         if ((ce = cudaMemsetAsync(ws.hist2, 0, (size_t)C.B * n * 512 * 4, st))) return record_cuda(ce);
+        const int sm2 = kCalCols * 2 * kCalStride * 4;
         if ((ce = cudaFuncSetAttribute(k_calib_hist, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kCalCols * 512 * 4)))
+                                       sm2)))
             return record_cuda(ce);
         const int groups = (n + kCalCols - 1) / kCalCols;
-        int splits = (4 * 148 + groups * C.B - 1) / (groups * C.B);
+        int splits = (6 * 148 + groups * C.B - 1) / (groups * C.B);
         splits = splits < 1 ? 1 : splits;
-        const int maxsp = (n_new + 255) / 256;
+        const int maxsp = (n_new + 1023) / 1024;
         splits = splits > maxsp ? (maxsp < 1 ? 1 : maxsp) : splits;
         dim3 gh(groups, splits, C.B);
         dim3 gs((n + 127) / 128, C.B);
-        k_calib_hist<<<gh, 256, kCalCols * 256 * 4, st>>>(C, k, n_new, ws, 1);
+        k_calib_hist<<<gh, kCalThreads, kCalCols * kCalStride * 4, st>>>(C, k, n_new, ws, 1);
         k_calib_select<<<gs, 128, 0, st>>>(C, K, ws, 1);
-        k_calib_hist<<<gh, 256, kCalCols * 512 * 4, st>>>(C, k, n_new, ws, 2);
+        k_calib_hist<<<gh, kCalThreads, sm2, st>>>(C, k, n_new, ws, 2);
         k_calib_select<<<gs, 128, 0, st>>>(C, K, ws, 2);
+        const size_t nrec = (size_t)C.B * (n / 2) * 16;
+        k_key_cuts<<<(unsigned)((nrec + 255) / 256), 256, 0, st>>>(C, K, *cbK, ws);
     }
-    dim3 gt(n_new, C.B);
-    k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
-    k_tok_scan<<<C.B * C.Hkv, kScanThreads, 0, st>>>(C, K, n_new, ws);
-    dim3 gw((n_new + 2) / 4 + 1, C.B, C.Hkv);
-    k_tok_write<<<gw, kWrThreads, 0, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
+    launch_tokens(C, K, *cbK, *cbV, k, v, n_new, calibrate != 0, ws, st);
     return record_cuda(cudaGetLastError());
 }
 
@@ -627,6 +1197,7 @@ extern "C" int kvq_quantize_append_noalloc(const kvq_cfg* cfg, const kvq_cache* 
     if (n_new < 0 || n_new > cfg->T_max) return KVQ_ERR_RANGE;
     if (n_new == 0) return KVQ_OK;
     if (!k || !v) return KVQ_ERR_NULL;
+    if (!aligned16(k) || !aligned16(v)) return KVQ_ERR_ALIGN;
     const WsPlan p = plan_ws(*cfg, n_new, 0);
     if (p.total > (size_t)KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_SCRATCH_LIMIT;
     void* scratch = nullptr;
@@ -635,11 +1206,11 @@ extern "C" int kvq_quantize_append_noalloc(const kvq_cfg* cfg, const kvq_cache* 
     cudaStream_t st = (cudaStream_t)stream;
     const kvq_cfg C = *cfg;
     const kvq_cache K = *cache;
+    if (n_new <= kSmallAppend && C.Hkv <= 32) {
+        launch_small(C, K, *cbK, *cbV, k, v, n_new, plen, st);
+        return record_cuda(cudaGetLastError());
+    }
     k_begin<<<(C.B + 127) / 128, 128, 0, st>>>(C, K, plen, n_new, 0, ws);
-    dim3 gt(n_new, C.B);
-    k_tok_stats<<<gt, kTokThreads, 0, st>>>(C, K, k, v, n_new, ws);
-    k_tok_scan<<<C.B * C.Hkv, kScanThreads, 0, st>>>(C, K, n_new, ws);
-    dim3 gw((n_new + 2) / 4 + 1, C.B, C.Hkv);
-    k_tok_write<<<gw, kWrThreads, 0, st>>>(C, K, *cbK, *cbV, k, v, n_new, ws);
+    launch_tokens(C, K, *cbK, *cbV, k, v, n_new, false, ws, st);
     return record_cuda(cudaGetLastError());
 }

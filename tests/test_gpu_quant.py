@@ -155,3 +155,82 @@ def test_device_generator_matches_numpy(name):
     assert np.array_equal(u16(k), K16[:, 50:90].view(np.uint16))
     assert np.array_equal(u16(v), V16[:, 50:90].view(np.uint16))
     assert np.array_equal(u16(q), synth.gen_q(w, 0, 3).view(np.uint16))
+
+
+@pytest.mark.parametrize("name,over,T,plen", [CASES[1], CASES[4], CASES[2]])
+def test_long_append_bit_exact(name, over, T, plen):
+    """Appends longer than the short-append path takes (a block of 37, then 23 tokens): the
+    general pipeline with keys encoded against the stored calibration, a first quad that is
+    partly filled already, chunks that straddle the call's start."""
+    w, K16, V16, cbK, cbV, o, g, dK, dV = _build(name, over, T, plen, extra=64)
+    B = w.B
+    pos = 0
+    for n_add in (37, 23):
+        lens = o.len.copy()
+        if any(int(lens[b]) + n_add > T + 64 for b in range(B)):
+            break
+        blk_k = np.stack([K16[b, T + pos: T + pos + n_add] for b in range(B)])
+        blk_v = np.stack([V16[b, T + pos: T + pos + n_add] for b in range(B)])
+        o.append(blk_k, blk_v, cbK, cbV)
+        gpu_quantize(g, dK, dV, blk_k, blk_v)
+        compare_cache(g, o, B)
+        pos += n_add
+
+
+@pytest.mark.parametrize("n_add", [1, 5, 40])
+def test_append_capacity_overflow(n_add):
+    """Lists that fill up during appends (short and general paths): the tokens whose outliers
+    do not fit drop them, the count stops at the last kept token, the status bit is set."""
+    import long_context_decode_nuq_b200 as K
+    w, K16, V16, cbK, cbV, o, g, dK, dV = _build("llama7b_layer_32k", dict(Hq=4, Hkv=4), 120,
+                                                  None, extra=128, cap=304)
+    assert not o.status & O.STATUS_OUTLIER_OVERFLOW
+    pos = 0
+    while pos + n_add <= 120 and not o.status & O.STATUS_OUTLIER_OVERFLOW:
+        blk_k = K16[:, 120 + pos: 120 + pos + n_add]
+        blk_v = V16[:, 120 + pos: 120 + pos + n_add]
+        o.append(blk_k, blk_v, cbK, cbV)
+        gpu_quantize(g, dK, dV, blk_k, blk_v)
+        compare_cache(g, o, w.B)
+        pos += n_add
+    assert o.status & O.STATUS_OUTLIER_OVERFLOW
+    assert K.kvq_get_status(g) & K.KVQ_STATUS_OUTLIER_OVERFLOW
+
+
+def _plant_specials(K16, V16, seed):
+    """Overwrite a seeded scatter of entries with fp16 specials, and make one key channel and
+    one token's value row constant (so that their half is 0)."""
+    rng = np.random.default_rng(seed)
+    specials = np.array([0x7E00, 0xFE00, 0x7C00, 0xFC00, 0x0000, 0x8000, 0x0001, 0x8001, 0x7BFF,
+                         0xFBFF, 0x03FF, 0x3C00], dtype=np.uint16)
+    for a in (K16, V16):
+        flat = a.reshape(-1).view(np.uint16)
+        idx = rng.choice(flat.size, size=max(1, flat.size // 400), replace=False)
+        flat[idx] = specials[rng.integers(0, specials.size, idx.size)]
+    K16[:, :, 0, 5] = np.float16(0.25)      # a constant key channel
+    V16[:, 3] = np.float16(-1.5)           # a constant value row
+    V16[:, 7, :, :64] = np.float16(np.nan)  # a row whose upper threshold is NaN
+    return K16, V16
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_special_values_bit_exact(bits):
+    """NaN, infinities, signed zeros, subnormals, fp16 extremes, constant channels and rows:
+    prefill, a short append and a long append all match the oracle bit for bit."""
+    import oracle as O2
+    w = synth.workload("llama7b_layer_32k", Hq=4, Hkv=4, bits=bits)
+    T, extra = 190, 64
+    K16, V16 = host_block(w, T + extra)
+    K16, V16 = _plant_specials(K16.copy(), V16.copy(), 7 + bits)
+    cbK, cbV = oracle_codebooks(w)
+    cap = 1 << 18
+    o = O2.QuantizedCache(w.B, w.Hkv, w.bits, T + extra, w.f, cap, cap)
+    o.prefill(K16[:, :T], V16[:, :T], [T] * w.B, cbK, cbV)
+    g = gpu_cache(w, T + extra, cap, cap)
+    dK, dV = to_dev_codebook(cbK), to_dev_codebook(cbV)
+    gpu_quantize(g, dK, dV, K16[:, :T], V16[:, :T], calibrate=1)
+    compare_cache(g, o, w.B)
+    for lo, hi in ((T, T + 3), (T + 3, T + 44)):
+        o.append(K16[:, lo:hi], V16[:, lo:hi], cbK, cbV)
+        gpu_quantize(g, dK, dV, K16[:, lo:hi], V16[:, lo:hi])
+        compare_cache(g, o, w.B)
