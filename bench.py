@@ -49,6 +49,7 @@ def parse():
     p.add_argument("--no-fp16", action="store_true")
     p.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
     p.add_argument("--tokens", type=int, default=0, help="override the cached token count")
+    p.add_argument("--bits", type=int, default=0, help="override the workload's code width")
     p.add_argument("--shard", default="tokens", choices=["tokens", "replicas"],
                    help="N > 1: tokens = one sequence of N x T tokens, rank r holding tokens "
                         "[r T, (r+1) T) (partials all-gathered and merged per layer); replicas = "
@@ -190,7 +191,8 @@ def cache_bytes_per_token(w, outlier_bytes=OUTLIER_ENTRY_BYTES, params=True):
 
 
 def bytes_model(w, T, kcount, vcount, path, outlier_bytes=OUTLIER_ENTRY_BYTES, logits=True):
-    """Algorithmic bytes of one layer's decode (attention part) over T tokens.
+    """Algorithmic bytes of one layer's decode (attention part) over T tokens of each of the
+    w.B sequences; kcount and vcount are the outlier entries of all the sequences.
 
     Key side (QK): packed key codes, key-outlier entries (outlier_bytes each: position and
     value), key chunk pointers (one list per kv head); value side (PV): packed value codes,
@@ -201,9 +203,9 @@ def bytes_model(w, T, kcount, vcount, path, outlier_bytes=OUTLIER_ENTRY_BYTES, l
     """
     code_row = w.Hkv * w.D * w.bits // 8
     nch = (T + 63) // 64 + 1
-    k_bytes = T * code_row + outlier_bytes * kcount + 4 * nch * w.Hkv
-    v_bytes = T * code_row + outlier_bytes * vcount + 8 * T + 4 * nch * w.Hkv
-    logit = 4 * w.Hq * T if logits else 0
+    k_bytes = w.B * (T * code_row + 4 * nch * w.Hkv) + outlier_bytes * kcount
+    v_bytes = w.B * (T * code_row + 8 * T + 4 * nch * w.Hkv) + outlier_bytes * vcount
+    logit = 4 * w.Hq * T * w.B if logits else 0
     if path == "split":
         return {"qk": k_bytes + logit, "pv": v_bytes + logit, "total": k_bytes + v_bytes + 2 * logit}
     if path == "one-call":
@@ -299,6 +301,8 @@ def run_kvq(args, rank, world):
         over["layers"] = args.layers
     if args.tokens:
         over["T"] = args.tokens
+    if args.bits:
+        over["bits"] = args.bits
     w = synth.workload(args.workload, **over)
     steps_total = args.warmup + args.steps
     e2e_steps = min(args.steps, 10)
@@ -369,8 +373,8 @@ def run_kvq(args, rank, world):
     if args.no_fp16:  # the staged K/V of the last layer serve only the fp16 comparison
         del kstage, vstage
         torch.cuda.empty_cache()
-    kcount = int(caches[0].kcount.cpu()[0].sum())
-    vcount = int(caches[0].vcount.cpu()[0].sum())
+    kcount = int(caches[0].kcount.cpu().sum())  # all sequences of the layer
+    vcount = int(caches[0].vcount.cpu().sum())
 
     # per-step inputs: appended token K/V and queries, per layer (device and pinned host)
     nL = layers * R

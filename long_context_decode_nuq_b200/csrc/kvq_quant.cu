@@ -29,7 +29,7 @@ struct QuantWs {
     uint32_t* hist1;  // [B][n][256]
     uint32_t* sel1;   // [B][n][4]  bin_lo, rem_lo, bin_hi, rem_hi
     uint32_t* hist2;  // [B][n][512]
-    uint32_t* kcut;   // [B][Hkv][64][16] key cut pairs (calibrating calls)
+    uint32_t* kcut;   // [B][n/2][16] key cut pairs of adjacent channels (calibrating calls)
     uint32_t* vthr;   // [B][n_new] fp16 t_lo | t_hi << 16
     uint16_t* vcut;   // [B][n_new][16] value cuts of each token, slot 15 force-zero flag
     uint32_t* kcc;    // [B*Hkv][nchc] outliers of this call in chunk cl of list (b, h)
@@ -118,6 +118,11 @@ __device__ uint32_t block_excl_scan(uint32_t v, uint32_t* sm, uint32_t* total) {
     return before + incl - v;
 }
 
+__device__ __forceinline__ uint32_t okey2(uint32_t w) {  // order keys of both halves of w
+    const uint32_t s = (w >> 15) & 0x00010001u;
+    return w ^ ((s * 0x7FFFu) | 0x80008000u);
+}
+
 // ---------------------------------------------------------------------------------
 __global__ void k_begin(kvq_cfg cfg, kvq_cache c, const int32_t* plen, int n_new, int calibrate,
                         QuantWs ws) {
@@ -148,27 +153,30 @@ __global__ void k_begin(kvq_cfg cfg, kvq_cache c, const int32_t* plen, int n_new
 
 // ---------------------------------------------------------------------------------
 // Key channel calibration: per-channel radix select (technique (i), pre-RoPE (ii)).  A block
-// takes kCalCols adjacent channels over a range of tokens; lane l of each warp reads channels
-// 2l and 2l + 1 of a token row (one 4-byte load, 128 bytes per warp and row), kCalU rows in
-// flight per warp; per-channel histograms in shared memory with a stride of 257 words (the
-// same bin of neighbouring channels falls in different banks), added to the global ones at
-// the end.  Pass 1 counts the high byte of the fp16 order key; pass 2 the low byte of the keys
-// whose high byte is the bin of t_lo (first 256 bins) or of t_hi (next 256).
+// takes kCalCols adjacent channels over a range of at most 65,535 tokens; lane l of each warp
+// reads channels 2l and 2l + 1 of a token row (one 4-byte load, 128 bytes per warp and row),
+// kCalU rows in flight per warp.  Per-channel histograms live in shared memory, 257 words per
+// channel (the same bin of neighbouring channels falls in different banks), and are added to
+// the global ones at the end.  Pass 1 counts the high byte of the fp16 order key (32-bit
+// counters); pass 2 the low byte of the keys whose high byte is the bin of t_lo (bins 0-255)
+// or of t_hi (bins 256-511), in 16-bit counters two to a word.
 constexpr int kCalCols = 64;
 constexpr int kCalThreads = 512;
 constexpr int kCalU = 8;
 constexpr int kCalStride = 257;
+constexpr int kCalRows = 65535;  // rows per block at most (16-bit counters of pass 2)
+constexpr int kCalSmem = kCalCols * kCalStride * 4;
 
+template <int PASS>
 __global__ void __launch_bounds__(kCalThreads) k_calib_hist(kvq_cfg cfg,
                                                             const uint16_t* __restrict__ k,
-                                                            int n_new, QuantWs ws, int pass) {
+                                                            int n_new, QuantWs ws) {
     extern __shared__ uint32_t sh[];
     const int b = blockIdx.z;
     if (!ws.calib[b]) return;
     const int n = cfg.Hkv * kD;
     const int N = ws.ntok[b];
-    const int nh = pass == 1 ? 1 : 2;  // histograms per channel
-    for (int i = threadIdx.x; i < kCalCols * nh * kCalStride; i += blockDim.x) sh[i] = 0;
+    for (int i = threadIdx.x; i < kCalCols * kCalStride; i += blockDim.x) sh[i] = 0;
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const int j0 = blockIdx.x * kCalCols + 2 * lane;  // this lane's first channel
@@ -177,43 +185,46 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_hist(kvq_cfg cfg,
     const int i1 = min(N, i0 + per);
     if (j0 < n) {
         uint32_t bl0 = 0, bh0 = 0, bl1 = 0, bh1 = 0;
-        if (pass == 2) {
+        if (PASS == 2) {
             const uint32_t* s0 = ws.sel1 + ((size_t)b * n + j0) * 4;
             bl0 = s0[0]; bh0 = s0[2]; bl1 = s0[4]; bh1 = s0[6];
         }
-        uint32_t* h0 = sh + (2 * lane) * nh * kCalStride;
-        uint32_t* h1 = h0 + nh * kCalStride;
+        uint32_t* h0 = sh + (2 * lane) * kCalStride;
+        uint32_t* h1 = h0 + kCalStride;
         const uint16_t* src = k + (size_t)b * n_new * n + j0;
-        for (int ib = i0 + warp; ib < i1; ib += nw * kCalU) {
-            uint32_t v[kCalU];
-#pragma unroll
-            for (int u = 0; u < kCalU; ++u) {
-                const int i = ib + u * nw;
-                v[u] = i < i1 ? *reinterpret_cast<const uint32_t*>(src + (size_t)i * n) : 0u;
+        auto count = [&](uint32_t w) {
+            const uint32_t key = okey2(w);
+            const uint32_t a0 = (key >> 8) & 0xFFu, a1 = key >> 24;
+            if (PASS == 1) {
+                atomicAdd(&h0[a0], 1u);
+                atomicAdd(&h1[a1], 1u);
+            } else {
+                const uint32_t l0 = key & 0xFFu, l1 = (key >> 16) & 0xFFu;
+                if (a0 == bl0) atomicAdd(&h0[l0 >> 1], 1u << (16 * (l0 & 1u)));
+                if (a0 == bh0) atomicAdd(&h0[128 + (l0 >> 1)], 1u << (16 * (l0 & 1u)));
+                if (a1 == bl1) atomicAdd(&h1[l1 >> 1], 1u << (16 * (l1 & 1u)));
+                if (a1 == bh1) atomicAdd(&h1[128 + (l1 >> 1)], 1u << (16 * (l1 & 1u)));
             }
+        };
+        int ib = i0 + warp;
+        for (; ib + (kCalU - 1) * nw < i1; ib += nw * kCalU) {
+            uint32_t w[kCalU];
 #pragma unroll
-            for (int u = 0; u < kCalU; ++u) {
-                if (ib + u * nw >= i1) break;
-                const uint32_t k0 = okey(v[u] & 0xFFFFu), k1 = okey(v[u] >> 16);
-                if (pass == 1) {
-                    atomicAdd(&h0[k0 >> 8], 1u);
-                    atomicAdd(&h1[k1 >> 8], 1u);
-                } else {
-                    if ((k0 >> 8) == bl0) atomicAdd(&h0[k0 & 255u], 1u);
-                    if ((k0 >> 8) == bh0) atomicAdd(&h0[kCalStride + (k0 & 255u)], 1u);
-                    if ((k1 >> 8) == bl1) atomicAdd(&h1[k1 & 255u], 1u);
-                    if ((k1 >> 8) == bh1) atomicAdd(&h1[kCalStride + (k1 & 255u)], 1u);
-                }
-            }
+            for (int u = 0; u < kCalU; ++u)
+                w[u] = *reinterpret_cast<const uint32_t*>(src + (size_t)(ib + u * nw) * n);
+#pragma unroll
+            for (int u = 0; u < kCalU; ++u) count(w[u]);
         }
+        for (; ib < i1; ib += nw) count(*reinterpret_cast<const uint32_t*>(src + (size_t)ib * n));
     }
     __syncthreads();
-    const int nb = 256 * nh;
-    uint32_t* gh = (pass == 1 ? ws.hist1 : ws.hist2) + ((size_t)b * n + blockIdx.x * kCalCols) * nb;
+    const int nb = PASS == 1 ? 256 : 512;
+    uint32_t* gh = (PASS == 1 ? ws.hist1 : ws.hist2) + ((size_t)b * n + blockIdx.x * kCalCols) * nb;
     for (int i = threadIdx.x; i < kCalCols * nb; i += blockDim.x) {
         const int col = i / nb, r = i % nb;
         if (blockIdx.x * kCalCols + col < n) {
-            const uint32_t v = sh[col * nh * kCalStride + (r >> 8) * kCalStride + (r & 255)];
+            const uint32_t* hc = sh + col * kCalStride;
+            const uint32_t v = PASS == 1 ? hc[r] : ((hc[r >> 1] >> (16 * (r & 1))) & 0xFFFFu);
             if (v) atomicAdd(&gh[i], v);
         }
     }
@@ -279,20 +290,41 @@ __global__ void k_calib_select(kvq_cfg cfg, kvq_cache c, QuantWs ws, int pass) {
 // every input, NaN included, normalize to 0: such a channel or token is flagged in slot 15 of
 // its record and its inputs are replaced by +0 before the comparison.
 
-// Least fp16 value in the fp16 total order whose normalized value exceeds `bound` (fp16 bits),
-// found by bisection over the order keys of -inf .. +inf; 0x7E00 (NaN) when none does.
+// Least fp16 value in the fp16 total order whose normalized value exceeds `bound` (fp16 bits);
+// 0x7E00 (NaN) when none does.  The walk starts at the fp16 value nearest off + bound * half,
+// which is within a step or two of the answer, and moves along the order keys until the test
+// changes; the test being monotone along the keys, that is the least passing key.  A long walk
+// (not expected) falls back to bisection over -inf .. +inf.
 __device__ uint32_t cut_of(float bound, float off, float half) {
     auto above = [&](uint32_t key) {
         return normalize(h2f((uint16_t)okey_inv(key)), off, half) > bound;
     };
-    uint32_t lo = 0x03FFu, hi = 0xFC00u;
-    if (!above(hi)) return 0x7E00u;
-    while (lo < hi) {
-        const uint32_t mid = (lo + hi) >> 1;
-        if (above(mid)) hi = mid;
-        else lo = mid + 1;
+    const uint32_t kmin = 0x03FFu, kmax = 0xFC00u;
+    if (!above(kmax)) return 0x7E00u;
+    if (above(kmin)) return okey_inv(kmin);
+    // here above(kmin) fails and above(kmax) passes
+    uint32_t key = kmin + 1;
+    const float x0 = __fadd_rn(off, __fmul_rn(bound, half));
+    if (isfinite(x0)) {
+        key = okey(__half_as_ushort(__float2half_rn(x0)));
+        key = key < kmin + 1 ? kmin + 1 : (key > kmax ? kmax : key);
     }
-    return okey_inv(lo);
+    int steps = 0;
+    if (above(key)) {
+        while (above(key - 1) && ++steps < 64) --key;  // key - 1 >= kmin, which fails
+    } else {
+        while (!above(key) && ++steps < 64) ++key;     // stops at kmax at the latest
+    }
+    if (steps >= 64) {
+        uint32_t lo = kmin, hi = kmax;  // above(lo) fails, above(hi) passes
+        while (hi - lo > 1) {
+            const uint32_t mid = (lo + hi) >> 1;
+            if (above(mid)) hi = mid;
+            else lo = mid;
+        }
+        key = hi;
+    }
+    return okey_inv(key);
 }
 
 __device__ __forceinline__ __half2 as_h2(uint32_t x) { return *reinterpret_cast<__half2*>(&x); }
@@ -325,20 +357,20 @@ __device__ __forceinline__ uint32_t enc_pair(uint32_t x, const uint32_t* C) {
     return code;
 }
 
-// Per key channel pair (c, c + 64) of every kv head, after calibration: record p of head h
-// holds word j = cut_j(c) | cut_j(c + 64) << 16 for c = 128h + p, p < 64; word 15 the
-// force-zero flags (0xFFFF per half whose channel has half == 0).
+// Per pair of adjacent key channels (2m, 2m + 1), after calibration: word j of record m holds
+// cut_j(2m) | cut_j(2m + 1) << 16; word 15 the force-zero flags (0xFFFF per half whose channel
+// has half == 0).
 __global__ void k_key_cuts(kvq_cfg cfg, kvq_cache c, kvq_codebook cbK, QuantWs ws) {
     const int n = cfg.Hkv * kD, nb = (1 << cfg.bits) - 1;
     const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= (size_t)cfg.B * (n / 2) * 16) return;
     const int j = (int)(gid & 15);
-    const size_t rec = gid >> 4;  // (b, h, p)
+    const size_t rec = gid >> 4;  // (b, m)
     const int b = (int)(rec / (n / 2));
     if (!ws.calib[b]) return;
-    const int hp = (int)(rec % (n / 2)), h = hp >> 6, p = hp & 63;
-    const float* kp0 = c.kparams + ((size_t)b * n + h * kD + p) * 2;
-    const float* kp1 = kp0 + 64 * 2;
+    const int m = (int)(rec % (n / 2));
+    const float* kp0 = c.kparams + ((size_t)b * n + 2 * m) * 2;
+    const float* kp1 = kp0 + 2;
     uint32_t word;
     if (j < nb) {
         const float bd = cbK.bounds[j];
@@ -386,7 +418,9 @@ __device__ inline void warp_rank(const uint32_t* hist, uint32_t r, uint32_t& bin
     rem = __shfl_sync(0xffffffffu, fr, src);
 }
 
-__global__ void __launch_bounds__(kStWarps * 32) k_tok_stats(kvq_cfg cfg, kvq_cache c,
+constexpr int kStRegs = 8;   // row words (16 bytes) a lane holds at once (all of it for n <= 2048)
+
+__global__ void __launch_bounds__(kStWarps * 32, 3) k_tok_stats(kvq_cfg cfg, kvq_cache c,
                                                             kvq_codebook cbV,
                                                             const uint16_t* __restrict__ k,
                                                             const uint16_t* __restrict__ v,
@@ -397,33 +431,59 @@ __global__ void __launch_bounds__(kStWarps * 32) k_tok_stats(kvq_cfg cfg, kvq_ca
     const int chk = t0 / kChunk + cl;
     const int ta = max(chk * kChunk, t0), tb = min(chk * kChunk + kChunk, t0 + nt);
     if (ta >= tb) return;
-    __shared__ __align__(16) uint32_t hist[kStWarps][512];
+    extern __shared__ __align__(16) uint32_t sst[];
+    const int Hkv = cfg.Hkv, n = Hkv * kD, n8 = n / 8;
+    uint32_t* hist = sst;                        // [kStWarps][512]
+    uint4* kth = reinterpret_cast<uint4*>(sst + kStWarps * 512);  // [n8][2]: t_lo and t_hi pairs
     __shared__ uint32_t ck[64], cv[64];
     __shared__ float bnd[16];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int Hkv = cfg.Hkv, n = Hkv * kD, n8 = n / 8;
     const int nb = (1 << cfg.bits) - 1;
-    for (int h = threadIdx.x; h < 64; h += blockDim.x) ck[h] = cv[h] = 0u;
+    for (int hh = threadIdx.x; hh < 64; hh += blockDim.x) ck[hh] = cv[hh] = 0u;
     if (threadIdx.x < nb) bnd[threadIdx.x] = cbV.bounds[threadIdx.x];
+    {
+        // key thresholds of 8 channels per entry, as (t_lo pairs, t_hi pairs) of half2 words
+        const uint4* kt4 = reinterpret_cast<const uint4*>(c.kthr + (size_t)b * n * 2);
+        for (int x = threadIdx.x; x < n8; x += blockDim.x) {
+            const uint4 p = kt4[2 * x], r = kt4[2 * x + 1];
+            kth[2 * x] = make_uint4(__byte_perm(p.x, p.y, 0x5410), __byte_perm(p.z, p.w, 0x5410),
+                                    __byte_perm(r.x, r.y, 0x5410), __byte_perm(r.z, r.w, 0x5410));
+            kth[2 * x + 1] = make_uint4(__byte_perm(p.x, p.y, 0x7632), __byte_perm(p.z, p.w, 0x7632),
+                                        __byte_perm(r.x, r.y, 0x7632), __byte_perm(r.z, r.w, 0x7632));
+        }
+    }
     __syncthreads();
-    uint32_t* hw = hist[warp];
+    uint32_t* hw = hist + warp * 512;
     const int kk = vector_k(cfg.outlier_frac, n);
     const uint32_t rl = kk, rh = n - 1 - kk;
-    const uint4* kt4 = reinterpret_cast<const uint4*>(c.kthr + (size_t)b * n * 2);
+    const int nrep = (n8 + 32 * kStRegs - 1) / (32 * kStRegs);
     for (int t = ta + warp; t < tb; t += kStWarps) {
         const int i = t - t0;
         const uint4* vr = reinterpret_cast<const uint4*>(v + ((size_t)b * n_new + i) * n);
         const uint4* kr = reinterpret_cast<const uint4*>(k + ((size_t)b * n_new + i) * n);
+        uint4 reg[kStRegs];
+        auto load = [&](int rep) {
+#pragma unroll
+            for (int r = 0; r < kStRegs; ++r) {
+                const int x = rep * 32 * kStRegs + 32 * r + lane;
+                reg[r] = x < n8 ? vr[x] : make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
         // pass 1: the high byte of each value's order key
         for (int q = lane; q < 512; q += 32) hw[q] = 0u;
         __syncwarp();
-        for (int x = lane; x < n8; x += 32) {
-            const uint4 w = vr[x];
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int rep = 0; rep < nrep; ++rep) {
+            load(rep);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                atomicAdd(&hw[okey(ww[e] & 0xFFFFu) >> 8], 1u);
-                atomicAdd(&hw[okey(ww[e] >> 16) >> 8], 1u);
+            for (int r = 0; r < kStRegs; ++r) {
+                if (rep * 32 * kStRegs + 32 * r + lane >= n8) continue;
+                const uint32_t ww[4] = {reg[r].x, reg[r].y, reg[r].z, reg[r].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t key = okey2(ww[e]);
+                    atomicAdd(&hw[(key >> 8) & 0xFFu], 1u);
+                    atomicAdd(&hw[key >> 24], 1u);
+                }
             }
         }
         __syncwarp();
@@ -434,16 +494,20 @@ __global__ void __launch_bounds__(kStWarps * 32) k_tok_stats(kvq_cfg cfg, kvq_ca
         for (int q = lane; q < 512; q += 32) hw[q] = 0u;
         __syncwarp();
         // pass 2: the low byte of the keys in the two selected bins
-        for (int x = lane; x < n8; x += 32) {
-            const uint4 w = vr[x];
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        for (int rep = 0; rep < nrep; ++rep) {
+            if (nrep > 1) load(rep);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
+            for (int r = 0; r < kStRegs; ++r) {
+                if (rep * 32 * kStRegs + 32 * r + lane >= n8) continue;
+                const uint32_t ww[4] = {reg[r].x, reg[r].y, reg[r].z, reg[r].w};
 #pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const uint32_t key = okey(hf ? (ww[e] >> 16) : (ww[e] & 0xFFFFu));
-                    if ((key >> 8) == bl) atomicAdd(&hw[key & 255u], 1u);
-                    if ((key >> 8) == bh) atomicAdd(&hw[256 + (key & 255u)], 1u);
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t key = okey2(ww[e]);
+                    const uint32_t h0 = (key >> 8) & 0xFFu, h1 = key >> 24;
+                    if (h0 == bl) atomicAdd(&hw[key & 255u], 1u);
+                    if (h0 == bh) atomicAdd(&hw[256 + (key & 255u)], 1u);
+                    if (h1 == bl) atomicAdd(&hw[(key >> 16) & 255u], 1u);
+                    if (h1 == bh) atomicAdd(&hw[256 + ((key >> 16) & 255u)], 1u);
                 }
             }
         }
@@ -468,38 +532,29 @@ __global__ void __launch_bounds__(kStWarps * 32) k_tok_stats(kvq_cfg cfg, kvq_ca
             else if (lane == 15) cut = half == 0.0f ? 0xFFFFu : 0u;
             ws.vcut[((size_t)b * n_new + i) * 16 + lane] = (uint16_t)cut;
         }
-        // outliers per kv head: lanes 0-15 of a pass lie in head x >> 4, lanes 16-31 in the next
+        // outliers per kv head (entry x of the row lies in head x >> 4)
         const uint32_t lo2 = lo_bits | (lo_bits << 16), hi2 = hi_bits | (hi_bits << 16);
-        for (int base = 0; base < n8; base += 32) {
-            const int x = base + lane;
-            uint32_t nv = 0, nk = 0;
-            if (x < n8) {
-                const uint4 w = vr[x];
-                nv = __popc(out2(w.x, lo2, hi2)) + __popc(out2(w.y, lo2, hi2)) +
-                     __popc(out2(w.z, lo2, hi2)) + __popc(out2(w.w, lo2, hi2));
-                const uint4 kw = kr[x];
-                const uint4 p = kt4[2 * x], q = kt4[2 * x + 1];  // (t_lo, t_hi) of 8 channels
-                nk = __popc(out2(kw.x, __byte_perm(p.x, p.y, 0x5410), __byte_perm(p.x, p.y, 0x7632))) +
-                     __popc(out2(kw.y, __byte_perm(p.z, p.w, 0x5410), __byte_perm(p.z, p.w, 0x7632))) +
-                     __popc(out2(kw.z, __byte_perm(q.x, q.y, 0x5410), __byte_perm(q.x, q.y, 0x7632))) +
-                     __popc(out2(kw.w, __byte_perm(q.z, q.w, 0x5410), __byte_perm(q.z, q.w, 0x7632)));
-            }
+        for (int rep = 0; rep < nrep; ++rep) {
+            if (nrep > 1) load(rep);
 #pragma unroll
-            for (int o = 8; o; o >>= 1) {
-                nv += __shfl_xor_sync(0xffffffffu, nv, o);
-                nk += __shfl_xor_sync(0xffffffffu, nk, o);
-            }
-            if ((lane & 15) == 0 && x < n8) {
+            for (int r = 0; r < kStRegs; ++r) {
+                const int x = rep * 32 * kStRegs + 32 * r + lane;
+                if (x >= n8) continue;
+                const uint32_t nv = __popc(out2(reg[r].x, lo2, hi2)) + __popc(out2(reg[r].y, lo2, hi2)) +
+                                    __popc(out2(reg[r].z, lo2, hi2)) + __popc(out2(reg[r].w, lo2, hi2));
+                const uint4 kw = kr[x], tl = kth[2 * x], th = kth[2 * x + 1];
+                const uint32_t nk = __popc(out2(kw.x, tl.x, th.x)) + __popc(out2(kw.y, tl.y, th.y)) +
+                                    __popc(out2(kw.z, tl.z, th.z)) + __popc(out2(kw.w, tl.w, th.w));
                 if (nv) atomicAdd(&cv[x >> 4], nv >> 4);
                 if (nk) atomicAdd(&ck[x >> 4], nk >> 4);
             }
         }
     }
     __syncthreads();
-    for (int h = threadIdx.x; h < Hkv; h += blockDim.x) {
-        const size_t li = (size_t)b * Hkv + h;
-        ws.kcc[li * nchc + cl] = ck[h];
-        ws.vcc[li * nchc + cl] = cv[h];
+    for (int hh = threadIdx.x; hh < Hkv; hh += blockDim.x) {
+        const size_t li = (size_t)b * Hkv + hh;
+        ws.kcc[li * nchc + cl] = ck[hh];
+        ws.vcc[li * nchc + cl] = cv[hh];
     }
 }
 
@@ -580,21 +635,28 @@ __global__ void k_tok_final(kvq_cfg cfg, kvq_cache c, QuantWs ws) {
 
 // ---------------------------------------------------------------------------------
 // Encode and pack.  One warp per (64-token chunk, kv head) of a sequence, two token quads at a
-// time: half-warp hw takes quad u + hw and lane i = lane & 15 builds the lane group i words
-// of that quad's key and value blocks itself.  Lane group i owns the channel pairs
-// (c, c + 64), c = i + 16kk (kk < 4), and holds token 4u + (s ^ (i >> 2)) in slot s, so every
-// field's bit offset is a constant.  The rows of the two quads (keys and values of one kv
-// head, 256 bytes per token) reach shared memory through a three-stage ring of 16-byte
-// asynchronous copies, a warp's own; quad 1's rows sit 32 bytes further on so that the two
-// half-warps read disjoint banks.  Outliers are written per token in channel order: channel
-// c = i + 16*k2 (k2 < 8) ranks after all flagged channels of the lower k2 and the lower
-// lanes of its own k2.
+// time; the rows of the two quads (keys and values of one kv head, 256 bytes per token) reach
+// shared memory through a two-stage ring of 16-byte asynchronous copies, a warp's own (the
+// encode of a stage takes longer than the copies of the next).
+//  - Encode: half-warp hw takes quad u0 + hw and lane q the channels 8q .. 8q + 7 of each of
+//    its four tokens (one 16-byte shared load per row), compares them two at a time against
+//    the thresholds and cuts, and stores the eight codes as bytes, row by row.
+//  - Outliers: the flagged channels of a lane are contiguous in channel order, so a token's
+//    entries are ranked by a prefix sum of the per-lane counts over the half-warp (the four
+//    tokens of a quad in one scan, one byte each); tokens go in order, quad u0 first.
+//  - Pack: lane i of half-warp hw builds the lane group i words of quad u0 + hw from the code
+//    bytes: slot s holds token s ^ (i >> 2), the field of pair (c, c + 64), c = i + 16kk, is
+//    code(c) | code(c + 64) << bits at bit 2 bits (4kk + s).
+// Quad 1's rows and codes sit 32 and 16 bytes further on, so the two half-warps read disjoint
+// banks.
 constexpr int kWrWarps = 4;
-constexpr int kWrStages = 3;
+constexpr int kWrStages = 2;
 constexpr int kQStride = 4 * 256 + 32;
 constexpr int kKVStride = 2 * kQStride;
 constexpr int kStageBytes = 2 * kKVStride;
-constexpr int kWrSmem = kWrWarps * kWrStages * kStageBytes;
+constexpr int kCQ = 4 * 128 + 16;
+constexpr int kWarpSmem = kWrStages * kStageBytes + 4 * kCQ;
+constexpr int kWrSmem = kWrWarps * kWarpSmem;
 
 __device__ __forceinline__ void cp16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -604,16 +666,13 @@ template <int N>
 __device__ __forceinline__ void cp_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-__device__ __forceinline__ uint32_t lds16(const unsigned char* p) {
-    return (uint32_t)*reinterpret_cast<const uint16_t*>(p);
-}
 
 template <int BITS, bool KCUTS>
-__global__ void __launch_bounds__(kWrWarps * 32) k_tok_write(kvq_cfg cfg, kvq_cache c,
-                                                            kvq_codebook cbK,
-                                                            const uint16_t* __restrict__ k,
-                                                            const uint16_t* __restrict__ v,
-                                                            int n_new, int nchc, QuantWs ws) {
+__global__ void __launch_bounds__(kWrWarps * 32, BITS == 4 ? 4 : 5) k_tok_write(kvq_cfg cfg, kvq_cache c,
+                                                               kvq_codebook cbK,
+                                                               const uint16_t* __restrict__ k,
+                                                               const uint16_t* __restrict__ v,
+                                                               int n_new, int nchc, QuantWs ws) {
     constexpr int NB = (1 << BITS) - 1;
     constexpr int W2 = 2 * BITS;
     extern __shared__ __align__(16) unsigned char wsm[];
@@ -626,26 +685,28 @@ __global__ void __launch_bounds__(kWrWarps * 32) k_tok_write(kvq_cfg cfg, kvq_ca
     const int chk = t0 / kChunk + cl;
     const int ta = max(chk * kChunk, t0), tb = min(chk * kChunk + kChunk, t0 + nt);
     if (ta >= tb) return;
-    const int n = Hkv * kD, i = lane & 15, hw = lane >> 4;
+    const int n = Hkv * kD, q = lane & 15, hw = lane >> 4;
     const size_t li = (size_t)b * Hkv + h;
-    unsigned char* ring = wsm + warp * (kWrStages * kStageBytes);
+    unsigned char* ring = wsm + warp * kWarpSmem;
+    unsigned char* codes = ring + kWrStages * kStageBytes;
     const uint32_t ring_s = (uint32_t)__cvta_generic_to_shared(ring);
     const int ua = ta >> 2, ub = (tb - 1) >> 2;
     const int nit = (ub - ua) / 2 + 1;
-    // stage `it`: rows of quads ua + 2it and ua + 2it + 1, keys then values
+    // stage `it`: rows of quads ua + 2it and ua + 2it + 1; piece r of a lane is (keys or
+    // values) r >> 2, quad (r >> 1) & 1, token (lane >> 4) + 2 (r & 1), bytes 16 (lane & 15)
+    const uint16_t* srcK = k + (size_t)b * n_new * n + h * kD + q * 8;
+    const uint16_t* srcV = v + (size_t)b * n_new * n + h * kD + q * 8;
+    const uint32_t dlane = (uint32_t)((lane >> 4) * 256 + q * 16);
     auto issue = [&](int it) {
         const int u0 = ua + 2 * it;
-        const uint32_t sb = ring_s + (it % kWrStages) * kStageBytes;
+        const uint32_t sb = ring_s + (it % kWrStages) * kStageBytes + dlane;
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-            const int pc = lane + 32 * r;
-            const int which = pc >> 7, hq = (pc >> 6) & 1, j = (pc >> 4) & 3, seg = pc & 15;
+            const int which = r >> 2, hq = (r >> 1) & 1, j = hw + 2 * (r & 1);
             const int t = 4 * (u0 + hq) + j;
-            if (t >= ta && t < tb) {
-                const uint16_t* src =
-                    (which ? v : k) + ((size_t)b * n_new + (t - t0)) * n + h * kD + seg * 8;
-                cp16(sb + which * kKVStride + hq * kQStride + j * 256 + seg * 16, src);
-            }
+            if (t >= ta && t < tb)
+                cp16(sb + which * kKVStride + hq * kQStride + 2 * (r & 1) * 256,
+                     (which ? srcV : srcK) + (size_t)(t - t0) * n);
         }
     };
 #pragma unroll
@@ -653,35 +714,43 @@ __global__ void __launch_bounds__(kWrWarps * 32) k_tok_write(kvq_cfg cfg, kvq_ca
         if (p < nit) issue(p);
         cp_commit();
     }
-    // key channel data of the lane's four pairs
-    uint32_t klo[4], khi[4], kz[4];
+    // the lane's key channels 8q .. 8q + 7 as four adjacent pairs
+    uint32_t KLO[4], KHI[4], KZ[4];
     uint32_t KC[4][KCUTS ? NB : 1];
-    float kof[4][2], khf[4][2], bK[KCUTS ? 1 : NB];
+    float kof[8], khf[8], bK[KCUTS ? 1 : NB];
+    {
+        const uint4* th = reinterpret_cast<const uint4*>(c.kthr + ((size_t)b * n + h * kD + 8 * q) * 2);
+        const uint4 t0v = th[0], t1v = th[1];
+        const uint32_t a[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-        const int p = i + 16 * kk;
-        const uint32_t* th = reinterpret_cast<const uint32_t*>(c.kthr) + (size_t)b * n + h * kD + p;
-        const uint32_t a0 = th[0], a1 = th[64];
-        klo[kk] = __byte_perm(a0, a1, 0x5410);
-        khi[kk] = __byte_perm(a0, a1, 0x7632);
-        if constexpr (KCUTS) {
-            const uint4* rec = reinterpret_cast<const uint4*>(ws.kcut + (li * 64 + p) * 16);
+        for (int e = 0; e < 4; ++e) {
+            KLO[e] = __byte_perm(a[2 * e], a[2 * e + 1], 0x5410);
+            KHI[e] = __byte_perm(a[2 * e], a[2 * e + 1], 0x7632);
+        }
+    }
+    if constexpr (KCUTS) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const uint4* rec =
+                reinterpret_cast<const uint4*>(ws.kcut + ((size_t)b * (n / 2) + h * 64 + 4 * q + e) * 16);
             const uint4 r0 = rec[0], r1 = rec[1], r2 = rec[2], r3 = rec[3];
             const uint32_t rw[16] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w,
                                      r2.x, r2.y, r2.z, r2.w, r3.x, r3.y, r3.z, r3.w};
 #pragma unroll
-            for (int j = 0; j < NB; ++j) KC[kk][j] = rw[j];
-            kz[kk] = rw[15];
-        } else {
-            const float* kp = c.kparams + ((size_t)b * n + h * kD + p) * 2;
-            kof[kk][0] = kp[0];
-            khf[kk][0] = kp[1];
-            kof[kk][1] = kp[128];
-            khf[kk][1] = kp[129];
-            kz[kk] = 0u;
+            for (int j = 0; j < NB; ++j) KC[e][j] = rw[j];
+            KZ[e] = rw[15];
         }
-    }
-    if constexpr (!KCUTS) {
+    } else {
+        const float4* kp = reinterpret_cast<const float4*>(c.kparams + ((size_t)b * n + h * kD + 8 * q) * 2);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float4 p = kp[e];
+            kof[2 * e] = p.x;
+            khf[2 * e] = p.y;
+            kof[2 * e + 1] = p.z;
+            khf[2 * e + 1] = p.w;
+            KZ[e] = 0u;
+        }
 #pragma unroll
         for (int j = 0; j < NB; ++j) bK[j] = cbK.bounds[j];
     }
@@ -703,112 +772,105 @@ __global__ void __launch_bounds__(kWrWarps * 32) k_tok_write(kvq_cfg cfg, kvq_ca
     uint32_t acc[2] = {inc[0], inc[1]};
     uint32_t* outl[2] = {c.kout + li * cfg.out_cap_k, c.vout + li * cfg.out_cap_v};
     const size_t blk0 = li * nquads(cfg.T_max);
+    unsigned char* cq = codes + hw * kCQ;  // this half-warp's quad: key code rows, then values
     for (int it = 0; it < nit; ++it) {
         if (it + kWrStages - 1 < nit) issue(it + kWrStages - 1);
         cp_commit();
         cp_wait<kWrStages - 1>();
         __syncwarp();
-        const unsigned char* sbuf = ring + (it % kWrStages) * kStageBytes;
+        const unsigned char* sq = ring + (it % kWrStages) * kStageBytes + hw * kQStride;
         const int u0 = ua + 2 * it, u = u0 + hw;
-        const unsigned char* qk = sbuf + hw * kQStride;  // this half-warp's quad, keys
-        const unsigned char* qv = qk + kKVStride;        // and values
-        uint32_t kw[BITS], vw[BITS], fm[BITS];
-#pragma unroll
-        for (int q = 0; q < BITS; ++q) kw[q] = vw[q] = fm[q] = 0u;
-        uint32_t FK = 0, FV = 0;  // outlier flags, bit 8s + k2
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int j = s ^ (i >> 2), t = 4 * u + j;
+        // ---- encode the four tokens of quad u
+        uint32_t F[2] = {0u, 0u};  // flags of the lane's 8 channels, byte j per token
+        uint32_t pres = 0;
+#pragma unroll 1
+        for (int j = 0; j < 4; ++j) {
+            const int t = 4 * u + j;
             const bool pr = u <= ub && t >= ta && t < tb;
-            const uint32_t pm = pr ? 0xFFFFFFFFu : 0u;
-            uint32_t vlo2, vhi2, VC[NB], vz;
+            pres |= (pr ? 1u : 0u) << j;
+            const uint4 xk = *reinterpret_cast<const uint4*>(sq + j * 256 + q * 16);
+            const uint4 xv = *reinterpret_cast<const uint4*>(sq + kKVStride + j * 256 + q * 16);
+            uint32_t VC[NB], VLO, VHI, VZ;
             {
                 const size_t ti = (size_t)b * n_new + (pr ? t - t0 : 0);
                 const uint32_t vt = ws.vthr[ti];
-                vlo2 = __byte_perm(vt, 0, 0x1010);
-                vhi2 = __byte_perm(vt, 0, 0x3232);
+                VLO = __byte_perm(vt, 0, 0x1010);
+                VHI = __byte_perm(vt, 0, 0x3232);
                 const uint4* cr = reinterpret_cast<const uint4*>(ws.vcut + ti * 16);
                 const uint4 c0v = cr[0], c1v = cr[1];
                 const uint32_t cw[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
 #pragma unroll
                 for (int jj = 0; jj < NB; ++jj)
                     VC[jj] = __byte_perm(cw[jj >> 1], 0, (jj & 1) ? 0x3232 : 0x1010);
-                vz = (cw[7] >> 16) ? 0xFFFFFFFFu : 0u;
+                VZ = (cw[7] >> 16) ? 0xFFFFFFFFu : 0u;
             }
-            const unsigned char* rk = qk + j * 256;
-            const unsigned char* rv = qv + j * 256;
+            const uint32_t xkw[4] = {xk.x, xk.y, xk.z, xk.w};
+            const uint32_t xvw[4] = {xv.x, xv.y, xv.z, xv.w};
+            uint32_t ck[4], cv[4], fk = 0, fv = 0;
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const int f = 4 * kk + s, off = f * W2, wd = off >> 5, bt = off & 31;
-                const int cb = 2 * (i + 16 * kk);
-                const uint32_t xk = pr ? (lds16(rk + cb) | (lds16(rk + cb + 128) << 16)) : 0u;
-                const uint32_t xv = pr ? (lds16(rv + cb) | (lds16(rv + cb + 128) << 16)) : 0u;
-                // keys
-                const uint32_t ok = out2(xk, klo[kk], khi[kk]) & pm;
-                FK |= ((ok & 1u) << (8 * s + kk)) | (((ok >> 16) & 1u) << (8 * s + kk + 4));
-                uint32_t cp;
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t ok = out2(xkw[e], KLO[e], KHI[e]);
+                fk |= ((ok & 1u) | ((ok >> 15) & 2u)) << (2 * e);
                 if constexpr (KCUTS) {
-                    cp = enc_pair<BITS>(xk & ~(ok | kz[kk]), KC[kk]);
+                    ck[e] = enc_pair<BITS>(xkw[e] & ~(ok | KZ[e]), KC[e]);
                 } else {
                     uint32_t c2[2];
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const float xf =
-                            ((ok >> (16 * e)) & 1u) ? 0.0f : h2f((uint16_t)(xk >> (16 * e)));
-                        c2[e] = encode(normalize(xf, kof[kk][e], khf[kk][e]), bK, NB);
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const float xf = ((ok >> (16 * hf)) & 1u) ? 0.0f : h2f((uint16_t)(xkw[e] >> (16 * hf)));
+                        c2[hf] = encode(normalize(xf, kof[2 * e + hf], khf[2 * e + hf]), bK, NB);
                     }
-                    cp = c2[0] | (c2[1] << 16);
+                    ck[e] = c2[0] | (c2[1] << 16);
                 }
-                const uint32_t fk = pr ? ((cp & 0xFFFFu) | ((cp >> 16) << BITS)) : 0u;
-                // values
-                const uint32_t ov = out2(xv, vlo2, vhi2) & pm;
-                FV |= ((ov & 1u) << (8 * s + kk)) | (((ov >> 16) & 1u) << (8 * s + kk + 4));
-                const uint32_t cq = enc_pair<BITS>(xv & ~(ov | vz), VC);
-                const uint32_t fv = pr ? ((cq & 0xFFFFu) | ((cq >> 16) << BITS)) : 0u;
-                const uint32_t fmask = pr ? ((1u << W2) - 1u) : 0u;
-                kw[wd] |= fk << bt;
-                vw[wd] |= fv << bt;
-                fm[wd] |= fmask << bt;
-                if (bt + W2 > 32) {
-                    kw[wd + 1] |= fk >> (32 - bt);
-                    vw[wd + 1] |= fv >> (32 - bt);
-                    fm[wd + 1] |= fmask >> (32 - bt);
-                }
+                const uint32_t ov = out2(xvw[e], VLO, VHI);
+                fv |= ((ov & 1u) | ((ov >> 15) & 2u)) << (2 * e);
+                cv[e] = enc_pair<BITS>(xvw[e] & ~(ov | VZ), VC);
             }
+            // code bytes of channels 8q .. 8q + 7 (zero for a token outside this call)
+            const uint32_t pm = pr ? 0xFFFFFFFFu : 0u;
+            *reinterpret_cast<uint2*>(cq + j * 128 + 8 * q) =
+                make_uint2(__byte_perm(ck[0], ck[1], 0x6420) & pm, __byte_perm(ck[2], ck[3], 0x6420) & pm);
+            *reinterpret_cast<uint2*>(cq + 2 * kCQ + j * 128 + 8 * q) =
+                make_uint2(__byte_perm(cv[0], cv[1], 0x6420) & pm, __byte_perm(cv[2], cv[3], 0x6420) & pm);
+            F[0] |= (fk & pm) << (8 * j);
+            F[1] |= (fv & pm) << (8 * j);
         }
-        // outlier entries, token by token in order (half 0's quad, then half 1's)
+        // ---- outlier entries, token by token (quad u0's four tokens, then quad u0 + 1's)
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
-            const uint32_t F = w ? FV : FK;
-            if (!__ballot_sync(0xffffffffu, F != 0u)) continue;
+            if (!__ballot_sync(0xffffffffu, F[w] != 0u)) continue;
+            // per-token counts of the lane (one byte each) and their inclusive prefix over
+            // the half-warp; a byte never exceeds 16 x 8
+            uint32_t c4 = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) c4 |= (uint32_t)__popc((F[w] >> (8 * j)) & 0xFFu) << (8 * j);
+            uint32_t in4 = c4;
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, in4, o, 16);
+                if (q >= o) in4 += y;
+            }
+            const uint32_t T0 = __shfl_sync(0xffffffffu, in4, 15);
+            const uint32_t T1 = __shfl_sync(0xffffffffu, in4, 31);
+#pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                const uint32_t hmask = hh ? 0xFFFF0000u : 0x0000FFFFu;
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const int s = j ^ (i >> 2);
-                    const uint32_t f8 = (F >> (8 * s)) & 0xFFu;
-                    if (!(__ballot_sync(0xffffffffu, f8 != 0u) & hmask)) continue;
-                    uint32_t bal[8], tot = 0;
-#pragma unroll
-                    for (int k2 = 0; k2 < 8; ++k2) {
-                        bal[k2] = __ballot_sync(0xffffffffu, (f8 >> k2) & 1u) & hmask;
-                        tot += __popc(bal[k2]);
-                    }
+                    const uint32_t tot = ((hh ? T1 : T0) >> (8 * j)) & 0xFFu;
+                    if (!tot) continue;
                     const uint32_t incl = inc[w] + tot;
                     const bool kept = incl <= room[w];
-                    if (kept && hw == hh) {
+                    const uint32_t f8 = (F[w] >> (8 * j)) & 0xFFu;
+                    if (kept && hw == hh && f8) {
+                        uint32_t r = start[w] + inc[w] + ((in4 >> (8 * j)) & 0xFFu) - __popc(f8);
                         const uint32_t tloc = (uint32_t)((4 * (u0 + hh) + j) % kChunk);
-                        const unsigned char* row = (w ? qv : qk) + j * 256;
-                        uint32_t before = 0;
+                        const unsigned char* row = sq + (w ? kKVStride : 0) + j * 256 + q * 16;
 #pragma unroll
-                        for (int k2 = 0; k2 < 8; ++k2) {
-                            if ((f8 >> k2) & 1u) {
-                                const uint32_t r = before + __popc(bal[k2] & ((1u << lane) - 1u));
-                                const uint32_t x16 = lds16(row + 2 * (i + 16 * k2));
-                                outl[w][start[w] + inc[w] + r] =
-                                    (x16 << 16) | (tloc << 7) | (uint32_t)(i + 16 * k2);
+                        for (int m = 0; m < 8; ++m) {
+                            if ((f8 >> m) & 1u) {
+                                const uint32_t x16 = *reinterpret_cast<const uint16_t*>(row + 2 * m);
+                                outl[w][r++] = (x16 << 16) | (tloc << 7) | (uint32_t)(8 * q + m);
                             }
-                            before += __popc(bal[k2]);
                         }
                     }
                     if (kept) acc[w] = incl;
@@ -816,23 +878,59 @@ __global__ void __launch_bounds__(kWrWarps * 32) k_tok_write(kvq_cfg cfg, kvq_ca
                 }
             }
         }
-        // the quad's blocks: fresh when the quad starts at or after this call's first token,
-        // else only the fields of this call's tokens replace the stored ones
+        __syncwarp();  // code bytes complete
+        // ---- the quad's blocks: lane group i = q
         if (u <= ub) {
-            const size_t o = (blk0 + u) * (16 * BITS) + BITS * i;
-            const bool fresh = 4 * u >= t0;
+            uint32_t kw[BITS], vw[BITS];
 #pragma unroll
-            for (int q = 0; q < BITS; ++q) {
-                if (fresh) {
-                    c.kcodes[o + q] = kw[q];
-                    c.vcodes[o + q] = vw[q];
-                } else {
-                    c.kcodes[o + q] = (c.kcodes[o + q] & ~fm[q]) | kw[q];
-                    c.vcodes[o + q] = (c.vcodes[o + q] & ~fm[q]) | vw[q];
+            for (int d = 0; d < BITS; ++d) kw[d] = vw[d] = 0u;
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                const unsigned char* rk = cq + (s ^ (q >> 2)) * 128 + q;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const int off = (4 * kk + s) * W2, wd = off >> 5, bt = off & 31;
+                    const uint32_t fk = (uint32_t)rk[16 * kk] | ((uint32_t)rk[16 * kk + 64] << BITS);
+                    const uint32_t fv = (uint32_t)rk[2 * kCQ + 16 * kk] |
+                                        ((uint32_t)rk[2 * kCQ + 16 * kk + 64] << BITS);
+                    kw[wd] |= fk << bt;
+                    vw[wd] |= fv << bt;
+                    if (bt + W2 > 32) {
+                        kw[wd + 1] |= fk >> (32 - bt);
+                        vw[wd + 1] |= fv >> (32 - bt);
+                    }
+                }
+            }
+            const size_t o = (blk0 + u) * (16 * BITS) + BITS * q;
+            if (4 * u >= t0) {
+#pragma unroll
+                for (int d = 0; d < BITS; ++d) {
+                    c.kcodes[o + d] = kw[d];
+                    c.vcodes[o + d] = vw[d];
+                }
+            } else {
+                // the quad holds earlier tokens: replace only the fields of this call's tokens
+                uint32_t fm[BITS];
+#pragma unroll
+                for (int d = 0; d < BITS; ++d) fm[d] = 0u;
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const uint32_t m = ((pres >> (s ^ (q >> 2))) & 1u) ? ((1u << W2) - 1u) : 0u;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const int off = (4 * kk + s) * W2, wd = off >> 5, bt = off & 31;
+                        fm[wd] |= m << bt;
+                        if (bt + W2 > 32) fm[wd + 1] |= m >> (32 - bt);
+                    }
+                }
+#pragma unroll
+                for (int d = 0; d < BITS; ++d) {
+                    c.kcodes[o + d] = (c.kcodes[o + d] & ~fm[d]) | kw[d];
+                    c.vcodes[o + d] = (c.vcodes[o + d] & ~fm[d]) | vw[d];
                 }
             }
         }
-        __syncwarp();
+        __syncwarp();  // the ring slot and the code rows are free again
     }
     cp_wait<0>();
     if (lane == 0) {
@@ -1082,7 +1180,9 @@ void launch_tokens(const kvq_cfg& C, const kvq_cache& K, const kvq_codebook& cbK
                    bool kcuts, const QuantWs& ws, cudaStream_t st) {
     const int nchc = call_chunks(n_new);
     dim3 gt(nchc, C.B);
-    k_tok_stats<<<gt, kStWarps * 32, 0, st>>>(C, K, cbV, k, v, n_new, nchc, ws);
+    const int smst = (kStWarps * 512 + C.Hkv * kD / 8 * 8) * 4;
+    cudaFuncSetAttribute(k_tok_stats, cudaFuncAttributeMaxDynamicSharedMemorySize, smst);
+    k_tok_stats<<<gt, kStWarps * 32, smst, st>>>(C, K, cbV, k, v, n_new, nchc, ws);
     k_tok_scan<<<C.B * C.Hkv, kScThreads, 0, st>>>(C, K, nchc, ws);
     switch (C.bits) {
         case 2: launch_write<2>(C, K, cbK, k, v, n_new, nchc, kcuts, ws, st); break;
@@ -1136,20 +1236,24 @@ extern "C" int kvq_quantize_append(const kvq_cfg* cfg, const kvq_cache* cache,
         cudaError_t ce;
         if ((ce = cudaMemsetAsync(ws.hist1, 0, (size_t)C.B * n * 256 * 4, st))) return record_cuda(ce);
         if ((ce = cudaMemsetAsync(ws.hist2, 0, (size_t)C.B * n * 512 * 4, st))) return record_cuda(ce);
-        const int sm2 = kCalCols * 2 * kCalStride * 4;
-        if ((ce = cudaFuncSetAttribute(k_calib_hist, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       sm2)))
+        if ((ce = cudaFuncSetAttribute(k_calib_hist<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kCalSmem)))
+            return record_cuda(ce);
+        if ((ce = cudaFuncSetAttribute(k_calib_hist<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kCalSmem)))
             return record_cuda(ce);
         const int groups = (n + kCalCols - 1) / kCalCols;
         int splits = (6 * 148 + groups * C.B - 1) / (groups * C.B);
-        splits = splits < 1 ? 1 : splits;
         const int maxsp = (n_new + 1023) / 1024;
-        splits = splits > maxsp ? (maxsp < 1 ? 1 : maxsp) : splits;
+        splits = splits > maxsp ? maxsp : splits;
+        const int minsp = (n_new + kCalRows - 1) / kCalRows;
+        splits = splits < minsp ? minsp : splits;
+        splits = splits < 1 ? 1 : splits;
         dim3 gh(groups, splits, C.B);
         dim3 gs((n + 127) / 128, C.B);
-        k_calib_hist<<<gh, kCalThreads, kCalCols * kCalStride * 4, st>>>(C, k, n_new, ws, 1);
+        k_calib_hist<1><<<gh, kCalThreads, kCalSmem, st>>>(C, k, n_new, ws);
         k_calib_select<<<gs, 128, 0, st>>>(C, K, ws, 1);
-        k_calib_hist<<<gh, kCalThreads, sm2, st>>>(C, k, n_new, ws, 2);
+        k_calib_hist<2><<<gh, kCalThreads, kCalSmem, st>>>(C, k, n_new, ws);
         k_calib_select<<<gs, 128, 0, st>>>(C, K, ws, 2);
         const size_t nrec = (size_t)C.B * (n / 2) * 16;
         k_key_cuts<<<(unsigned)((nrec + 255) / 256), 256, 0, st>>>(C, K, *cbK, ws);

@@ -65,15 +65,17 @@ def test_closed_form_per_token(name, over, expect):
     # the decode traffic per token equals the stored bytes plus the chunk pointers (one uint32
     # per 64 tokens per kv head, K and V) for the fused path, and adds the logits (4 B per
     # query head, written then read) for the split kernels (three calls or one)
+    # (outlier counts are totals over the batch's w.B sequences)
     T = 1 << 16
+    BT = w.B * T
     k_out, v_out = bench.expected_outliers_per_token(w)
-    fused = bench.bytes_model(w, T, k_out * T, v_out * T, "fused", outlier_bytes=6)["total"]
-    ptr = 2 * 4 * w.Hkv * ((T + 63) // 64 + 1)
-    assert (fused - ptr) / T == pytest.approx(got, rel=1e-12)
-    split = bench.bytes_model(w, T, k_out * T, v_out * T, "split", outlier_bytes=6)
-    assert split["total"] - fused == 2 * 4 * w.Hq * T
+    fused = bench.bytes_model(w, T, k_out * BT, v_out * BT, "fused", outlier_bytes=6)["total"]
+    ptr = 2 * 4 * w.Hkv * ((T + 63) // 64 + 1) * w.B
+    assert (fused - ptr) / BT == pytest.approx(got, rel=1e-12)
+    split = bench.bytes_model(w, T, k_out * BT, v_out * BT, "split", outlier_bytes=6)
+    assert split["total"] - fused == 2 * 4 * w.Hq * BT
     assert split["qk"] + split["pv"] == split["total"]
-    one = bench.bytes_model(w, T, k_out * T, v_out * T, "one-call", outlier_bytes=6)["total"]
+    one = bench.bytes_model(w, T, k_out * BT, v_out * BT, "one-call", outlier_bytes=6)["total"]
     assert one == split["total"]
 
 
