@@ -617,6 +617,241 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 }
 
 // ---------------------------------------------------------------------------------
+// QK for kv heads that serve G query heads (grouped-query attention), codes of 2 or 3 bits:
+// one CTA per (split, sequence, kv head).  The table holds, for each pair p and code pair, the
+// dequantized key pair (off + half L[code], for channels p and p + 64) turned by j theta_p for
+// the four token offsets j of a quad -- no query folded in -- so a kv head's codes are looked
+// up once for all G query heads.  Per (token, pair): one lookup, the turn by the quad's phase
+// (four scalar multiply-adds) and one packed multiply-add per query head.  Stages, ring,
+// streaming warp and lane mapping are those of k_qk_quad.  The reduction over the 16 lane
+// groups first folds the lane bits that pick a lane's token slots (slot s of lane group i
+// holds token s ^ (i >> 2), so the partner's slot s ^ 2 or s ^ 1 holds the same token and no
+// selection is needed), then the bits over the heads; lane i ends with token i >> 2 and head
+// i & 3 (G = 4) or head (i >> 1) & 1 (G = 2).
+template <int BITS, int G>
+__global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
+    k_qk_grp(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ qr_all,
+             const float2* __restrict__ thi, const float2* __restrict__ tlo, int Ls,
+             int max_len, float* __restrict__ logits) {
+    static_assert(G == 2 || G == 4, "two or four query heads per kv head");
+    using F = Fmt<BITS>;
+    constexpr int NC = kQWarps * 32;
+    constexpr int P = 9;                         // entry bit of a table byte offset
+    constexpr int JS = P + F::FW;                // j bit of a table byte offset
+    constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << P;
+    extern __shared__ __align__(128) uint8_t sm[];
+    const QQPlan L = qq_plan(BITS);
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t tpos = (sbase + L.pre + L.jslice - 1) & ~(uint32_t)(L.jslice - 1);
+    uint8_t* tab = sm + (tpos - sbase);
+    uint8_t* ring = sm + L.ring;
+    float4* base = (float4*)(sm + L.base);
+    float* lev = (float*)(sm + L.lev);
+    uint64_t* full = (uint64_t*)(sm + L.bar);
+    uint64_t* empty = full + kStages;
+    int* flag = (int*)(sm + L.flag);
+
+    const int tid = threadIdx.x;
+    const int i = tid & 15, x = i >> 2, lane = tid & 31, warp = tid >> 5;
+    const int s = blockIdx.x, b = blockIdx.y, kvh = blockIdx.z;
+    const int Hq = cfg.Hq, Hkv = cfg.Hkv, hq0 = kvh * G;
+    int len = c.len[b];
+    if (len > max_len) {
+        if (tid == 0 && s == 0 && kvh == 0) set_status(c.status, KVQ_STATUS_LEN_OVERFLOW);
+        len = max_len;
+    }
+    const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
+    if (t_begin >= t_end) return;
+    const int nst = (t_end - t_begin + kQTokens - 1) / kQTokens;
+    if (tid == 0) {
+        for (int k = 0; k < kStages; ++k) {
+            mbar_init(full + k, 1);
+            mbar_init(empty + k, kQWarps);
+        }
+        flag[0] = 0;
+        flag[1] = 0;
+        fence_mbar_init();
+    }
+    // ---- tables: the dequantized key pair of each entry turned by j theta_p.  Thread (p, r)
+    // of the first 512 writes entries r, r + 8, ... of pair p for every j.
+    if (tid < (1 << BITS)) lev[tid] = cb.levels[tid];
+    __syncthreads();
+    if (tid < 512) {
+        const int p = tid & 63, r0 = tid >> 6;
+        const float* kp = c.kparams + ((size_t)b * Hkv + kvh) * kD * 2;
+        const float offa = kp[2 * p], halfa = kp[2 * p + 1];
+        const float offb = kp[2 * (p + 64)], halfb = kp[2 * (p + 64) + 1];
+        float2 rj[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) rj[j] = tlo[j * 64 + p];
+        unsigned long long* t64 = reinterpret_cast<unsigned long long*>(tab);
+        for (int idx = r0; idx < F::NT; idx += 8) {
+            const float ka = fmaf(halfa, lev[idx & ((1 << BITS) - 1)], offa);
+            const float kb = fmaf(halfb, lev[idx >> BITS], offb);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                t64[(j * F::NT + idx) * 64 + p] =
+                    pk(fmaf(rj[j].x, ka, -rj[j].y * kb), fmaf(rj[j].y, ka, rj[j].x * kb));
+        }
+    }
+    __syncthreads();  // tables complete, barriers initialised
+
+    if (tid >= NC) {
+        // ================= streaming warp (as in k_qk_quad)
+        const int pl = tid - NC;
+        const uint32_t* src = c.kcodes + ((size_t)b * Hkv + kvh) * nquads(cfg.T_max) * F::BW;
+        int cc = 0;
+        for (; cc < nst; ++cc) {
+            const int slot = cc % kStages;
+            if (cc >= kStages && !mbar_wait(empty + slot, (uint32_t)(cc / kStages - 1) & 1u)) {
+                if (pl == 0) {
+                    atomicOr(flag, 1);
+                    set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+                }
+                break;
+            }
+            if (*flag) break;
+            const int tc = t_begin + cc * kQTokens;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const float2 cs = trig_at(thi, tlo, tc, pl + 32 * u);
+                base[slot * 64 + pl + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
+            }
+            __syncwarp();
+            __threadfence_block();
+            if (pl == 0) {
+                fence_proxy_async();
+                const int q0 = tc >> 2, q1 = (min(tc + kQTokens, t_end) + 3) >> 2;
+                const uint32_t bytes = (uint32_t)(q1 - q0) * F::BW * 4;
+                mbar_arrive_expect_tx(full + slot, bytes);
+                bulk_load(ring + (size_t)slot * L.stage, src + (size_t)q0 * F::BW, bytes,
+                          full + slot);
+            }
+            __syncwarp();
+        }
+        if (pl == 0) flag[1] = cc;
+    } else {
+        // ================= consumer warps: half-warp hh takes quads 4 warp + hh and + 2
+        const int qbase = 4 * warp + ((tid >> 4) & 1);
+        uint32_t lb[4], woff[2];
+#pragma unroll
+        for (int sl = 0; sl < 4; ++sl)
+            lb[sl] = tpos + ((uint32_t)(sl ^ x) << JS) + ((uint32_t)i << 3);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) woff[u] = (uint32_t)((qbase + 2 * u) * F::BW + i * BITS) * 4;
+        unsigned long long Q[G][4];  // (q_p, q_{p+64}) of each query head, p = i + 16 k
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float* qv = qr_all + ((size_t)b * Hq + hq0 + h) * kD;
+                Q[h][k] = pk(qv[i + 16 * k], qv[i + 16 * k + 64]);
+            }
+        const int hown = G == 4 ? (i & 3) : ((i >> 1) & 1);
+        const bool owner = G == 4 ? true : !(i & 1);
+        float* lrow = logits + ((size_t)b * Hq + hq0 + hown) * cfg.T_max;
+        for (int st = 0; st < nst; ++st) {
+            const int slot = st % kStages;
+            if (!mbar_wait(full + slot, (uint32_t)(st / kStages) & 1u)) {
+                atomicOr(flag, 1);
+                set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+            }
+            if (*flag) break;
+            const uint8_t* stage = ring + (size_t)slot * L.stage;
+            uint32_t w[2][BITS];
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int d = 0; d < BITS; ++d)
+                    w[u][d] = *reinterpret_cast<const uint32_t*>(stage + woff[u] + 4 * d);
+            float bc[4], bs[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float4 bq = base[slot * 64 + i + 16 * k];
+                bc[k] = bq.x;
+                bs[k] = bq.z;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
+#pragma unroll 1
+            for (int u = 0; u < 2; ++u) {
+                unsigned long long acc[4][G];
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl)
+#pragma unroll
+                    for (int h = 0; h < G; ++h) acc[sl][h] = 0ull;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    // the quad's phase for pair i + 16 k: the stage start's turned by 4 q theta_p
+                    // (read again each stage: an L1 hit, and no registers held across stages)
+                    const float2 r = __ldg(tlo + (4 * (qbase + 2 * u)) * 64 + i + 16 * k);
+                    const float pc = fmaf(bc[k], r.x, -bs[k] * r.y);
+                    const float ps = fmaf(bc[k], r.y, bs[k] * r.x);
+#pragma unroll
+                    for (int sl = 0; sl < 4; ++sl) {
+                        uint32_t fs;
+                        switch (4 * k + sl) {
+#define KVQ_FS(N) case N: fs = field_to<BITS, N, P>(w[u]); break;
+                            KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5)
+                            KVQ_FS(6) KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11)
+                            KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
+#undef KVQ_FS
+                        }
+                        const uint32_t a = (fs & MASK) | lb[sl];
+                        const unsigned long long T = k == 0 ? lds64<0>(a)
+                                                   : k == 1 ? lds64<128>(a)
+                                                   : k == 2 ? lds64<256>(a) : lds64<384>(a);
+                        const f2 t = upk(T);
+                        const unsigned long long K2 =
+                            pk(fmaf(pc, t.x, -ps * t.y), fmaf(ps, t.x, pc * t.y));
+#pragma unroll
+                        for (int h = 0; h < G; ++h) acc[sl][h] = fma2(Q[h][k], K2, acc[sl][h]);
+                    }
+                }
+                // token slots: fold lane bit 3 (slots 2, 3 go to the partner), then bit 2
+                float v[2][G];
+#pragma unroll
+                for (int sl = 0; sl < 2; ++sl)
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const f2 a0 = upk(acc[sl][h]), a1 = upk(acc[sl + 2][h]);
+                        v[sl][h] = (a0.x + a0.y) + __shfl_xor_sync(0xffffffffu, a1.x + a1.y, 8);
+                    }
+                float hv[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) hv[h] = v[0][h] + __shfl_xor_sync(0xffffffffu, v[1][h], 4);
+                // heads: lane bit 1, then bit 0
+                float r;
+                if constexpr (G == 4) {
+                    const bool b1 = (i >> 1) & 1, b0 = i & 1;
+                    float h2[2];
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const float keep = b1 ? hv[t + 2] : hv[t];
+                        const float send = b1 ? hv[t] : hv[t + 2];
+                        h2[t] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                    }
+                    const float keep = b0 ? h2[1] : h2[0];
+                    const float send = b0 ? h2[0] : h2[1];
+                    r = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+                } else {
+                    const bool b1 = (i >> 1) & 1;
+                    const float keep = b1 ? hv[1] : hv[0];
+                    const float send = b1 ? hv[0] : hv[1];
+                    r = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+                    r += __shfl_xor_sync(0xffffffffu, r, 1);
+                }
+                const int t = t_begin + st * kQTokens + 4 * (qbase + 2 * u) + x;
+                if (owner && t < t_end) lrow[t] = r;
+            }
+        }
+    }
+    __syncthreads();
+    // after an abandoned wait, copies of the last stages issued may still be in flight
+    if (*flag && tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1], kStages);
+}
+
+// ---------------------------------------------------------------------------------
 // Outlier kernels.  A block takes up to kOutChunks 64-token chunks of one (sequence, kv head)
 // list and stages their chunk pointers in shared memory; a warp walks a contiguous range of
 // the block's entries, 32 kOutBatch at a time.  An entry holds only its token's offset within
@@ -1083,12 +1318,12 @@ constexpr int kPTokens = 4 * kPQuads;        // tokens per stage
 struct PQPlan {
     int ring, stage, wsm, bar, flag, pre, tsize, total;
 };
-__host__ __device__ inline PQPlan pq_plan(int bits) {
+__host__ __device__ inline PQPlan pq_plan(int bits, int g = 1) {
     PQPlan p;
     int o = 0;
     p.stage = kPQuads * 16 * bits * 4;
     p.ring = o;  o += kStages * p.stage;                     // reused by the final reduction
-    p.wsm = o;   o += kQWarps * 32 * 8;                      // [warp][token] (w, w)
+    p.wsm = o;   o += kQWarps * g * 32 * 8;                  // [warp][head][token] (w, w)
     p.bar = o;   o += 2 * kStages * 8;
     p.flag = o;  o += 16;
     p.pre = o;
@@ -1278,6 +1513,220 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
         float o = 0.0f;
         for (int w2 = 0; w2 < kQWarps; ++w2) o += pored[w2];
         po_out[e] = a + o;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// PV for kv heads that serve G query heads (grouped-query attention), codes of 2 or 3 bits:
+// one CTA per (split, sequence, kv head).  Stages, ring, streaming warp, lane mapping and the
+// 16-bit (La, Lb) table are those of k_pv_quad; each (La, Lb) lookup serves all G heads, one
+// packed multiply-add per head with that head's weight p half of the token.  The per-warp
+// weights sit in shared memory as [head][token] (w, w); the split's outputs are reduced head
+// by head through the idle ring at the end.
+template <int BITS, int G>
+__global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
+    k_pv_grp(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
+             const float2* __restrict__ ml, int Ls, int S, int max_len,
+             float* __restrict__ part) {
+    static_assert(G == 2 || G == 4, "two or four query heads per kv head");
+    using F = Fmt<BITS>;
+    constexpr int NC = kQWarps * 32;
+    constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << 7;
+    extern __shared__ __align__(128) uint8_t sm[];
+    const PQPlan L = pq_plan(BITS, G);
+    const uint32_t sbase = smem_u32(sm);
+    const uint32_t tpos = (sbase + L.pre + L.tsize - 1) & ~(uint32_t)(L.tsize - 1);
+    uint8_t* tab = sm + (tpos - sbase);
+    uint8_t* ring = sm + L.ring;
+    unsigned long long* wsm = (unsigned long long*)(sm + L.wsm);
+    uint64_t* full = (uint64_t*)(sm + L.bar);
+    uint64_t* empty = full + kStages;
+    int* flag = (int*)(sm + L.flag);
+
+    const int tid = threadIdx.x, nthr = blockDim.x;
+    const int i = tid & 15, x = i >> 2, lane = tid & 31, warp = tid >> 5, hh = (tid >> 4) & 1;
+    const int s = blockIdx.x, b = blockIdx.y, kvh = blockIdx.z;
+    const int Hq = cfg.Hq, Hkv = cfg.Hkv, hq0 = kvh * G;
+    const int len = min(c.len[b], max_len);
+    const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
+    if (t_begin >= t_end) {
+        for (int e = tid; e < G * kD; e += nthr)
+            part[(((size_t)b * Hq + hq0 + e / kD) * S + s) * kD + e % kD] = 0.0f;
+        return;
+    }
+    const int nst = (t_end - t_begin + kPTokens - 1) / kPTokens;
+    if (tid == 0) {
+        for (int k = 0; k < kStages; ++k) {
+            mbar_init(full + k, 1);
+            mbar_init(empty + k, kQWarps);
+        }
+        flag[0] = 0;
+        flag[1] = 0;
+        fence_mbar_init();
+    }
+    const int nb = (1 << BITS) - 1;
+    for (int e = tid; e < F::NT * 32; e += nthr) {
+        const int idx = e >> 5;
+        const uint32_t ua = __float_as_uint(cb.levels[idx & nb]);
+        const uint32_t ub = __float_as_uint(cb.levels[idx >> BITS]);
+        reinterpret_cast<uint32_t*>(tab)[e] = (ua & 0xFFFFu) | (ub << 16);
+    }
+    if (tid <= nb) {
+        const uint32_t u = __float_as_uint(cb.levels[tid]);
+        if ((u >> 16) != (u & 0xFFFFu)) set_status(c.status, KVQ_STATUS_CODEBOOK);
+    }
+    __syncthreads();  // tables complete, barriers initialised
+
+    unsigned long long O[G][4];
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) O[h][k] = 0ull;
+    float po[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) po[h] = 0.0f;
+    if (tid >= NC) {
+        // ================= streaming warp
+        const int pl = tid - NC;
+        const uint32_t* src = c.vcodes + ((size_t)b * Hkv + kvh) * nquads(cfg.T_max) * F::BW;
+        int cc = 0;
+        for (; cc < nst; ++cc) {
+            const int slot = cc % kStages;
+            if (cc >= kStages && !mbar_wait(empty + slot, (uint32_t)(cc / kStages - 1) & 1u)) {
+                if (pl == 0) {
+                    atomicOr(flag, 1);
+                    set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+                }
+                break;
+            }
+            if (*flag) break;
+            if (pl == 0) {
+                fence_proxy_async();
+                const int tc = t_begin + cc * kPTokens;
+                const int q0 = tc >> 2, q1 = (min(tc + kPTokens, t_end) + 3) >> 2;
+                const uint32_t bytes = (uint32_t)(q1 - q0) * F::BW * 4;
+                mbar_arrive_expect_tx(full + slot, bytes);
+                bulk_load(ring + (size_t)slot * L.stage, src + (size_t)q0 * F::BW, bytes,
+                          full + slot);
+            }
+            __syncwarp();
+        }
+        if (pl == 0) flag[1] = cc;  // stages issued
+    } else {
+        // ================= consumer warps
+        float mM[G], invL[G], lg[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            const float2 mL = ml[(size_t)b * Hq + hq0 + h];
+            mM[h] = mL.x;
+            invL[h] = mL.y > 0.0f ? 1.0f / mL.y : 0.0f;
+        }
+        const float* lrow0 = logits + ((size_t)b * Hq + hq0) * cfg.T_max;
+        const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
+        float2 vp = make_float2(0.0f, 0.0f);
+        auto fetch = [&](int st) {
+            const int t = t_begin + st * kPTokens + 32 * warp + lane;
+            const bool ok = t < t_end;
+#pragma unroll
+            for (int h = 0; h < G; ++h) lg[h] = ok ? lrow0[(size_t)h * cfg.T_max + t] : -INFINITY;
+            vp = ok ? vpar[t] : make_float2(0.0f, 0.0f);
+        };
+        fetch(0);
+        uint32_t woff[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            woff[u] = (uint32_t)((8 * warp + 2 * u + hh) * F::BW + i * BITS) * 4;
+        const uint32_t lanebits = tpos | ((uint32_t)lane << 2);
+        unsigned long long* wsw = wsm + 32 * G * warp;  // [head][32 tokens]
+        for (int st = 0; st < nst; ++st) {
+            const int slot = st % kStages;
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float p = (lg[h] > -INFINITY) ? __expf(lg[h] - mM[h]) * invL[h] : 0.0f;
+                const float wv = p * vp.y;
+                po[h] = fmaf(p, vp.x, po[h]);
+                wsw[32 * h + lane] = pk(wv, wv);
+            }
+            __syncwarp();
+            if (st + 1 < nst) fetch(st + 1);
+            if (!mbar_wait(full + slot, (uint32_t)(st / kStages) & 1u)) {
+                atomicOr(flag, 1);
+                set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
+            }
+            if (*flag) break;
+            const uint8_t* stage = ring + (size_t)slot * L.stage;
+            uint32_t w[4][BITS];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int d = 0; d < BITS; ++d)
+                    w[u][d] = *reinterpret_cast<const uint32_t*>(stage + woff[u] + 4 * d);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int sl = 0; sl < 4; ++sl) {
+                    // token 4 (2 u + hh) + (sl ^ x) of the warp's 32
+                    unsigned long long ww[G];
+#pragma unroll
+                    for (int h = 0; h < G; ++h) ww[h] = wsw[32 * h + 8 * u + 4 * hh + (sl ^ x)];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint32_t fs = 0;
+                        switch (4 * k + sl) {
+#define KVQ_FS(N) case N: fs = field_to<BITS, N, 7>(w[u]); break;
+                            KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5)
+                            KVQ_FS(6) KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11)
+                            KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
+#undef KVQ_FS
+                        }
+                        const uint32_t lv = lds32((fs & MASK) | lanebits);
+                        const unsigned long long LL =
+                            pk(__uint_as_float(__byte_perm(lv, 0u, 0x1010)),
+                               __uint_as_float(__byte_perm(lv, 0u, 0x3232)));
+#pragma unroll
+                        for (int h = 0; h < G; ++h) O[h][k] = fma2(ww[h], LL, O[h][k]);
+                    }
+                }
+            }
+            __syncwarp();  // wsw is rewritten for the next stage
+        }
+    }
+    __syncthreads();
+    if (*flag) {
+        if (tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1], kStages);
+        return;
+    }
+    // per head: the two half-warps of a warp hold the same pairs; fold them, then sum the 16
+    // warps' rows through the idle ring
+    float* red = (float*)ring;
+    float* pored = red + kQWarps * kD;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+        if (tid < NC) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                f2 o = upk(O[h][k]);
+                o.x += __shfl_xor_sync(0xffffffffu, o.x, 16);
+                o.y += __shfl_xor_sync(0xffffffffu, o.y, 16);
+                if (!hh) {
+                    red[warp * kD + i + 16 * k] = o.x;
+                    red[warp * kD + i + 16 * k + 64] = o.y;
+                }
+            }
+            const float pw = warp_sum(po[h]);  // sum_t p_t off_t over the warp's tokens
+            if (lane == 0) pored[warp] = pw;
+        }
+        __syncthreads();
+        for (int e = tid; e < kD; e += nthr) {
+            float a = 0.0f;
+            for (int r = 0; r < kQWarps; ++r) a += red[r * kD + e];
+            float o = 0.0f;
+            for (int w2 = 0; w2 < kQWarps; ++w2) o += pored[w2];
+            part[(((size_t)b * Hq + hq0 + h) * S + s) * kD + e] = a + o;
+        }
+        __syncthreads();
     }
 }
 
@@ -1663,15 +2112,31 @@ static int kvb_of(const kvq_cfg* cfg, int hpc) {
     return m;
 }
 
+// Splits of the decode grid.  The CTAs of a split are one per (sequence, kv head) for the
+// table kernels of 2- and 3-bit codes with 1, 2 or 4 query heads per kv head, else one per
+// (sequence, group of hpc query heads); each CTA holds an SM.  The count minimises
+// waves x (setup + stages): waves of 148 CTAs, stages of 256 tokens per CTA, and a setup
+// (tables, barriers) worth about two stages -- so short caches get few long splits instead of
+// many CTAs that mostly build tables.
 static int auto_splits(const kvq_cfg* cfg, int max_len) {
-    // two waves of one CTA per SM over (splits x sequences x head groups), >= 256 tokens each
-    const int groups = cfg->B * (cfg->Hq / hpc_of(cfg));
-    int S = (2 * 148 + groups - 1) / groups;
-    const int maxs = (max_len + 255) / 256;
-    if (S > maxs) S = maxs;
-    if (S < 1) S = 1;
-    if (S > 4096) S = 4096;
-    return S;
+    const int g = cfg->Hq / cfg->Hkv;
+    const bool tab = cfg->bits <= 3 && (g == 1 || g == 2 || g == 4);
+    const long long groups = tab ? (long long)cfg->B * cfg->Hkv : (long long)cfg->B * (cfg->Hq / hpc_of(cfg));
+    int maxs = (max_len + 255) / 256;
+    if (maxs > 4096) maxs = 4096;
+    if (maxs < 1) maxs = 1;
+    long long best = -1;
+    int bestS = 1;
+    for (int S = 1; S <= maxs; ++S) {
+        const long long waves = (S * groups + 147) / 148;
+        const long long stages = (((long long)max_len + S - 1) / S + 255) / 256;
+        const long long cost = waves * (2 + stages);
+        if (best < 0 || cost < best) {
+            best = cost;
+            bestS = S;
+        }
+    }
+    return bestS;
 }
 
 static int resolve_splits(const kvq_cfg* cfg, int max_len, int splits, int* S, int* Ls) {
@@ -1756,12 +2221,15 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
         k_decode_prep<<<(n + 255) / 256, 256, 0, st>>>(*cfg, *cache, *cbK, q, qpos, T.nhi,
                                                         pos_off, T.qr, T.thi, T.tlo, T.zk);
     }
-    if (cfg->bits <= 3 && cfg->Hq == cfg->Hkv) {
-        QKQKernel kq = cfg->bits == 2 ? k_qk_quad<2> : k_qk_quad<3>;
+    const int g = cfg->Hq / cfg->Hkv;
+    if (cfg->bits <= 3 && (g == 1 || g == 2 || g == 4)) {
+        QKQKernel kq = g == 1 ? (cfg->bits == 2 ? k_qk_quad<2> : k_qk_quad<3>)
+                     : g == 2 ? (cfg->bits == 2 ? k_qk_grp<2, 2> : k_qk_grp<3, 2>)
+                              : (cfg->bits == 2 ? k_qk_grp<2, 4> : k_qk_grp<3, 4>);
         const int smem = qq_plan(cfg->bits).total;
         cudaError_t ce = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (ce) return record_cuda(ce);
-        dim3 grid(S, cfg->B, cfg->Hq);
+        dim3 grid(S, cfg->B, cfg->Hkv);
         kq<<<grid, kQWarps * 32 + 32, smem, st>>>(*cfg, *cache, *cbK, T.qr, T.thi, T.tlo, Ls,
                                                     max_len, logits);
     } else {
@@ -1834,6 +2302,16 @@ static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
         if (ce) return record_cuda(ce);
         dim3 grid(S, cfg->B, cfg->Hq);
         kq<<<grid, kQWarps * 32 + 32, smem, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls,
+                                                    S, max_len, part);
+    } else if (cfg->Hq == 2 * cfg->Hkv || cfg->Hq == 4 * cfg->Hkv) {
+        const int g = cfg->Hq / cfg->Hkv;
+        PVQKernel kg = g == 2 ? (cfg->bits == 2 ? k_pv_grp<2, 2> : cfg->bits == 3 ? k_pv_grp<3, 2> : k_pv_grp<4, 2>)
+                              : (cfg->bits == 2 ? k_pv_grp<2, 4> : cfg->bits == 3 ? k_pv_grp<3, 4> : k_pv_grp<4, 4>);
+        const int smem = pq_plan(cfg->bits, g).total;
+        cudaError_t ce = cudaFuncSetAttribute(kg, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (ce) return record_cuda(ce);
+        dim3 grid(S, cfg->B, cfg->Hkv);
+        kg<<<grid, kQWarps * 32 + 32, smem, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls,
                                                     S, max_len, part);
     } else {
     const int hpc = hpc_of(cfg);

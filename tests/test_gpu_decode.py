@@ -29,6 +29,9 @@ CASES = [
     ("llama3_8b_gqa_128k", dict(B=2, Hq=8, Hkv=2, bits=4), 330, [330, 97], 1),
     # an empty sequence between two others (its output is defined as 0)
     ("batched_8x8k", dict(B=3, Hq=4, Hkv=4, bits=3), 260, [260, 0, 5], 0),
+    # grouped-query table kernels at 2 bits: four and two query heads per kv head
+    ("llama3_8b_gqa_128k", dict(B=1, Hq=8, Hkv=2, bits=2), 410, None, 1),
+    ("batched_8x8k", dict(B=2, Hq=4, Hkv=2, bits=2), 300, [300, 123], 0),
 ]
 
 
