@@ -1012,6 +1012,34 @@ __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
             const int tn = __shfl_down_sync(0xffffffffu, tu, 1);
             const bool tail = tu >= 0 && lane < 31 && tn != tu;
             const bool flush = ct >= 0 && t0 != ct;  // the carried token ended with the last slice
+            if constexpr (G > 1) {
+                // all heads in one segmented scan: the token ids move once per step
+                float v[G];
+#pragma unroll
+                for (int a = 0; a < G; ++a) {
+                    v[a] = d * fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
+                    if (ct >= 0 && lane == 0) {
+                        const float cv = carry[warp][a];
+                        if (flush) atomicAdd(&lb0[a * T_max + ct], cv);
+                        else v[a] += cv;
+                    }
+                }
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int tt = __shfl_up_sync(0xffffffffu, tu, off);
+                    const bool same = lane >= off && tt == tu;
+#pragma unroll
+                    for (int a = 0; a < G; ++a) {
+                        const float vv = __shfl_up_sync(0xffffffffu, v[a], off);
+                        if (same) v[a] += vv;
+                    }
+                }
+#pragma unroll
+                for (int a = 0; a < G; ++a) {
+                    if (tail) atomicAdd(&lb0[a * T_max + tu], v[a]);
+                    if (lane == 31) carry[warp][a] = v[a];
+                }
+            } else {
             for (int a = 0; a < g; ++a) {
                 float v = d * fmaf(sa, qs[a * kD + p], sb * qs[a * kD + p + 64]);
                 if (ct >= 0 && lane == 0) {
@@ -1022,6 +1050,7 @@ __global__ void __launch_bounds__(kOutThreads) k_key_outliers(
                 v = seg_scan(v, tu, lane);
                 if (tail) atomicAdd(&lb0[a * T_max + tu], v);
                 if (lane == 31) carry[warp][a] = v;
+            }
             }
             __syncwarp();
             ct = __shfl_sync(0xffffffffu, tu, 31);
@@ -1778,13 +1807,15 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
         while (wk.next(cps, ent, t, w)) {
             bool ok[kOutBatch];
             float2 vp[kOutBatch];
-            float l0[kOutBatch];
+            constexpr int GP = G ? G : 1;  // heads whose logits are gathered up front
+            float l0[kOutBatch][GP];
 #pragma unroll
             for (int u = 0; u < kOutBatch; ++u) {
                 ok[u] = (unsigned)t[u] < (unsigned)len;
                 const int tt = ok[u] ? t[u] : 0;
                 vp[u] = vpar[tt];
-                l0[u] = lrow[tt];
+#pragma unroll
+                for (int a = 0; a < GP; ++a) l0[u][a] = lrow[a * T_max + tt];
             }
 #pragma unroll
             for (int u = 0; u < kOutBatch; ++u) {
@@ -1797,7 +1828,7 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
                 const int ch = (int)(w[u] & 127u);
                 for (int a = 0; a < g; ++a) {
                     const float2 mi = mls[a];
-                    const float la = a == 0 ? l0[u] : lrow[a * T_max + (ok[u] ? t[u] : 0)];
+                    const float la = a < GP ? l0[u][a < GP ? a : 0] : lrow[a * T_max + (ok[u] ? t[u] : 0)];
                     if (ok[u] && mi.y > 0.0f) {
                         const float v = __expf(la - mi.x) * mi.y * d;
                         atomicAdd(&acc[a * kD + ch], (unsigned long long)__float2ll_rn(v * kFixScale));
@@ -2247,7 +2278,9 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     }
     const int nch = (max_len + kChunk - 1) / kChunk;
     dim3 go((nch + kOutChunks - 1) / kOutChunks, cfg->B * cfg->Hkv);
-    auto ko = cfg->Hq == cfg->Hkv ? k_key_outliers<1> : k_key_outliers<0>;
+    const int gq = cfg->Hq / cfg->Hkv;
+    auto ko = gq == 1 ? k_key_outliers<1> : gq == 2 ? k_key_outliers<2>
+            : gq == 4 ? k_key_outliers<4> : k_key_outliers<0>;
     ko<<<go, kOutThreads, 0, st>>>(*cfg, *cache, T.qr, T.thi, T.tlo, T.zk, max_len, logits);
     dim3 gs(S, cfg->B * cfg->Hq);
     k_logit_stats<<<gs, kStatThreads, 0, st>>>(*cfg, cache->len, logits, Ls, S, max_len, (float2*)stats);
@@ -2329,9 +2362,10 @@ static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     }
     dim3 go(S, cfg->B * cfg->Hkv);
     const bool mha = cfg->Hq == cfg->Hkv;
-    auto vo = cfg->bits == 2 ? (mha ? k_value_outliers<2, 1> : k_value_outliers<2, 0>)
-            : cfg->bits == 3 ? (mha ? k_value_outliers<3, 1> : k_value_outliers<3, 0>)
-                             : (mha ? k_value_outliers<4, 1> : k_value_outliers<4, 0>);
+    const int gq = cfg->Hq / cfg->Hkv;
+    auto vo = cfg->bits == 2 ? (mha ? k_value_outliers<2, 1> : gq == 2 ? k_value_outliers<2, 2> : gq == 4 ? k_value_outliers<2, 4> : k_value_outliers<2, 0>)
+            : cfg->bits == 3 ? (mha ? k_value_outliers<3, 1> : gq == 2 ? k_value_outliers<3, 2> : gq == 4 ? k_value_outliers<3, 4> : k_value_outliers<3, 0>)
+                             : (mha ? k_value_outliers<4, 1> : gq == 2 ? k_value_outliers<4, 2> : gq == 4 ? k_value_outliers<4, 4> : k_value_outliers<4, 0>);
     vo<<<go, kOutThreads, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls, S, max_len,
                                    part);
     k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);

@@ -636,8 +636,7 @@ __global__ void k_tok_final(kvq_cfg cfg, kvq_cache c, QuantWs ws) {
 // ---------------------------------------------------------------------------------
 // Encode and pack.  One warp per (64-token chunk, kv head) of a sequence, two token quads at a
 // time; the rows of the two quads (keys and values of one kv head, 256 bytes per token) reach
-// shared memory through a two-stage ring of 16-byte asynchronous copies, a warp's own (the
-// encode of a stage takes longer than the copies of the next).
+// shared memory through a three-stage ring of 16-byte asynchronous copies, a warp's own.
 //  - Encode: half-warp hw takes quad u0 + hw and lane q the channels 8q .. 8q + 7 of each of
 //    its four tokens (one 16-byte shared load per row), compares them two at a time against
 //    the thresholds and cuts, and stores the eight codes as bytes, row by row.
@@ -650,7 +649,7 @@ __global__ void k_tok_final(kvq_cfg cfg, kvq_cache c, QuantWs ws) {
 // Quad 1's rows and codes sit 32 and 16 bytes further on, so the two half-warps read disjoint
 // banks.
 constexpr int kWrWarps = 4;
-constexpr int kWrStages = 2;
+constexpr int kWrStages = 3;
 constexpr int kQStride = 4 * 256 + 32;
 constexpr int kKVStride = 2 * kQStride;
 constexpr int kStageBytes = 2 * kKVStride;
@@ -668,7 +667,7 @@ __device__ __forceinline__ void cp_wait() {
 }
 
 template <int BITS, bool KCUTS>
-__global__ void __launch_bounds__(kWrWarps * 32, BITS == 4 ? 4 : 5) k_tok_write(kvq_cfg cfg, kvq_cache c,
+__global__ void __launch_bounds__(kWrWarps * 32, 3) k_tok_write(kvq_cfg cfg, kvq_cache c,
                                                                kvq_codebook cbK,
                                                                const uint16_t* __restrict__ k,
                                                                const uint16_t* __restrict__ v,
@@ -783,7 +782,7 @@ __global__ void __launch_bounds__(kWrWarps * 32, BITS == 4 ? 4 : 5) k_tok_write(
         // ---- encode the four tokens of quad u
         uint32_t F[2] = {0u, 0u};  // flags of the lane's 8 channels, byte j per token
         uint32_t pres = 0;
-#pragma unroll 1
+#pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int t = 4 * u + j;
             const bool pr = u <= ub && t >= ta && t < tb;
