@@ -834,7 +834,10 @@ __global__ void __launch_bounds__(kWrWarps * 32, 3) k_tok_write(kvq_cfg cfg, kvq
             F[0] |= (fk & pm) << (8 * j);
             F[1] |= (fv & pm) << (8 * j);
         }
-        // ---- outlier entries, token by token (quad u0's four tokens, then quad u0 + 1's)
+        // ---- outlier entries.  The list order is token by token (quad u0's four tokens, then
+        // quad u0 + 1's) and channel by channel; a token's place in its list follows from the
+        // per-token totals, a lane's place within the token from the prefix sum of the lanes'
+        // counts.  Each lane then writes its own entries, set bit by set bit.
 #pragma unroll
         for (int w = 0; w < 2; ++w) {
             if (!__ballot_sync(0xffffffffu, F[w] != 0u)) continue;
@@ -851,30 +854,38 @@ __global__ void __launch_bounds__(kWrWarps * 32, 3) k_tok_write(kvq_cfg cfg, kvq
             }
             const uint32_t T0 = __shfl_sync(0xffffffffu, in4, 15);
             const uint32_t T1 = __shfl_sync(0xffffffffu, in4, 31);
+            // the eight tokens in list order: running counts and the capacity rule (warp-
+            // uniform); before = the list offset at the start of this half-warp's quad
+            uint32_t keep4 = 0, before = 0;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
+                if (hh == hw) before = inc[w];
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const uint32_t tot = ((hh ? T1 : T0) >> (8 * j)) & 0xFFu;
-                    if (!tot) continue;
                     const uint32_t incl = inc[w] + tot;
                     const bool kept = incl <= room[w];
-                    const uint32_t f8 = (F[w] >> (8 * j)) & 0xFFu;
-                    if (kept && hw == hh && f8) {
-                        uint32_t r = start[w] + inc[w] + ((in4 >> (8 * j)) & 0xFFu) - __popc(f8);
-                        const uint32_t tloc = (uint32_t)((4 * (u0 + hh) + j) % kChunk);
-                        const unsigned char* row = sq + (w ? kKVStride : 0) + j * 256 + q * 16;
-#pragma unroll
-                        for (int m = 0; m < 8; ++m) {
-                            if ((f8 >> m) & 1u) {
-                                const uint32_t x16 = *reinterpret_cast<const uint16_t*>(row + 2 * m);
-                                outl[w][r++] = (x16 << 16) | (tloc << 7) | (uint32_t)(8 * q + m);
-                            }
-                        }
-                    }
                     if (kept) acc[w] = incl;
+                    if (hh == hw && kept) keep4 |= 1u << j;
                     inc[w] = incl;
                 }
+            }
+            uint32_t m = F[w];
+            const unsigned char* rows = sq + (w ? kKVStride : 0) + q * 16;
+            while (m) {
+                const int bit = __ffs(m) - 1;
+                m &= m - 1;
+                const int j = bit >> 3, ch = bit & 7;
+                if (!((keep4 >> j) & 1u)) continue;
+                const uint32_t tj = (hw ? T1 : T0);
+                uint32_t pos = before;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) pos += jj < j ? ((tj >> (8 * jj)) & 0xFFu) : 0u;
+                const uint32_t f8 = (F[w] >> (8 * j)) & 0xFFu;
+                pos += ((in4 >> (8 * j)) & 0xFFu) - __popc(f8) + __popc(f8 & ((1u << ch) - 1u));
+                const uint32_t x16 = *reinterpret_cast<const uint16_t*>(rows + j * 256 + 2 * ch);
+                const uint32_t tloc = (uint32_t)((4 * (u0 + hw) + j) % kChunk);
+                outl[w][start[w] + pos] = (x16 << 16) | (tloc << 7) | (uint32_t)(8 * q + ch);
             }
         }
         __syncwarp();  // code bytes complete
