@@ -362,9 +362,9 @@ int kvq_fit_codebook(const uint16_t* samples, int32_t n_vec, int32_t vec_len, do
  * file-scope device array of KVQ_NOALLOC_SCRATCH_BYTES that the library owns; every GPU
  * that loads libkvq.so holds that array until the process exits.
  *   - Limit: the scratch that kvq_quantize_workspace(cfg, n_new, 0) reports must fit in
- *     KVQ_NOALLOC_SCRATCH_BYTES (1 MiB).  A call needs about 36 bytes per (sequence, new
+ *     KVQ_NOALLOC_SCRATCH_BYTES (1 MiB).  A call needs about 80 bytes per (sequence, new
  *     token) and 16*(n_new/64 + 2) + 32 bytes per (sequence, kv head): 256 sequences with
- *     32 kv heads fit appending up to 56 tokens each; larger requests return
+ *     32 kv heads fit appending up to 25 tokens each; larger requests return
  *     KVQ_ERR_SCRATCH_LIMIT and launch nothing.  Use kvq_quantize_append with a caller
  *     workspace for prefills.
  *   - The first call on a device looks up the array's device address

@@ -30,8 +30,8 @@ struct QuantWs {
     uint32_t* sel1;   // [B][n][4]  bin_lo, rem_lo, bin_hi, rem_hi
     uint32_t* hist2;  // [B][n][512]
     uint32_t* kcut;   // [B][n/2][16] key cut pairs of adjacent channels (calibrating calls)
-    uint32_t* vthr;   // [B][n_new] fp16 t_lo | t_hi << 16
-    uint16_t* vcut;   // [B][n_new][16] value cuts of each token, slot 15 force-zero flag
+    uint32_t* vrec;   // [B][n_new][kVRec] per token: force-zero mask, (t_lo, t_lo), (t_hi, t_hi),
+                      // then (cut_j, cut_j) for j < 2^bits - 1, fp16 pairs ready for half2 compares
     uint32_t* kcc;    // [B*Hkv][nchc] outliers of this call in chunk cl of list (b, h)
     uint32_t* vcc;
     uint32_t* kce;    // [B*Hkv][nchc] their exclusive prefix
@@ -39,7 +39,8 @@ struct QuantWs {
     int32_t* lst;     // [B*Hkv][8] start K/V, first overflowing chunk K/V (-1: none), kept K/V
 };
 
-constexpr int kWsParts = 14;
+constexpr int kWsParts = 13;
+constexpr int kVRec = 20;  // words of a token's value record (3 + up to 15 cuts, padded)
 
 struct WsPlan {
     size_t off[kWsParts];
@@ -58,7 +59,7 @@ WsPlan plan_ws(const kvq_cfg& cfg, int n_new, int calibrate) {
                               calibrate ? B * n * 4 * 4 : 0,
                               calibrate ? B * n * 512 * 4 : 0,
                               calibrate ? B * n * 32 : 0,
-                              B * T * 4, B * T * 32,
+                              B * T * kVRec * 4,
                               L * C * 4, L * C * 4, L * C * 4, L * C * 4,
                               L * 8 * 4};
     WsPlan p;
@@ -80,13 +81,12 @@ QuantWs bind_ws(char* base, const WsPlan& p) {
     w.sel1 = (uint32_t*)(base + p.off[4]);
     w.hist2 = (uint32_t*)(base + p.off[5]);
     w.kcut = (uint32_t*)(base + p.off[6]);
-    w.vthr = (uint32_t*)(base + p.off[7]);
-    w.vcut = (uint16_t*)(base + p.off[8]);
-    w.kcc = (uint32_t*)(base + p.off[9]);
-    w.vcc = (uint32_t*)(base + p.off[10]);
-    w.kce = (uint32_t*)(base + p.off[11]);
-    w.vce = (uint32_t*)(base + p.off[12]);
-    w.lst = (int32_t*)(base + p.off[13]);
+    w.vrec = (uint32_t*)(base + p.off[7]);
+    w.kcc = (uint32_t*)(base + p.off[8]);
+    w.vcc = (uint32_t*)(base + p.off[9]);
+    w.kce = (uint32_t*)(base + p.off[10]);
+    w.vce = (uint32_t*)(base + p.off[11]);
+    w.lst = (int32_t*)(base + p.off[12]);
     return w;
 }
 
@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kCalThreads) k_calib_hist(kvq_cfg cfg,
             const uint32_t* s0 = ws.sel1 + ((size_t)b * n + j0) * 4;
             bl0 = s0[0]; bh0 = s0[2]; bl1 = s0[4]; bh1 = s0[6];
         }
+
         uint32_t* h0 = sh + (2 * lane) * kCalStride;
         uint32_t* h1 = h0 + kCalStride;
         const uint16_t* src = k + (size_t)b * n_new * n + j0;
@@ -521,16 +522,17 @@ __global__ void __launch_bounds__(kStWarps * 32, 3) k_tok_stats(kvq_cfg cfg, kvq
         const float vlo = h2f((uint16_t)lo_bits), vhi = h2f((uint16_t)hi_bits);
         const float off = __fmul_rn(__fadd_rn(vlo, vhi), 0.5f);
         const float half = __fmul_rn(__fsub_rn(vhi, vlo), 0.5f);
+        uint32_t* rec = ws.vrec + ((size_t)b * n_new + i) * kVRec;
         if (lane == 0) {
             c.vparams[((size_t)b * cfg.T_max + t) * 2 + 0] = off;
             c.vparams[((size_t)b * cfg.T_max + t) * 2 + 1] = half;
-            ws.vthr[(size_t)b * n_new + i] = lo_bits | (hi_bits << 16);
+            rec[0] = half == 0.0f ? 0xFFFFFFFFu : 0u;
+            rec[1] = lo_bits | (lo_bits << 16);
+            rec[2] = hi_bits | (hi_bits << 16);
         }
-        if (lane < 16) {
-            uint32_t cut = 0x7E00u;
-            if (lane < nb) cut = cut_of(bnd[lane], off, half);
-            else if (lane == 15) cut = half == 0.0f ? 0xFFFFu : 0u;
-            ws.vcut[((size_t)b * n_new + i) * 16 + lane] = (uint16_t)cut;
+        if (lane < nb) {
+            const uint32_t cut = cut_of(bnd[lane], off, half);
+            rec[3 + lane] = cut | (cut << 16);
         }
         // outliers per kv head (entry x of the row lies in head x >> 4)
         const uint32_t lo2 = lo_bits | (lo_bits << 16), hi2 = hi_bits | (hi_bits << 16);
@@ -791,25 +793,28 @@ __global__ void __launch_bounds__(kWrWarps * 32, 3) k_tok_write(kvq_cfg cfg, kvq
             const uint4 xv = *reinterpret_cast<const uint4*>(sq + kKVStride + j * 256 + q * 16);
             uint32_t VC[NB], VLO, VHI, VZ;
             {
-                const size_t ti = (size_t)b * n_new + (pr ? t - t0 : 0);
-                const uint32_t vt = ws.vthr[ti];
-                VLO = __byte_perm(vt, 0, 0x1010);
-                VHI = __byte_perm(vt, 0, 0x3232);
-                const uint4* cr = reinterpret_cast<const uint4*>(ws.vcut + ti * 16);
-                const uint4 c0v = cr[0], c1v = cr[1];
-                const uint32_t cw[8] = {c0v.x, c0v.y, c0v.z, c0v.w, c1v.x, c1v.y, c1v.z, c1v.w};
+                constexpr int NW = (3 + NB + 3) / 4;  // record words read, in 16-byte loads
+                const uint4* cr = reinterpret_cast<const uint4*>(
+                    ws.vrec + ((size_t)b * n_new + (pr ? t - t0 : 0)) * kVRec);
+                uint32_t rw[4 * NW];
 #pragma unroll
-                for (int jj = 0; jj < NB; ++jj)
-                    VC[jj] = __byte_perm(cw[jj >> 1], 0, (jj & 1) ? 0x3232 : 0x1010);
-                VZ = (cw[7] >> 16) ? 0xFFFFFFFFu : 0u;
+                for (int r = 0; r < NW; ++r) {
+                    const uint4 x4 = cr[r];
+                    rw[4 * r] = x4.x; rw[4 * r + 1] = x4.y; rw[4 * r + 2] = x4.z; rw[4 * r + 3] = x4.w;
+                }
+                VZ = rw[0];
+                VLO = rw[1];
+                VHI = rw[2];
+#pragma unroll
+                for (int jj = 0; jj < NB; ++jj) VC[jj] = rw[3 + jj];
             }
             const uint32_t xkw[4] = {xk.x, xk.y, xk.z, xk.w};
             const uint32_t xvw[4] = {xv.x, xv.y, xv.z, xv.w};
-            uint32_t ck[4], cv[4], fk = 0, fv = 0;
+            uint32_t ck[4], cv[4], okk[4], okv[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const uint32_t ok = out2(xkw[e], KLO[e], KHI[e]);
-                fk |= ((ok & 1u) | ((ok >> 15) & 2u)) << (2 * e);
+                okk[e] = ok;
                 if constexpr (KCUTS) {
                     ck[e] = enc_pair<BITS>(xkw[e] & ~(ok | KZ[e]), KC[e]);
                 } else {
@@ -822,8 +827,18 @@ __global__ void __launch_bounds__(kWrWarps * 32, 3) k_tok_write(kvq_cfg cfg, kvq
                     ck[e] = c2[0] | (c2[1] << 16);
                 }
                 const uint32_t ov = out2(xvw[e], VLO, VHI);
-                fv |= ((ov & 1u) | ((ov >> 15) & 2u)) << (2 * e);
+                okv[e] = ov;
                 cv[e] = enc_pair<BITS>(xvw[e] & ~(ov | VZ), VC);
+            }
+            // flag bits (channel 8q + m at bit m), built only when the lane has an outlier
+            uint32_t fk = 0, fv = 0;
+            if (okk[0] | okk[1] | okk[2] | okk[3]) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) fk |= ((okk[e] & 1u) | ((okk[e] >> 15) & 2u)) << (2 * e);
+            }
+            if (okv[0] | okv[1] | okv[2] | okv[3]) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) fv |= ((okv[e] & 1u) | ((okv[e] >> 15) & 2u)) << (2 * e);
             }
             // code bytes of channels 8q .. 8q + 7 (zero for a token outside this call)
             const uint32_t pm = pr ? 0xFFFFFFFFu : 0u;
