@@ -15,6 +15,8 @@
 // outlier lists chunk by chunk: key outliers add (x - zhat) times the rotated query component
 // to the logits before the softmax statistics are taken, value outliers add
 // p (x - zhat) to the output after the merge.
+#include <cooperative_groups.h>
+
 #include "kvq_common.cuh"
 #include "kvq_device.cuh"
 
@@ -388,7 +390,6 @@ __global__ void __launch_bounds__(qk_warps(HPC) * 32 + 32, 1)
 constexpr int kQQuads = 64;                  // token quads per stage
 constexpr int kQTokens = 4 * kQQuads;        // tokens per stage
 constexpr int kQWarps = 16;                  // consumer warps
-constexpr bool kQKHalfTables = false;        // QK tables of fp16 pairs (k_qk_quadh) for one-head kv heads
 
 // The table goes last, at the first shared-window address past `pre` that is a multiple of
 // its j-slice (64 pairs x NT entries x 8 bytes): a lookup address is then one OR of the
@@ -589,250 +590,6 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
                         const unsigned long long T = k == 0 ? lds64<0>(a)
                                                    : k == 1 ? lds64<128>(a)
                                                    : k == 2 ? lds64<256>(a) : lds64<384>(a);
-                        acc[sl][u] = fma2(Pc, T, acc[sl][u]);
-                    }
-                }
-            }
-            float v[8];
-#pragma unroll
-            for (int sl = 0; sl < 4; ++sl)
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const f2 a = upk(acc[sl][u]);
-                    v[2 * sl + u] = a.x + a.y;
-                }
-            int mk = 8;
-#pragma unroll
-            for (int half = 4; half >= 1; half >>= 1, mk >>= 1)
-#pragma unroll
-                for (int t = 0; t < half; ++t)
-                    v[t] += __shfl_xor_sync(0xffffffffu, v[t + half], mk);
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-            const int t = t_begin + st * kQTokens + tq;
-            if (owner && t < t_end) lrow[t] = v[0];
-        }
-    }
-    __syncthreads();
-    // after an abandoned wait, copies of the last stages issued may still be in flight
-    if (*flag && tid == 0) drain_chunks(full, max(0, flag[1] - kStages), flag[1], kStages);
-}
-
-// The lane group's 16 fields with groups k and k ^ 1 (four fields each, pairs i + 16 k)
-// exchanged in place.
-template <int BITS>
-__device__ __forceinline__ void swap_groups(uint32_t (&w)[BITS]) {
-    if constexpr (BITS == 2) {
-        w[0] = __byte_perm(w[0], 0u, 0x1032);
-        w[1] = __byte_perm(w[1], 0u, 0x1032);
-    } else {
-        static_assert(BITS == 3, "2 or 3 bits");
-        const unsigned long long lo = ((unsigned long long)w[1] << 32) | w[0];
-        const uint32_t g0 = (uint32_t)lo & 0xFFFFFFu;
-        const uint32_t g1 = (uint32_t)(lo >> 24) & 0xFFFFFFu;
-        const uint32_t g2 = ((uint32_t)(lo >> 48) | (w[2] << 16)) & 0xFFFFFFu;
-        const uint32_t g3 = w[2] >> 8;
-        w[0] = g1 | (g0 << 24);
-        w[1] = (g0 >> 8) | (g3 << 16);
-        w[2] = (g3 >> 16) | (g2 << 8);
-    }
-}
-
-// QK as k_qk_quad with the (X, Y) table entries stored as fp16 pairs (4 bytes): half the
-// lookup bytes, two conversions per lookup.  Built for measurement against the binary32
-// tables; the decode path uses k_qk_quad unless kQKHalfTables is set.
-template <int BITS>
-__global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
-    k_qk_quadh(kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ qr_all,
-              const float2* __restrict__ thi, const float2* __restrict__ tlo, int Ls,
-              int max_len, float* __restrict__ logits) {
-    using F = Fmt<BITS>;
-    constexpr int NC = kQWarps * 32;
-    constexpr int P = 8;                         // entry bit of a table byte offset (4-byte entries)
-    constexpr int JS = P + F::FW;                // j bit of a table byte offset
-    constexpr uint32_t MASK = (uint32_t)(F::NT - 1) << P;
-    extern __shared__ __align__(128) uint8_t sm[];
-    const QQPlan L = qq_plan(BITS);
-    const uint32_t sbase = smem_u32(sm);
-    const int JSL = L.jslice / 2;                // half2 entries: half the j-slice
-    const uint32_t tpos = (sbase + L.pre + JSL - 1) & ~(uint32_t)(JSL - 1);
-    uint8_t* tab = sm + (tpos - sbase);
-    uint8_t* ring = sm + L.ring;
-    float4* base = (float4*)(sm + L.base);
-    float* lev = (float*)(sm + L.lev);
-    uint64_t* full = (uint64_t*)(sm + L.bar);
-    uint64_t* empty = full + kStages;
-    int* flag = (int*)(sm + L.flag);
-
-    const int tid = threadIdx.x;
-    const int i = tid & 15, x = i >> 2, lane = tid & 31, warp = tid >> 5;
-    const int s = blockIdx.x, b = blockIdx.y, hq = blockIdx.z;
-    const int Hq = cfg.Hq, Hkv = cfg.Hkv, kvh = hq / (Hq / Hkv);
-    int len = c.len[b];
-    if (len > max_len) {
-        if (tid == 0 && s == 0 && hq == 0) set_status(c.status, KVQ_STATUS_LEN_OVERFLOW);
-        len = max_len;
-    }
-    const int t_begin = s * Ls, t_end = min(len, t_begin + Ls);
-    if (t_begin >= t_end) return;
-    const int nst = (t_end - t_begin + kQTokens - 1) / kQTokens;
-    if (tid == 0) {
-        for (int k = 0; k < kStages; ++k) {
-            mbar_init(full + k, 1);
-            mbar_init(empty + k, kQWarps);
-        }
-        flag[0] = 0;
-        flag[1] = 0;
-        fence_mbar_init();
-    }
-    // ---- tables: (X, Y) of Z_p(entry) turned by j theta_p.  Thread (p, r) of the first 512
-    // holds pair p's constants and writes entries r, r + 8, ... for every j.
-    if (tid < (1 << BITS)) lev[tid] = cb.levels[tid];
-    __syncthreads();
-    if (tid < 512) {
-        const int p = tid & 63, r0 = tid >> 6;
-        const float* kp = c.kparams + ((size_t)b * Hkv + kvh) * kD * 2;
-        const float* qv = qr_all + ((size_t)b * Hq + hq) * kD;
-        const float offa = kp[2 * p], halfa = kp[2 * p + 1];
-        const float offb = kp[2 * (p + 64)], halfb = kp[2 * (p + 64) + 1];
-        const float qa = qv[p], qb = qv[p + 64];
-        const float A1 = qa * halfa, B1 = qb * halfb, C1 = qa * offa + qb * offb;
-        const float A2 = qb * halfa, B2 = -qa * halfb, C2 = qb * offa - qa * offb;
-        float2 rj[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) rj[j] = tlo[j * 64 + p];
-        uint32_t* t32 = reinterpret_cast<uint32_t*>(tab);
-        for (int idx = r0; idx < F::NT; idx += 8) {
-            const float La = lev[idx & ((1 << BITS) - 1)], Lb = lev[idx >> BITS];
-            const float X = fmaf(B1, Lb, fmaf(A1, La, C1));
-            const float Y = fmaf(B2, Lb, fmaf(A2, La, C2));
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-            {
-                const __half2 hv = __floats2half2_rn(fmaf(rj[j].x, X, rj[j].y * Y),
-                                                     fmaf(rj[j].x, Y, -rj[j].y * X));
-                t32[(j * F::NT + idx) * 64 + p] = *reinterpret_cast<const uint32_t*>(&hv);
-            }
-        }
-    }
-    __syncthreads();  // tables complete, barriers initialised
-
-    if (tid >= NC) {
-        // ================= streaming warp
-        const int pl = tid - NC;
-        const uint32_t* src = c.kcodes + ((size_t)b * Hkv + kvh) * nquads(cfg.T_max) * F::BW;
-        int cc = 0;
-        for (; cc < nst; ++cc) {
-            const int slot = cc % kStages;
-            if (cc >= kStages && !mbar_wait(empty + slot, (uint32_t)(cc / kStages - 1) & 1u)) {
-                if (pl == 0) {
-                    atomicOr(flag, 1);
-                    set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
-                }
-                break;
-            }
-            if (*flag) break;
-            const int tc = t_begin + cc * kQTokens;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const float2 cs = trig_at(thi, tlo, tc, pl + 32 * u);
-                base[slot * 64 + pl + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
-            }
-            __syncwarp();
-            __threadfence_block();
-            if (pl == 0) {
-                fence_proxy_async();
-                const int q0 = tc >> 2, q1 = (min(tc + kQTokens, t_end) + 3) >> 2;
-                const uint32_t bytes = (uint32_t)(q1 - q0) * F::BW * 4;
-                mbar_arrive_expect_tx(full + slot, bytes);
-                bulk_load(ring + (size_t)slot * L.stage, src + (size_t)q0 * F::BW, bytes,
-                          full + slot);
-            }
-            __syncwarp();
-        }
-        if (pl == 0) flag[1] = cc;  // stages issued
-    } else {
-        // ================= consumer warps
-        const int uperm = (i >> 1) & 1;     // partial u of the lane holds quad u ^ uperm
-        const bool owner = !(i & 1);
-        // quads 4 warp + hh and 4 warp + hh + 2 (hh the half-warp): the code words of the two
-        // half-warps then sit 16 banks apart
-        const int qbase = 4 * warp + ((tid >> 4) & 1);
-        // half-warp 1 takes pair group k ^ 1 where half-warp 0 takes k: the two read disjoint
-        // banks.  Even k: immediate 64 k, half-warp 1 adds 64; odd k: immediate 64 (k - 1),
-        // half-warp 0 adds 64.
-        const int hw = (tid >> 4) & 1;
-        uint32_t lbE[4], lbO[4], woff[2];
-#pragma unroll
-        for (int sl = 0; sl < 4; ++sl) {
-            const uint32_t lb = tpos + ((uint32_t)(sl ^ x) << JS) + ((uint32_t)i << 2);
-            lbE[sl] = lb | (hw ? 64u : 0u);
-            lbO[sl] = lb | (hw ? 0u : 64u);
-        }
-        // phase from the stage start to the quad, pair i + 16 k, as (c, s) and (-s, c)
-        unsigned long long RQ[2][4], RQp[2][4];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int q = qbase + 2 * (u ^ uperm);
-            woff[u] = (uint32_t)(q * F::BW + i * BITS) * 4;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 r = tlo[(4 * q) * 64 + i + 16 * (k ^ hw)];
-                RQ[u][k] = pk(r.x, r.y);
-                RQp[u][k] = pk(-r.y, r.x);
-            }
-        }
-        const int tq = 4 * (qbase + 2 * uperm) + x;
-        float* lrow = logits + ((size_t)b * Hq + hq) * cfg.T_max;
-        for (int st = 0; st < nst; ++st) {
-            const int slot = st % kStages;
-            if (!mbar_wait(full + slot, (uint32_t)(st / kStages) & 1u)) {
-                atomicOr(flag, 1);
-                set_status(c.status, KVQ_STATUS_WAIT_TIMEOUT);
-            }
-            if (*flag) break;
-            const uint8_t* stage = ring + (size_t)slot * L.stage;
-            uint32_t w[2][BITS];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-#pragma unroll
-                for (int d = 0; d < BITS; ++d)
-                    w[u][d] = *reinterpret_cast<const uint32_t*>(stage + woff[u] + 4 * d);
-                if (hw) swap_groups<BITS>(w[u]);  // fields of pair group k ^ 1 in group k's place
-            }
-            unsigned long long Bc[4], Bs[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float4 bq = base[slot * 64 + i + 16 * (k ^ hw)];
-                Bc[k] = pk(bq.x, bq.y);
-                Bs[k] = pk(bq.z, bq.w);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
-            unsigned long long acc[4][2];
-#pragma unroll
-            for (int sl = 0; sl < 4; ++sl) acc[sl][0] = acc[sl][1] = 0ull;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    // (c_b c_q - s_b s_q, c_b s_q + s_b c_q) in two packed instructions
-                    const unsigned long long Pc = fma2(Bc[k], RQ[u][k], mul2(Bs[k], RQp[u][k]));
-#pragma unroll
-                    for (int sl = 0; sl < 4; ++sl) {
-                        uint32_t fs;
-                        switch (4 * k + sl) {
-#define KVQ_FS(N) case N: fs = field_to<BITS, N, P>(w[u]); break;
-                            KVQ_FS(0) KVQ_FS(1) KVQ_FS(2) KVQ_FS(3) KVQ_FS(4) KVQ_FS(5)
-                            KVQ_FS(6) KVQ_FS(7) KVQ_FS(8) KVQ_FS(9) KVQ_FS(10) KVQ_FS(11)
-                            KVQ_FS(12) KVQ_FS(13) KVQ_FS(14) KVQ_FS(15)
-#undef KVQ_FS
-                        }
-                        const uint32_t a = (fs & MASK) | ((k & 1) ? lbO[sl] : lbE[sl]);
-                        const uint32_t hv = k == 0 ? lds32<0>(a)
-                                          : k == 1 ? lds32<0>(a)
-                                          : k == 2 ? lds32<128>(a) : lds32<128>(a);
-                        const float2 tf = __half22float2(*reinterpret_cast<const __half2*>(&hv));
-                        const unsigned long long T = pk(tf.x, tf.y);
                         acc[sl][u] = fma2(Pc, T, acc[sl][u]);
                     }
                 }
@@ -2016,7 +1773,12 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
     kvq_cfg cfg, kvq_cache c, kvq_codebook cb, const float* __restrict__ logits,
     const float2* __restrict__ ml, int Ls, int S, int max_len, float* __restrict__ part) {
     constexpr int NB = (1 << BITS) - 1;
-    const int s = blockIdx.x, li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
+    // a cluster of blocks along x shares one split: block `rank` walks its share of the
+    // split's chunks, and rank 0 adds the blocks' integer sums (read through distributed
+    // shared memory) once into the split's partial
+    cooperative_groups::cluster_group cluster = cooperative_groups::this_cluster();
+    const int nsub = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
+    const int s = blockIdx.x / nsub, li = blockIdx.y, b = li / cfg.Hkv, h = li % cfg.Hkv;
     const int g = G ? G : cfg.Hq / cfg.Hkv;
     const int len = min(c.len[b], max_len);
     const uint32_t* cp = c.vchunk + (size_t)li * (nchunks(cfg.T_max) + 1);
@@ -2035,14 +1797,14 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
     const float2* vpar = reinterpret_cast<const float2*>(c.vparams) + (size_t)b * cfg.T_max;
     const float* lrow = logits + ((size_t)b * cfg.Hq + h * g) * cfg.T_max;
     const size_t T_max = cfg.T_max;
-    const int mb = s * (Ls / kChunk), me = min(mb + Ls / kChunk, (len + kChunk - 1) / kChunk);
+    const int mb0 = s * (Ls / kChunk), me0 = min(mb0 + Ls / kChunk, (len + kChunk - 1) / kChunk);
+    const int span = max(0, (me0 - mb0 + nsub - 1) / nsub);
+    const int mb = mb0 + rank * span, me = min(me0, mb + span);
     const uint32_t cnt = c.vcount[li];
-    bool any = false;
     for (int m0 = mb; m0 < me; m0 += kOutChunks) {
         __syncthreads();  // the previous window's cps are no longer read
         const OutRange r = stage_chunks(cp, cnt, len, m0, me, cps);  // barrier covers the above
         if (r.lo >= r.hi) continue;
-        any = true;
         float bd[NB];
 #pragma unroll
         for (int j = 0; j < NB; ++j) bd[j] = bnd[j];
@@ -2082,15 +1844,18 @@ __global__ void __launch_bounds__(kOutThreads) k_value_outliers(
             }
         }
     }
-    __syncthreads();
-    if (!any) return;
-    for (int e = threadIdx.x; e < g * kD; e += blockDim.x) {
-        const long long v = (long long)acc[e];
-        if (v != 0) {
-            float* pp = part + (((size_t)b * cfg.Hq + h * g + e / kD) * S + s) * kD + e % kD;
-            *pp += (float)((double)v * kFixInv);
+    cluster.sync();  // every block's sums are complete (and visible across the cluster)
+    if (rank == 0) {
+        for (int e = threadIdx.x; e < g * kD; e += blockDim.x) {
+            long long v = 0;
+            for (int r = 0; r < nsub; ++r) v += (long long)cluster.map_shared_rank(acc, r)[e];
+            if (v != 0) {
+                float* pp = part + (((size_t)b * cfg.Hq + h * g + e / kD) * S + s) * kD + e % kD;
+                *pp += (float)((double)v * kFixInv);
+            }
         }
     }
+    cluster.sync();  // the other blocks' shared memory stays until rank 0 has read it
 }
 
 __global__ void k_softmax_merge(int BH, int S, const float2* __restrict__ stats,
@@ -2499,8 +2264,7 @@ static int run_qk(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
     }
     const int g = cfg->Hq / cfg->Hkv;
     if (cfg->bits <= 3 && (g == 1 || g == 2 || g == 4)) {
-        QKQKernel kq = g == 1 ? (kQKHalfTables ? (cfg->bits == 2 ? k_qk_quadh<2> : k_qk_quadh<3>)
-                                               : (cfg->bits == 2 ? k_qk_quad<2> : k_qk_quad<3>))
+        QKQKernel kq = g == 1 ? (cfg->bits == 2 ? k_qk_quad<2> : k_qk_quad<3>)
                      : g == 2 ? (cfg->bits == 2 ? k_qk_grp<2, 2> : k_qk_grp<3, 2>)
                               : (cfg->bits == 2 ? k_qk_grp<2, 4> : k_qk_grp<3, 4>);
         const int smem = qq_plan(cfg->bits).total;
@@ -2606,14 +2370,33 @@ static int run_pv(const kvq_cfg* cfg, const kvq_cache* cache, const kvq_codebook
                                                             (const float2*)ml, Ls, S, max_len,
                                                             kvb, part);
     }
-    dim3 go(S, cfg->B * cfg->Hkv);
+
     const bool mha = cfg->Hq == cfg->Hkv;
     const int gq = cfg->Hq / cfg->Hkv;
     auto vo = cfg->bits == 2 ? (mha ? k_value_outliers<2, 1> : gq == 2 ? k_value_outliers<2, 2> : gq == 4 ? k_value_outliers<2, 4> : k_value_outliers<2, 0>)
             : cfg->bits == 3 ? (mha ? k_value_outliers<3, 1> : gq == 2 ? k_value_outliers<3, 2> : gq == 4 ? k_value_outliers<3, 4> : k_value_outliers<3, 0>)
                              : (mha ? k_value_outliers<4, 1> : gq == 2 ? k_value_outliers<4, 2> : gq == 4 ? k_value_outliers<4, 4> : k_value_outliers<4, 0>);
-    vo<<<go, kOutThreads, 0, st>>>(*cfg, *cache, *cbV, logits, (const float2*)ml, Ls, S, max_len,
-                                   part);
+    {
+        // blocks per split: enough for about four per SM, at most a portable cluster of 8
+        const long long base = (long long)S * cfg->B * cfg->Hkv;
+        int nsub = (int)((4 * 148 + base - 1) / base);
+        nsub = nsub < 1 ? 1 : (nsub > 8 ? 8 : nsub);
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(S * nsub, cfg->B * cfg->Hkv);
+        lc.blockDim = dim3(kOutThreads);
+        lc.dynamicSmemBytes = 0;
+        lc.stream = st;
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = nsub;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        lc.attrs = at;
+        lc.numAttrs = 1;
+        cudaError_t ce = cudaLaunchKernelEx(&lc, vo, *cfg, *cache, *cbV, logits, (const float2*)ml,
+                                            Ls, S, max_len, part);
+        if (ce) return record_cuda(ce);
+    }
     k_pv_reduce<<<cfg->B * cfg->Hq, kD, 0, st>>>(S, part, out);
     return record_cuda(cudaGetLastError());
 }

@@ -125,14 +125,6 @@ __device__ __forceinline__ unsigned long long lds64(uint32_t addr) {
     return d;
 }
 
-// 32-bit shared-memory load at a shared-window address plus an immediate byte offset.
-template <int IMM>
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
-    uint32_t d;
-    asm("ld.shared.b32 %0, [%1+%2];" : "=r"(d) : "r"(addr), "n"(IMM));
-    return d;
-}
-
 // 32-bit shared-memory load at a shared-window address.
 __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     uint32_t d;
