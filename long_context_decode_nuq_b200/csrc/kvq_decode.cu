@@ -6,7 +6,8 @@
 // The two streaming kernels share one shape.  A CTA covers HPC query heads over one split of
 // the tokens and walks it in 64-token chunks.  The chunk's code blocks (one contiguous run of
 // 16 blocks per kv head) arrive in a ring of shared-memory stages filled by bulk copies
-// (cp.async.bulk, completion counted on an mbarrier; no multicast) that the last warp issues.
+// (cp.async.bulk into the CTA's own shared memory, completion counted on an mbarrier) that
+// the last warp issues.
 // Half-warp qd of a consumer warp takes token quad qd of the chunk and lane i of the
 // half-warp the rotate-half pairs (c, c + 64), c = i + 16k: exactly the lane group i of the
 // code block, whose token slot s holds token s ^ (i >> 2) (the rotation that lets QK reduce

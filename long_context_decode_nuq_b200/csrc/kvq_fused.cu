@@ -8,7 +8,7 @@
 // A CTA has 16 consumer warps and three helper warps and walks its split in 256-token stages
 // through a ring of kFSlots shared-memory slots.
 //  - Issuing warp: per stage, bulk copies (cp.async.bulk, completion counted on an mbarrier;
-//    no multicast) of the key code blocks, the tokens' value (off, half), and the stage's key-
+//    one destination CTA) of the key code blocks, the tokens' value (off, half), and the stage's key-
 //    and value-outlier entries (up to kFEnt of each; entries past that are read from global
 //    memory).  It waits only for the slot to be released, so copies run a full ring ahead.
 //  - Key warp: per stage, the (cos, sin) of the stage start for the 64 RoPE pairs and, once
