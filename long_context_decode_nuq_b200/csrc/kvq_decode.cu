@@ -873,7 +873,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 // associative, so their order does not matter), then adds each block sum once into its
 // split's PV partial before the partials are summed in split order.
 constexpr int kOutThreads = 256;  // threads per block of the outlier kernels
-constexpr int kOutChunks = 64;    // chunks per staged window of chunk pointers
+constexpr int kOutChunks = 128;   // chunks per staged window of chunk pointers
 constexpr int kOutBatch = 4;      // entries a lane gathers at once
 constexpr float kFixScale = 1099511627776.0f;      // 2^40
 constexpr double kFixInv = 1.0 / 1099511627776.0;  // 2^-40
