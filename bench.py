@@ -47,6 +47,10 @@ def parse():
                         "kvq_decode_attention_fused (one kernel per split, no logits)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-fp16", action="store_true")
+    p.add_argument("--no-graph", action="store_true",
+                   help="time the per-layer calls only (by default the headline is the whole "
+                        "step, every layer's append and attention, replayed as one CUDA graph "
+                        "through kvq_step_launch)")
     p.add_argument("--layers", type=int, default=0, help="override the workload's layer count")
     p.add_argument("--tokens", type=int, default=0, help="override the cached token count")
     p.add_argument("--bits", type=int, default=0, help="override the workload's code width")
@@ -109,6 +113,10 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            # the timed region starts once the sampler runs (first sample, at most 5 s)
+            t_end = time.time() + 5.0
+            while not self.lines and time.time() < t_end and self.proc.poll() is None:
+                time.sleep(0.02)
         except Exception:
             self.proc = None
         return self
@@ -319,7 +327,10 @@ def run_kvq(args, rank, world):
     t_base = rank * T0 if sharded else 0          # position of this rank's first token
     pos0 = shard_n * T0                            # position of the first appended token
     appends_here = (not sharded) or rank == world - 1
-    T_max = T0 + steps_total + e2e_steps + 64
+    # the graph-replayed step (not with token sharding, whose merge is a collective) runs first
+    use_graph = not args.no_graph and not sharded
+    graph_steps = steps_total if use_graph else 0
+    T_max = T0 + graph_steps + steps_total + e2e_steps + 64
     # outlier lists are per (sequence, kv head): a key channel keeps ~f*T outliers, a token's
     # 2k value outliers spread over the Hkv heads; capacities are multiples of 8
     ceil8 = lambda x: (int(x) + 7) // 8 * 8  # noqa: E731
@@ -391,8 +402,9 @@ def run_kvq(args, rank, world):
             gen.fill_v(tmp, pos0 + s, 1)
             vnew[i, s] = tmp
             gen.fill_q(qall[i, s], step=s)
-    qpos = torch.tensor([[pos0 + s] * w.B for s in range(steps_total)], dtype=torch.int32,
-                        device=dev)
+    # the per-layer region appends after the graph region's tokens
+    qpos = torch.tensor([[pos0 + graph_steps + s] * w.B for s in range(steps_total)],
+                        dtype=torch.int32, device=dev)
     sdec = None
     if sharded:
         from long_context_decode_nuq_b200.shard import ShardedDecode
@@ -417,7 +429,7 @@ def run_kvq(args, rank, world):
         return e
 
     def local_len(s):
-        return T0 + s + 1 if appends_here else T0
+        return T0 + graph_steps + s + 1 if appends_here else T0
 
     def layer_step(i, s, timing):
         c = caches[i]
@@ -456,10 +468,73 @@ def run_kvq(args, rank, world):
             marks[4].record()
         return marks
 
+    # ---- the whole step (every layer's append + attention) replayed as one CUDA graph
+    appended = [0] * R  # tokens appended so far to each replica's caches
+
+    def step_record(s, r, qp):
+        """Packed kvq_step input record: per layer k, v, q (fp16 bytes), then qpos (int32 [B],
+        padded to 16 bytes)."""
+        parts = []
+        for i in range(r * layers, (r + 1) * layers):
+            parts += [knew[i, s].reshape(-1).view(torch.uint8),
+                      vnew[i, s].reshape(-1).view(torch.uint8),
+                      qall[i, s].reshape(-1).view(torch.uint8)]
+        qp_t = torch.zeros((w.B * 4 + 15) // 16 * 4, dtype=torch.int32, device=dev)
+        qp_t[:w.B] = qp
+        parts.append(qp_t.view(torch.uint8))
+        return torch.cat(parts)
+
+    graph = None
+    if use_graph:
+        g_max_len = T0 + graph_steps + steps_total + e2e_steps  # bounds every graph launch
+        g_in = torch.empty(K.kvq_step_input_bytes(cfg, layers, 1), dtype=torch.uint8, device=dev)
+        g_ws = torch.empty(K.kvq_step_workspace(cfg, 1, g_max_len, S,
+                                                1 if args.path == "fused" else 0),
+                           dtype=torch.uint8, device=dev)
+        gsteps = [K.kvq_step_create(cfg, caches[r * layers:(r + 1) * layers],
+                                    [cb[0] for cb in cbs[r * layers:(r + 1) * layers]],
+                                    [cb[1] for cb in cbs[r * layers:(r + 1) * layers]], 1,
+                                    g_max_len, g_in, outs[r * layers:(r + 1) * layers], g_ws, S,
+                                    1 if args.path == "fused" else 0)
+                  for r in range(R)]
+        # the launch schedule: warm-up launches every replica per step, a timed step one
+        plan = [(s, r) for s in range(args.warmup) for r in range(R)] + [
+            (s, s % R) for s in range(args.warmup, steps_total)]
+        recs, g_tok = [], []
+        for s, r in plan:
+            recs.append(step_record(s, r, pos0 + appended[r]))
+            appended[r] += 1
+            g_tok.append(T0 + appended[r])
+        recs = torch.stack(recs)
+        n_warm = args.warmup * R
+        torch.cuda.synchronize()
+        for j in range(n_warm):
+            K.kvq_step_launch(gsteps[plan[j][1]], recs[j])
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(dev.index) as clk_g:
+            g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            g0.record()
+            for j in range(n_warm, len(plan)):
+                K.kvq_step_launch(gsteps[plan[j][1]], recs[j])
+            g1.record()
+            torch.cuda.synchronize()
+        g_ms = g0.elapsed_time(g1)
+        for c in caches:
+            if K.kvq_get_status(c):
+                raise RuntimeError("cache status set after the graph-replayed steps")
+        graph = {"ms": g_ms, "tokens": w.B * layers * sum(g_tok[n_warm:]), "clk": clk_g}
+        del recs
+
+    # ---- the same step as per-layer calls, with events between the kernels of each layer
     # warm-up
     for s in range(args.warmup):
         for i in range(nL):
             layer_step(i, s, False)
+        for r in range(R):
+            appended[r] += 1
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -468,27 +543,36 @@ def run_kvq(args, rank, world):
     with ClockSampler(dev.index) as clk:
         t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t_start.record()
+        m_tok, m_len = [], []
         for s in range(args.warmup, steps_total):
             rep = s % R
             for i in range(rep * layers, (rep + 1) * layers):
                 marks.append(layer_step(i, s, True))
+            appended[rep] += 1  # the sequence grows (on the last rank when sharded)
+            m_len.append(T0 + appended[rep] if appends_here else T0)
+            m_tok.append(w.B * layers * (shard_n * T0 + appended[rep]) *
+                         (1 if sharded else world))
         t_end.record()
         torch.cuda.synchronize()
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world, dev)
     if world > 1:
         dist.barrier()
     n_layer_steps = len(marks)
-    # KV tokens attended per layer-step over the whole job: replicas, each rank its own
-    # sequence of T0 + s + 1 tokens; sharded, one sequence of N T0 + s + 1 tokens
-    tok_job = [(shard_n * T0 + s + 1) * (1 if sharded else world)
-               for s in range(args.warmup, steps_total) for _ in range(layers)]
-    value = w.B * sum(tok_job) / (elapsed_ms / 1e3)
+    # KV tokens attended over the whole job: replicas, each rank its own sequence; sharded,
+    # one sequence of N T0 + appended tokens
+    m_value = sum(m_tok) / (elapsed_ms / 1e3)
+    if graph is not None:
+        graph["ms"] = max_over_ranks(graph["ms"], world, dev)
+        value = graph["tokens"] * world / (graph["ms"] / 1e3)
+        ms_per_step = graph["ms"] / args.steps
+    else:
+        value, ms_per_step = m_value, elapsed_ms / args.steps
     # per-kernel times
     t_app = sum(m[0].elapsed_time(m[1]) for m in marks)
     t_qk = sum(m[1].elapsed_time(m[2]) for m in marks)
     t_merge = sum(m[2].elapsed_time(m[3]) for m in marks)
     t_pv = sum(m[3].elapsed_time(m[4]) for m in marks)
-    Tmid = T0 + (args.warmup + args.steps // 2 + 1 if appends_here else 0)
+    Tmid = int(round(statistics.mean(m_len)))  # this rank's cache length, mid-region
     bm = bytes_model(w, Tmid, kcount, vcount, "one-call" if sharded else args.path)
     hbm, peak_kind = peaks()
     if args.path == "split" and not sharded:
@@ -502,58 +586,80 @@ def run_kvq(args, rank, world):
     step_attn_ms = (t_qk + t_merge + t_pv) / n_layer_steps
     attn_gbs = bm["total"] / (step_attn_ms / 1e3) / 1e9
 
-    # ---- end-to-end through the public API with host buffers
-    h_q = torch.empty_like(qall, device="cpu").pin_memory()
-    h_k = torch.empty_like(knew, device="cpu").pin_memory()
-    h_v = torch.empty_like(vnew, device="cpu").pin_memory()
-    h_q.copy_(qall)
-    h_k.copy_(knew)
-    h_v.copy_(vnew)
-    h_out = torch.empty((nL, w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
-    d_q = torch.empty((nL, w.B, w.Hq, w.D), dtype=torch.float16, device=dev)
-    d_k = torch.empty((nL, w.B, 1, w.Hkv, w.D), dtype=torch.float16, device=dev)
-    d_v = torch.empty_like(d_k)
-    # the e2e leg appends at fresh positions after the timed steps (replica 0)
-    qpos_e2e = torch.tensor([[pos0 + steps_total + j] * w.B for j in range(e2e_steps)],
-                            dtype=torch.int32, device=dev)
-    torch.cuda.synchronize()
-    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h2d = d2h = 0
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    e_s.record()
+    # ---- end-to-end through the public API with host buffers: every step copies its inputs
+    # from pinned host memory and reads its outputs back (replica 0, fresh positions)
+    e2e_app = []
     for j in range(e2e_steps):
-        s = args.warmup + j
-        ml_len = T0 + steps_total + j + 1 if appends_here else T0
-        d_q.copy_(h_q[:, s], non_blocking=True)
-        d_k.copy_(h_k[:, s], non_blocking=True)
-        d_v.copy_(h_v[:, s], non_blocking=True)
-        for i in range(layers):
-            c = caches[i]
-            if appends_here:
-                K.kvq_quantize_append(c, cbs[i][0], cbs[i][1], d_k[i], d_v[i], 1, None, 0, aws)
-            if sharded:
-                sdec(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j], ml_len, t_base, outs[i], dws, S)
-            elif args.path == "split":
-                K.kvq_decode_qk(c, cbs[i][0], d_q[i], qpos_e2e[j], ml_len, logits, stats, S, qkws)
-                K.kvq_softmax_merge(cfg, stats, S, mlb)
-                K.kvq_decode_pv(c, cbs[i][1], logits, mlb, ml_len, outs[i], part, S)
-            elif args.path == "fused":
-                K.kvq_decode_attention_fused(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j],
-                                             ml_len, outs[i], dws, S)
-            else:
-                K.kvq_decode_attention(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j], ml_len,
-                                       outs[i], dws, S)
-        h_out.copy_(outs, non_blocking=True)
-        h2d = (d_q[:layers].numel() + d_k[:layers].numel() + d_v[:layers].numel()) * 2
-        d2h = h_out[:layers].numel() * 4
-    e_e.record()
-    torch.cuda.synchronize()
+        appended[0] += 1
+        e2e_app.append(appended[0])
+    e2e_tokens = w.B * layers * sum(shard_n * T0 + a for a in e2e_app) * (1 if sharded else world)
+    h_out = torch.empty((layers, w.B, w.Hq, w.D), dtype=torch.float32).pin_memory()
+    e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if graph is not None:
+        h_rec = torch.stack([step_record(args.warmup + j, 0, pos0 + a - 1)
+                             for j, a in enumerate(e2e_app)]).cpu().pin_memory()
+        h2d = h_rec[0].numel()
+        d2h = h_out.numel() * 4
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_s.record()
+        for j in range(e2e_steps):
+            K.kvq_step_launch(gsteps[0], h_rec[j])
+            h_out.copy_(outs[:layers], non_blocking=True)
+        e_e.record()
+        torch.cuda.synchronize()
+    else:
+        h_q = torch.empty_like(qall, device="cpu").pin_memory()
+        h_k = torch.empty_like(knew, device="cpu").pin_memory()
+        h_v = torch.empty_like(vnew, device="cpu").pin_memory()
+        h_q.copy_(qall)
+        h_k.copy_(knew)
+        h_v.copy_(vnew)
+        d_q = torch.empty((layers, w.B, w.Hq, w.D), dtype=torch.float16, device=dev)
+        d_k = torch.empty((layers, w.B, 1, w.Hkv, w.D), dtype=torch.float16, device=dev)
+        d_v = torch.empty_like(d_k)
+        qpos_e2e = torch.tensor([[pos0 + a - 1] * w.B for a in e2e_app], dtype=torch.int32,
+                                device=dev)
+        h2d = (d_q.numel() + d_k.numel() + d_v.numel()) * 2
+        d2h = h_out.numel() * 4
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_s.record()
+        for j in range(e2e_steps):
+            s = args.warmup + j
+            ml_len = T0 + e2e_app[j] if appends_here else T0
+            d_q.copy_(h_q[:layers, s], non_blocking=True)
+            d_k.copy_(h_k[:layers, s], non_blocking=True)
+            d_v.copy_(h_v[:layers, s], non_blocking=True)
+            for i in range(layers):
+                c = caches[i]
+                if appends_here:
+                    K.kvq_quantize_append(c, cbs[i][0], cbs[i][1], d_k[i], d_v[i], 1, None, 0,
+                                          aws)
+                if sharded:
+                    sdec(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j], ml_len, t_base, outs[i],
+                         dws, S)
+                elif args.path == "split":
+                    K.kvq_decode_qk(c, cbs[i][0], d_q[i], qpos_e2e[j], ml_len, logits, stats, S,
+                                    qkws)
+                    K.kvq_softmax_merge(cfg, stats, S, mlb)
+                    K.kvq_decode_pv(c, cbs[i][1], logits, mlb, ml_len, outs[i], part, S)
+                elif args.path == "fused":
+                    K.kvq_decode_attention_fused(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j],
+                                                 ml_len, outs[i], dws, S)
+                else:
+                    K.kvq_decode_attention(c, cbs[i][0], cbs[i][1], d_q[i], qpos_e2e[j], ml_len,
+                                           outs[i], dws, S)
+            h_out.copy_(outs[:layers], non_blocking=True)
+        e_e.record()
+        torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e_s.elapsed_time(e_e), world, dev)
-    e2e_tokens = w.B * sum((shard_n * T0 + steps_total + j + 1) * (1 if sharded else world)
-                           for j in range(e2e_steps)) * layers
     e2e_value = e2e_tokens / (e2e_ms / 1e3)
+    if graph is not None:
+        for st in gsteps:
+            K.kvq_step_destroy(st)
 
     # ---- uncompressed fp16 comparison kernel on one layer (last staged K/V)
     fp16 = None
@@ -596,16 +702,19 @@ def run_kvq(args, rank, world):
 
     if rank != 0:
         return 0
-    # append: begin, stats, scan, write; split kernels: qk (tables, qk, key outliers, split
-    # stats), merge, pv (pv, value outliers, split sum); fused: tables, fused kernel, merge;
-    # sharded: the split kernels and the conversion to a partial, then one merge of the
-    # gathered partials
+    # append of one token: the short-append kernel (up to 32 kv heads), else begin, statistics,
+    # scan, write, final; split kernels: qk (tables, qk, key outliers, split stats), merge, pv
+    # (pv, value outliers, split sum); fused: tables, fused kernel, merge; sharded: the split
+    # kernels and the conversion to a partial, then one merge of the gathered partials.  The
+    # graph replays exactly these launches.
     fused_path = args.path == "fused" and not sharded
-    launches_per_layer_step = (4 if appends_here else 0) + (3 if fused_path else 8) + (
-        2 if sharded else 0)
+    launches_per_layer_step = ((1 if w.Hkv <= 32 else 5) if appends_here else 0) + (
+        3 if fused_path else 8) + (2 if sharded else 0)
+    per_layer_calls = {"value": m_value, "ms_per_step": elapsed_ms / args.steps,
+                       "clocks": clk.summary()}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded Philox4x32-10; LLaMA-7B-shaped K/V distributions)",
         "config": {"workload": w.name, "layers": layers, "B": w.B, "q_heads": w.Hq,
@@ -613,6 +722,10 @@ def run_kvq(args, rank, world):
                    "outlier_frac": w.f, "rope_theta": w.rope_theta,
                    "path": "sharded (partial + all-gather + merge)" if sharded else args.path,
                    "splits": S, "cache_replicas": R,
+                   "step": ("one CUDA graph per step: every layer's append + attention "
+                            "(kvq_step_create / kvq_step_launch; the step's packed inputs "
+                            "copied in by each launch)") if graph is not None
+                           else "per-layer calls",
                    "parallelism": (f"token-sharded x{world}: one sequence of {shard_n * T0} "
                                    "tokens, rank r holding [r T, (r+1) T)") if sharded
                                   else (f"replicas x{world}" if world > 1 else "1 GPU"),
@@ -633,8 +746,9 @@ def run_kvq(args, rank, world):
                 "d2h_bytes_per_step": d2h},
         "fp16_attention": fp16,
         "cpu_baseline": cpu,
+        "per_layer_calls": per_layer_calls if graph is not None else None,
         "gpu_launches": launches_per_layer_step * n_layer_steps,
-        "clocks": clk.summary(),
+        "clocks": graph["clk"].summary() if graph is not None else clk.summary(),
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -17,8 +17,9 @@
  * Conventions (every entry point):
  *   - Buffers are DEVICE pointers owned by the caller unless a parameter says
  *     "host".  Cache and workspace buffers must be 16-byte aligned.  The library
- *     allocates no memory; its only global state is the fixed scratch array of
- *     kvq_quantize_append_noalloc and the per-thread text of the last CUDA error.
+ *     allocates no device buffer; its only global state is the fixed scratch array of
+ *     kvq_quantize_append_noalloc and the per-thread text of the last CUDA error
+ *     (a kvq_step owns host memory and an instantiated CUDA graph).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
  *     Calls only enqueue work; none synchronizes except kvq_get_status.
  *   - Return value: KVQ_OK (0) or a negative KVQ_ERR_* code.  Argument checks are
@@ -381,6 +382,76 @@ int kvq_quantize_append_noalloc(const kvq_cfg* cfg, const kvq_cache* cache,
                                 const kvq_codebook* cbK, const kvq_codebook* cbV,
                                 const uint16_t* k, const uint16_t* v, int32_t n_new,
                                 const int32_t* plen, void* stream);
+
+/*
+ * Whole-model decode step as one CUDA graph.  The pages use the cache for token-by-token
+ * generation over a long context on one GPU (study.space summary: LLaMA-7B served with a
+ * context of a million tokens on a single GPU; phantomic12 research note, the paper's own
+ * claim): for every generated token, every layer appends that token's key and value to its
+ * cache and attends over the whole cache.  kvq_step_create records that step for `layers`
+ * caches in one CUDA graph -- for l = 0 .. layers-1 in order, kvq_quantize_append
+ * (calibrate = 0) of n_new tokens per sequence into caches[l] (nothing when n_new = 0), then
+ * kvq_decode_attention (kvq_decode_attention_fused when desc->fused = 1) over caches[l] into
+ * out[l] -- and kvq_step_launch replays it: one graph launch in place of about ten kernel
+ * launches per layer.  A launch gives the same bits as those calls made one by one on the
+ * same inputs.  (The layers' query, key and value inputs arrive together; the projections
+ * that would produce them from the previous layer are model code, outside this library.)
+ *
+ * Inputs of a launch: one packed record of kvq_step_input_bytes bytes, which
+ * kvq_step_launch copies into desc->inputs (the graph reads its inputs only there):
+ *   for l = 0 .. layers-1:  k fp16 [B][n_new][Hkv][D], v fp16 [B][n_new][Hkv][D],
+ *                           q fp16 [B][Hq][D]   (each part a multiple of 256 bytes)
+ *   then qpos int32 [B] (each sequence's query position), padded to 16 bytes.
+ * Each launch advances len[b] of every cache by n_new on the device.  desc->max_len sizes
+ * the grids once, at create: it must bound len[b] after the append at every launch (a
+ * longer sequence is clipped and sets KVQ_STATUS_LEN_OVERFLOW, as in kvq_decode_qk), and a
+ * max_len far above the actual lengths costs empty splits.  Launches of one step share
+ * desc->inputs, desc->out and the workspace: issue them on one stream, in order.
+ */
+typedef struct kvq_step kvq_step; /* opaque: the instantiated graph and its buffers */
+
+typedef struct kvq_step_desc {
+    int32_t layers;              /* 1 .. 4096 */
+    const kvq_cache* caches;     /* host array [layers]; read during kvq_step_create only */
+    const kvq_codebook* cbK;     /* host array [layers] (key datatypes) */
+    const kvq_codebook* cbV;     /* host array [layers] (value datatypes) */
+    int32_t n_new;               /* tokens appended per sequence and launch, 0 .. T_max */
+    int32_t max_len;             /* 1 .. T_max, see above */
+    int32_t splits;              /* as for kvq_decode_attention (0 = the library's choice) */
+    int32_t fused;               /* 0 or 1 (kvq_decode_attention_fused) */
+    void* inputs;                /* device, kvq_step_input_bytes bytes, 16-byte aligned */
+    float* out;                  /* device float [layers][B][Hq][D], 16-byte aligned */
+    void* workspace;             /* device scratch of kvq_step_workspace bytes, 16-byte aligned */
+    size_t workspace_bytes;
+} kvq_step_desc;
+
+/* Bytes of one packed input record. */
+int kvq_step_input_bytes(const kvq_cfg* cfg, int32_t layers, int32_t n_new, size_t* bytes);
+
+/* Workspace bytes of a step: the append's scratch, then the attention's (layers share both,
+ * since the recorded calls run one after another). */
+int kvq_step_workspace(const kvq_cfg* cfg, int32_t n_new, int32_t max_len, int32_t splits,
+                       int32_t fused, size_t* bytes);
+
+/*
+ * Record and instantiate the step.  Every recorded call checks its arguments here; on an
+ * error the code is returned, *step is NULL and nothing has run on the GPU (recording runs
+ * nothing).  The step owns host memory and the instantiated graph until kvq_step_destroy;
+ * the library allocates no device buffer for it.  Must not be called while another stream
+ * capture is in progress on the calling thread.
+ */
+int kvq_step_create(const kvq_cfg* cfg, const kvq_step_desc* desc, kvq_step** step);
+
+/*
+ * One step: copy the packed record `inputs` (host or device memory; NULL if the caller has
+ * already written desc->inputs) into desc->inputs with cudaMemcpyAsync on `stream`, then
+ * launch the graph on `stream`.  Enqueue only (a pageable host record is copied before the
+ * call returns; a pinned one asynchronously, so keep it unchanged until the step completes).
+ */
+int kvq_step_launch(kvq_step* step, const void* inputs, void* stream);
+
+/* Release the step.  Call it after the step's launches have completed. */
+int kvq_step_destroy(kvq_step* step);
 
 /* Read the sticky status word into *out (host).  Synchronizes `stream`. */
 int kvq_get_status(const kvq_cache* cache, int32_t* out, void* stream);

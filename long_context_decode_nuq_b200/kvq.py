@@ -30,6 +30,8 @@ EXPORTS = (
     "kvq_dequantize", "kvq_fp16_decode_attention", "kvq_fit_workspace", "kvq_fit_codebook",
     "kvq_get_status", "kvq_quantize_append_noalloc", "kvq_decode_partial", "kvq_merge_partials",
     "kvq_decode_attention_fused", "kvq_decode_fused_workspace",
+    "kvq_step_input_bytes", "kvq_step_workspace", "kvq_step_create", "kvq_step_launch",
+    "kvq_step_destroy",
 )
 
 
@@ -60,6 +62,14 @@ class CodebookStruct(ctypes.Structure):
 
 class Sizes(ctypes.Structure):
     _fields_ = [(f, c_size_t) for f in _CACHE_FIELDS]
+
+
+class StepDesc(ctypes.Structure):
+    _fields_ = [("layers", c_int32), ("caches", POINTER(CacheStruct)),
+                ("cbK", POINTER(CodebookStruct)), ("cbV", POINTER(CodebookStruct)),
+                ("n_new", c_int32), ("max_len", c_int32), ("splits", c_int32), ("fused", c_int32),
+                ("inputs", c_void_p), ("out", c_void_p), ("workspace", c_void_p),
+                ("workspace_bytes", c_size_t)]
 
 
 _lib = None
@@ -116,6 +126,12 @@ def load():
         "kvq_quantize_append_noalloc": ([POINTER(Cfg), POINTER(CacheStruct),
                                          POINTER(CodebookStruct), POINTER(CodebookStruct), P, P,
                                          c_int32, P, P], c_int),
+        "kvq_step_input_bytes": ([POINTER(Cfg), c_int32, c_int32, POINTER(c_size_t)], c_int),
+        "kvq_step_workspace": ([POINTER(Cfg), c_int32, c_int32, c_int32, c_int32,
+                                POINTER(c_size_t)], c_int),
+        "kvq_step_create": ([POINTER(Cfg), POINTER(StepDesc), POINTER(c_void_p)], c_int),
+        "kvq_step_launch": ([P, P, P], c_int),
+        "kvq_step_destroy": ([P], c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -340,6 +356,60 @@ def kvq_quantize_append_noalloc(cache: Cache, cbK: Codebook, cbV: Codebook, k, v
         ctypes.byref(cache.cfg), ctypes.byref(cache.struct), ctypes.byref(cbK.struct),
         ctypes.byref(cbV.struct), _ptr(k), _ptr(v), n_new, _ptr(plen), _stream(stream)),
         "kvq_quantize_append_noalloc")
+
+
+def kvq_step_input_bytes(cfg: Cfg, layers: int, n_new: int) -> int:
+    b = c_size_t()
+    _check(load().kvq_step_input_bytes(ctypes.byref(cfg), layers, n_new, ctypes.byref(b)),
+           "kvq_step_input_bytes")
+    return b.value
+
+
+def kvq_step_workspace(cfg: Cfg, n_new: int, max_len: int, splits: int = 0,
+                       fused: int = 0) -> int:
+    b = c_size_t()
+    _check(load().kvq_step_workspace(ctypes.byref(cfg), n_new, max_len, splits, fused,
+                                     ctypes.byref(b)), "kvq_step_workspace")
+    return b.value
+
+
+class Step:
+    """Handle of a recorded whole-model step (kvq_step_create); keeps its buffers alive."""
+
+    def __init__(self, handle, keep):
+        self.handle = handle
+        self._keep = keep
+
+    def destroy(self) -> None:
+        if self.handle:
+            _check(load().kvq_step_destroy(self.handle), "kvq_step_destroy")
+            self.handle = None
+
+
+def kvq_step_create(cfg: Cfg, caches, cbK, cbV, n_new: int, max_len: int, inputs, out,
+                    workspace, splits: int = 0, fused: int = 0) -> Step:
+    """caches, cbK, cbV: one Cache / Codebook per layer, in layer order."""
+    L = len(caches)
+    carr = (CacheStruct * L)(*[c.struct for c in caches])
+    karr = (CodebookStruct * L)(*[c.struct for c in cbK])
+    varr = (CodebookStruct * L)(*[c.struct for c in cbV])
+    desc = StepDesc(L, carr, karr, varr, n_new, max_len, splits, fused, inputs.data_ptr(),
+                    out.data_ptr(), workspace.data_ptr(),
+                    workspace.numel() * workspace.element_size())
+    h = c_void_p()
+    _check(load().kvq_step_create(ctypes.byref(cfg), ctypes.byref(desc), ctypes.byref(h)),
+           "kvq_step_create")
+    return Step(h, (inputs, out, workspace, list(caches), list(cbK), list(cbV)))
+
+
+def kvq_step_launch(step: Step, inputs=None, stream=None) -> None:
+    """inputs: a packed input record (host or device tensor), or None if already in place."""
+    _check(load().kvq_step_launch(step.handle, _ptr(inputs), _stream(stream)),
+           "kvq_step_launch")
+
+
+def kvq_step_destroy(step: Step) -> None:
+    step.destroy()
 
 
 def kvq_get_status(cache: Cache, stream=None) -> int:

@@ -107,3 +107,48 @@ def test_noalloc_append_argument_errors_without_gpu():
     rc = lib.kvq_quantize_append_noalloc(ctypes.byref(cfg), ctypes.byref(fake), ctypes.byref(cb),
                                          ctypes.byref(cb), 0x1000, 0x1000, 257, null, null)
     assert rc == -5
+
+
+def test_step_sizes_and_argument_errors_without_gpu():
+    """The whole-model step's record size is the closed form of its packed layout, and bad
+    descriptors are refused before any CUDA call."""
+    lib = K.load()
+    cfg = K.make_cfg(2, 8, 4, 3, 512, 0.01, 1e4, 64, 64)
+    # per layer: k and v fp16 [B][n_new][Hkv][D], q fp16 [B][Hq][D]; then qpos int32 [B]
+    # padded to 16 bytes
+    assert K.kvq_step_input_bytes(cfg, 3, 1) == 3 * (2 * 2 * 1 * 4 * 128 * 2 + 2 * 8 * 128 * 2) + 16
+    assert K.kvq_step_input_bytes(cfg, 1, 0) == 2 * 8 * 128 * 2 + 16
+    assert K.kvq_step_input_bytes(cfg, 2, 5) == 2 * (2 * 2 * 5 * 4 * 128 * 2 + 2 * 8 * 128 * 2) + 16
+    ws = K.kvq_step_workspace(cfg, 1, 400)
+    assert ws >= K.kvq_decode_workspace(cfg, 400, 0)
+    assert ws >= K.kvq_quantize_workspace(cfg, 1, 0)
+    assert K.kvq_step_workspace(cfg, 0, 400) == K.kvq_decode_workspace(cfg, 400, 0)
+    n = ctypes.c_size_t()
+    assert lib.kvq_step_input_bytes(ctypes.byref(cfg), 0, 1, ctypes.byref(n)) == -3
+    assert lib.kvq_step_input_bytes(ctypes.byref(cfg), 1, -1, ctypes.byref(n)) == -3
+    assert lib.kvq_step_workspace(ctypes.byref(cfg), 1, 400, 0, 2, ctypes.byref(n)) == -3
+    # fused attention needs one query head per kv head
+    assert lib.kvq_step_workspace(ctypes.byref(cfg), 1, 400, 0, 1, ctypes.byref(n)) == -4
+
+    caches = (K.CacheStruct * 1)()
+    cbs = (K.CodebookStruct * 1)()
+    h = ctypes.c_void_p()
+
+    def desc(**kw):
+        d = dict(layers=1, caches=caches, cbK=cbs, cbV=cbs, n_new=1, max_len=400, splits=0,
+                 fused=0, inputs=0x10000, out=0x20000, workspace=0x30000, workspace_bytes=ws)
+        d.update(kw)
+        return K.StepDesc(**d)
+
+    def create(d):
+        return lib.kvq_step_create(ctypes.byref(cfg), ctypes.byref(d), ctypes.byref(h))
+
+    assert lib.kvq_step_create(ctypes.byref(cfg), None, ctypes.byref(h)) == -1
+    assert create(desc(inputs=None)) == -1 and h.value is None
+    assert create(desc(out=0x20004)) == -2
+    assert create(desc(workspace=0x30008)) == -2
+    assert create(desc(layers=0)) == -3
+    assert create(desc(max_len=600)) < 0      # past T_max
+    assert create(desc(workspace_bytes=ws - 16)) == -6
+    assert lib.kvq_step_launch(None, None, None) == -1
+    assert lib.kvq_step_destroy(None) == -1
