@@ -403,7 +403,7 @@ __host__ __device__ inline QQPlan qq_plan(int bits) {
     int o = 0;
     p.stage = kQQuads * 16 * bits * 4;                       // code blocks of 64 quads
     p.ring = o;  o += kStages * p.stage;
-    p.base = o;  o += kStages * 64 * 16;                     // [stage][pair] (c, c, s, s) at stage start
+    p.base = o;  o += kStages * 64 * 8;                      // [stage][pair] (cos, sin) at stage start
     p.lev = o;   o += 16 * 4;                                // codebook levels
     p.bar = o;   o += 2 * kStages * 8;
     p.flag = o;  o += 16;
@@ -429,7 +429,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
     const uint32_t tpos = (sbase + L.pre + L.jslice - 1) & ~(uint32_t)(L.jslice - 1);
     uint8_t* tab = sm + (tpos - sbase);
     uint8_t* ring = sm + L.ring;
-    float4* base = (float4*)(sm + L.base);
+    float2* base = (float2*)(sm + L.base);
     float* lev = (float*)(sm + L.lev);
     uint64_t* full = (uint64_t*)(sm + L.bar);
     uint64_t* empty = full + kStages;
@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const float2 cs = trig_at(thi, tlo, tc, pl + 32 * u);
-                base[slot * 64 + pl + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
+                base[slot * 64 + pl + 32 * u] = cs;
             }
             __syncwarp();
             __threadfence_block();
@@ -530,18 +530,14 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 #pragma unroll
         for (int sl = 0; sl < 4; ++sl)
             lb[sl] = tpos + ((uint32_t)(sl ^ x) << JS) + ((uint32_t)i << 3);
-        // phase from the stage start to the quad, pair i + 16 k, as (c, s) and (-s, c)
-        unsigned long long RQ[2][4], RQp[2][4];
+        // phase from the stage start to the quad, pair i + 16 k, as (c, s)
+        float2 RQ[2][4];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             const int q = qbase + 2 * (u ^ uperm);
             woff[u] = (uint32_t)(q * F::BW + i * BITS) * 4;
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float2 r = tlo[(4 * q) * 64 + i + 16 * k];
-                RQ[u][k] = pk(r.x, r.y);
-                RQp[u][k] = pk(-r.y, r.x);
-            }
+            for (int k = 0; k < 4; ++k) RQ[u][k] = tlo[(4 * q) * 64 + i + 16 * k];
         }
         const int tq = 4 * (qbase + 2 * uperm) + x;
         float* lrow = logits + ((size_t)b * Hq + hq) * cfg.T_max;
@@ -559,13 +555,10 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 #pragma unroll
                 for (int d = 0; d < BITS; ++d)
                     w[u][d] = *reinterpret_cast<const uint32_t*>(stage + woff[u] + 4 * d);
-            unsigned long long Bc[4], Bs[4];
+            // the stage start's (cos, sin) of pairs i + 16 k: one 8-byte read per pair
+            float2 B[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float4 bq = base[slot * 64 + i + 16 * k];
-                Bc[k] = pk(bq.x, bq.y);
-                Bs[k] = pk(bq.z, bq.w);
-            }
+            for (int k = 0; k < 4; ++k) B[k] = base[slot * 64 + i + 16 * k];
             __syncwarp();
             if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
             unsigned long long acc[4][2];
@@ -575,8 +568,10 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
             for (int u = 0; u < 2; ++u) {
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    // (c_b c_q - s_b s_q, c_b s_q + s_b c_q) in two packed instructions
-                    const unsigned long long Pc = fma2(Bc[k], RQ[u][k], mul2(Bs[k], RQp[u][k]));
+                    // (c_b c_q - s_b s_q, c_b s_q + s_b c_q)
+                    const float2 r = RQ[u][k];
+                    const unsigned long long Pc = pk(fmaf(B[k].x, r.x, -B[k].y * r.y),
+                                                     fmaf(B[k].x, r.y, B[k].y * r.x));
 #pragma unroll
                     for (int sl = 0; sl < 4; ++sl) {
                         uint32_t fs;
@@ -648,7 +643,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
     const uint32_t tpos = (sbase + L.pre + L.jslice - 1) & ~(uint32_t)(L.jslice - 1);
     uint8_t* tab = sm + (tpos - sbase);
     uint8_t* ring = sm + L.ring;
-    float4* base = (float4*)(sm + L.base);
+    float2* base = (float2*)(sm + L.base);
     float* lev = (float*)(sm + L.lev);
     uint64_t* full = (uint64_t*)(sm + L.bar);
     uint64_t* empty = full + kStages;
@@ -718,7 +713,7 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
                 const float2 cs = trig_at(thi, tlo, tc, pl + 32 * u);
-                base[slot * 64 + pl + 32 * u] = make_float4(cs.x, cs.x, cs.y, cs.y);
+                base[slot * 64 + pl + 32 * u] = cs;
             }
             __syncwarp();
             __threadfence_block();
@@ -770,9 +765,9 @@ __global__ void __launch_bounds__(kQWarps * 32 + 32, 1)
             float bc[4], bs[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const float4 bq = base[slot * 64 + i + 16 * k];
+                const float2 bq = base[slot * 64 + i + 16 * k];
                 bc[k] = bq.x;
-                bs[k] = bq.z;
+                bs[k] = bq.y;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty + slot);  // the stage may be refilled
