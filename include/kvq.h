@@ -437,8 +437,10 @@ int kvq_step_workspace(const kvq_cfg* cfg, int32_t n_new, int32_t max_len, int32
  * Record and instantiate the step.  Every recorded call checks its arguments here; on an
  * error the code is returned, *step is NULL and nothing has run on the GPU (recording runs
  * nothing).  The step owns host memory and the instantiated graph until kvq_step_destroy;
- * the library allocates no device buffer for it.  Must not be called while another stream
- * capture is in progress on the calling thread.
+ * the library allocates no device buffer for it.  The graph is recorded (by stream capture in
+ * relaxed mode, on a stream the call creates and destroys) for the calling thread's current
+ * CUDA device, which must hold every buffer the descriptor names; launch it on a stream of
+ * that device.
  */
 int kvq_step_create(const kvq_cfg* cfg, const kvq_step_desc* desc, kvq_step** step);
 
