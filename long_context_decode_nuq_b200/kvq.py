@@ -390,6 +390,9 @@ def kvq_step_create(cfg: Cfg, caches, cbK, cbV, n_new: int, max_len: int, inputs
                     workspace, splits: int = 0, fused: int = 0) -> Step:
     """caches, cbK, cbV: one Cache / Codebook per layer, in layer order."""
     L = len(caches)
+    if len(cbK) != L or len(cbV) != L:
+        raise ValueError(f"kvq_step_create: {L} caches but {len(cbK)} key and {len(cbV)} value "
+                         "codebooks")
     carr = (CacheStruct * L)(*[c.struct for c in caches])
     karr = (CodebookStruct * L)(*[c.struct for c in cbK])
     varr = (CodebookStruct * L)(*[c.struct for c in cbV])

@@ -152,3 +152,15 @@ def test_step_sizes_and_argument_errors_without_gpu():
     assert create(desc(workspace_bytes=ws - 16)) == -6
     assert lib.kvq_step_launch(None, None, None) == -1
     assert lib.kvq_step_destroy(None) == -1
+
+
+def test_step_binding_checks_layer_lists():
+    """The binding refuses per-layer lists of different lengths before calling the library."""
+    cfg = K.make_cfg(1, 4, 4, 3, 256, 0.01, 1e4, 64, 64)
+
+    class _Fake:
+        struct = K.CacheStruct()
+
+    with pytest.raises(ValueError):
+        K.kvq_step_create(cfg, [_Fake(), _Fake()], [_Fake()], [_Fake(), _Fake()], 1, 200,
+                          None, None, None)
